@@ -1,0 +1,230 @@
+"""Pins for the oracle's KV-size arithmetic and decode attention.
+
+Each test ties the oracle to something other than itself: numbers printed on
+the pages (tests/golden), closed forms, invariants the method states, a
+brute-force loop written independently, or torch's own attention routine.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as A
+from oracle import kv_size as K
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- KV size --
+
+def test_worked_example_llama2_7b_4k():
+    g = _golden("kv_size_worked_example.json")
+    got = K.kv_cache_bytes(g["n_layers"], g["n_kv_heads"], g["head_dim"], g["seq_len"],
+                           g["batch"], g["bytes_per_elt"])
+    assert got == g["kv_bytes"]
+
+
+def test_worked_example_batch16_is_32gb():
+    g = _golden("kv_size_worked_example.json")
+    got = K.kv_cache_bytes(g["n_layers"], g["n_kv_heads"], g["head_dim"], g["seq_len"],
+                           g["batch16"], g["bytes_per_elt"])
+    assert got == g["batch16_kv_gb_printed"] * 2 ** 30
+
+
+def test_decode_bound_about_140():
+    g = _golden("decode_bound.json")
+    v = K.decode_tokens_per_s_bound(g["bandwidth_gb_s"], g["weights_gb"])
+    assert abs(v - g["printed_tokens_per_s_approx"]) < 5
+
+
+def test_paged_waste_below_one_block():
+    # "at most one block is wasted per sequence" (LLM 推理优化深度解析, §PagedAttention table)
+    for n in range(0, 2000):
+        w = K.paged_waste_tokens(n)
+        assert 0 <= w < 16
+        assert K.paged_blocks_needed(n) * 16 >= n
+
+
+def test_gqa_shrinks_kv_by_group_factor():
+    # 32 q heads over 8 KV heads cut the cache 4x (LLM 推理优化深度解析, §MQA 与 GQA)
+    mha = K.kv_cache_bytes(32, 32, 128, 4096)
+    gqa = K.kv_cache_bytes(32, 8, 128, 4096)
+    mqa = K.kv_cache_bytes(32, 1, 128, 4096)
+    assert mha == 4 * gqa and mha == 32 * mqa
+
+
+# ------------------------------------------------------------- attention --
+
+def _scatter(K_log, perm_blocks, bs=16):
+    """Place logical [ctx, H, D] rows into a pool so that logical block j lives
+    in physical block perm_blocks[j] (test-side helper)."""
+    ctx, H, D = K_log.shape
+    nb = int(max(perm_blocks)) + 1
+    pool = np.full((nb, H, bs, D), np.nan)
+    for j in range(ctx):
+        pool[perm_blocks[j // bs], :, j % bs, :] = K_log[j]
+    return pool
+
+
+def _brute(q, K_log, V_log, scale):
+    """Triple loop with math.exp, no numpy reductions."""
+    Hq, D = len(q), len(q[0])
+    ctx, Hkv = len(K_log), len(K_log[0])
+    G = Hq // Hkv
+    out = []
+    for i in range(Hq):
+        h = i // G
+        logits = []
+        for j in range(ctx):
+            acc = 0.0
+            for d in range(D):
+                acc += q[i][d] * K_log[j][h][d]
+            logits.append(scale * acc)
+        mx = max(logits)
+        w = [math.exp(x - mx) for x in logits]
+        tot = sum(w)
+        row = []
+        for d in range(D):
+            acc = 0.0
+            for j in range(ctx):
+                acc += w[j] / tot * V_log[j][h][d]
+            row.append(acc)
+        out.append(row)
+    return np.array(out)
+
+
+@pytest.mark.parametrize("ctx,hq,hkv,d", [(1, 2, 1, 4), (15, 4, 2, 8), (16, 2, 2, 8),
+                                          (17, 4, 1, 8), (40, 8, 2, 4)])
+def test_paged_equals_contiguous_bitwise(ctx, hq, hkv, d):
+    rng = np.random.default_rng(ctx * 100 + hq)
+    K_log = rng.standard_normal((ctx, hkv, d))
+    V_log = rng.standard_normal((ctx, hkv, d))
+    q = rng.standard_normal((1, hq, d))
+    nblk = (ctx + 15) // 16
+    perm = rng.permutation(nblk + 3)[:nblk]
+    kc, vc = _scatter(K_log, perm), _scatter(V_log, perm)
+    bt = np.array([perm])
+    paged = A.paged_decode_attention(q, kc, vc, bt, [ctx], 0.3)
+    contig = A.contiguous_attention(q[0], K_log, V_log, 0.3)
+    assert np.array_equal(paged[0], contig)
+
+
+def test_block_permutation_invariance():
+    rng = np.random.default_rng(7)
+    nb, hkv, d, hq = 12, 2, 8, 4
+    kc = rng.standard_normal((nb, hkv, 16, d))
+    vc = rng.standard_normal((nb, hkv, 16, d))
+    q = rng.standard_normal((2, hq, d))
+    bt = np.array([[3, 7, 1, 0], [5, 2, 9, 11]])
+    ctx = [50, 61]
+    ref = A.paged_decode_attention(q, kc, vc, bt, ctx, 0.5)
+    perm = rng.permutation(nb)            # new physical position of old block b is perm[b]
+    kc2 = np.empty_like(kc)
+    vc2 = np.empty_like(vc)
+    kc2[perm] = kc
+    vc2[perm] = vc
+    got = A.paged_decode_attention(q, kc2, vc2, perm[bt], ctx, 0.5)
+    assert np.array_equal(ref, got)
+
+
+@pytest.mark.parametrize("ctx,hq,hkv,d", [(1, 2, 2, 3), (7, 4, 2, 8), (16, 2, 1, 4),
+                                          (33, 6, 3, 5), (40, 8, 8, 2)])
+def test_against_brute_force(ctx, hq, hkv, d):
+    rng = np.random.default_rng(1 + ctx + d)
+    K_log = rng.standard_normal((ctx, hkv, d))
+    V_log = rng.standard_normal((ctx, hkv, d))
+    q = rng.standard_normal((hq, d))
+    nblk = (ctx + 15) // 16
+    perm = rng.permutation(nblk)
+    got = A.paged_decode_attention(q[None], _scatter(K_log, perm), _scatter(V_log, perm),
+                                   np.array([perm]), [ctx], 0.7)[0]
+    ref = _brute(q.tolist(), K_log.tolist(), V_log.tolist(), 0.7)
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("hq,hkv", [(8, 8), (8, 2), (4, 1)])
+def test_against_torch_sdpa(hq, hkv):
+    ctx, d = 100, 16
+    g = torch.Generator().manual_seed(11)
+    K_log = torch.randn(ctx, hkv, d, generator=g, dtype=torch.float64)
+    V_log = torch.randn(ctx, hkv, d, generator=g, dtype=torch.float64)
+    q = torch.randn(hq, d, generator=g, dtype=torch.float64)
+    scale = 1 / math.sqrt(d)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q[:, None, :], K_log.permute(1, 0, 2), V_log.permute(1, 0, 2),
+        scale=scale, enable_gqa=True)[:, 0, :]
+    perm = np.arange(7)[::-1]
+    got = A.paged_decode_attention(q.numpy()[None], _scatter(K_log.numpy(), perm),
+                                   _scatter(V_log.numpy(), perm), np.array([perm]), [ctx], scale)[0]
+    np.testing.assert_allclose(got, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_ctx1_returns_v0_exactly():
+    rng = np.random.default_rng(3)
+    kc = rng.standard_normal((4, 2, 16, 8))
+    vc = rng.standard_normal((4, 2, 16, 8))
+    q = rng.standard_normal((1, 4, 8)) * 100
+    out = A.paged_decode_attention(q, kc, vc, np.array([[2]]), [1], 1.0)
+    assert np.array_equal(out[0, 0], vc[2, 0, 0]) and np.array_equal(out[0, 3], vc[2, 1, 0])
+
+
+def test_identical_keys_give_mean_of_values():
+    rng = np.random.default_rng(4)
+    kc = np.broadcast_to(rng.standard_normal((1, 1, 1, 8)), (3, 1, 16, 8)).copy()
+    vc = rng.standard_normal((3, 1, 16, 8))
+    q = rng.standard_normal((1, 2, 8))
+    ctx = 37
+    out = A.paged_decode_attention(q, kc, vc, np.array([[1, 0, 2]]), [ctx], 0.9)
+    V = np.concatenate([vc[1, 0], vc[0, 0], vc[2, 0]])[:ctx]
+    np.testing.assert_allclose(out[0, 0], V.mean(0), atol=1e-14)
+
+
+def test_one_hot_query_large_scale_selects_argmax_key():
+    rng = np.random.default_rng(5)
+    kc = rng.standard_normal((2, 1, 16, 8))
+    vc = rng.standard_normal((2, 1, 16, 8))
+    q = np.zeros((1, 1, 8))
+    q[0, 0, 3] = 1.0
+    out = A.paged_decode_attention(q, kc, vc, np.array([[1, 0]]), [32], 1e4)
+    K_log = np.concatenate([kc[1, 0], kc[0, 0]])
+    V_log = np.concatenate([vc[1, 0], vc[0, 0]])
+    np.testing.assert_allclose(out[0, 0], V_log[np.argmax(K_log[:, 3])], atol=1e-9)
+
+
+def test_ctx0_gives_zero_row():
+    kc = np.ones((2, 1, 16, 4))
+    out = A.paged_decode_attention(np.ones((2, 1, 4)), kc, kc, np.array([[0], [1]]), [0, 3], 1.0)
+    assert np.all(out[0] == 0) and np.allclose(out[1], 1.0)
+
+
+def test_dequantised_gather_matches_scaled_codes():
+    rng = np.random.default_rng(6)
+    codes = rng.integers(-127, 128, size=(3, 2, 16, 4)).astype(np.int8)
+    sc = rng.random((3, 2, 16)).astype(np.float32)
+    K_log = A.gather_sequence(codes, [2, 0], 20, sc)
+    for j in range(20):
+        b = [2, 0][j // 16]
+        for h in range(2):
+            assert np.array_equal(K_log[j, h], codes[b, h, j % 16].astype(np.float64) * np.float64(sc[b, h, j % 16]))
+
+
+def test_head_sample_matches_full_oracle():
+    rng = np.random.default_rng(8)
+    kc = rng.standard_normal((10, 2, 16, 8))
+    vc = rng.standard_normal((10, 2, 16, 8))
+    q = rng.standard_normal((3, 4, 8))
+    bt = np.array([[0, 1, 2], [3, 4, 5], [9, 8, 7]])
+    ctx = [33, 48, 5]
+    full = A.paged_decode_attention(q, kc, vc, bt, ctx, 0.4)
+    pairs = [(0, 0), (2, 3), (1, 2), (1, 1)]
+    part = A.paged_decode_attention_heads(q, kc, vc, bt, ctx, 0.4, pairs)
+    for n, (s, i) in enumerate(pairs):
+        np.testing.assert_allclose(part[n], full[s, i], rtol=0, atol=1e-14)
