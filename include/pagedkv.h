@@ -1,0 +1,260 @@
+/*
+ * pagedkv.h -- C ABI of libpagedkv.so: paged KV-cache decode for NVIDIA B200
+ * (sm_100a).
+ *
+ * The library implements the data-parallel hot path of PagedAttention: the
+ * KV cache lives in fixed-size physical blocks of 16 tokens, each sequence
+ * owns a block table that maps its logical blocks to physical ones, and
+ * decode attention gathers a sequence's keys and values through that table.
+ * Pages this follows (cited by title and section):
+ *   [P-ASC] ascendai.csdn.net article on KV Cache and PagedAttention,
+ *           §二 核心突破：PagedAttention与虚拟内存 (Fig. 2, copy-on-write),
+ *           §三 进阶优化：KV Cache量化与压缩.
+ *   [P-WIKI] "KV Cache 与 PagedAttention" (ai-infra-wiki), §KV cache 有多大,
+ *           §碎片问题, §三个直接推论 (KV 量化 FP8/INT8).
+ *   [P-WMRH] "大模型推理的KV Cache管理从内存碎片到前缀缓存的优化实战" (wmrh.cn),
+ *           §二 (KVCacheBlock, BlockTable, PagedKVCache.append_slot, copy_prefix),
+ *           §四 (KV quantisation).
+ *   [P-LJT] "LLM 推理优化深度解析：KV Cache、Continuous Batching、PagedAttention
+ *           与量化" (blog.longjiangtao.top), §KV Cache 的本质, §MQA 与 GQA,
+ *           §PagedAttention：vLLM 的显存碎片治理.
+ *
+ * Conventions (every function):
+ *   - returns PKV_OK (0) or a negative PKV_ERR_* code; on error nothing is
+ *     launched and pkv_last_error() holds a message (thread-local);
+ *   - device memory is owned by the caller; the library never allocates or
+ *     frees device memory and never synchronises the stream (except the
+ *     explicitly synchronous pkv_device_status and validation mode);
+ *   - kernels are launched on `stream` (a cudaStream_t; NULL = legacy default
+ *     stream) on the CUDA device that is current for the calling thread;
+ *   - all tensors are dense, row-major, without padding, in the layouts given;
+ *   - block_size must be 16 and head_dim 64 or 128.
+ *
+ * Cache layout (per [P-WMRH] §二 KVCacheBlock: one block stores
+ * [num_heads, block_size, head_dim]):
+ *   k_cache, v_cache : [num_blocks, num_kv_heads, 16, head_dim] of cache_dtype
+ *   k_scale, v_scale : [num_blocks, num_kv_heads, 16] fp32 (quantised caches
+ *                      only; one scale per token and KV head)
+ * Token at flat slot `slot` of KV head h is row cache[slot / 16][h][slot % 16].
+ *
+ * Device-side checks never fault: an out-of-range slot, block id, copy pair or
+ * context length is skipped (or clamped) and a bit is set in a device status
+ * word that pkv_device_status() reads.
+ */
+#ifndef PAGEDKV_H
+#define PAGEDKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------ */
+#define PKV_OK               0
+#define PKV_ERR_INVALID_ARG (-1)  /* bad pointer, size, shape or alignment */
+#define PKV_ERR_UNSUPPORTED (-2)  /* dtype / head_dim / group size not built */
+#define PKV_ERR_NO_BLOCKS   (-3)  /* block allocator out of free blocks     */
+#define PKV_ERR_CUDA        (-4)  /* a CUDA runtime/driver call failed      */
+#define PKV_ERR_NOT_FOUND   (-5)  /* unknown sequence id                    */
+#define PKV_ERR_EXISTS      (-6)  /* sequence id already present            */
+
+/* ---- element types ------------------------------------------------------ */
+#define PKV_F16     0   /* IEEE binary16                                   */
+#define PKV_BF16    1   /* bfloat16                                        */
+#define PKV_I8      2   /* int8 codes, symmetric absmax, range [-127, 127] */
+#define PKV_FP8E4M3 3   /* OCP FP8 E4M3 (e4m3fn) codes, absmax maps to 448 */
+
+/* ---- device status bits (pkv_device_status) ----------------------------- */
+#define PKV_DEV_BAD_SLOT     1u   /* slot >= num_blocks * 16 (write skipped)       */
+#define PKV_DEV_BAD_BLOCK    2u   /* block-table entry outside [0, num_blocks)     */
+#define PKV_DEV_BAD_CONTEXT  4u   /* context_len > max_context_len or table width  */
+#define PKV_DEV_TIMEOUT      8u   /* a bounded wait on a copy barrier gave up      */
+#define PKV_DEV_BAD_PAIR    16u   /* copy pair outside [0, num_blocks)             */
+
+/* Thread-local message describing the last error of this thread. */
+const char* pkv_last_error(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int pkv_version(void);
+
+/*
+ * pkv_kv_cache_write -- slot-mapped write of new tokens' K and V.
+ *   [P-WMRH] §二 append_slot: token_idx lives in logical block
+ *   token_idx // block_size; the slot number slot = physical * 16 + offset
+ *   names that row.  [P-LJT] §KV Cache 的本质: each decode step appends the
+ *   new token's K/V to the cache.
+ * k, v          : device, [num_tokens, num_kv_heads, head_dim] of in_dtype
+ *                 (PKV_F16 or PKV_BF16).
+ * k_cache, v_cache : device, cache layout above, cache_dtype.
+ * k_scale, v_scale : device fp32 scale arrays; required (non-NULL) iff
+ *                 cache_dtype is PKV_I8 or PKV_FP8E4M3, else ignored.
+ * slot_mapping  : device int64 [num_tokens]; -1 skips the token.  Slots of
+ *                 one call must be distinct (duplicates race).
+ * For a 16-bit cache in_dtype must equal cache_dtype and the write is a bit
+ * copy.  For a quantised cache each (token, head) row x is stored as
+ *   a = max|x| (fp32), s = a / 127 (INT8) or a / 448 (FP8), code = round-to-
+ *   nearest-even of x / s (IEEE fp32 division), clamped to +-127 / +-448
+ *   before the e4m3 conversion; a = 0 stores s = 0 and zero codes.
+ * Alignment: k, v, k_cache, v_cache 16 bytes; scales 4 bytes.
+ */
+int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
+                       float* k_scale, float* v_scale,
+                       const int64_t* slot_mapping, int num_tokens,
+                       int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                       int in_dtype, int cache_dtype, void* stream);
+
+/*
+ * pkv_decode_plan -- how pkv_paged_attention_decode will split the work.
+ *   The long-context split (token partitions whose partial softmax results
+ *   are merged by a log-sum-exp reduce) is this library's choice; the pages
+ *   do not prescribe one.
+ * partition_tokens : 0 = automatic, else a multiple of 16 (tokens per
+ *                 partition).  Pass the same value to the decode call.
+ * num_partitions_out, partition_tokens_out : the chosen split (1 partition
+ *                 means a single pass with no workspace).
+ * workspace_bytes_out : device workspace decode needs (0 for one partition).
+ * Depends only on its arguments and the current device's SM count.
+ */
+int pkv_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                    int max_context_len, int cache_dtype, int partition_tokens,
+                    int* num_partitions_out, int* partition_tokens_out,
+                    size_t* workspace_bytes_out);
+
+/* Workspace bytes for the automatic plan (pkv_decode_plan with partition_tokens 0). */
+int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                              int max_context_len, int cache_dtype, size_t* bytes);
+
+/*
+ * pkv_paged_attention_decode -- single-query GQA decode attention through
+ * block tables.
+ *   [P-LJT] §KV Cache 的本质 (one query per step attends to all cached K/V),
+ *   §PagedAttention (logical blocks map to scattered physical blocks),
+ *   §MQA 与 GQA (query head i uses KV head i / (num_q_heads / num_kv_heads)).
+ * For every sequence s and query head i, with h = i / G, G = Hq / Hkv and
+ * K_s[j], V_s[j] the rows of token j < context_lens[s] found through
+ * block_tables[s][j / 16]:
+ *   out[s][i] = sum_j softmax_j(scale * q[s][i] . K_s[j]) V_s[j]
+ * (quantised caches are read as code * scale of that token and head).  A
+ * context length of 0 gives a zero row.
+ * out            : device, [num_seqs, num_q_heads, head_dim] of q_dtype.
+ * q              : device, [num_seqs, num_q_heads, head_dim] of q_dtype
+ *                  (PKV_F16 or PKV_BF16; equal to cache_dtype for 16-bit
+ *                  caches; for quantised caches q is converted to fp16 and
+ *                  must lie within fp16 range).
+ * k_cache, v_cache, k_scale, v_scale : as for pkv_kv_cache_write.
+ * block_tables   : device int32 [num_seqs, max_blocks_per_seq].
+ * context_lens   : device int32 [num_seqs], each in [0, max_context_len] and
+ *                  <= max_blocks_per_seq * 16.
+ * num_blocks     : physical blocks in the pool (entries of block_tables must
+ *                  lie in [0, num_blocks)).
+ * max_context_len: host-side upper bound of context_lens (sizes the grid).
+ * num_q_heads / num_kv_heads = G must be an integer in [1, 16].
+ * partition_tokens: as for pkv_decode_plan.
+ * workspace      : device scratch of at least the planned bytes (may be NULL
+ *                  when the plan has one partition); 16-byte aligned.
+ * Alignment: k_cache, v_cache, scales and workspace 16 bytes; q, out 4 bytes.
+ */
+int pkv_paged_attention_decode(void* out, const void* q,
+                               const void* k_cache, const void* v_cache,
+                               const float* k_scale, const float* v_scale,
+                               const int32_t* block_tables, const int32_t* context_lens,
+                               int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                               int block_size, int num_blocks, int max_blocks_per_seq,
+                               int max_context_len, float scale, int q_dtype, int cache_dtype,
+                               int partition_tokens, void* workspace, size_t workspace_bytes,
+                               void* stream);
+
+/*
+ * pkv_copy_blocks -- copy whole physical blocks (K, V and, for quantised
+ * caches, their scales): for each pair p, block src_dst_pairs[2p+1] becomes a
+ * copy of block src_dst_pairs[2p].  This is the copy behind copy-on-write
+ * prefix sharing ([P-ASC] §二 写时复制; [P-LJT] §意外的收获：prefix sharing).
+ * src_dst_pairs : device int32 [num_pairs, 2].  Destinations must be
+ *                 distinct and no destination may also be a source in the
+ *                 same call (then the result equals copying all pairs at once).
+ * k_scale, v_scale : required iff cache_dtype is quantised.
+ */
+int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale,
+                    const int32_t* src_dst_pairs, int num_pairs,
+                    int num_kv_heads, int head_dim, int block_size, int num_blocks,
+                    int cache_dtype, void* stream);
+
+/*
+ * pkv_device_status -- read (and optionally clear) the device status word of
+ * the current device: an OR of PKV_DEV_* bits set by kernels since the last
+ * clear.  Synchronous (waits for the device).
+ */
+int pkv_device_status(unsigned int* status_out, int clear);
+
+/*
+ * pkv_set_validation -- when on, every launch first copies its index arrays
+ * (slot_mapping, block_tables, context_lens, src_dst_pairs) to the host,
+ * synchronously, and rejects invalid entries with PKV_ERR_INVALID_ARG before
+ * launching anything.  Off by default (the hot path stays asynchronous).
+ * Process-wide.
+ */
+int pkv_set_validation(int on);
+
+/* ======================================================================= *
+ * Host block allocator (CPU only; no device memory).  [P-WMRH] §二:
+ * BlockTable keeps a free list and allocate() pops its end (LIFO), returning
+ * failure when empty; free() pushes back; append_slot() maps logical block
+ * token // 16 and allocates on demand; copy_prefix() lets a child alias the
+ * parent's first ceil(prefix / 16) blocks and bumps their reference counts.
+ * Copy-on-write ([P-ASC] §二; [P-LJT] §prefix sharing): appending into a
+ * block with reference count > 1 takes a fresh block, reports (old, new) for
+ * pkv_copy_blocks and drops the old count; the last holder writes in place.
+ * A handle is not thread-safe; use one per thread or lock around it.
+ * ======================================================================= */
+
+/* Create an allocator over blocks [0, num_blocks).  initial_free_order
+ * (host, may be NULL) gives the free list, popped from its end; NULL means
+ * 0, 1, ..., num_blocks-1 (so block num_blocks-1 is handed out first). */
+int pkv_alloc_create(int num_blocks, int block_size, const int32_t* initial_free_order,
+                     void** handle_out);
+int pkv_alloc_destroy(void* handle);
+
+/* Register an empty sequence. */
+int pkv_seq_add(void* handle, int64_t seq_id);
+
+/* child shares parent's first ceil(prefix_len / 16) blocks and has length
+ * prefix_len (prefix_len = -1: the whole parent). */
+int pkv_seq_fork(void* handle, int64_t parent, int64_t child, int prefix_len);
+
+/* Append n_tokens to a sequence.  slots_out (host int64 [n_tokens]) receives
+ * each token's slot; cow_pairs_out (host int32 [cow_cap, 2]) the (src, dst)
+ * block copies that must run before the tokens are written; num_cow_out their
+ * count.  Transactional: on PKV_ERR_NO_BLOCKS nothing changed. */
+int pkv_seq_append(void* handle, int64_t seq_id, int n_tokens, int64_t* slots_out,
+                   int32_t* cow_pairs_out, int cow_cap, int* num_cow_out);
+
+/* One token for each of n sequences (a decode step), transactional over the
+ * whole batch.  slots_out [n]; cow pairs as above. */
+int pkv_batch_append(void* handle, const int64_t* seq_ids, int n, int64_t* slots_out,
+                     int32_t* cow_pairs_out, int cow_cap, int* num_cow_out);
+
+/* Export block tables (host int32 [n, max_blocks], unused entries 0) and
+ * context lengths (host int32 [n]) of n sequences. */
+int pkv_batch_tables(void* handle, const int64_t* seq_ids, int n, int32_t* block_tables_out,
+                     int max_blocks, int32_t* context_lens_out);
+
+/* Release a sequence: every block's count drops by one; blocks reaching 0
+ * return to the free list in table order. */
+int pkv_seq_free(void* handle, int64_t seq_id);
+
+int pkv_seq_block_table(void* handle, int64_t seq_id, int32_t* out, int cap, int* n_out);
+int pkv_seq_len(void* handle, int64_t seq_id, int* len_out);
+int pkv_block_refcount(void* handle, int32_t block, int* rc_out);
+
+/* Free blocks, blocks shared by more than one sequence, and the longest run
+ * of consecutive free block ids ([P-WMRH] §三 metrics table: fragmentation =
+ * total free / largest contiguous free run). */
+int pkv_alloc_stats(void* handle, int* num_free, int* num_shared, int* largest_free_run);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PAGEDKV_H */

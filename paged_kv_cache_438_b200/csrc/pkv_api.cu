@@ -1,0 +1,448 @@
+// C-ABI entry points of libpagedkv: argument checks, launch planning, TMA
+// tensor maps and kernel launches.  The single CUDA translation unit of the
+// library (the kernels live in the included headers), so the device status
+// word exists once per device.  Compiled without fast-math: the quantising
+// write relies on IEEE fp32 division and round-to-nearest-even.
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <mutex>
+#include <unordered_set>
+#include <vector>
+
+#include "pkv_decode.cuh"
+#include "pkv_error.h"
+#include "pkv_write.cuh"
+
+using pkv::fail;
+using pkv::ok;
+
+namespace {
+
+std::atomic<int> g_validate{0};
+
+bool is16(int dt) { return dt == PKV_F16 || dt == PKV_BF16; }
+bool is8(int dt) { return dt == PKV_I8 || dt == PKV_FP8E4M3; }
+int elt_size(int dt) { return is16(dt) ? 2 : 1; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int cuda_fail(cudaError_t e, const char* what) {
+  return fail(PKV_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// Copies a device array to the host (validation mode only; synchronous).
+template <class T>
+int fetch(std::vector<T>* dst, const T* src, size_t n, cudaStream_t st) {
+  dst->resize(n);
+  if (n == 0) return PKV_OK;
+  cudaError_t e = cudaMemcpyAsync(dst->data(), src, n * sizeof(T), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  return e == cudaSuccess ? PKV_OK : cuda_fail(e, "validation copy");
+}
+
+// ---------------------------------------------------------- tensor maps --
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// 2-D view of a cache: rows of head_dim elements, one row per (block, head,
+// token); box = one 16-token block x (128 bytes or the whole row) with the
+// matching swizzle.
+int make_cache_map(CUtensorMap* map, const void* cache, int head_dim, int elt, long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int row_bytes = head_dim * elt;
+  const int tile_bytes = row_bytes < 128 ? row_bytes : 128;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(tile_bytes / elt), 16u};
+  cuuint32_t estr[2] = {1u, 1u};
+  const CUtensorMapSwizzle swz = tile_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  CUresult r = fn(map, elt == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                  const_cast<void*>(cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled failed (CUresult %d)", static_cast<int>(r));
+  return PKV_OK;
+}
+
+// ------------------------------------------------------------ planning --
+constexpr int kMaxPartitionBlocks = 2048;
+
+struct Plan {
+  int num_partitions;
+  int partition_blocks;
+  size_t workspace;
+};
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Split the token range of each (sequence, KV head) into partitions so that
+// the grid holds enough CTAs to cover all SMs a few times over, with
+// partitions as long as that allows (fewer partials, less per-CTA setup).
+int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int req_tokens, Plan* out) {
+  const int blocks_max = std::max(1, (max_ctx + 15) / 16);
+  int pb;
+  if (req_tokens > 0) {
+    if (req_tokens % 16 != 0) return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d is not a multiple of 16", req_tokens);
+    pb = std::min(req_tokens / 16, blocks_max);
+    if (pb > kMaxPartitionBlocks && pb < blocks_max)
+      return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d exceeds %d", req_tokens, kMaxPartitionBlocks * 16);
+  } else {
+    const long long target = 8LL * 2 * sm_count();  // ~8 waves of 2 resident CTAs per SM
+    const long long pairs = static_cast<long long>(B) * Hkv;
+    pb = 16;
+    while (pb < blocks_max && pairs * ((blocks_max + pb - 1) / pb) > target) pb *= 2;
+    pb = std::min(pb, blocks_max);
+  }
+  if (pb > kMaxPartitionBlocks) pb = kMaxPartitionBlocks;
+  const int np = (blocks_max + pb - 1) / pb;
+  out->num_partitions = np;
+  out->partition_blocks = np == 1 ? std::max(pb, blocks_max) : pb;
+  if (np == 1 && out->partition_blocks > kMaxPartitionBlocks) out->partition_blocks = blocks_max;
+  if (np > 1) {
+    const size_t rows = static_cast<size_t>(B) * Hq * np;
+    out->workspace = align_up(rows * 4, 256) * 2 + rows * static_cast<size_t>(D) * 4;
+  } else {
+    out->workspace = 0;
+  }
+  return PKV_OK;
+}
+
+template <class T>
+int set_smem_once(T* kernel, size_t bytes) {
+  // cudaFuncSetAttribute is per device; remember (device, kernel) pairs done.
+  static std::mutex mu;
+  static std::unordered_set<unsigned long long> done;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const unsigned long long key = (reinterpret_cast<uintptr_t>(kernel) << 8) ^ static_cast<unsigned>(dev);
+  std::lock_guard<std::mutex> lk(mu);
+  if (done.count(key)) return PKV_OK;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
+  done.insert(key);
+  return PKV_OK;
+}
+
+template <int kD, int kCT>
+size_t decode_smem_bytes(int partition_blocks) {
+  using Tr = pkv::DecodeTraits<kD, kCT>;
+  return 1024 + static_cast<size_t>(Tr::kWarps) * Tr::kRing * Tr::kStageBytes + Tr::kWarps * Tr::kRing * 8 +
+         static_cast<size_t>(partition_blocks) * 4;
+}
+
+template <int kD, int kCT, int kNT, bool kQBF16>
+int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, int num_seqs,
+                  cudaStream_t st) {
+  using Tr = pkv::DecodeTraits<kD, kCT>;
+  auto kernel = pkv::paged_decode_kernel<kD, kCT, kNT, kQBF16>;
+  const size_t smem = decode_smem_bytes<kD, kCT>(p.partition_blocks);
+  const size_t smem_max = decode_smem_bytes<kD, kCT>(kMaxPartitionBlocks);
+  int rc = set_smem_once(kernel, smem_max);
+  if (rc != PKV_OK) return rc;
+  dim3 grid(p.num_partitions, p.num_kv_heads, num_seqs);
+  kernel<<<grid, Tr::kWarps * 32, smem, st>>>(km, vm, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  if (p.num_partitions > 1) {
+    constexpr bool kOutBF16 = (kCT == pkv::kI8 || kCT == pkv::kFP8) ? kQBF16 : (kCT == pkv::kBF16);
+    dim3 rgrid(p.num_q_heads, num_seqs);
+    pkv::paged_reduce_kernel<kD, kOutBF16><<<rgrid, kD, 0, st>>>(p);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return cuda_fail(e, "reduce launch");
+  }
+  return PKV_OK;
+}
+
+template <int kD, int kCT>
+int dispatch_nt_q(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, int num_seqs,
+                  bool q_bf16, cudaStream_t st) {
+  const bool nt2 = p.group > 8;
+  if constexpr (kCT == pkv::kI8 || kCT == pkv::kFP8) {
+    if (q_bf16)
+      return nt2 ? launch_decode<kD, kCT, 2, true>(km, vm, p, num_seqs, st)
+                 : launch_decode<kD, kCT, 1, true>(km, vm, p, num_seqs, st);
+    return nt2 ? launch_decode<kD, kCT, 2, false>(km, vm, p, num_seqs, st)
+               : launch_decode<kD, kCT, 1, false>(km, vm, p, num_seqs, st);
+  } else {
+    (void)q_bf16;
+    constexpr bool kQ = (kCT == pkv::kBF16);
+    return nt2 ? launch_decode<kD, kCT, 2, kQ>(km, vm, p, num_seqs, st)
+               : launch_decode<kD, kCT, 1, kQ>(km, vm, p, num_seqs, st);
+  }
+}
+
+template <int kD>
+int dispatch_ct(int ct, const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, int num_seqs,
+                bool q_bf16, cudaStream_t st) {
+  switch (ct) {
+    case PKV_F16: return dispatch_nt_q<kD, pkv::kF16>(km, vm, p, num_seqs, q_bf16, st);
+    case PKV_BF16: return dispatch_nt_q<kD, pkv::kBF16>(km, vm, p, num_seqs, q_bf16, st);
+    case PKV_I8: return dispatch_nt_q<kD, pkv::kI8>(km, vm, p, num_seqs, q_bf16, st);
+    case PKV_FP8E4M3: return dispatch_nt_q<kD, pkv::kFP8>(km, vm, p, num_seqs, q_bf16, st);
+  }
+  return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", ct);
+}
+
+int grid_for(long long work, int per_cta) {
+  const long long ctas = (work + per_cta - 1) / per_cta;
+  const long long cap = 16LL * sm_count();
+  return static_cast<int>(std::max(1LL, std::min(ctas, cap)));
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_set_validation(int on) {
+  g_validate.store(on ? 1 : 0);
+  return ok();
+}
+
+int pkv_device_status(unsigned int* status_out, int clear) {
+  if (!status_out) return fail(PKV_ERR_INVALID_ARG, "status_out is NULL");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_fail(e, "cudaDeviceSynchronize");
+  e = cudaMemcpyFromSymbol(status_out, pkv::g_status, sizeof(unsigned int));
+  if (e != cudaSuccess) return cuda_fail(e, "read status");
+  if (clear) {
+    const unsigned int zero = 0;
+    e = cudaMemcpyToSymbol(pkv::g_status, &zero, sizeof(unsigned int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear status");
+  }
+  return ok();
+}
+
+int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache, float* k_scale, float* v_scale,
+                       const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                       int num_blocks, int in_dtype, int cache_dtype, void* stream) {
+  if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0)
+    return fail(PKV_ERR_INVALID_ARG, "bad sizes (num_tokens %d, num_kv_heads %d, num_blocks %d)", num_tokens,
+                num_kv_heads, num_blocks);
+  if (block_size != 16) return fail(PKV_ERR_UNSUPPORTED, "block_size must be 16 (got %d)", block_size);
+  if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (!is16(in_dtype)) return fail(PKV_ERR_UNSUPPORTED, "input dtype %d (need PKV_F16 or PKV_BF16)", in_dtype);
+  if (is16(cache_dtype) && cache_dtype != in_dtype)
+    return fail(PKV_ERR_UNSUPPORTED, "a 16-bit cache must have the input's dtype");
+  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  if (num_tokens == 0) return ok();
+  if (!k || !v || !k_cache || !v_cache || !slot_mapping) return fail(PKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
+    return fail(PKV_ERR_INVALID_ARG, "k, v and caches must be 16-byte aligned");
+  if (is8(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4)))
+    return fail(PKV_ERR_INVALID_ARG, "quantised caches need k_scale and v_scale");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (g_validate.load()) {
+    std::vector<int64_t> sl;
+    int rc = fetch(&sl, slot_mapping, static_cast<size_t>(num_tokens), st);
+    if (rc != PKV_OK) return rc;
+    std::unordered_set<int64_t> seen;
+    const int64_t lim = static_cast<int64_t>(num_blocks) * 16;
+    for (int t = 0; t < num_tokens; ++t) {
+      if (sl[t] == -1) continue;
+      if (sl[t] < -1 || sl[t] >= lim) return fail(PKV_ERR_INVALID_ARG, "slot_mapping[%d] = %lld out of range", t, (long long)sl[t]);
+      if (!seen.insert(sl[t]).second) return fail(PKV_ERR_INVALID_ARG, "slot %lld appears twice", (long long)sl[t]);
+    }
+  }
+  const long long rows = static_cast<long long>(num_tokens) * num_kv_heads;
+  if (is16(cache_dtype)) {
+    const int chunks = head_dim * 2 / 16;
+    const int grid = grid_for(rows * chunks, 256);
+    if (chunks == 16)
+      pkv::kv_write_copy_kernel<16><<<grid, 256, 0, st>>>(
+          static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
+          static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, num_blocks);
+    else
+      pkv::kv_write_copy_kernel<8><<<grid, 256, 0, st>>>(
+          static_cast<const uint4*>(k), static_cast<const uint4*>(v), static_cast<uint4*>(k_cache),
+          static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, num_blocks);
+  } else {
+    const int grid = grid_for(rows, 8);  // 8 warps per CTA, one row per warp
+    const bool fp8 = cache_dtype == PKV_FP8E4M3;
+    const bool bf = in_dtype == PKV_BF16;
+    auto* kc = static_cast<uint8_t*>(k_cache);
+    auto* vc = static_cast<uint8_t*>(v_cache);
+#define PKV_QW(D, F, B) \
+  pkv::kv_write_quant_kernel<D, F, B><<<grid, 256, 0, st>>>(k, v, kc, vc, k_scale, v_scale, slot_mapping, num_tokens, num_kv_heads, num_blocks)
+    if (head_dim == 128) {
+      if (fp8) { if (bf) PKV_QW(128, true, true); else PKV_QW(128, true, false); }
+      else { if (bf) PKV_QW(128, false, true); else PKV_QW(128, false, false); }
+    } else {
+      if (fp8) { if (bf) PKV_QW(64, true, true); else PKV_QW(64, true, false); }
+      else { if (bf) PKV_QW(64, false, true); else PKV_QW(64, false, false); }
+    }
+#undef PKV_QW
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "kv_cache_write launch");
+  return ok();
+}
+
+int pkv_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                    int cache_dtype, int partition_tokens, int* num_partitions_out, int* partition_tokens_out,
+                    size_t* workspace_bytes_out) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0)
+    return fail(PKV_ERR_INVALID_ARG, "bad sizes");
+  if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  Plan pl{};
+  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, &pl);
+  if (rc != PKV_OK) return rc;
+  if (num_partitions_out) *num_partitions_out = pl.num_partitions;
+  if (partition_tokens_out) *partition_tokens_out = pl.partition_blocks * 16;
+  if (workspace_bytes_out) *workspace_bytes_out = pl.workspace;
+  return ok();
+}
+
+int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                              int cache_dtype, size_t* bytes) {
+  if (!bytes) return fail(PKV_ERR_INVALID_ARG, "bytes is NULL");
+  return pkv_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, 0, nullptr,
+                         nullptr, bytes);
+}
+
+int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                               const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
+                               int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
+                               int max_context_len, float scale, int q_dtype, int cache_dtype, int partition_tokens,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
+      max_context_len < 0)
+    return fail(PKV_ERR_INVALID_ARG, "bad sizes");
+  if (block_size != 16) return fail(PKV_ERR_UNSUPPORTED, "block_size must be 16 (got %d)", block_size);
+  if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  if (num_q_heads % num_kv_heads != 0) return fail(PKV_ERR_INVALID_ARG, "num_q_heads %% num_kv_heads != 0");
+  const int G = num_q_heads / num_kv_heads;
+  if (G > 16) return fail(PKV_ERR_UNSUPPORTED, "query group %d > 16", G);
+  if (!is16(q_dtype)) return fail(PKV_ERR_UNSUPPORTED, "q dtype %d", q_dtype);
+  if (is16(cache_dtype) && q_dtype != cache_dtype) return fail(PKV_ERR_UNSUPPORTED, "q dtype must match a 16-bit cache");
+  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "scale is not finite");
+  if (static_cast<long long>(num_blocks) * num_kv_heads * 16 >= (1LL << 31))
+    return fail(PKV_ERR_UNSUPPORTED, "pool too large for 32-bit copy coordinates");
+  if (static_cast<long long>(max_context_len) > static_cast<long long>(max_blocks_per_seq) * 16)
+    return fail(PKV_ERR_INVALID_ARG, "max_context_len %d exceeds max_blocks_per_seq * 16", max_context_len);
+  if (num_seqs == 0) return ok();
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+    return fail(PKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(PKV_ERR_INVALID_ARG, "caches must be 16-byte aligned");
+  if (!aligned(q, 4) || !aligned(out, 4)) return fail(PKV_ERR_INVALID_ARG, "q and out must be 4-byte aligned");
+  if (is8(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 16) || !aligned(v_scale, 16)))
+    return fail(PKV_ERR_INVALID_ARG, "quantised caches need 16-byte aligned k_scale and v_scale");
+  Plan pl{};
+  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, &pl);
+  if (rc != PKV_OK) return rc;
+  if (pl.num_partitions > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned(workspace, 16)))
+    return fail(PKV_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu", pl.workspace,
+                workspace ? workspace_bytes : 0);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (g_validate.load()) {
+    std::vector<int32_t> ctx, bt;
+    rc = fetch(&ctx, context_lens, static_cast<size_t>(num_seqs), st);
+    if (rc == PKV_OK) rc = fetch(&bt, block_tables, static_cast<size_t>(num_seqs) * max_blocks_per_seq, st);
+    if (rc != PKV_OK) return rc;
+    for (int s = 0; s < num_seqs; ++s) {
+      if (ctx[s] < 0 || ctx[s] > max_context_len)
+        return fail(PKV_ERR_INVALID_ARG, "context_lens[%d] = %d outside [0, %d]", s, ctx[s], max_context_len);
+      for (int j = 0; j < (ctx[s] + 15) / 16; ++j) {
+        const int32_t b = bt[static_cast<size_t>(s) * max_blocks_per_seq + j];
+        if (b < 0 || b >= num_blocks) return fail(PKV_ERR_INVALID_ARG, "block_tables[%d][%d] = %d out of range", s, j, b);
+      }
+    }
+  }
+  CUtensorMap km, vm;
+  const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * 16;
+  rc = make_cache_map(&km, k_cache, head_dim, elt_size(cache_dtype), rows);
+  if (rc == PKV_OK) rc = make_cache_map(&vm, v_cache, head_dim, elt_size(cache_dtype), rows);
+  if (rc != PKV_OK) return rc;
+
+  pkv::DecodeParams p{};
+  p.out = out;
+  p.q = q;
+  p.k_scale = k_scale;
+  p.v_scale = v_scale;
+  p.block_tables = block_tables;
+  p.context_lens = context_lens;
+  if (pl.num_partitions > 1) {
+    const size_t rowsp = static_cast<size_t>(num_seqs) * num_q_heads * pl.num_partitions;
+    auto* ws = static_cast<uint8_t*>(workspace);
+    p.part_m = reinterpret_cast<float*>(ws);
+    p.part_l = reinterpret_cast<float*>(ws + align_up(rowsp * 4, 256));
+    p.part_o = reinterpret_cast<float*>(ws + 2 * align_up(rowsp * 4, 256));
+  }
+  p.num_q_heads = num_q_heads;
+  p.num_kv_heads = num_kv_heads;
+  p.group = G;
+  p.max_blocks_per_seq = max_blocks_per_seq;
+  p.num_blocks = num_blocks;
+  p.partition_blocks = pl.partition_blocks;
+  p.num_partitions = pl.num_partitions;
+  p.max_context_len = max_context_len;
+  p.qk_scale_log2 = scale * 1.4426950408889634f;
+  const bool q_bf16 = q_dtype == PKV_BF16;
+  rc = head_dim == 128 ? dispatch_ct<128>(cache_dtype, km, vm, p, num_seqs, q_bf16, st)
+                       : dispatch_ct<64>(cache_dtype, km, vm, p, num_seqs, q_bf16, st);
+  if (rc != PKV_OK) return rc;
+  return ok();
+}
+
+int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale, const int32_t* src_dst_pairs,
+                    int num_pairs, int num_kv_heads, int head_dim, int block_size, int num_blocks, int cache_dtype,
+                    void* stream) {
+  if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "bad sizes");
+  if (block_size != 16) return fail(PKV_ERR_UNSUPPORTED, "block_size must be 16 (got %d)", block_size);
+  if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  if (num_pairs == 0) return ok();
+  if (!k_cache || !v_cache || !src_dst_pairs) return fail(PKV_ERR_INVALID_ARG, "NULL pointer");
+  if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(PKV_ERR_INVALID_ARG, "caches must be 16-byte aligned");
+  const bool q8 = is8(cache_dtype);
+  if (q8 && (!k_scale || !v_scale || !aligned(k_scale, 16) || !aligned(v_scale, 16)))
+    return fail(PKV_ERR_INVALID_ARG, "quantised caches need 16-byte aligned k_scale and v_scale");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (g_validate.load()) {
+    std::vector<int32_t> pr;
+    int rc = fetch(&pr, src_dst_pairs, static_cast<size_t>(num_pairs) * 2, st);
+    if (rc != PKV_OK) return rc;
+    std::unordered_set<int32_t> dsts, srcs;
+    for (int i = 0; i < num_pairs; ++i) {
+      const int32_t a = pr[2 * i], b = pr[2 * i + 1];
+      if (a < 0 || a >= num_blocks || b < 0 || b >= num_blocks)
+        return fail(PKV_ERR_INVALID_ARG, "pair %d (%d, %d) out of range", i, a, b);
+      if (!dsts.insert(b).second) return fail(PKV_ERR_INVALID_ARG, "destination %d appears twice", b);
+      srcs.insert(a);
+    }
+    for (int32_t b : dsts)
+      if (srcs.count(b)) return fail(PKV_ERR_INVALID_ARG, "block %d is both a source and a destination", b);
+  }
+  const long long words = static_cast<long long>(num_kv_heads) * 16 * head_dim * elt_size(cache_dtype) / 16;
+  const int swords = q8 ? num_kv_heads * 4 : 0;
+  const int grid = std::min(num_pairs, 16 * sm_count());
+  pkv::copy_blocks_kernel<<<grid, 256, 0, st>>>(static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
+                                                reinterpret_cast<uint4*>(k_scale), reinterpret_cast<uint4*>(v_scale),
+                                                src_dst_pairs, num_pairs, num_blocks, words, swords);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, "copy_blocks launch");
+  return ok();
+}
+
+}  // extern "C"

@@ -1,0 +1,166 @@
+// Slot-mapped KV write and physical block copy.
+//
+// Write ("大模型推理的KV Cache管理…优化实战" §二 append_slot; "LLM 推理优化深度解析"
+// §KV Cache 的本质): row t of k / v [T, Hkv, D] goes to
+// cache[slot / 16][h][slot % 16][:], slot = slot_mapping[t]; -1 skips.
+// Quantised caches store per-(token, head) absmax codes (ascendai.csdn.net
+// article §三 1. KV Cache量化; "KV Cache 与 PagedAttention" §三个直接推论):
+// a = max|x|, s = a / 127 or a / 448, code = RNE(x / s) clamped, with IEEE
+// fp32 divisions (this translation unit is compiled without fast-math).
+//
+// Copy (ascendai.csdn.net article §二 写时复制): block dst := block src for K,
+// V and scales.
+#pragma once
+
+#include "pkv_device.cuh"
+
+namespace pkv {
+
+constexpr int kBlockTokens = 16;
+
+// 16-bit caches: a bit copy, one thread per 16-byte chunk of a (token, head)
+// row; consecutive threads touch consecutive chunks of the same row.
+template <int kChunks>
+__global__ void __launch_bounds__(256) kv_write_copy_kernel(const uint4* __restrict__ k, const uint4* __restrict__ v,
+                                                            uint4* __restrict__ kc, uint4* __restrict__ vc,
+                                                            const int64_t* __restrict__ slots, int num_tokens,
+                                                            int num_kv_heads, int num_blocks) {
+  const long long total = static_cast<long long>(num_tokens) * num_kv_heads * kChunks;
+  const long long slot_limit = static_cast<long long>(num_blocks) * kBlockTokens;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const int c = static_cast<int>(i % kChunks);
+    const long long row = i / kChunks;  // t * Hkv + h
+    const int h = static_cast<int>(row % num_kv_heads);
+    const long long t = row / num_kv_heads;
+    const long long slot = slots[t];
+    if (slot < 0) continue;
+    if (slot >= slot_limit) {
+      if (c == 0) raise_status(PKV_DEV_BAD_SLOT);
+      continue;
+    }
+    const long long blk = slot / kBlockTokens;
+    const int off = static_cast<int>(slot % kBlockTokens);
+    const long long dst = ((blk * num_kv_heads + h) * kBlockTokens + off) * kChunks + c;
+    const uint4 kv = __ldg(k + i);
+    const uint4 vv = __ldg(v + i);
+    kc[dst] = kv;
+    vc[dst] = vv;
+  }
+}
+
+template <bool kInBF16>
+__device__ __forceinline__ float load_in(const void* p, long long idx) {
+  if constexpr (kInBF16) {
+    return __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(p)[idx]);
+  } else {
+    return __half2float(reinterpret_cast<const __half*>(p)[idx]);
+  }
+}
+
+__device__ __forceinline__ float warp_max(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// One quantised code from x given scale s (s > 0).
+template <bool kFP8>
+__device__ __forceinline__ uint32_t quantize_one(float x, float s) {
+  const float y = __fdiv_rn(x, s);
+  if constexpr (kFP8) {
+    const float yc = fminf(fmaxf(y, -448.0f), 448.0f);
+    return static_cast<uint32_t>(__nv_cvt_float_to_fp8(yc, __NV_SATFINITE, __NV_E4M3));
+  } else {
+    int q = __float2int_rn(y);
+    q = max(-127, min(127, q));
+    return static_cast<uint32_t>(q) & 0xFFu;
+  }
+}
+
+// Quantising write: one warp per (token, head) row, D / 32 elements per lane.
+template <int kD, bool kFP8, bool kInBF16>
+__global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restrict__ k, const void* __restrict__ v,
+                                                             uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
+                                                             float* __restrict__ ks, float* __restrict__ vs,
+                                                             const int64_t* __restrict__ slots, int num_tokens,
+                                                             int num_kv_heads, int num_blocks) {
+  constexpr int kE = kD / 32;
+  const int lane = threadIdx.x & 31;
+  const long long rows = static_cast<long long>(num_tokens) * num_kv_heads;
+  const long long slot_limit = static_cast<long long>(num_blocks) * kBlockTokens;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long row = (blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x) >> 5; row < rows;
+       row += warps) {
+    const long long t = row / num_kv_heads;
+    const int h = static_cast<int>(row % num_kv_heads);
+    const long long slot = slots[t];
+    if (slot < 0) continue;
+    if (slot >= slot_limit) {
+      if (lane == 0) raise_status(PKV_DEV_BAD_SLOT);
+      continue;
+    }
+    const long long blk = slot / kBlockTokens;
+    const int off = static_cast<int>(slot % kBlockTokens);
+    const long long dst_row = (blk * num_kv_heads + h) * kBlockTokens + off;
+#pragma unroll
+    for (int which = 0; which < 2; ++which) {
+      const void* src = which == 0 ? k : v;
+      uint8_t* cache = which == 0 ? kc : vc;
+      float* scales = which == 0 ? ks : vs;
+      float x[kE];
+      float a = 0.0f;
+#pragma unroll
+      for (int e = 0; e < kE; ++e) {
+        x[e] = load_in<kInBF16>(src, row * kD + lane * kE + e);
+        a = fmaxf(a, fabsf(x[e]));
+      }
+      a = warp_max(a);
+      const float s = __fdiv_rn(a, kFP8 ? 448.0f : 127.0f);
+      uint32_t packed = 0;
+      if (a > 0.0f) {
+#pragma unroll
+        for (int e = 0; e < kE; ++e) packed |= quantize_one<kFP8>(x[e], s) << (8 * e);
+      }
+      if constexpr (kE == 4) {
+        reinterpret_cast<uint32_t*>(cache + dst_row * kD)[lane] = packed;
+      } else {
+        reinterpret_cast<uint16_t*>(cache + dst_row * kD)[lane] = static_cast<uint16_t>(packed);
+      }
+      if (lane == 0) scales[dst_row] = s;
+    }
+  }
+}
+
+// Block copy: grid.x walks pairs, each CTA copies whole blocks with 16-byte
+// vectors.  `words` = 16-byte units per block of one cache; `swords` = 16-byte
+// units of one block's scales (0 for 16-bit caches).
+__global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ vc,
+                                                          uint4* __restrict__ ks, uint4* __restrict__ vs,
+                                                          const int32_t* __restrict__ pairs, int num_pairs,
+                                                          int num_blocks, long long words, int swords) {
+  for (int p = blockIdx.x; p < num_pairs; p += gridDim.x) {
+    const int src = pairs[2 * p];
+    const int dst = pairs[2 * p + 1];
+    if (src < 0 || src >= num_blocks || dst < 0 || dst >= num_blocks) {
+      if (threadIdx.x == 0) raise_status(PKV_DEV_BAD_PAIR);
+      continue;
+    }
+    const uint4* ks_src = kc + src * words;
+    const uint4* vs_src = vc + src * words;
+    uint4* kd = kc + dst * words;
+    uint4* vd = vc + dst * words;
+    for (long long i = threadIdx.x; i < words; i += blockDim.x) {
+      const uint4 a = ks_src[i];
+      const uint4 b = vs_src[i];
+      kd[i] = a;
+      vd[i] = b;
+    }
+    for (int i = threadIdx.x; i < swords; i += blockDim.x) {
+      ks[static_cast<long long>(dst) * swords + i] = ks[static_cast<long long>(src) * swords + i];
+      vs[static_cast<long long>(dst) * swords + i] = vs[static_cast<long long>(src) * swords + i];
+    }
+  }
+}
+
+}  // namespace pkv

@@ -123,15 +123,18 @@ def random_scales(shape, gen, kind):
     return (2.0 + 2.0 * u) / qmax
 
 
-def decode_case(name, seed=None, batch=None, ctx_override=None, cache_kind=None, num_blocks=None):
+def decode_case(name, seed=None, batch=None, ctx_override=None, cache_kind=None, num_blocks=None,
+                **shape):
     """A complete random decode problem for workload ``name`` on the CPU.
 
     Returns a dict with q [B, Hq, D], k_cache / v_cache [NB, Hkv, 16, D]
     (values, or codes for int8 / fp8 with k_scale / v_scale [NB, Hkv, 16]),
     block_tables [B, MB] int32, context_lens [B] int32, scale and the shape
-    fields.  ``ctx_override`` replaces the drawn context lengths.
+    fields.  ``ctx_override`` replaces the drawn context lengths; ``shape``
+    may override hq, hkv, d and dtype.
     """
     spec = dict(WORKLOADS[name])
+    spec.update(shape)
     if batch is not None:
         spec["batch"] = batch
     gen = generator(spec["seed"] if seed is None else seed)
@@ -180,3 +183,55 @@ def distinct_slots(n_tokens, num_blocks, seed, skip_every=0):
     if skip_every:
         perm[::skip_every] = -1
     return perm
+
+
+def device_decode_case(name, device, seed=None, batch=None, cache_kind=None, ctx_override=None):
+    """Like ``decode_case`` but the large arrays (q and the caches) are drawn
+    directly on ``device`` from a seeded CUDA generator, so full-size
+    workloads need no host copy.  Context lengths and block tables are drawn
+    on the CPU exactly as in ``decode_case`` and then moved to the device."""
+    spec = dict(WORKLOADS[name])
+    if batch is not None:
+        spec["batch"] = batch
+    base_seed = spec["seed"] if seed is None else seed
+    gen = generator(base_seed)
+    B, hq, hkv, d = spec["batch"], spec["hq"], spec["hkv"], spec["d"]
+    if ctx_override is not None:
+        ctx = torch.as_tensor(ctx_override, dtype=torch.int32).reshape(-1)
+        B = ctx.numel()
+        prefix = 0
+    else:
+        ctx = context_lens(spec, gen, B)
+        prefix = spec.get("prefix", 0)
+        ctx = ctx + prefix
+    need = sum(blocks_for(int(c)) for c in ctx.tolist())
+    if prefix:
+        need -= (B - 1) * blocks_for(prefix)
+    nb = max(pool_size(spec, max(need, 1)), need, 1)
+    bt = random_block_tables(ctx, nb, gen, shared_prefix_tokens=prefix)
+    dg = torch.Generator(device=device)
+    dg.manual_seed(base_seed + 7919)
+    kind = cache_kind or "float"
+    dt = TORCH_DTYPES[spec["dtype"]]
+    out = dict(name=name, batch=B, hq=hq, hkv=hkv, d=d, block_size=BLOCK_SIZE, num_blocks=nb,
+               dtype=spec["dtype"], cache_kind=kind, scale=1.0 / math.sqrt(d),
+               block_tables=bt.to(device), context_lens=ctx.to(device),
+               block_tables_cpu=bt, context_lens_cpu=ctx)
+    out["q"] = torch.randn((B, hq, d), generator=dg, device=device, dtype=dt)
+    shape = (nb, hkv, BLOCK_SIZE, d)
+    if kind == "float":
+        out["k_cache"] = torch.randn(shape, generator=dg, device=device, dtype=dt)
+        out["v_cache"] = torch.randn(shape, generator=dg, device=device, dtype=dt)
+    else:
+        for key in ("k_cache", "v_cache"):
+            x = torch.randn(shape, generator=dg, device=device, dtype=torch.float16)
+            if kind == "int8":
+                out[key] = (x * (127.0 / 3.0)).round().clamp(-127, 127).to(torch.int8)
+            else:
+                out[key] = (x.float() * (448.0 / 3.0)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+            del x
+        qmax = 127.0 if kind == "int8" else 448.0
+        for key in ("k_scale", "v_scale"):
+            u = torch.rand((nb, hkv, BLOCK_SIZE), generator=dg, device=device, dtype=torch.float32)
+            out[key] = (2.0 + 2.0 * u) / qmax
+    return out

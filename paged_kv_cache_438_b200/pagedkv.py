@@ -1,0 +1,330 @@
+"""ctypes binding of libpagedkv.so (C ABI declared in include/pagedkv.h).
+
+Argument marshalling only: every computation runs in the library's CUDA
+kernels (or, for the block allocator, its C++ code).  torch provides device
+memory and streams.  If the shared library is missing, every call raises.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpagedkv.so")
+
+PKV_OK = 0
+PKV_ERR_INVALID_ARG = -1
+PKV_ERR_UNSUPPORTED = -2
+PKV_ERR_NO_BLOCKS = -3
+PKV_ERR_CUDA = -4
+PKV_ERR_NOT_FOUND = -5
+PKV_ERR_EXISTS = -6
+
+PKV_F16, PKV_BF16, PKV_I8, PKV_FP8E4M3 = 0, 1, 2, 3
+
+DEV_BAD_SLOT, DEV_BAD_BLOCK, DEV_BAD_CONTEXT, DEV_TIMEOUT, DEV_BAD_PAIR = 1, 2, 4, 8, 16
+
+EXPORTS = [
+    "pkv_last_error", "pkv_version", "pkv_kv_cache_write", "pkv_decode_plan", "pkv_decode_workspace_size",
+    "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_device_status", "pkv_set_validation",
+    "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_fork", "pkv_seq_append",
+    "pkv_batch_append", "pkv_batch_tables", "pkv_seq_free", "pkv_seq_block_table", "pkv_seq_len",
+    "pkv_block_refcount", "pkv_alloc_stats",
+]
+
+
+class PagedKVError(RuntimeError):
+    def __init__(self, code, msg):
+        super().__init__(f"libpagedkv error {code}: {msg}")
+        self.code = code
+
+
+class NoBlocksError(PagedKVError):
+    pass
+
+
+_lib_handle = None
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_I64 = ctypes.c_int64
+_SZ = ctypes.c_size_t
+_F = ctypes.c_float
+
+
+def _signatures(lib):
+    sig = {
+        "pkv_last_error": ([], ctypes.c_char_p),
+        "pkv_version": ([], _I),
+        "pkv_kv_cache_write": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
+        "pkv_decode_plan": ([_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
+                             ctypes.POINTER(_SZ)], _I),
+        "pkv_decode_workspace_size": ([_I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
+        "pkv_paged_attention_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
+                                        _I, _I, _I, _P, _SZ, _P], _I),
+        "pkv_copy_blocks": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P], _I),
+        "pkv_device_status": ([ctypes.POINTER(ctypes.c_uint), _I], _I),
+        "pkv_set_validation": ([_I], _I),
+        "pkv_alloc_create": ([_I, _I, _P, ctypes.POINTER(_P)], _I),
+        "pkv_alloc_destroy": ([_P], _I),
+        "pkv_seq_add": ([_P, _I64], _I),
+        "pkv_seq_fork": ([_P, _I64, _I64, _I], _I),
+        "pkv_seq_append": ([_P, _I64, _I, _P, _P, _I, ctypes.POINTER(_I)], _I),
+        "pkv_batch_append": ([_P, _P, _I, _P, _P, _I, ctypes.POINTER(_I)], _I),
+        "pkv_batch_tables": ([_P, _P, _I, _P, _I, _P], _I),
+        "pkv_seq_free": ([_P, _I64], _I),
+        "pkv_seq_block_table": ([_P, _I64, _P, _I, ctypes.POINTER(_I)], _I),
+        "pkv_seq_len": ([_P, _I64, ctypes.POINTER(_I)], _I),
+        "pkv_block_refcount": ([_P, ctypes.c_int32, ctypes.POINTER(_I)], _I),
+        "pkv_alloc_stats": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+
+
+def lib():
+    """The loaded library; raises if libpagedkv.so has not been built."""
+    global _lib_handle
+    if _lib_handle is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m paged_kv_cache_438_b200.build`")
+        h = ctypes.CDLL(LIB_PATH)
+        _signatures(h)
+        _lib_handle = h
+    return _lib_handle
+
+
+def _check(rc):
+    if rc != PKV_OK:
+        msg = lib().pkv_last_error().decode(errors="replace")
+        if rc == PKV_ERR_NO_BLOCKS:
+            raise NoBlocksError(rc, msg)
+        raise PagedKVError(rc, msg)
+
+
+# ------------------------------------------------------------------ helpers --
+
+def dtype_code(t):
+    d = t.dtype if isinstance(t, torch.Tensor) else t
+    if d == torch.float16:
+        return PKV_F16
+    if d == torch.bfloat16:
+        return PKV_BF16
+    if d == torch.int8:
+        return PKV_I8
+    if d in (torch.uint8, torch.float8_e4m3fn):
+        return PKV_FP8E4M3
+    raise TypeError(f"unsupported dtype {d}")
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _need(t, name, device=None, dtype=None, contiguous=True):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if dtype is not None and t.dtype not in (dtype if isinstance(dtype, tuple) else (dtype,)):
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+# ---------------------------------------------------------------- kernels ----
+
+def version():
+    return lib().pkv_version()
+
+
+def set_validation(on):
+    _check(lib().pkv_set_validation(1 if on else 0))
+
+
+def device_status(clear=True):
+    v = ctypes.c_uint(0)
+    _check(lib().pkv_device_status(ctypes.byref(v), 1 if clear else 0))
+    return v.value
+
+
+def kv_cache_write(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=None, stream=None):
+    """Writes rows k, v [T, Hkv, D] into the paged caches at slot_mapping [T]
+    (int64, -1 skips).  Quantised caches (int8 / float8_e4m3fn) need the
+    fp32 scale arrays [NB, Hkv, 16]."""
+    for n, t in (("k", k), ("v", v), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need(t, n, device=k.device)
+    _need(slot_mapping, "slot_mapping", device=k.device, dtype=torch.int64)
+    if k.dim() != 3 or v.shape != k.shape or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("k, v must be [T, Hkv, D]; caches [NB, Hkv, 16, D]")
+    T, hkv, d = k.shape
+    nb = k_cache.shape[0]
+    if k_cache.shape[1] != hkv or k_cache.shape[3] != d or slot_mapping.numel() != T:
+        raise ValueError("shape mismatch between k and the caches")
+    ct = dtype_code(k_cache)
+    if ct in (PKV_I8, PKV_FP8E4M3):
+        _need(k_scale, "k_scale", device=k.device, dtype=torch.float32)
+        _need(v_scale, "v_scale", device=k.device, dtype=torch.float32)
+    _check(lib().pkv_kv_cache_write(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
+                                    _ptr(slot_mapping), T, hkv, d, k_cache.shape[2], nb, dtype_code(k), ct,
+                                    _stream(stream)))
+
+
+def decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens=0):
+    """(num_partitions, partition_tokens, workspace_bytes) the decode call uses."""
+    npart, ptok, ws = _I(0), _I(0), _SZ(0)
+    ct = cache_dtype if isinstance(cache_dtype, int) else dtype_code(cache_dtype)
+    _check(lib().pkv_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, ct,
+                                 partition_tokens, ctypes.byref(npart), ctypes.byref(ptok), ctypes.byref(ws)))
+    return npart.value, ptok.value, ws.value
+
+
+def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale=None, v_scale=None,
+                           max_context_len=None, out=None, workspace=None, partition_tokens=0, stream=None):
+    """out[s, i] = softmax(scale * q[s, i] . K_s) V_s through block tables.
+
+    q [B, Hq, D] fp16/bf16; caches [NB, Hkv, 16, D]; block_tables [B, MB]
+    int32; context_lens [B] int32.  ``max_context_len`` is a host-side upper
+    bound on context_lens (if None it is read from the device, which
+    synchronises).  Returns ``out`` [B, Hq, D] in q's dtype."""
+    dev = q.device
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need(t, n, device=dev)
+    _need(block_tables, "block_tables", device=dev, dtype=torch.int32)
+    _need(context_lens, "context_lens", device=dev, dtype=torch.int32)
+    if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q must be [B, Hq, D]; caches [NB, Hkv, 16, D]")
+    B, hq, d = q.shape
+    nb, hkv, bs, dk = k_cache.shape
+    if dk != d or block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.numel() != B:
+        raise ValueError("shape mismatch")
+    ct = dtype_code(k_cache)
+    if ct in (PKV_I8, PKV_FP8E4M3):
+        _need(k_scale, "k_scale", device=dev, dtype=torch.float32)
+        _need(v_scale, "v_scale", device=dev, dtype=torch.float32)
+    if max_context_len is None:
+        max_context_len = int(context_lens.max().item()) if B else 0
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", device=dev, dtype=q.dtype)
+    npart, _, ws_bytes = decode_plan(B, hq, hkv, d, max_context_len, ct, partition_tokens)
+    if npart > 1 and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
+        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pkv_paged_attention_decode(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], max_context_len, float(scale),
+        dtype_code(q), ct, partition_tokens, _ptr(workspace), ws_len, _stream(stream)))
+    return out
+
+
+def copy_blocks(k_cache, v_cache, src_dst_pairs, k_scale=None, v_scale=None, stream=None):
+    """Block dst := block src for every row (src, dst) of src_dst_pairs
+    [N, 2] int32 (device), for K, V and the scales of quantised caches."""
+    dev = k_cache.device
+    _need(k_cache, "k_cache", device=dev)
+    _need(v_cache, "v_cache", device=dev)
+    _need(src_dst_pairs, "src_dst_pairs", device=dev, dtype=torch.int32)
+    nb, hkv, bs, d = k_cache.shape
+    ct = dtype_code(k_cache)
+    n = src_dst_pairs.numel() // 2
+    _check(lib().pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(src_dst_pairs),
+                                 n, hkv, d, bs, nb, ct, _stream(stream)))
+
+
+# --------------------------------------------------------- block allocator --
+
+class BlockAllocator:
+    """Host block manager (C++): LIFO free list, reference counts, fork and
+    copy-on-write, slot and block-table production."""
+
+    def __init__(self, num_blocks, block_size=16, initial_free_order=None):
+        self._h = ctypes.c_void_p()
+        order = None
+        if initial_free_order is not None:
+            self._order = torch.as_tensor(initial_free_order, dtype=torch.int32).contiguous()
+            order = ctypes.c_void_p(self._order.data_ptr())
+        _check(lib().pkv_alloc_create(num_blocks, block_size, order, ctypes.byref(self._h)))
+        self.num_blocks = num_blocks
+        self.block_size = block_size
+
+    def close(self):
+        if self._h:
+            lib().pkv_alloc_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def add(self, seq_id):
+        _check(lib().pkv_seq_add(self._h, seq_id))
+
+    def fork(self, parent, child, prefix_len=-1):
+        _check(lib().pkv_seq_fork(self._h, parent, child, prefix_len))
+
+    def append(self, seq_id, n_tokens):
+        """Returns (slots int64 tensor [n_tokens], cow pairs int32 tensor [k, 2])."""
+        slots = torch.empty(n_tokens, dtype=torch.int64)
+        pairs = torch.empty((max(n_tokens, 1), 2), dtype=torch.int32)
+        npairs = _I(0)
+        _check(lib().pkv_seq_append(self._h, seq_id, n_tokens, _ptr(slots), _ptr(pairs), pairs.shape[0],
+                                    ctypes.byref(npairs)))
+        return slots, pairs[:npairs.value].clone()
+
+    def batch_append(self, seq_ids):
+        """One token for each sequence; returns (slots [n], cow pairs [k, 2])."""
+        ids = torch.as_tensor(seq_ids, dtype=torch.int64).contiguous()
+        n = ids.numel()
+        slots = torch.empty(n, dtype=torch.int64)
+        pairs = torch.empty((max(n, 1), 2), dtype=torch.int32)
+        npairs = _I(0)
+        _check(lib().pkv_batch_append(self._h, _ptr(ids), n, _ptr(slots), _ptr(pairs), pairs.shape[0],
+                                      ctypes.byref(npairs)))
+        return slots, pairs[:npairs.value].clone()
+
+    def batch_tables(self, seq_ids, max_blocks, out_tables=None, out_lens=None):
+        ids = torch.as_tensor(seq_ids, dtype=torch.int64).contiguous()
+        n = ids.numel()
+        bt = torch.empty((n, max_blocks), dtype=torch.int32) if out_tables is None else out_tables
+        cl = torch.empty(n, dtype=torch.int32) if out_lens is None else out_lens
+        _check(lib().pkv_batch_tables(self._h, _ptr(ids), n, _ptr(bt), max_blocks, _ptr(cl)))
+        return bt, cl
+
+    def free(self, seq_id):
+        _check(lib().pkv_seq_free(self._h, seq_id))
+
+    def block_table(self, seq_id):
+        n = _I(0)
+        length = self.seq_len(seq_id)
+        cap = (length + self.block_size - 1) // self.block_size
+        out = torch.empty(max(cap, 1), dtype=torch.int32)
+        _check(lib().pkv_seq_block_table(self._h, seq_id, _ptr(out), out.numel(), ctypes.byref(n)))
+        return out[:n.value].tolist()
+
+    def seq_len(self, seq_id):
+        n = _I(0)
+        _check(lib().pkv_seq_len(self._h, seq_id, ctypes.byref(n)))
+        return n.value
+
+    def refcount(self, block):
+        rc = _I(0)
+        _check(lib().pkv_block_refcount(self._h, block, ctypes.byref(rc)))
+        return rc.value
+
+    def stats(self):
+        a, b, c = _I(0), _I(0), _I(0)
+        _check(lib().pkv_alloc_stats(self._h, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+        return a.value, b.value, c.value

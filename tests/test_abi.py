@@ -1,0 +1,111 @@
+"""The C-ABI library loads without a GPU, exports every entry point that
+include/pagedkv.h declares, and rejects bad arguments on the host before any
+launch (these calls need no device)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from paged_kv_cache_438_b200 import pagedkv as P
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "pagedkv.h")) as f:
+        src = f.read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(pkv_[a-z0-9_]+)\s*\(", src)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from paged_kv_cache_438_b200 import build
+    build.build()
+    return P.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    declared = _declared()
+    assert len(declared) >= 20
+    raw = ctypes.CDLL(P.LIB_PATH)
+    for name in declared:
+        assert hasattr(raw, name), name
+    assert sorted(P.EXPORTS) == declared
+
+
+def test_version(lib):
+    assert lib.pkv_version() >= 10000
+
+
+def _err(rc, code):
+    assert rc == code, (rc, P.lib().pkv_last_error())
+
+
+def test_write_rejects_bad_block_size_and_dtypes(lib):
+    n = ctypes.c_void_p(16)
+    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, n, 4, 2, 64, 8, 10, P.PKV_F16, P.PKV_F16, None),
+         P.PKV_ERR_UNSUPPORTED)
+    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, n, 4, 2, 96, 16, 10, P.PKV_F16, P.PKV_F16, None),
+         P.PKV_ERR_UNSUPPORTED)
+    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, n, 4, 2, 64, 16, 10, P.PKV_BF16, P.PKV_F16, None),
+         P.PKV_ERR_UNSUPPORTED)
+    # quantised cache without scale arrays
+    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, n, 4, 2, 64, 16, 10, P.PKV_BF16, P.PKV_I8, None),
+         P.PKV_ERR_INVALID_ARG)
+    # misaligned cache pointer
+    m = ctypes.c_void_p(18)
+    _err(lib.pkv_kv_cache_write(n, n, m, n, None, None, n, 4, 2, 64, 16, 10, P.PKV_F16, P.PKV_F16, None),
+         P.PKV_ERR_INVALID_ARG)
+    assert b"aligned" in lib.pkv_last_error()
+
+
+def test_write_zero_tokens_is_a_noop(lib):
+    _err(lib.pkv_kv_cache_write(None, None, None, None, None, None, None, 0, 2, 64, 16, 10, P.PKV_F16, P.PKV_F16,
+                                None), P.PKV_OK)
+
+
+def _decode(lib, **kw):
+    n = ctypes.c_void_p(256)
+    a = dict(out=n, q=n, kc=n, vc=n, ks=None, vs=None, bt=n, cl=n, B=2, hq=8, hkv=2, d=128, bs=16, nb=100, mb=4,
+             maxc=64, scale=0.1, qd=P.PKV_BF16, cd=P.PKV_BF16, pt=0, ws=None, wsb=0)
+    a.update(kw)
+    return lib.pkv_paged_attention_decode(a["out"], a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["bt"], a["cl"],
+                                          a["B"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["mb"], a["maxc"],
+                                          a["scale"], a["qd"], a["cd"], a["pt"], a["ws"], a["wsb"], None)
+
+
+def test_decode_host_rejections(lib):
+    _err(_decode(lib, hq=7), P.PKV_ERR_INVALID_ARG)              # Hq % Hkv != 0
+    _err(_decode(lib, hq=64, hkv=2), P.PKV_ERR_UNSUPPORTED)       # G = 32 > 16
+    _err(_decode(lib, d=80), P.PKV_ERR_UNSUPPORTED)
+    _err(_decode(lib, bs=32), P.PKV_ERR_UNSUPPORTED)
+    _err(_decode(lib, qd=P.PKV_F16), P.PKV_ERR_UNSUPPORTED)       # q dtype must match a 16-bit cache
+    _err(_decode(lib, maxc=65), P.PKV_ERR_INVALID_ARG)            # > max_blocks * 16
+    _err(_decode(lib, scale=float("nan")), P.PKV_ERR_INVALID_ARG)
+    _err(_decode(lib, cd=P.PKV_I8), P.PKV_ERR_INVALID_ARG)        # quantised without scales
+    _err(_decode(lib, pt=24), P.PKV_ERR_INVALID_ARG)              # partition not a multiple of 16
+    # split plan needs a workspace
+    _err(_decode(lib, maxc=64, pt=16), P.PKV_ERR_INVALID_ARG)
+    assert b"workspace" in lib.pkv_last_error()
+    _err(_decode(lib, B=0), P.PKV_OK)
+
+
+def test_plan_is_consistent(lib):
+    for (B, hq, hkv, d, ctx) in [(4, 8, 2, 64, 256), (64, 32, 8, 128, 4096), (32, 64, 8, 128, 32768),
+                                 (256, 32, 32, 128, 8192), (1, 8, 8, 128, 1)]:
+        np_, pt, ws = P.decode_plan(B, hq, hkv, d, ctx, P.PKV_BF16)
+        assert pt % 16 == 0 and np_ * pt >= ctx and (np_ - 1) * pt < max(ctx, 1)
+        assert (ws == 0) == (np_ == 1)
+        if np_ > 1:
+            assert ws >= B * hq * np_ * (d + 2) * 4
+    np_, pt, ws = P.decode_plan(2, 8, 2, 128, 1000, P.PKV_BF16, partition_tokens=64)
+    assert (np_, pt) == (16, 64)
+
+
+def test_copy_rejections(lib):
+    n = ctypes.c_void_p(256)
+    _err(lib.pkv_copy_blocks(n, n, None, None, n, 3, 2, 128, 16, 10, P.PKV_FP8E4M3, None), P.PKV_ERR_INVALID_ARG)
+    _err(lib.pkv_copy_blocks(n, n, None, None, n, 3, 2, 128, 12, 10, P.PKV_BF16, None), P.PKV_ERR_UNSUPPORTED)
+    _err(lib.pkv_copy_blocks(n, n, None, None, n, 0, 2, 128, 16, 10, P.PKV_BF16, None), P.PKV_OK)
