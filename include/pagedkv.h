@@ -167,6 +167,40 @@ int pkv_paged_attention_decode(void* out, const void* q,
                                void* stream);
 
 /*
+ * pkv_paged_attention_decode_noalloc -- pkv_paged_attention_decode for
+ * callers that cannot allocate device memory (no counterpart on the pages;
+ * this is a library convenience).  Typical such callers: a plugin inside a
+ * host framework that owns every device allocation and passes the plugin only
+ * its input and output buffers, or a latency-critical loop in which a
+ * cudaMalloc could synchronise the device.  The arguments mean what they mean
+ * for pkv_paged_attention_decode; there is no workspace argument.
+ *   - The split-KV partials go to one library-owned device array of
+ *     PKV_NOALLOC_SCRATCH_BYTES (a file-scope __device__ array: every GPU that
+ *     loads the library holds it until the process exits).  A call whose plan
+ *     needs more (pkv_decode_plan's workspace_bytes_out) is rejected with
+ *     PKV_ERR_INVALID_ARG before anything is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make
+ *     that first call before any stream capture.
+ *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
+ *   - All calls on a device share the one array and it keeps the last call's
+ *     contents.  Nothing in it needs to start at zero (every partial is written
+ *     before it is read), but calls that overlap on the GPU (concurrent
+ *     streams, or other threads) race on it and give wrong results; serialise
+ *     them, e.g. on one stream.
+ */
+#define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+int pkv_paged_attention_decode_noalloc(void* out, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const float* k_scale, const float* v_scale,
+                                       const int32_t* block_tables, const int32_t* context_lens,
+                                       int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                       int block_size, int num_blocks, int max_blocks_per_seq,
+                                       int max_context_len, float scale, int q_dtype, int cache_dtype,
+                                       int partition_tokens, void* stream);
+
+/*
  * pkv_copy_blocks -- copy whole physical blocks (K, V and, for quantised
  * caches, their scales): for each pair p, block src_dst_pairs[2p+1] becomes a
  * copy of block src_dst_pairs[2p].  This is the copy behind copy-on-write

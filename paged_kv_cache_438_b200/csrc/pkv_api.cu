@@ -446,3 +446,75 @@ int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free decode.  Some callers cannot allocate device memory at all:
+// a plugin whose host framework owns every device allocation and hands it
+// only its input and output buffers, or a latency-critical loop where a
+// cudaMalloc could synchronise the device.  For them the split-KV partials
+// live in one library-owned device array instead of a caller workspace.
+// The array is file-scope, so every GPU that loads this library holds it
+// (PKV_NOALLOC_SCRATCH_BYTES) until the process exits.  Host code must not
+// use the array's name as a device address: it is a host-side stand-in, so
+// its device address is fetched once per device with cudaGetSymbolAddress.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(PKV_NOALLOC_SCRATCH_BYTES);
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device, looked up on
+// the first call for that device (with that device current) and cached.
+int noalloc_scratch_address(void** out) {
+  static std::mutex mu;
+  static std::vector<void*> by_device;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  std::lock_guard<std::mutex> lk(mu);
+  if (static_cast<size_t>(dev) < by_device.size() && by_device[dev] != nullptr) {
+    *out = by_device[dev];
+    return PKV_OK;
+  }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
+  if (p == nullptr) return fail(PKV_ERR_CUDA, "cudaGetSymbolAddress returned NULL for the no-alloc scratch");
+  if (by_device.size() <= static_cast<size_t>(dev)) by_device.resize(dev + 1, nullptr);
+  by_device[dev] = p;
+  *out = p;
+  return PKV_OK;
+}
+
+}  // namespace
+
+extern "C" int pkv_paged_attention_decode_noalloc(void* out, const void* q, const void* k_cache,
+                                                  const void* v_cache, const float* k_scale, const float* v_scale,
+                                                  const int32_t* block_tables, const int32_t* context_lens,
+                                                  int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                                                  int block_size, int num_blocks, int max_blocks_per_seq,
+                                                  int max_context_len, float scale, int q_dtype, int cache_dtype,
+                                                  int partition_tokens, void* stream) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0)
+    return fail(PKV_ERR_INVALID_ARG, "bad sizes");
+  if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
+  Plan pl{};
+  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, &pl);
+  if (rc != PKV_OK) return rc;
+  if (pl.workspace > kNoAllocScratchBytes)
+    return fail(PKV_ERR_INVALID_ARG,
+                "this decode needs %zu bytes of split-KV scratch but the built-in array holds %zu "
+                "(PKV_NOALLOC_SCRATCH_BYTES); use fewer sequences per call, a larger partition_tokens, "
+                "or pkv_paged_attention_decode with a caller workspace",
+                pl.workspace, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  if (pl.workspace > 0) {
+    rc = noalloc_scratch_address(&scratch);
+    if (rc != PKV_OK) return rc;
+  }
+  return pkv_paged_attention_decode(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+                                    num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
+                                    max_blocks_per_seq, max_context_len, scale, q_dtype, cache_dtype,
+                                    partition_tokens, scratch, pl.workspace > 0 ? kNoAllocScratchBytes : 0, stream);
+}

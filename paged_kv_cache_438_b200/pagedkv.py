@@ -26,7 +26,7 @@ DEV_BAD_SLOT, DEV_BAD_BLOCK, DEV_BAD_CONTEXT, DEV_TIMEOUT, DEV_BAD_PAIR = 1, 2, 
 
 EXPORTS = [
     "pkv_last_error", "pkv_version", "pkv_kv_cache_write", "pkv_decode_plan", "pkv_decode_workspace_size",
-    "pkv_paged_attention_decode", "pkv_copy_blocks", "pkv_device_status", "pkv_set_validation",
+    "pkv_paged_attention_decode", "pkv_paged_attention_decode_noalloc", "pkv_copy_blocks", "pkv_device_status", "pkv_set_validation",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_fork", "pkv_seq_append",
     "pkv_batch_append", "pkv_batch_tables", "pkv_seq_free", "pkv_seq_block_table", "pkv_seq_len",
     "pkv_block_refcount", "pkv_alloc_stats",
@@ -62,6 +62,8 @@ def _signatures(lib):
         "pkv_decode_workspace_size": ([_I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
         "pkv_paged_attention_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
                                         _I, _I, _I, _P, _SZ, _P], _I),
+        "pkv_paged_attention_decode_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                                                _F, _I, _I, _I, _P], _I),
         "pkv_copy_blocks": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P], _I),
         "pkv_device_status": ([ctypes.POINTER(ctypes.c_uint), _I], _I),
         "pkv_set_validation": ([_I], _I),
@@ -225,6 +227,33 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
         _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], max_context_len, float(scale),
         dtype_code(q), ct, partition_tokens, _ptr(workspace), ws_len, _stream(stream)))
+    return out
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
+                                   out, k_scale=None, v_scale=None, partition_tokens=0, stream=None):
+    """paged_attention_decode for callers that cannot allocate device memory
+    (for instance a plugin whose host framework owns every allocation and
+    hands it only input and output buffers): ``out`` must be given, no
+    workspace is taken, and the split-KV partials use the library's own
+    device array of NOALLOC_SCRATCH_BYTES.  Work that needs more scratch is
+    rejected with an error.  Calls that overlap on the GPU share that array
+    and race; keep them on one stream.  The first call on a device looks up
+    the array's address, so make it before any stream capture."""
+    dev = q.device
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache), ("out", out)):
+        _need(t, n, device=dev)
+    _need(block_tables, "block_tables", device=dev, dtype=torch.int32)
+    _need(context_lens, "context_lens", device=dev, dtype=torch.int32)
+    B, hq, d = q.shape
+    nb, hkv, bs, _ = k_cache.shape
+    _check(lib().pkv_paged_attention_decode_noalloc(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
+        _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], int(max_context_len), float(scale),
+        dtype_code(q), dtype_code(k_cache), partition_tokens, _stream(stream)))
     return out
 
 

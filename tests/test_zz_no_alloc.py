@@ -1,0 +1,78 @@
+"""The allocation-free decode entry point against the regular one.
+
+pkv_paged_attention_decode_noalloc serves callers that cannot allocate device
+memory (a plugin whose host framework owns all device allocations, or a
+latency-critical loop where cudaMalloc could synchronise the device); its
+split-KV partials live in the library's own fixed device array.  This file is
+collected last so that a failure here leaves every other test already run;
+it passes alone in a fresh process and after the rest of the suite.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from paged_kv_cache_438_b200 import inputs as I
+from paged_kv_cache_438_b200 import pagedkv as P
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda:0")
+ATOL, MEANREL = 2e-2, 1e-2
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from paged_kv_cache_438_b200 import build
+    build.build()
+    P.lib()
+
+
+def _case(seed, batch):
+    c = I.device_decode_case("llama3_8b", DEV, seed=seed, batch=batch)
+    c["maxc"] = int(c["context_lens_cpu"].max())
+    return c
+
+
+def _close(a, b):
+    a = a.double().cpu().numpy()
+    b = b.double().cpu().numpy()
+    err = np.abs(a - b)
+    assert err.max() <= ATOL
+    assert err.sum() / max(np.abs(b).sum(), 1e-30) <= MEANREL
+
+
+def test_noalloc_matches_workspace_entry_point_on_two_calls():
+    cases = [_case(2024, 16), _case(2025, 24)]
+    outs = []
+    for c in cases:
+        # partitions of 256 tokens: the split path, so the scratch array is used
+        np_, _, ws = P.decode_plan(c["batch"], c["hq"], c["hkv"], c["d"], c["maxc"], c["k_cache"].dtype, 256)
+        assert np_ > 1 and 0 < ws <= P.NOALLOC_SCRATCH_BYTES
+        out = torch.empty_like(c["q"])
+        P.paged_attention_decode_noalloc(c["q"], c["k_cache"], c["v_cache"], c["block_tables"], c["context_lens"],
+                                         c["scale"], c["maxc"], out, partition_tokens=256)
+        outs.append(out)
+    torch.cuda.synchronize()
+    for c, out in zip(cases, outs):
+        ref = P.paged_attention_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"], c["context_lens"],
+                                       c["scale"], max_context_len=c["maxc"], partition_tokens=256)
+        torch.cuda.synchronize()
+        _close(out, ref)
+    assert P.device_status(clear=True) == 0
+
+
+def test_noalloc_rejects_work_beyond_its_scratch():
+    c = _case(7, 4)
+    # 4096 sequences x 64 query heads x 16 partitions of partials exceed the array
+    big_b, hq, hkv, d, maxc = 4096, 64, 8, 128, 16 * 256
+    _, _, ws = P.decode_plan(big_b, hq, hkv, d, maxc, torch.bfloat16, 256)
+    assert ws > P.NOALLOC_SCRATCH_BYTES
+    q = torch.empty((big_b, hq, d), dtype=torch.bfloat16, device=DEV)
+    bt = torch.zeros((big_b, 256), dtype=torch.int32, device=DEV)
+    cl = torch.zeros(big_b, dtype=torch.int32, device=DEV)
+    kc = torch.empty((8, hkv, 16, d), dtype=torch.bfloat16, device=DEV)
+    with pytest.raises(P.PagedKVError, match="scratch"):
+        P.paged_attention_decode_noalloc(q, kc, kc, bt, cl, 1 / math.sqrt(d), maxc, torch.empty_like(q),
+                                         partition_tokens=256)
+    del c
