@@ -59,6 +59,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     return ap.parse_args()
 
 
@@ -167,11 +168,13 @@ class DecodeWorkload:
     """A batch of sequences living in a paged cache on one GPU, advanced one
     decode step at a time through the library's public API."""
 
-    def __init__(self, name, cache, device, seed_offset=0):
+    def __init__(self, name, cache, device, seed_offset=0, batch=None):
         from paged_kv_cache_438_b200 import pagedkv as P
         self.P = P
         self.name = name
         spec = dict(I.WORKLOADS[name])
+        if batch is not None:
+            spec["batch"] = batch
         self.spec = spec
         self.dev = device
         seed = spec["seed"] + seed_offset
@@ -250,23 +253,22 @@ class DecodeWorkload:
         v = torch.randn((self.B, self.hkv, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
         return q, k, v
 
-    def device_step(self, q, k, v, slots, pairs, bt, cl, maxc, out, ws, ev=None):
-        """Launches of one step; returns the number of kernels launched."""
+    def device_step(self, q, k, v, slots, pairs, bt, cl, maxc, out, ws):
+        """Launches of one step; returns the number of kernels launched.  No
+        event sits between the write and the decode launch, so the decode may
+        start its prologue while the write finishes."""
         P = self.P
         n = 0
         if pairs is not None and pairs.numel():
             P.copy_blocks(self.k_cache, self.v_cache, pairs, self.k_scale, self.v_scale)
             n += 1
         P.kv_cache_write(k, v, self.k_cache, self.v_cache, slots, self.k_scale, self.v_scale)
-        n += 1
-        if ev is not None:
-            ev[0].record()
-        P.paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.scale, self.k_scale, self.v_scale,
-                                 max_context_len=maxc, out=out, workspace=ws)
-        if ev is not None:
-            ev[1].record()
-        npart = P.decode_plan(self.B, self.hq, self.hkv, self.d, maxc, self.k_cache.dtype)[0]
-        return n + (2 if npart > 1 else 1)
+        self.decode(q, bt, cl, maxc, out, ws)
+        return n + 2
+
+    def decode(self, q, bt, cl, maxc, out, ws):
+        self.P.paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.scale, self.k_scale,
+                                      self.v_scale, max_context_len=maxc, out=out, workspace=ws)
 
 
 # ------------------------------------------------------------------ ours --
@@ -276,7 +278,7 @@ def run_ours(args, rank, world, device):
     from paged_kv_cache_438_b200 import pagedkv as P
     build.build()
     P.lib()
-    wl = DecodeWorkload(args.workload, args.cache, device, seed_offset=1000 * rank)
+    wl = DecodeWorkload(args.workload, args.cache, device, seed_offset=1000 * rank, batch=args.batch)
     K, W = args.steps, args.warmup
     # host allocator outputs of every step, staged in HBM before timing
     staged = []
@@ -288,7 +290,7 @@ def run_ours(args, rank, world, device):
                            kv=wl.kv_bytes(cl)))
     maxc_all = max(s["maxc"] for s in staged)
     _, _, ws_bytes = P.decode_plan(wl.B, wl.hq, wl.hkv, wl.d, maxc_all, wl.k_cache.dtype)
-    ws = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=device)
+    ws = P.new_workspace(device, ws_bytes)
     out = torch.empty((wl.B, wl.hq, wl.d), dtype=wl.dtype, device=device)
     kv_step = staged[0]["kv"]
     flush = kv_step < 4 * L2_BYTES
@@ -309,7 +311,6 @@ def run_ours(args, rank, world, device):
     sampler.wait_ready()
     roll(wl, staged[:W], out, ws, flush, scrub, device, seconds=0.4)   # busy window before the timed steps
     step_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
-    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     launches = 0
     kv_total = 0
     torch.cuda.synchronize(device)
@@ -320,7 +321,7 @@ def run_ours(args, rank, world, device):
         st = staged[W + i]
         step_ev[i][0].record(stream)
         launches += wl.device_step(st["q"], st["k"], st["v"], st["slots"], st["pairs"], st["bt"], st["cl"],
-                                   st["maxc"], out, ws, ev=dec_ev[i])
+                                   st["maxc"], out, ws)
         step_ev[i][1].record(stream)
         kv_total += st["kv"]
         if flush:
@@ -331,6 +332,17 @@ def run_ours(args, rank, world, device):
     clocks = sampler.stop()
     wall_ms = t0.elapsed_time(t1)
     step_ms = sum(a.elapsed_time(b) for a, b in step_ev)       # excludes L2 scrubs
+    # the decode kernel alone, for its roofline: the timed steps' decode calls
+    # again, each bracketed by events on the launching stream
+    dec_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for i in range(K):
+        st = staged[W + i]
+        if flush:
+            scrub.zero_()
+        dec_ev[i][0].record(stream)
+        wl.decode(st["q"], st["bt"], st["cl"], st["maxc"], out, ws)
+        dec_ev[i][1].record(stream)
+    torch.cuda.synchronize(device)
     dec_ms = sum(a.elapsed_time(b) for a, b in dec_ev)
     timed_ms = step_ms if flush else wall_ms
     status = P.device_status(clear=True)
@@ -532,9 +544,10 @@ def main():
     seqsteps = r["seqsteps_all"] / (r["timed_ms"] * 1e-3)
     # roofline of the decode call (decode kernel + reduce when split) on this rank
     dec_ms = r["dec_ms"] / r["K"]
-    npart, ptok, ws_bytes = wl.P.decode_plan(wl.B, wl.hq, wl.hkv, wl.d, r["maxc"], wl.k_cache.dtype)
+    nstreams, stream_tokens, ws_bytes = wl.P.decode_plan(wl.B, wl.hq, wl.hkv, wl.d, r["maxc"], wl.k_cache.dtype)
     kv_call = r["kv_rank"] / r["K"]
-    small = wl.B * wl.hq * wl.d * 2 * 2 + wl.B * wl.max_blocks * 4 // 16 + (2 * ws_bytes if npart > 1 else 0)
+    # q read + out written + the block-table entries the step reads
+    small = wl.B * wl.hq * wl.d * 2 * 2 + (kv_call // (wl.hkv * wl.d * 2 * wl.elt * 16)) * 4
     alg_bytes = kv_call + small
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
     traffic = recorded_traffic(args.workload, args.cache)
@@ -547,16 +560,17 @@ def main():
         "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload, "batch": wl.B,
                    "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.d, "block_size": 16,
                    "cache": args.cache or ("bf16" if wl.dtype == torch.bfloat16 else "f16"),
-                   "kv_bytes_per_step": r["kv_step"], "partitions": npart, "partition_tokens": ptok,
+                   "kv_bytes_per_step": r["kv_step"], "decode_warp_streams": nstreams,
                    "l2": "L2 scrubbed (512 MiB) between steps, outside the step events" if r["flush"]
                    else "inputs larger than L2 (KV read per step > 4 x 126 MB)",
                    "parallelism": f"replicas x{world} (independent batches)"},
         "seq_steps_per_s": round(seqsteps, 1),
         "pct_of_hbm_measured": round(100 * value / (peak * world), 2),
         "pct_of_hbm_nominal_8tbs": round(100 * value / (NOMINAL_HBM_GBS * world), 2),
-        "roofline": {"kernel": "paged_attention_decode (decode kernel + split reduce)", "bound": "hbm",
+        "roofline": {"kernel": "paged_decode_kernel (one launch per decode call)", "bound": "hbm",
                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                      "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
+                     "timing": "decode-only launches of the timed steps' inputs, CUDA events on the launching stream",
                      "traffic": traffic, "algorithmic_bytes_per_call": int(alg_bytes),
                      "ms_per_call": round(dec_ms, 4)},
         "gpu_launches": r["launches"],

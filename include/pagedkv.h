@@ -106,15 +106,22 @@ int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cach
                        int in_dtype, int cache_dtype, void* stream);
 
 /*
- * pkv_decode_plan -- how pkv_paged_attention_decode will split the work.
- *   The long-context split (token partitions whose partial softmax results
- *   are merged by a log-sum-exp reduce) is this library's choice; the pages
- *   do not prescribe one.
- * partition_tokens : 0 = automatic, else a multiple of 16 (tokens per
- *                 partition).  Pass the same value to the decode call.
- * num_partitions_out, partition_tokens_out : the chosen split (1 partition
- *                 means a single pass with no workspace).
- * workspace_bytes_out : device workspace decode needs (0 for one partition).
+ * pkv_decode_plan -- how pkv_paged_attention_decode will divide the work.
+ *   The decode streams the ordered list of (sequence, KV head, block) items
+ *   through warps that each own an equal contiguous share of it (a persistent
+ *   grid of about two CTAs per SM by default).  A (sequence, head) pair whose
+ *   blocks span several warps is merged from per-warp partial softmax results
+ *   by a log-sum-exp rule.  This split is the library's choice; the pages do
+ *   not prescribe one.
+ * partition_tokens : 0 = automatic, else a multiple of 16 capping the tokens
+ *                 one warp processes (more warps, more merging).  Pass the
+ *                 same value to the decode call.
+ * num_partitions_out   : the number of warp streams.
+ * partition_tokens_out : the most tokens one stream processes (bounded with
+ *                 max_context_len).
+ * workspace_bytes_out : device workspace the decode needs: arrival counters
+ *                 and partial results; needed whenever there is more than one
+ *                 stream.
  * Depends only on its arguments and the current device's SM count.
  */
 int pkv_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
@@ -152,9 +159,19 @@ int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, i
  * max_context_len: host-side upper bound of context_lens (sizes the grid).
  * num_q_heads / num_kv_heads = G must be an integer in [1, 16].
  * partition_tokens: as for pkv_decode_plan.
- * workspace      : device scratch of at least the planned bytes (may be NULL
- *                  when the plan has one partition); 16-byte aligned.
- * Alignment: k_cache, v_cache, scales and workspace 16 bytes; q, out 4 bytes.
+ * workspace      : device scratch of at least the planned bytes, 256-byte
+ *                  aligned (may be NULL when the plan has one stream).  It
+ *                  must be zero-filled before its first use; afterwards the
+ *                  library leaves it valid for the next call (its counters are
+ *                  tagged with a per-call epoch).  One workspace serves one
+ *                  call at a time: calls that overlap on the GPU need separate
+ *                  workspaces.
+ * The kernel is launched with programmatic stream serialisation: it may
+ * start while the immediately preceding kernel on the stream is finishing,
+ * and waits for that kernel to complete before it reads q, the caches, or
+ * writes out.  (This library's KV write kernel allows that early start; any
+ * other preceding kernel completes first as usual.)
+ * Alignment: k_cache, v_cache and scales 16 bytes; q, out 4 bytes.
  */
 int pkv_paged_attention_decode(void* out, const void* q,
                                const void* k_cache, const void* v_cache,
@@ -184,8 +201,9 @@ int pkv_paged_attention_decode(void* out, const void* q,
  *     that first call before any stream capture.
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents.  Nothing in it needs to start at zero (every partial is written
- *     before it is read), but calls that overlap on the GPU (concurrent
+ *     contents.  The array starts zero-filled (as a __device__ array does at
+ *     load), which is the only state its arrival counters need; partials are
+ *     written before they are read.  Calls that overlap on the GPU (concurrent
  *     streams, or other threads) race on it and give wrong results; serialise
  *     them, e.g. on one stream.
  */

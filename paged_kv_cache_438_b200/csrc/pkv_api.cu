@@ -9,6 +9,7 @@
 #include <atomic>
 #include <cmath>
 #include <mutex>
+#include <unordered_map>
 #include <unordered_set>
 #include <vector>
 
@@ -84,120 +85,142 @@ int make_cache_map(CUtensorMap* map, const void* cache, int head_dim, int elt, l
 }
 
 // ------------------------------------------------------------ planning --
-constexpr int kMaxPartitionBlocks = 2048;
+constexpr int kDecodeWarps = 4;          // warps per decode CTA (DecodeTraits::kWarps)
+constexpr int kMaxCtaSmem = 227 * 1024;  // opt-in shared memory per CTA on sm_100
 
 struct Plan {
-  int num_partitions;
-  int partition_blocks;
-  size_t workspace;
+  int num_streams;     // warps that share the (sequence, head, block) work list
+  int stream_tokens;   // upper bound of tokens one stream processes
+  size_t workspace;    // arrival counters + partial slots
+  size_t counter_bytes;
+  int slot_floats;
 };
+
+// One partial: m[G] and l[G] padded to a multiple of 4 floats, then o[G][D];
+// every slot and its o rows stay 16-byte aligned.
+int slot_floats(int G, int D) { return (2 * G + 3) / 4 * 4 + G * D; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// Split the token range of each (sequence, KV head) into partitions so that
-// the grid holds enough CTAs to cover all SMs a few times over, with
-// partitions as long as that allows (fewer partials, less per-CTA setup).
-int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int req_tokens, Plan* out) {
-  const int blocks_max = std::max(1, (max_ctx + 15) / 16);
-  int pb;
+// The work list has at most B * Hkv * ceil(max_ctx / 16) items.  By default
+// it is spread over the warps of the resident CTAs (one per SM for 16-bit
+// caches, two for 8-bit: a persistent grid)
+// but never thinner than 16 blocks per warp; partition_tokens > 0 instead caps
+// the items per warp at partition_tokens / 16.
+int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int req_tokens, Plan* out) {
+  const long long blocks_max = std::max(1, (max_ctx + 15) / 16);
+  const long long t_max = static_cast<long long>(std::max(B, 1)) * Hkv * blocks_max;
+  if (t_max >= (1LL << 31)) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31 (sequence, head, block) items");
+  long long nw;
   if (req_tokens > 0) {
     if (req_tokens % 16 != 0) return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d is not a multiple of 16", req_tokens);
-    pb = std::min(req_tokens / 16, blocks_max);
-    if (pb > kMaxPartitionBlocks && pb < blocks_max)
-      return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d exceeds %d", req_tokens, kMaxPartitionBlocks * 16);
+    const long long per = req_tokens / 16;
+    nw = (t_max + per - 1) / per;
   } else {
-    const long long target = 8LL * 2 * sm_count();  // ~8 waves of 2 resident CTAs per SM
-    const long long pairs = static_cast<long long>(B) * Hkv;
-    pb = 16;
-    while (pb < blocks_max && pairs * ((blocks_max + pb - 1) / pb) > target) pb *= 2;
-    pb = std::min(pb, blocks_max);
+    const long long resident = static_cast<long long>(is8(cache_dtype) ? 2 : 1) * kDecodeWarps * sm_count();
+    nw = std::min(resident, (t_max + 15) / 16);
   }
-  if (pb > kMaxPartitionBlocks) pb = kMaxPartitionBlocks;
-  const int np = (blocks_max + pb - 1) / pb;
-  out->num_partitions = np;
-  out->partition_blocks = np == 1 ? std::max(pb, blocks_max) : pb;
-  if (np == 1 && out->partition_blocks > kMaxPartitionBlocks) out->partition_blocks = blocks_max;
-  if (np > 1) {
-    const size_t rows = static_cast<size_t>(B) * Hq * np;
-    out->workspace = align_up(rows * 4, 256) * 2 + rows * static_cast<size_t>(D) * 4;
-  } else {
-    out->workspace = 0;
-  }
+  nw = std::max(1LL, std::min(nw, t_max));
+  if (nw > (1LL << 24)) return fail(PKV_ERR_UNSUPPORTED, "more than 2^24 decode streams");
+  const int G = Hq / Hkv;
+  out->num_streams = static_cast<int>(nw);
+  out->stream_tokens = static_cast<int>((t_max + nw - 1) / nw * 16);
+  out->counter_bytes = align_up(static_cast<size_t>(std::max(B, 1)) * Hkv * 8, 256);
+  out->slot_floats = slot_floats(G, D);
+  out->workspace = out->counter_bytes + 2 * static_cast<size_t>(nw) * out->slot_floats * 4;
   return PKV_OK;
 }
 
+// Monotonic epoch of decode calls (40 bits, never 0): tags the arrival
+// counters so a workspace needs zeroing only before its first use.
+unsigned long long next_epoch() {
+  static std::atomic<unsigned long long> epoch{0};
+  unsigned long long e;
+  do {
+    e = (epoch.fetch_add(1) + 1) & ((1ull << 40) - 1);
+  } while (e == 0);
+  return e;
+}
+
 template <class T>
-int set_smem_once(T* kernel, size_t bytes) {
-  // cudaFuncSetAttribute is per device; remember (device, kernel) pairs done.
+int set_smem(T* kernel, size_t bytes) {
+  // cudaFuncSetAttribute is per device; remember the largest value set for
+  // each (device, kernel).
   static std::mutex mu;
-  static std::unordered_set<unsigned long long> done;
+  static std::unordered_map<unsigned long long, size_t> done;
   int dev = 0;
   cudaGetDevice(&dev);
   const unsigned long long key = (reinterpret_cast<uintptr_t>(kernel) << 8) ^ static_cast<unsigned>(dev);
   std::lock_guard<std::mutex> lk(mu);
-  if (done.count(key)) return PKV_OK;
+  auto it = done.find(key);
+  if (it != done.end() && it->second >= bytes) return PKV_OK;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes));
   if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute");
-  done.insert(key);
+  done[key] = bytes;
   return PKV_OK;
 }
 
 template <int kD, int kCT>
-size_t decode_smem_bytes(int partition_blocks) {
+size_t decode_smem_bytes(int num_seqs) {
   using Tr = pkv::DecodeTraits<kD, kCT>;
   return 1024 + static_cast<size_t>(Tr::kWarps) * Tr::kRing * Tr::kStageBytes + Tr::kWarps * Tr::kRing * 8 +
-         static_cast<size_t>(partition_blocks) * 4;
+         (static_cast<size_t>(num_seqs) + 1) * 4;
 }
 
 template <int kD, int kCT, int kNT, bool kQBF16>
-int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, int num_seqs,
-                  cudaStream_t st) {
+int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, cudaStream_t st) {
   using Tr = pkv::DecodeTraits<kD, kCT>;
+  static_assert(Tr::kWarps == kDecodeWarps, "plan and kernel disagree on warps per CTA");
+  static_assert(Tr::kCtasPerSm == (Tr::k8bit ? 2 : 1), "plan and kernel disagree on CTAs per SM");
   auto kernel = pkv::paged_decode_kernel<kD, kCT, kNT, kQBF16>;
-  const size_t smem = decode_smem_bytes<kD, kCT>(p.partition_blocks);
-  const size_t smem_max = decode_smem_bytes<kD, kCT>(kMaxPartitionBlocks);
-  int rc = set_smem_once(kernel, smem_max);
+  const size_t smem = decode_smem_bytes<kD, kCT>(p.num_seqs);
+  if (smem > static_cast<size_t>(kMaxCtaSmem))
+    return fail(PKV_ERR_UNSUPPORTED, "batch of %d sequences needs %zu bytes of shared memory", p.num_seqs, smem);
+  int rc = set_smem(kernel, smem);
   if (rc != PKV_OK) return rc;
-  dim3 grid(p.num_partitions, p.num_kv_heads, num_seqs);
-  kernel<<<grid, Tr::kWarps * 32, smem, st>>>(km, vm, p);
-  cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((p.num_streams + Tr::kWarps - 1) / Tr::kWarps);
+  cfg.blockDim = dim3(Tr::kWarps * 32);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  // may start while the preceding kernel (the KV write) finishes; the kernel
+  // waits for it (griddepcontrol.wait) before reading the cache
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, km, vm, p);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  if (p.num_partitions > 1) {
-    constexpr bool kOutBF16 = (kCT == pkv::kI8 || kCT == pkv::kFP8) ? kQBF16 : (kCT == pkv::kBF16);
-    dim3 rgrid(p.num_q_heads, num_seqs);
-    pkv::paged_reduce_kernel<kD, kOutBF16><<<rgrid, kD, 0, st>>>(p);
-    e = cudaGetLastError();
-    if (e != cudaSuccess) return cuda_fail(e, "reduce launch");
-  }
   return PKV_OK;
 }
 
 template <int kD, int kCT>
-int dispatch_nt_q(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, int num_seqs,
-                  bool q_bf16, cudaStream_t st) {
+int dispatch_nt_q(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, bool q_bf16,
+                  cudaStream_t st) {
   const bool nt2 = p.group > 8;
   if constexpr (kCT == pkv::kI8 || kCT == pkv::kFP8) {
     if (q_bf16)
-      return nt2 ? launch_decode<kD, kCT, 2, true>(km, vm, p, num_seqs, st)
-                 : launch_decode<kD, kCT, 1, true>(km, vm, p, num_seqs, st);
-    return nt2 ? launch_decode<kD, kCT, 2, false>(km, vm, p, num_seqs, st)
-               : launch_decode<kD, kCT, 1, false>(km, vm, p, num_seqs, st);
+      return nt2 ? launch_decode<kD, kCT, 2, true>(km, vm, p, st)
+                 : launch_decode<kD, kCT, 1, true>(km, vm, p, st);
+    return nt2 ? launch_decode<kD, kCT, 2, false>(km, vm, p, st)
+               : launch_decode<kD, kCT, 1, false>(km, vm, p, st);
   } else {
     (void)q_bf16;
     constexpr bool kQ = (kCT == pkv::kBF16);
-    return nt2 ? launch_decode<kD, kCT, 2, kQ>(km, vm, p, num_seqs, st)
-               : launch_decode<kD, kCT, 1, kQ>(km, vm, p, num_seqs, st);
+    return nt2 ? launch_decode<kD, kCT, 2, kQ>(km, vm, p, st)
+               : launch_decode<kD, kCT, 1, kQ>(km, vm, p, st);
   }
 }
 
 template <int kD>
-int dispatch_ct(int ct, const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, int num_seqs,
-                bool q_bf16, cudaStream_t st) {
+int dispatch_ct(int ct, const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, bool q_bf16,
+                cudaStream_t st) {
   switch (ct) {
-    case PKV_F16: return dispatch_nt_q<kD, pkv::kF16>(km, vm, p, num_seqs, q_bf16, st);
-    case PKV_BF16: return dispatch_nt_q<kD, pkv::kBF16>(km, vm, p, num_seqs, q_bf16, st);
-    case PKV_I8: return dispatch_nt_q<kD, pkv::kI8>(km, vm, p, num_seqs, q_bf16, st);
-    case PKV_FP8E4M3: return dispatch_nt_q<kD, pkv::kFP8>(km, vm, p, num_seqs, q_bf16, st);
+    case PKV_F16: return dispatch_nt_q<kD, pkv::kF16>(km, vm, p, q_bf16, st);
+    case PKV_BF16: return dispatch_nt_q<kD, pkv::kBF16>(km, vm, p, q_bf16, st);
+    case PKV_I8: return dispatch_nt_q<kD, pkv::kI8>(km, vm, p, q_bf16, st);
+    case PKV_FP8E4M3: return dispatch_nt_q<kD, pkv::kFP8>(km, vm, p, q_bf16, st);
   }
   return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", ct);
 }
@@ -304,10 +327,10 @@ int pkv_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
   if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
   if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
   Plan pl{};
-  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, &pl);
+  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens, &pl);
   if (rc != PKV_OK) return rc;
-  if (num_partitions_out) *num_partitions_out = pl.num_partitions;
-  if (partition_tokens_out) *partition_tokens_out = pl.partition_blocks * 16;
+  if (num_partitions_out) *num_partitions_out = pl.num_streams;
+  if (partition_tokens_out) *partition_tokens_out = pl.stream_tokens;
   if (workspace_bytes_out) *workspace_bytes_out = pl.workspace;
   return ok();
 }
@@ -349,10 +372,10 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   if (is8(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 16) || !aligned(v_scale, 16)))
     return fail(PKV_ERR_INVALID_ARG, "quantised caches need 16-byte aligned k_scale and v_scale");
   Plan pl{};
-  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, &pl);
+  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens, &pl);
   if (rc != PKV_OK) return rc;
-  if (pl.num_partitions > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned(workspace, 16)))
-    return fail(PKV_ERR_INVALID_ARG, "workspace of %zu bytes (16-byte aligned) required, got %zu", pl.workspace,
+  if (pl.num_streams > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned(workspace, 256)))
+    return fail(PKV_ERR_INVALID_ARG, "workspace of %zu bytes (256-byte aligned) required, got %zu", pl.workspace,
                 workspace ? workspace_bytes : 0);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (g_validate.load()) {
@@ -382,25 +405,25 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   p.v_scale = v_scale;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
-  if (pl.num_partitions > 1) {
-    const size_t rowsp = static_cast<size_t>(num_seqs) * num_q_heads * pl.num_partitions;
+  if (pl.num_streams > 1) {
     auto* ws = static_cast<uint8_t*>(workspace);
-    p.part_m = reinterpret_cast<float*>(ws);
-    p.part_l = reinterpret_cast<float*>(ws + align_up(rowsp * 4, 256));
-    p.part_o = reinterpret_cast<float*>(ws + 2 * align_up(rowsp * 4, 256));
+    p.counters = reinterpret_cast<unsigned long long*>(ws);
+    p.slots = reinterpret_cast<float*>(ws + pl.counter_bytes);
   }
+  p.num_seqs = num_seqs;
   p.num_q_heads = num_q_heads;
   p.num_kv_heads = num_kv_heads;
   p.group = G;
   p.max_blocks_per_seq = max_blocks_per_seq;
   p.num_blocks = num_blocks;
-  p.partition_blocks = pl.partition_blocks;
-  p.num_partitions = pl.num_partitions;
   p.max_context_len = max_context_len;
+  p.num_streams = pl.num_streams;
+  p.slot_floats = pl.slot_floats;
+  p.epoch = next_epoch();
   p.qk_scale_log2 = scale * 1.4426950408889634f;
   const bool q_bf16 = q_dtype == PKV_BF16;
-  rc = head_dim == 128 ? dispatch_ct<128>(cache_dtype, km, vm, p, num_seqs, q_bf16, st)
-                       : dispatch_ct<64>(cache_dtype, km, vm, p, num_seqs, q_bf16, st);
+  rc = head_dim == 128 ? dispatch_ct<128>(cache_dtype, km, vm, p, q_bf16, st)
+                       : dispatch_ct<64>(cache_dtype, km, vm, p, q_bf16, st);
   if (rc != PKV_OK) return rc;
   return ok();
 }
@@ -500,21 +523,22 @@ extern "C" int pkv_paged_attention_decode_noalloc(void* out, const void* q, cons
     return fail(PKV_ERR_INVALID_ARG, "bad sizes");
   if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
   Plan pl{};
-  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, partition_tokens, &pl);
+  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens, &pl);
   if (rc != PKV_OK) return rc;
-  if (pl.workspace > kNoAllocScratchBytes)
+  const bool needs_scratch = pl.num_streams > 1;
+  if (needs_scratch && pl.workspace > kNoAllocScratchBytes)
     return fail(PKV_ERR_INVALID_ARG,
                 "this decode needs %zu bytes of split-KV scratch but the built-in array holds %zu "
                 "(PKV_NOALLOC_SCRATCH_BYTES); use fewer sequences per call, a larger partition_tokens, "
                 "or pkv_paged_attention_decode with a caller workspace",
                 pl.workspace, kNoAllocScratchBytes);
   void* scratch = nullptr;
-  if (pl.workspace > 0) {
+  if (needs_scratch) {
     rc = noalloc_scratch_address(&scratch);
     if (rc != PKV_OK) return rc;
   }
   return pkv_paged_attention_decode(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
                                     num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                     max_blocks_per_seq, max_context_len, scale, q_dtype, cache_dtype,
-                                    partition_tokens, scratch, pl.workspace > 0 ? kNoAllocScratchBytes : 0, stream);
+                                    partition_tokens, scratch, needs_scratch ? kNoAllocScratchBytes : 0, stream);
 }

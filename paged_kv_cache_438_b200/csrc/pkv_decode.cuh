@@ -1,30 +1,45 @@
 // Single-query GQA decode attention over a block-table-indexed KV cache.
 //
-// Method ("LLM 推理优化深度解析" §KV Cache 的本质, §MQA 与 GQA, §PagedAttention；
+// Method ("LLM 推理优化深度解析" §KV Cache 的本质, §MQA 与 GQA, §PagedAttention;
 // ascendai.csdn.net article §二 Fig. 2): every sequence's one new query per
 // head attends to all of its cached keys/values; the cache lives in 16-token
 // physical blocks reached through the sequence's block table; query head i
 // reads KV head i / G.
 //
 // Design for sm_100a (HBM-bound: every K/V byte is read once):
-//   * grid = (partition, kv_head, sequence); one CTA serves the whole GQA
-//     group of a KV head, so the group's G queries share one read of K/V;
-//   * each warp owns a ring of kR shared-memory stages fed by TMA: per
-//     16-token block, 2-D tiled tensor copies of the K and V rows (128-byte
-//     swizzle, so ldmatrix reads are bank-conflict free) plus untiled bulk
-//     copies of the per-token scales of quantised caches, completing on one
-//     mbarrier per stage; waits are bounded;
-//   * both contractions run on the tensor cores with the block's 16 tokens
-//     as the M dimension and the (zero-padded) query group as N = 8:
+//   * Work list.  All (sequence, KV head, block) triples form one ordered
+//     list (sequence-major).  Each warp of a persistent grid (one CTA of four
+//     warps per SM for 16-bit caches, two for 8-bit) owns an equal contiguous
+//     share of it and streams
+//     through that share, crossing (sequence, head) boundaries without
+//     stopping its copy pipeline.  The G query heads of a KV head are served
+//     together, so the group shares one read of K/V.
+//   * Copies.  Each warp owns a ring of shared-memory stages fed by TMA: per
+//     block, 2-D tiled tensor copies of the 16-token K and V tiles (128-byte
+//     swizzle, 64-byte for 64-byte rows, so ldmatrix reads are bank-conflict
+//     free) plus untiled bulk copies of the per-token scales of quantised
+//     caches, completing on one mbarrier per stage.  Block ids and copy
+//     coordinates for the next 32-block chunk are computed ahead by the lanes.
+//     Waits are bounded.
+//   * Math.  Both contractions run on the tensor cores with the block's 16
+//     tokens as M and the zero-padded query group as N = 8:
 //       S^T[16 tok x 8 g]  = K[16 x D] . Q^T[D x 8]         (mma.m16n8k16)
 //       O^T[D x 8 g]      += V^T[D x 16 tok] . P^T[16 x 8]
-//     P^T is built from the S^T accumulators in registers with movmatrix;
-//     8-bit codes are widened to fp16 in registers (int8 exactly through the
-//     0x6400 exponent trick, e4m3 with the hardware converter) and their
-//     per-token scales fold into S (keys) and P (values);
-//   * online softmax in fp32 (base-2 exponentials), per warp; warps merge
-//     through shared memory with a log-sum-exp rule; long contexts split into
-//     token partitions whose (m, l, o) partials a reduce kernel merges.
+//     P^T comes from the S^T accumulators through movmatrix.  8-bit codes
+//     are widened to fp16 in registers (int8 exactly through the 0x6400
+//     exponent trick, e4m3 with the hardware converter); per-token scales
+//     fold into S (keys) and P (values).  Online softmax in fp32, base 2.
+//   * Merge.  A warp that saw a whole (sequence, head) writes the output
+//     directly.  A pair split across warps gets one fp32 partial (m, l, o/l)
+//     per contributing warp; the last contributor to arrive (an epoch-tagged
+//     counter per pair, so nothing needs zeroing between calls) merges them
+//     with the log-sum-exp rule.  No warp ever waits for another.  Each warp
+//     processes the pair at the end of its share first (it is the one shared
+//     with the next warp), so merges happen early, not at the kernel's end.
+//   * The kernel may launch while the preceding KV write kernel still runs
+//     (programmatic dependent launch): it scans the context lengths, reads the
+//     block tables and q, and waits for the write only before its first copy
+//     from the cache.
 #pragma once
 
 #include "pkv_device.cuh"
@@ -49,8 +64,18 @@ struct DecodeTraits {
   static constexpr int kStageTx = 2 * kKVBytes + 2 * kScaleBytes;   // bytes landing per stage
   static constexpr int kStageBytes = round_up_c(kStageTx, 1024);    // keeps every tile 1024-aligned
   static constexpr int kWarps = 4;
-  static constexpr int kRing = (24 * 1024) / kStageBytes < 2 ? 2 : (24 * 1024) / kStageBytes;
+  // 16-bit caches run one CTA per SM with 4 stages of 8 KiB per warp; 8-bit
+  // caches (more conversion work per byte) run two CTAs per SM with ~24 KiB
+  // of ring per warp.
+  static constexpr int kRingBytes = k8bit ? 24 * 1024 : 32 * 1024;
+  static constexpr int kRing = kRingBytes / kStageBytes < 2 ? 2 : kRingBytes / kStageBytes;
+  static constexpr int kCtasPerSm = k8bit ? 2 : 1;
 };
+
+// Epoch-tagged arrival counters: bits 63..24 hold the epoch of the call that
+// last touched the counter, bits 23..0 the arrivals of that call.
+constexpr int kEpochShift = 24;
+constexpr unsigned long long kCountMask = (1ull << kEpochShift) - 1;
 
 struct DecodeParams {
   void* out;
@@ -59,22 +84,23 @@ struct DecodeParams {
   const float* v_scale;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  float* part_m;   // [B, Hq, NP]   (split only)
-  float* part_l;   // [B, Hq, NP]
-  float* part_o;   // [B, Hq, NP, D]
+  unsigned long long* counters;  // [B * Hkv] arrival counters (workspace)
+  float* slots;                  // [2 * num_streams][slot_floats] partials (workspace)
+  int num_seqs;
   int num_q_heads;
   int num_kv_heads;
   int group;
   int max_blocks_per_seq;
   int num_blocks;
-  int partition_blocks;
-  int num_partitions;
   int max_context_len;
-  float qk_scale_log2;  // softmax scale * log2(e)
+  int num_streams;   // warps sharing the work list
+  int slot_floats;   // ml + G * D: m[G], l[G] padded to ml = round_up(2G, 4), then o[G][D]
+  unsigned long long epoch;  // this call's epoch, nonzero, < 2^40
+  float qk_scale_log2;       // softmax scale * log2(e)
 };
 
 // Context length of sequence s as the kernels use it: clamped to what the
-// grid and the block table can cover (an out-of-range value raises a bit).
+// block table can hold (an out-of-range value raises a status bit).
 __device__ __forceinline__ int clamp_context(int ctx, int max_ctx, int max_blocks, bool report) {
   const int cap = min(max_ctx, max_blocks * 16);
   if (ctx < 0 || ctx > cap) {
@@ -123,6 +149,78 @@ __device__ __forceinline__ uint32_t load_q_pair(const void* q, long long idx) {
   return raw;
 }
 
+__device__ __forceinline__ int blocks_of(const DecodeParams& p, int s, bool report) {
+  return (clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, report) + 15) >> 4;
+}
+
+// cum[s] = sum over sequences s' < s of blocks(s') * Hkv, for s = 0..B; one
+// entry per (sequence, KV head, block) work item before sequence s.
+__device__ __forceinline__ void scan_work(const DecodeParams& p, int32_t* cum) {
+  __shared__ int warp_sums[32];
+  const int B = p.num_seqs;
+  const int nthreads = blockDim.x;
+  const int tid = threadIdx.x;
+  const int lane = tid & 31;
+  const int warp = tid >> 5;
+  const int per = (B + nthreads - 1) / nthreads;
+  const int s0 = min(tid * per, B);
+  const int s1 = min(s0 + per, B);
+  const bool report = blockIdx.x == 0;
+  int local = 0;
+  for (int s = s0; s < s1; ++s) local += blocks_of(p, s, report) * p.num_kv_heads;
+  int x = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  int run = x - local;
+  for (int w = 0; w < warp; ++w) run += warp_sums[w];
+  if (tid == 0) cum[0] = 0;
+  for (int s = s0; s < s1; ++s) {
+    run += blocks_of(p, s, false) * p.num_kv_heads;
+    cum[s + 1] = run;
+  }
+  __syncthreads();
+}
+
+// Largest s with cum[s] <= g (g < cum[B]); never lands on an empty sequence.
+__device__ __forceinline__ int find_seq(const int32_t* cum, int B, int g) {
+  int lo = 0, hi = B;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (cum[mid] <= g) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+// TMA row coordinate (block * Hkv + head) * 16 of work item g.
+__device__ __forceinline__ int item_row(const DecodeParams& p, const int32_t* cum, int g) {
+  const int s = find_seq(cum, p.num_seqs, g);
+  const int nb = (cum[s + 1] - cum[s]) / p.num_kv_heads;
+  const int off = g - cum[s];
+  const int h = off / nb;
+  const int j = off - h * nb;
+  int id = p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + j];
+  if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
+    raise_status(PKV_DEV_BAD_BLOCK);
+    id = 0;
+  }
+  return (id * p.num_kv_heads + h) * 16;
+}
+
+// First work item of stream w among T items split over nw streams.
+__device__ __forceinline__ int stream_start(long long T, long long w, long long nw) {
+  return static_cast<int>(T * w / nw);
+}
+
+// Stream holding work item g.
+__device__ __forceinline__ int stream_of(long long T, long long g, long long nw) {
+  return static_cast<int>(((g + 1) * nw - 1) / T);
+}
+
 template <int kD, int kCT, int kNT, bool kQBF16>
 __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -135,70 +233,72 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
   constexpr int kR = Tr::kRing;
   constexpr int kKS = kD / 16;  // k-steps of S^T = K Q^T
   constexpr int kMT = kD / 16;  // m-tiles of O^T = V^T P^T
-  constexpr int kGP = 8 * kNT;  // padded group
-  static_assert(kR * Tr::kStageBytes >= (2 * kGP + kGP * kD) * 4, "warp ring too small for the merge");
+  static_assert(kR <= 32, "ring deeper than a prefetch chunk");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
   const uint32_t base = (raw_addr + 1023u) & ~1023u;
   uint8_t* const base_ptr = smem_raw + (base - raw_addr);
   const uint32_t bar_base = base + kW * kR * Tr::kStageBytes;
-  int32_t* const blk_ids = reinterpret_cast<int32_t*>(base_ptr + kW * kR * Tr::kStageBytes + kW * kR * 8);
+  int32_t* const cum = reinterpret_cast<int32_t*>(base_ptr + kW * kR * Tr::kStageBytes + kW * kR * 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int r = lane >> 2;
   const int q4 = lane & 3;
-  const int part = blockIdx.x;
-  const int h = blockIdx.y;
-  const int s = blockIdx.z;
   const int G = p.group;
   const int Hq = p.num_q_heads;
-  const bool split = p.num_partitions > 1;
+  const int Hkv = p.num_kv_heads;
+  const int B = p.num_seqs;
 
-  const int ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq,
-                                threadIdx.x == 0 && part == 0 && h == 0);
-  const int tok_begin = part * p.partition_blocks * 16;
-  const int tok_end = min(ctx, tok_begin + p.partition_blocks * 16);
-  const int nblk = tok_end > tok_begin ? (tok_end - tok_begin + 15) / 16 : 0;
-  const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
-
-  if (nblk == 0) {
-    if (!split) {  // empty sequence: zero output rows
-      for (int idx = threadIdx.x; idx < G * kD; idx += blockDim.x)
-        store_out<kOutBF16>(p.out, head_row0 * kD + idx, 0.0f);
-    }
-    return;
-  }
-
-  // ---- block ids of this partition, barriers ----
-  const int32_t* bt = p.block_tables + static_cast<long long>(s) * p.max_blocks_per_seq +
-                      static_cast<long long>(part) * p.partition_blocks;
-  for (int i = threadIdx.x; i < nblk; i += blockDim.x) {
-    int id = bt[i];
-    if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
-      raise_status(PKV_DEV_BAD_BLOCK);
-      id = 0;
-    }
-    blk_ids[i] = id;
-  }
   if (lane == 0) {
 #pragma unroll
     for (int j = 0; j < kR; ++j) mbar_init(bar_base + (warp * kR + j) * 8, 1);
     fence_barrier_init();
   }
-  __syncthreads();
+  scan_work(p, cum);  // ends with __syncthreads (barrier init visible too)
 
-  const int count = nblk > warp ? (nblk - warp + kW - 1) / kW : 0;  // blocks of this warp
+  // Sequences without context get zero rows.  (Only the caches and scales can
+  // still be in flight from a KV write launched just before this kernel; the
+  // wait for it comes right before the first copy is issued.)
+  for (int s = blockIdx.x; s < B; s += gridDim.x) {
+    if (cum[s + 1] == cum[s]) {
+      for (int idx = threadIdx.x; idx < Hq * kD; idx += blockDim.x)
+        store_out<kOutBF16>(p.out, static_cast<long long>(s) * Hq * kD + idx, 0.0f);
+    }
+  }
+
+  const long long T = cum[B];
+  const long long nw = min(static_cast<long long>(p.num_streams), T);
+  const int gw = blockIdx.x * kW + warp;
+  if (gw >= nw) return;  // warps are independent from here on
+  const int g0 = stream_start(T, gw, nw);
+  const int g1 = stream_start(T, gw + 1, nw);
+  const int count = g1 - g0;
+  // The stream's last pair is usually shared with the next stream: process it
+  // first (then wrap to g0), so shared pairs finish early and their merges
+  // stay off the end of the kernel.  `offset` = local position of the start
+  // of the pair holding item g1 - 1 (0 if that pair began before g0).
+  int offset;
+  {
+    const int sl = find_seq(cum, B, g1 - 1);
+    const int nbl = (cum[sl + 1] - cum[sl]) / Hkv;
+    const int gpl = cum[sl] + ((g1 - 1 - cum[sl]) / nbl) * nbl;
+    offset = gpl > g0 ? gpl - g0 : 0;
+  }
+  auto item_of = [&](int k) { return g0 + (k + offset < count ? k + offset : k + offset - count); };
+
   const uint32_t ring = base + warp * kR * Tr::kStageBytes;
   const uint32_t bars = bar_base + warp * kR * 8;
 
-  auto issue = [&](int k) {
+  // Copy coordinates of this warp's items, 32 at a time, two chunks ahead.
+  int pre0 = lane < count ? item_row(p, cum, item_of(lane)) : 0;
+  int pre1 = 32 + lane < count ? item_row(p, cum, item_of(32 + lane)) : 0;
+
+  auto issue = [&](int k, int row0) {
     const int stage = k % kR;
     const uint32_t st = ring + stage * Tr::kStageBytes;
     const uint32_t bar = bars + stage * 8;
-    const int phys = blk_ids[warp + k * kW];
-    const int row0 = (phys * p.num_kv_heads + h) * 16;
     mbar_arrive_expect_tx(bar, Tr::kStageTx);
 #pragma unroll
     for (int ct = 0; ct < Tr::kNumColTiles; ++ct) {
@@ -207,97 +307,116 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
       tma_load_2d(st + Tr::kKVBytes + ct * Tr::kColTileBytes, &vmap, x, row0, bar);
     }
     if constexpr (k8) {
-      const long long so = static_cast<long long>(row0);
-      bulk_load(st + 2 * Tr::kKVBytes, p.k_scale + so, 64, bar);
-      bulk_load(st + 2 * Tr::kKVBytes + 64, p.v_scale + so, 64, bar);
+      bulk_load(st + 2 * Tr::kKVBytes, p.k_scale + row0, 64, bar);
+      bulk_load(st + 2 * Tr::kKVBytes + 64, p.v_scale + row0, 64, bar);
     }
   };
 
-  if (lane == 0) {
-    const int pre = count < kR ? count : kR;
-    for (int k = 0; k < pre; ++k) issue(k);
+  // the caches may still be being written by the preceding kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+#pragma unroll 1
+  for (int k = 0; k < kR && k < count; ++k) {
+    const int row0 = __shfl_sync(0xffffffffu, pre0, k);
+    if (lane == 0) issue(k, row0);
   }
 
-  // ---- query fragments: B operand of S^T = K Q^T (Q^T is D x 8 per n-tile) ----
+  // ---- cursor over (sequence, head, block), in processing order ----
+  int s, nb, h, j, ctx;
+  auto locate = [&](int g) {
+    s = find_seq(cum, B, g);
+    nb = (cum[s + 1] - cum[s]) / Hkv;
+    h = (g - cum[s]) / nb;
+    j = (g - cum[s]) - h * nb;
+    ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false);
+  };
+  locate(item_of(0));
+
   uint32_t qf[kNT][kKS][2];
-#pragma unroll
-  for (int nt = 0; nt < kNT; ++nt) {
-    const int g = nt * 8 + r;
-    const bool valid = g < G;
-    const long long qrow = (head_row0 + (valid ? g : 0)) * kD;
-#pragma unroll
-    for (int j = 0; j < kKS; ++j) {
-      // 16-bit K: k-index 2q,2q+1 -> d 16j+2q.. ; 2q+8.. -> d 16j+8+2q..
-      // 8-bit K:  k-index 2q,2q+1 -> d 16j+4q.. ; 2q+8.. -> d 16j+4q+2..
-      const int da = k8 ? 16 * j + 4 * q4 : 16 * j + 2 * q4;
-      const int db = k8 ? da + 2 : da + 8;
-      qf[nt][j][0] = valid ? load_q_pair<kCT, kQBF16>(p.q, qrow + da) : 0u;
-      qf[nt][j][1] = valid ? load_q_pair<kCT, kQBF16>(p.q, qrow + db) : 0u;
-    }
-  }
-
   float o[kMT][kNT][4];
   float m_run[kNT][2], l_run[kNT][2];
-#pragma unroll
-  for (int nt = 0; nt < kNT; ++nt) {
-    m_run[nt][0] = m_run[nt][1] = -INFINITY;
-    l_run[nt][0] = l_run[nt][1] = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kMT; ++i) o[i][nt][0] = o[i][nt][1] = o[i][nt][2] = o[i][nt][3] = 0.0f;
-  }
 
-  bool timed_out = false;
+  auto begin_pair = [&]() {
+    const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      const int g = nt * 8 + r;
+      const bool valid = g < G;
+      const long long qrow = (head_row0 + (valid ? g : 0)) * kD;
+#pragma unroll
+      for (int jj = 0; jj < kKS; ++jj) {
+        // 16-bit K: k-index 2q,2q+1 -> d 16jj+2q.. ; 2q+8.. -> d 16jj+8+2q..
+        // 8-bit K:  k-index 2q,2q+1 -> d 16jj+4q.. ; 2q+8.. -> d 16jj+4q+2..
+        const int da = k8 ? 16 * jj + 4 * q4 : 16 * jj + 2 * q4;
+        const int db = k8 ? da + 2 : da + 8;
+        qf[nt][jj][0] = valid ? load_q_pair<kCT, kQBF16>(p.q, qrow + da) : 0u;
+        qf[nt][jj][1] = valid ? load_q_pair<kCT, kQBF16>(p.q, qrow + db) : 0u;
+      }
+      m_run[nt][0] = m_run[nt][1] = -INFINITY;
+      l_run[nt][0] = l_run[nt][1] = 0.0f;
+#pragma unroll
+      for (int i = 0; i < kMT; ++i) o[i][nt][0] = o[i][nt][1] = o[i][nt][2] = o[i][nt][3] = 0.0f;
+    }
+  };
+  begin_pair();
+
+#pragma unroll 1
   for (int k = 0; k < count; ++k) {
     const int stage = k % kR;
     const uint32_t st = ring + stage * Tr::kStageBytes;
     const bool landed = mbar_wait(bars + stage * 8, (k / kR) & 1);
     if (__any_sync(0xffffffffu, !landed)) {  // warp-uniform: never split the warp before ldmatrix/mma
-      timed_out = true;
-      break;
+      // let copies already in flight land (bounded) before the warp leaves
+      for (int kk = k + 1; kk < count && kk < k + kR; ++kk) mbar_wait(bars + (kk % kR) * 8, (kk / kR) & 1);
+      return;
     }
-    const int tok0 = tok_begin + (warp + k * kW) * 16;
-    const int valid = tok_end - tok0;  // >= 1 tokens of this block count
+    const int valid = ctx - j * 16;  // >= 1 tokens of this block count
 
-    // ---- S^T = K . Q^T ----
-    float sacc[kNT][4];
+    // ---- S^T = K . Q^T (two independent accumulation chains, summed) ----
+    float sacc[kNT][4], sacc2[kNT][4];
 #pragma unroll
-    for (int nt = 0; nt < kNT; ++nt) sacc[nt][0] = sacc[nt][1] = sacc[nt][2] = sacc[nt][3] = 0.0f;
+    for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0.0f;
     if constexpr (!k8) {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int j = 0; j < kKS; ++j) {
+      for (int jj = 0; jj < kKS; ++jj) {
         uint32_t a0, a1, a2, a3;
-        ldsm_x4(st + swz<Tr>(t, 2 * j + (lane >> 4)), a0, a1, a2, a3);
+        ldsm_x4(st + swz<Tr>(t, 2 * jj + (lane >> 4)), a0, a1, a2, a3);
 #pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) mma_16816<kMmaBF16>(sacc[nt], a0, a1, a2, a3, qf[nt][j][0], qf[nt][j][1]);
+        for (int nt = 0; nt < kNT; ++nt)
+          mma_16816<kMmaBF16>((jj & 1) ? sacc2[nt] : sacc[nt], a0, a1, a2, a3, qf[nt][jj][0], qf[nt][jj][1]);
       }
     } else {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-      for (int j = 0; j < kKS; j += 2) {
+      for (int jj = 0; jj < kKS; jj += 2) {
         uint32_t w[4];
-        ldsm_x4(st + swz<Tr>(t, j + (lane >> 4)), w[0], w[1], w[2], w[3]);
+        ldsm_x4(st + swz<Tr>(t, jj + (lane >> 4)), w[0], w[1], w[2], w[3]);
 #pragma unroll
-        for (int jj = 0; jj < 2; ++jj) {
+        for (int j2 = 0; j2 < 2; ++j2) {
           uint32_t lo_r, hi_r, lo_r8, hi_r8;  // (d 4q,4q+1) and (d 4q+2,4q+3) of tokens r and r+8
           if constexpr (kCT == kI8) {
-            const uint32_t u0 = w[2 * jj] ^ 0x80808080u, u1 = w[2 * jj + 1] ^ 0x80808080u;
+            const uint32_t u0 = w[2 * j2] ^ 0x80808080u, u1 = w[2 * j2 + 1] ^ 0x80808080u;
             lo_r = i8pair_to_h2(u0, 0x4140u);
             hi_r = i8pair_to_h2(u0, 0x4342u);
             lo_r8 = i8pair_to_h2(u1, 0x4140u);
             hi_r8 = i8pair_to_h2(u1, 0x4342u);
           } else {
-            lo_r = e4m3pair_to_h2(w[2 * jj]);
-            hi_r = e4m3pair_to_h2(w[2 * jj] >> 16);
-            lo_r8 = e4m3pair_to_h2(w[2 * jj + 1]);
-            hi_r8 = e4m3pair_to_h2(w[2 * jj + 1] >> 16);
+            e4m3x4_to_h2x2(w[2 * j2], lo_r, hi_r);
+            e4m3x4_to_h2x2(w[2 * j2 + 1], lo_r8, hi_r8);
           }
 #pragma unroll
           for (int nt = 0; nt < kNT; ++nt)
-            mma_16816<false>(sacc[nt], lo_r, lo_r8, hi_r, hi_r8, qf[nt][j + jj][0], qf[nt][j + jj][1]);
+            mma_16816<false>(j2 ? sacc2[nt] : sacc[nt], lo_r, lo_r8, hi_r, hi_r8, qf[nt][jj + j2][0],
+                             qf[nt][jj + j2][1]);
         }
       }
     }
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
 
     // ---- scale, mask, online softmax (base 2) ----
     float f_r = p.qk_scale_log2, f_r8 = p.qk_scale_log2;
@@ -381,12 +500,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
             y0 = i8pair_to_h2(u1, 0x4240u);
             y1 = i8pair_to_h2(u1, 0x4341u);
           } else {
-            const uint32_t t0 = prmt(w[2 * ii], w[2 * ii], 0x3120u);
-            const uint32_t t1 = prmt(w[2 * ii + 1], w[2 * ii + 1], 0x3120u);
-            x0 = e4m3pair_to_h2(t0);
-            x1 = e4m3pair_to_h2(t0 >> 16);
-            y0 = e4m3pair_to_h2(t1);
-            y1 = e4m3pair_to_h2(t1 >> 16);
+            e4m3x4_to_h2x2(prmt(w[2 * ii], w[2 * ii], 0x3120u), x0, x1);
+            e4m3x4_to_h2x2(prmt(w[2 * ii + 1], w[2 * ii + 1], 0x3120u), y0, y1);
           }
 #pragma unroll
           for (int nt = 0; nt < kNT; ++nt) mma_16816<false>(o[i + ii][nt], x0, x1, y0, y1, pb[nt][0], pb[nt][1]);
@@ -394,108 +509,181 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
       }
     }
 
+    // ---- refill this stage with item k + kR ----
     __syncwarp();
-    if (lane == 0 && k + kR < count) issue(k + kR);
-  }
+    const int kn = k + kR;
+    if (kn < count) {
+      const int chunk = kn >> 5;
+      if ((kn & 31) == 0) {
+        // entering chunk `chunk` (held in pre[chunk & 1]); chunk - 1 is spent,
+        // so its register takes chunk + 1
+        const int ki = (chunk + 1) * 32 + lane;
+        const int nxt = ki < count ? item_row(p, cum, item_of(ki)) : 0;
+        if (chunk & 1) pre0 = nxt; else pre1 = nxt;
+      }
+      const int row0 = __shfl_sync(0xffffffffu, (chunk & 1) ? pre1 : pre0, kn & 31);
+      if (lane == 0) issue(kn, row0);
+    }
 
-  // ---- merge the warps of this CTA (log-sum-exp), then write ----
-  const bool any_timeout = __syncthreads_or(timed_out) != 0;
-  float* const wbase = reinterpret_cast<float*>(base_ptr);
-  const int region = kR * Tr::kStageBytes / 4;  // floats per warp region
-  if (!any_timeout) {
-    float* mw = wbase + warp * region;
-    float* lw = mw + kGP;
-    float* ow = lw + kGP;
+    // ---- advance; finish the (sequence, head) pair at its end or the stream's ----
+    ++j;
+    const bool wrap_next = offset > 0 && k + 1 == count - offset;  // next item is g0
+    if (j == nb || wrap_next || k == count - 1) {
+      float lsum[kNT][2];
 #pragma unroll
-    for (int nt = 0; nt < kNT; ++nt) {
-      float la = l_run[nt][0], lb = l_run[nt][1];
+      for (int nt = 0; nt < kNT; ++nt) {
+        float la = l_run[nt][0], lb = l_run[nt][1];
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        la += __shfl_xor_sync(0xffffffffu, la, off);
-        lb += __shfl_xor_sync(0xffffffffu, lb, off);
+        for (int off = 4; off < 32; off <<= 1) {
+          la += __shfl_xor_sync(0xffffffffu, la, off);
+          lb += __shfl_xor_sync(0xffffffffu, lb, off);
+        }
+        lsum[nt][0] = la;
+        lsum[nt][1] = lb;
       }
-      const int ga = nt * 8 + 2 * q4;
-      if (r == 0) {
-        mw[ga] = m_run[nt][0];
-        mw[ga + 1] = m_run[nt][1];
-        lw[ga] = la;
-        lw[ga + 1] = lb;
-      }
+      const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
+      const int gp0 = cum[s] + h * nb;  // the pair's first and last items
+      const int gpe = gp0 + nb - 1;
+      if (gp0 >= g0 && gpe < g1) {
+        // the whole pair went through this warp: write the output
 #pragma unroll
-      for (int i = 0; i < kMT; ++i) {
-        // output row d of the C fragment halves (c0,c1) and (c2,c3)
-        const int d0 = k8 ? 16 * i + 2 * r : 16 * i + r;
-        const int d1 = k8 ? d0 + 1 : d0 + 8;
-        ow[ga * kD + d0] = o[i][nt][0];
-        ow[(ga + 1) * kD + d0] = o[i][nt][1];
-        ow[ga * kD + d1] = o[i][nt][2];
-        ow[(ga + 1) * kD + d1] = o[i][nt][3];
+        for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int g = nt * 8 + 2 * q4 + c;
+            if (g >= G) continue;
+            const float inv = 1.0f / lsum[nt][c];
+#pragma unroll
+            for (int i = 0; i < kMT; ++i) {
+              const int d0 = k8 ? 16 * i + 2 * r : 16 * i + r;
+              const int d1 = k8 ? d0 + 1 : d0 + 8;
+              store_out<kOutBF16>(p.out, (head_row0 + g) * kD + d0, o[i][nt][c] * inv);
+              store_out<kOutBF16>(p.out, (head_row0 + g) * kD + d1, o[i][nt][2 + c] * inv);
+            }
+          }
+      } else {
+        // a share of a split pair: publish (m, l, o / l), then count arrivals
+        const int ml = p.slot_floats - G * kD;
+        float* slot = p.slots + static_cast<long long>(2 * gw + (gp0 <= g0 && g0 <= gpe ? 0 : 1)) * p.slot_floats;
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+          for (int c = 0; c < 2; ++c) {
+            const int g = nt * 8 + 2 * q4 + c;
+            if (g >= G) continue;
+            const float inv = 1.0f / lsum[nt][c];
+            if (r == 0) {
+              slot[g] = m_run[nt][c];
+              slot[G + g] = lsum[nt][c];
+            }
+            float* og = slot + ml + g * kD;
+#pragma unroll
+            for (int i = 0; i < kMT; ++i) {
+              const int d0 = k8 ? 16 * i + 2 * r : 16 * i + r;
+              const int d1 = k8 ? d0 + 1 : d0 + 8;
+              og[d0] = o[i][nt][c] * inv;
+              og[d1] = o[i][nt][2 + c] * inv;
+            }
+          }
+        __threadfence();
+        __syncwarp();
+        const int w_first = stream_of(T, gp0, nw);
+        const int n_c = stream_of(T, gpe, nw) - w_first + 1;
+        int last = 0;
+        if (lane == 0) {
+          unsigned long long* ctr = p.counters + static_cast<long long>(s) * Hkv + h;
+          const unsigned long long E = p.epoch;
+          unsigned long long old = atomicAdd(ctr, 0ull), assumed, next;
+          do {
+            assumed = old;
+            next = ((assumed >> kEpochShift) == E) ? assumed + 1 : ((E << kEpochShift) | 1ull);
+            old = atomicCAS(ctr, assumed, next);
+          } while (old != assumed);
+          last = static_cast<int>(next & kCountMask) == n_c;
+        }
+        last = __shfl_sync(0xffffffffu, last, 0);
+        if (last) {
+          __threadfence();
+          // contributor c = w_first + c keeps its share in slot 2w (the pair
+          // holds the stream's first item) or 2w + 1 (it does not)
+          auto slot_of = [&](int c) -> const float* {
+            const int w = w_first + c;
+            const int idx = 2 * w + (stream_start(T, w, nw) >= gp0 ? 0 : 1);
+            return p.slots + static_cast<long long>(idx) * p.slot_floats;
+          };
+          // Two rounds of independent loads: lane g (< G) first finds
+          // M[g] = max_c m_c[g]; then, per contributor, lanes g compute
+          // w_c[g] = 2^(m_c[g] - M[g]) l_c[g] (l_c[g] sits at lane G + g) and
+          // every lane accumulates w_c[g] o_c[g][its kV columns] for all g.
+          constexpr int kV = kD / 32;  // output columns per lane
+          constexpr int kG = 8 * kNT;
+          float Mv = -INFINITY;
+          for (int c = 0; c < n_c; ++c) {
+            const float v = lane < G ? __ldcg(slot_of(c) + lane) : -INFINITY;
+            Mv = fmaxf(Mv, v);
+          }
+          float Lv = 0.0f;
+          float acc[kG][kV];
+#pragma unroll
+          for (int g = 0; g < kG; ++g)
+#pragma unroll
+            for (int e = 0; e < kV; ++e) acc[g][e] = 0.0f;
+#pragma unroll 2
+          for (int c = 0; c < n_c; ++c) {
+            const float* sl = slot_of(c);
+            const float v = lane < 2 * G ? __ldcg(sl + lane) : 0.0f;
+            const float lc = __shfl_sync(0xffffffffu, v, (lane + G) & 31);
+            const float w = lane < G ? fast_exp2(v - Mv) * lc : 0.0f;
+            Lv += w;
+#pragma unroll
+            for (int g = 0; g < kG; ++g) {
+              if (g < G) {
+                const float wg = __shfl_sync(0xffffffffu, w, g);
+                const float* og = sl + ml + g * kD + lane * kV;
+                if constexpr (kV == 4) {
+                  const float4 ov = __ldcg(reinterpret_cast<const float4*>(og));
+                  acc[g][0] += wg * ov.x;
+                  acc[g][1] += wg * ov.y;
+                  acc[g][2] += wg * ov.z;
+                  acc[g][3] += wg * ov.w;
+                } else {
+                  const float2 ov = __ldcg(reinterpret_cast<const float2*>(og));
+                  acc[g][0] += wg * ov.x;
+                  acc[g][1] += wg * ov.y;
+                }
+              }
+            }
+          }
+#pragma unroll
+          for (int g = 0; g < kG; ++g) {
+            if (g < G) {
+              const float Lg = __shfl_sync(0xffffffffu, Lv, g);
+              const float inv = Lg > 0.0f ? 1.0f / Lg : 0.0f;
+#pragma unroll
+              for (int e = 0; e < kV; ++e)
+                store_out<kOutBF16>(p.out, (head_row0 + g) * kD + lane * kV + e, acc[g][e] * inv);
+            }
+          }
+        }
+      }
+      if (k + 1 < count) {  // the stream continues: back to g0, or the next non-empty pair
+        if (wrap_next) {
+          locate(g0);
+        } else {
+          j = 0;
+          if (++h == Hkv) {
+            h = 0;
+            do {
+              ++s;
+            } while (cum[s + 1] == cum[s]);
+            nb = (cum[s + 1] - cum[s]) / Hkv;
+            ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false);
+          }
+        }
+        begin_pair();
       }
     }
   }
-  __syncthreads();
-
-  const long long np = p.num_partitions;
-  for (int idx = threadIdx.x; idx < G * kD; idx += blockDim.x) {
-    const int g = idx / kD;
-    const int d = idx - g * kD;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kW; ++w) {
-      const float* mw = wbase + w * region;
-      if (w < nblk && !any_timeout) M = fmaxf(M, mw[g]);
-    }
-    float L = 0.0f, O = 0.0f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kW; ++w) {
-        if (w >= nblk) continue;
-        const float* mw = wbase + w * region;
-        const float e = fast_exp2(mw[g] - M);
-        L += e * mw[kGP + g];
-        O += e * mw[2 * kGP + g * kD + d];
-      }
-    }
-    const float val = L > 0.0f ? O / L : 0.0f;
-    const long long hrow = head_row0 + g;
-    if (!split) {
-      store_out<kOutBF16>(p.out, hrow * kD + d, val);
-    } else {
-      p.part_o[(hrow * np + part) * kD + d] = val;
-      if (d == 0) {
-        p.part_m[hrow * np + part] = M;
-        p.part_l[hrow * np + part] = L;
-      }
-    }
-  }
-}
-
-// Merges the partitions of each (sequence, query head):
-//   M = max_p m_p, w_p = 2^(m_p - M) l_p, out = sum_p w_p o_p / sum_p w_p.
-template <int kD, bool kOutBF16>
-__global__ void __launch_bounds__(kD) paged_reduce_kernel(DecodeParams p) {
-  const int i = blockIdx.x;
-  const int s = blockIdx.y;
-  const int d = threadIdx.x;
-  const int ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false);
-  const int ptok = p.partition_blocks * 16;
-  const int n = (ctx + ptok - 1) / ptok;
-  const long long hrow = static_cast<long long>(s) * p.num_q_heads + i;
-  const long long np = p.num_partitions;
-  const float* m = p.part_m + hrow * np;
-  const float* l = p.part_l + hrow * np;
-  const float* o = p.part_o + hrow * np * kD + d;
-  float M = -INFINITY;
-  for (int j = 0; j < n; ++j) M = fmaxf(M, m[j]);
-  float W = 0.0f, O = 0.0f;
-  if (M != -INFINITY) {
-    for (int j = 0; j < n; ++j) {
-      const float w = fast_exp2(m[j] - M) * l[j];
-      W += w;
-      O += w * o[j * kD];
-    }
-  }
-  store_out<kOutBF16>(p.out, hrow * kD + d, W > 0.0f ? O / W : 0.0f);
 }
 
 }  // namespace pkv

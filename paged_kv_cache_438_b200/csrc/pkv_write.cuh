@@ -25,6 +25,9 @@ __global__ void __launch_bounds__(256) kv_write_copy_kernel(const uint4* __restr
                                                             uint4* __restrict__ kc, uint4* __restrict__ vc,
                                                             const int64_t* __restrict__ slots, int num_tokens,
                                                             int num_kv_heads, int num_blocks) {
+  // a decode launched behind this write may start its prologue now; it waits
+  // for this grid to finish before it reads the cache
+  asm volatile("griddepcontrol.launch_dependents;");
   const long long total = static_cast<long long>(num_tokens) * num_kv_heads * kChunks;
   const long long slot_limit = static_cast<long long>(num_blocks) * kBlockTokens;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
@@ -86,6 +89,7 @@ __global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restr
                                                              const int64_t* __restrict__ slots, int num_tokens,
                                                              int num_kv_heads, int num_blocks) {
   constexpr int kE = kD / 32;
+  asm volatile("griddepcontrol.launch_dependents;");  // see kv_write_copy_kernel
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(num_tokens) * num_kv_heads;
   const long long slot_limit = static_cast<long long>(num_blocks) * kBlockTokens;

@@ -182,12 +182,35 @@ def kv_cache_write(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=N
 
 
 def decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens=0):
-    """(num_partitions, partition_tokens, workspace_bytes) the decode call uses."""
+    """(num_streams, tokens_per_stream_bound, workspace_bytes) the decode call
+    uses: the warps sharing the (sequence, head, block) work list, the most
+    tokens one of them processes, and the workspace it needs."""
     npart, ptok, ws = _I(0), _I(0), _SZ(0)
     ct = cache_dtype if isinstance(cache_dtype, int) else dtype_code(cache_dtype)
     _check(lib().pkv_decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, ct,
                                  partition_tokens, ctypes.byref(npart), ctypes.byref(ptok), ctypes.byref(ws)))
     return npart.value, ptok.value, ws.value
+
+
+_WORKSPACES = {}
+
+
+def _cached_workspace(device, stream, nbytes):
+    """A decode workspace for (device, stream): zero-filled when created (the
+    library needs zeros only before a workspace's first use) and grown on
+    demand.  One per stream, so calls on different streams never share one."""
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    key = (device.index, s.cuda_stream)
+    ws = _WORKSPACES.get(key)
+    if ws is None or ws.numel() < nbytes:
+        ws = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+        _WORKSPACES[key] = ws
+    return ws
+
+
+def new_workspace(device, nbytes):
+    """A zero-filled decode workspace of at least ``nbytes`` (see decode_plan)."""
+    return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale=None, v_scale=None,
@@ -197,7 +220,10 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     q [B, Hq, D] fp16/bf16; caches [NB, Hkv, 16, D]; block_tables [B, MB]
     int32; context_lens [B] int32.  ``max_context_len`` is a host-side upper
     bound on context_lens (if None it is read from the device, which
-    synchronises).  Returns ``out`` [B, Hq, D] in q's dtype."""
+    synchronises).  ``workspace`` (uint8, from ``new_workspace``) must be
+    zero-filled before its first use and serve one call at a time; when None
+    a cached per-stream workspace is used.  Returns ``out`` [B, Hq, D] in q's
+    dtype."""
     dev = q.device
     for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _need(t, n, device=dev)
@@ -219,9 +245,9 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         out = torch.empty_like(q)
     else:
         _need(out, "out", device=dev, dtype=q.dtype)
-    npart, _, ws_bytes = decode_plan(B, hq, hkv, d, max_context_len, ct, partition_tokens)
-    if npart > 1 and (workspace is None or workspace.numel() * workspace.element_size() < ws_bytes):
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    nstreams, _, ws_bytes = decode_plan(B, hq, hkv, d, max_context_len, ct, partition_tokens)
+    if nstreams > 1 and workspace is None:
+        workspace = _cached_workspace(dev, stream, ws_bytes)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().pkv_paged_attention_decode(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),

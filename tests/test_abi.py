@@ -95,13 +95,14 @@ def test_decode_host_rejections(lib):
 def test_plan_is_consistent(lib):
     for (B, hq, hkv, d, ctx) in [(4, 8, 2, 64, 256), (64, 32, 8, 128, 4096), (32, 64, 8, 128, 32768),
                                  (256, 32, 32, 128, 8192), (1, 8, 8, 128, 1)]:
-        np_, pt, ws = P.decode_plan(B, hq, hkv, d, ctx, P.PKV_BF16)
-        assert pt % 16 == 0 and np_ * pt >= ctx and (np_ - 1) * pt < max(ctx, 1)
-        assert (ws == 0) == (np_ == 1)
-        if np_ > 1:
-            assert ws >= B * hq * np_ * (d + 2) * 4
-    np_, pt, ws = P.decode_plan(2, 8, 2, 128, 1000, P.PKV_BF16, partition_tokens=64)
-    assert (np_, pt) == (16, 64)
+        nw, per, ws = P.decode_plan(B, hq, hkv, d, ctx, P.PKV_BF16)
+        items = B * hkv * ((ctx + 15) // 16)
+        assert 1 <= nw <= items and per % 16 == 0 and nw * per >= items * 16
+        G = hq // hkv
+        if nw > 1:
+            assert ws >= B * hkv * 8 + 2 * nw * (2 * G + G * d) * 4
+    nw, per, ws = P.decode_plan(2, 8, 2, 128, 1000, P.PKV_BF16, partition_tokens=64)
+    assert nw == (2 * 2 * 63 + 3) // 4 and per == 64
 
 
 def test_copy_rejections(lib):

@@ -46,17 +46,17 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
     cases = [_case(2024, 16), _case(2025, 24)]
     outs = []
     for c in cases:
-        # partitions of 256 tokens: the split path, so the scratch array is used
-        np_, _, ws = P.decode_plan(c["batch"], c["hq"], c["hkv"], c["d"], c["maxc"], c["k_cache"].dtype, 256)
+        # at most 1024 tokens per warp stream: many pairs split, so the scratch array is used
+        np_, _, ws = P.decode_plan(c["batch"], c["hq"], c["hkv"], c["d"], c["maxc"], c["k_cache"].dtype, 1024)
         assert np_ > 1 and 0 < ws <= P.NOALLOC_SCRATCH_BYTES
         out = torch.empty_like(c["q"])
         P.paged_attention_decode_noalloc(c["q"], c["k_cache"], c["v_cache"], c["block_tables"], c["context_lens"],
-                                         c["scale"], c["maxc"], out, partition_tokens=256)
+                                         c["scale"], c["maxc"], out, partition_tokens=1024)
         outs.append(out)
     torch.cuda.synchronize()
     for c, out in zip(cases, outs):
         ref = P.paged_attention_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"], c["context_lens"],
-                                       c["scale"], max_context_len=c["maxc"], partition_tokens=256)
+                                       c["scale"], max_context_len=c["maxc"], partition_tokens=1024)
         torch.cuda.synchronize()
         _close(out, ref)
     assert P.device_status(clear=True) == 0
@@ -64,7 +64,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 
 def test_noalloc_rejects_work_beyond_its_scratch():
     c = _case(7, 4)
-    # 4096 sequences x 64 query heads x 16 partitions of partials exceed the array
+    # 4096 sequences x 8 KV heads x 256 blocks split into 16-block streams need far more partials
     big_b, hq, hkv, d, maxc = 4096, 64, 8, 128, 16 * 256
     _, _, ws = P.decode_plan(big_b, hq, hkv, d, maxc, torch.bfloat16, 256)
     assert ws > P.NOALLOC_SCRATCH_BYTES
