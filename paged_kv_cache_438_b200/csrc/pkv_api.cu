@@ -85,10 +85,11 @@ int make_cache_map(CUtensorMap* map, const void* cache, int head_dim, int elt, l
 }
 
 // ------------------------------------------------------------ planning --
-constexpr int kDecodeWarps = 4;          // warps per decode CTA (DecodeTraits::kWarps)
+constexpr int kLongStreamBlocks = 256;   // streams at least this long use 4 warps with deep rings
 constexpr int kMaxCtaSmem = 227 * 1024;  // opt-in shared memory per CTA on sm_100
 
 struct Plan {
+  int warps;           // warps per CTA (one CTA per SM)
   int num_streams;     // warps that share the (sequence, head, block) work list
   int stream_tokens;   // upper bound of tokens one stream processes
   size_t workspace;    // arrival counters + partial slots
@@ -111,18 +112,25 @@ int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int r
   const long long blocks_max = std::max(1, (max_ctx + 15) / 16);
   const long long t_max = static_cast<long long>(std::max(B, 1)) * Hkv * blocks_max;
   if (t_max >= (1LL << 31)) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31 (sequence, head, block) items");
+  // One CTA per SM.  8-bit caches always use 8 warps (more conversion work per
+  // byte); 16-bit caches use 4 warps with twice the ring depth when each of 8
+  // warps per SM would still get at least kLongStreamBlocks blocks (measured:
+  // long contexts keep HBM busiest that way, short or L2-resident work wants
+  // the extra warps).
+  const long long sms = sm_count();
+  const int warps = (!is8(cache_dtype) && t_max / (8 * sms) >= kLongStreamBlocks) ? 4 : 8;
   long long nw;
   if (req_tokens > 0) {
     if (req_tokens % 16 != 0) return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d is not a multiple of 16", req_tokens);
     const long long per = req_tokens / 16;
     nw = (t_max + per - 1) / per;
   } else {
-    const long long resident = static_cast<long long>(is8(cache_dtype) ? 2 : 1) * kDecodeWarps * sm_count();
-    nw = std::min(resident, (t_max + 15) / 16);
+    nw = std::min(static_cast<long long>(warps) * sms, (t_max + 15) / 16);
   }
   nw = std::max(1LL, std::min(nw, t_max));
   if (nw > (1LL << 24)) return fail(PKV_ERR_UNSUPPORTED, "more than 2^24 decode streams");
   const int G = Hq / Hkv;
+  out->warps = warps;
   out->num_streams = static_cast<int>(nw);
   out->stream_tokens = static_cast<int>((t_max + nw - 1) / nw * 16);
   out->counter_bytes = align_up(static_cast<size_t>(std::max(B, 1)) * Hkv * 8, 256);
@@ -161,26 +169,29 @@ int set_smem(T* kernel, size_t bytes) {
 }
 
 template <int kD, int kCT>
-size_t decode_smem_bytes(int num_seqs) {
+size_t decode_smem_bytes(int num_seqs, int warps) {
   using Tr = pkv::DecodeTraits<kD, kCT>;
-  return 1024 + static_cast<size_t>(Tr::kWarps) * Tr::kRing * Tr::kStageBytes + Tr::kWarps * Tr::kRing * 8 +
+  const int ring = Tr::ring_depth(warps);
+  return 1024 + static_cast<size_t>(warps) * ring * Tr::kStageBytes + static_cast<size_t>(warps) * ring * 8 +
          (static_cast<size_t>(num_seqs) + 1) * 4;
 }
 
 template <int kD, int kCT, int kNT, bool kQBF16>
 int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, cudaStream_t st) {
   using Tr = pkv::DecodeTraits<kD, kCT>;
-  static_assert(Tr::kWarps == kDecodeWarps, "plan and kernel disagree on warps per CTA");
-  static_assert(Tr::kCtasPerSm == (Tr::k8bit ? 2 : 1), "plan and kernel disagree on CTAs per SM");
   auto kernel = pkv::paged_decode_kernel<kD, kCT, kNT, kQBF16>;
-  const size_t smem = decode_smem_bytes<kD, kCT>(p.num_seqs);
+  const int warps = p.ring_warps;
+  if (warps < 1 || warps > Tr::kMaxWarps) return fail(PKV_ERR_INVALID_ARG, "bad warp count %d", warps);
+  pkv::DecodeParams q = p;
+  q.ring = Tr::ring_depth(warps);
+  const size_t smem = decode_smem_bytes<kD, kCT>(p.num_seqs, warps);
   if (smem > static_cast<size_t>(kMaxCtaSmem))
     return fail(PKV_ERR_UNSUPPORTED, "batch of %d sequences needs %zu bytes of shared memory", p.num_seqs, smem);
   int rc = set_smem(kernel, smem);
   if (rc != PKV_OK) return rc;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3((p.num_streams + Tr::kWarps - 1) / Tr::kWarps);
-  cfg.blockDim = dim3(Tr::kWarps * 32);
+  cfg.gridDim = dim3((p.num_streams + warps - 1) / warps);
+  cfg.blockDim = dim3(warps * 32);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   // may start while the preceding kernel (the KV write) finishes; the kernel
@@ -190,7 +201,7 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::Decod
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, km, vm, p);
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, km, vm, q);
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return PKV_OK;
 }
@@ -418,6 +429,7 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   p.num_blocks = num_blocks;
   p.max_context_len = max_context_len;
   p.num_streams = pl.num_streams;
+  p.ring_warps = pl.warps;
   p.slot_floats = pl.slot_floats;
   p.epoch = next_epoch();
   p.qk_scale_log2 = scale * 1.4426950408889634f;

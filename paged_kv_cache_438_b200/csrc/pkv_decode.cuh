@@ -63,13 +63,15 @@ struct DecodeTraits {
   static constexpr int kScaleBytes = k8bit ? 64 : 0;                // 16 fp32 scales
   static constexpr int kStageTx = 2 * kKVBytes + 2 * kScaleBytes;   // bytes landing per stage
   static constexpr int kStageBytes = round_up_c(kStageTx, 1024);    // keeps every tile 1024-aligned
-  static constexpr int kWarps = 4;
-  // 16-bit caches run one CTA per SM with 4 stages of 8 KiB per warp; 8-bit
-  // caches (more conversion work per byte) run two CTAs per SM with ~24 KiB
-  // of ring per warp.
-  static constexpr int kRingBytes = k8bit ? 24 * 1024 : 32 * 1024;
-  static constexpr int kRing = kRingBytes / kStageBytes < 2 ? 2 : kRingBytes / kStageBytes;
-  static constexpr int kCtasPerSm = k8bit ? 2 : 1;
+  static constexpr int kMaxWarps = 8;
+  // One CTA per SM.  Its warps (4 or 8, chosen per call) share this many
+  // bytes of copy ring: 4 warps x 4 stages or 8 warps x 2 stages of 8 KiB for
+  // bf16 / fp16 at head_dim 128; 8-bit caches keep 8 warps and more stages.
+  static constexpr int kRingBudget = k8bit ? 160 * 1024 : 128 * 1024;
+  static int ring_depth(int warps) {
+    const int r = kRingBudget / (warps * kStageBytes);
+    return r < 2 ? 2 : (r > 8 ? 8 : r);
+  }
 };
 
 // Epoch-tagged arrival counters: bits 63..24 hold the epoch of the call that
@@ -94,6 +96,8 @@ struct DecodeParams {
   int num_blocks;
   int max_context_len;
   int num_streams;   // warps sharing the work list
+  int ring;          // copy stages per warp (set at launch from ring_warps)
+  int ring_warps;    // warps per CTA
   int slot_floats;   // ml + G * D: m[G], l[G] padded to ml = round_up(2G, 4), then o[G][D]
   unsigned long long epoch;  // this call's epoch, nonzero, < 2^40
   float qk_scale_log2;       // softmax scale * log2(e)
@@ -222,18 +226,17 @@ __device__ __forceinline__ int stream_of(long long T, long long g, long long nw)
 }
 
 template <int kD, int kCT, int kNT, bool kQBF16>
-__global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
+__global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                         const DecodeParams p) {
   using Tr = DecodeTraits<kD, kCT>;
   constexpr bool k8 = Tr::k8bit;
   constexpr bool kMmaBF16 = (kCT == kBF16);
   constexpr bool kOutBF16 = k8 ? kQBF16 : (kCT == kBF16);
-  constexpr int kW = Tr::kWarps;
-  constexpr int kR = Tr::kRing;
+  const int kW = blockDim.x >> 5;  // warps of this CTA
+  const int kR = p.ring;           // stages per warp (<= 8)
   constexpr int kKS = kD / 16;  // k-steps of S^T = K Q^T
   constexpr int kMT = kD / 16;  // m-tiles of O^T = V^T P^T
-  static_assert(kR <= 32, "ring deeper than a prefetch chunk");
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
@@ -252,7 +255,6 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
   const int B = p.num_seqs;
 
   if (lane == 0) {
-#pragma unroll
     for (int j = 0; j < kR; ++j) mbar_init(bar_base + (warp * kR + j) * 8, 1);
     fence_barrier_init();
   }
@@ -295,8 +297,10 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
   int pre0 = lane < count ? item_row(p, cum, item_of(lane)) : 0;
   int pre1 = 32 + lane < count ? item_row(p, cum, item_of(32 + lane)) : 0;
 
-  auto issue = [&](int k, int row0) {
-    const int stage = k % kR;
+  int istage = 0;  // ring stage of the next item to issue (only lane 0 issues)
+  auto issue = [&](int row0) {
+    const int stage = istage;
+    istage = istage + 1 == kR ? 0 : istage + 1;
     const uint32_t st = ring + stage * Tr::kStageBytes;
     const uint32_t bar = bars + stage * 8;
     mbar_arrive_expect_tx(bar, Tr::kStageTx);
@@ -317,7 +321,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
 #pragma unroll 1
   for (int k = 0; k < kR && k < count; ++k) {
     const int row0 = __shfl_sync(0xffffffffu, pre0, k);
-    if (lane == 0) issue(k, row0);
+    if (lane == 0) issue(row0);
   }
 
   // ---- cursor over (sequence, head, block), in processing order ----
@@ -359,11 +363,17 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
   };
   begin_pair();
 
+  int cstage = 0;        // ring stage of item k
+  uint32_t cphase = 0;   // its barrier phase
 #pragma unroll 1
   for (int k = 0; k < count; ++k) {
-    const int stage = k % kR;
+    const int stage = cstage;
     const uint32_t st = ring + stage * Tr::kStageBytes;
-    const bool landed = mbar_wait(bars + stage * 8, (k / kR) & 1);
+    const bool landed = mbar_wait(bars + stage * 8, cphase);
+    if (++cstage == kR) {
+      cstage = 0;
+      cphase ^= 1u;
+    }
     if (__any_sync(0xffffffffu, !landed)) {  // warp-uniform: never split the warp before ldmatrix/mma
       // let copies already in flight land (bounded) before the warp leaves
       for (int kk = k + 1; kk < count && kk < k + kR; ++kk) mbar_wait(bars + (kk % kR) * 8, (kk / kR) & 1);
@@ -522,7 +532,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kWarps * 32)
         if (chunk & 1) pre0 = nxt; else pre1 = nxt;
       }
       const int row0 = __shfl_sync(0xffffffffu, (chunk & 1) ? pre1 : pre0, kn & 31);
-      if (lane == 0) issue(kn, row0);
+      if (lane == 0) issue(row0);
     }
 
     // ---- advance; finish the (sequence, head) pair at its end or the stream's ----

@@ -431,3 +431,29 @@ def test_validation_mode_rejects_bad_indices_before_launch():
     finally:
         P.set_validation(False)
     torch.cuda.synchronize()
+
+
+# ------------------------------------------------- workspace reuse, determinism --
+
+def test_workspace_reused_across_shapes_matches_fresh_workspaces():
+    """One workspace serving calls of different shapes (the arrival counters,
+    the claim counter and the partial slots of one call overlap different
+    fields of the next) must give exactly what a fresh zero-filled workspace
+    gives.  The shapes are large enough for dynamically claimed tail chunks."""
+    cases = [I.device_decode_case("llama3_8b", DEV, batch=32, seed=5),
+             I.device_decode_case("prefix_shared", DEV, batch=48, seed=6),
+             I.device_decode_case("quant_mha", DEV, batch=64, cache_kind="int8", seed=7)]
+    shared = P.new_workspace(DEV, 256 << 20)
+    for c in cases + cases[:1]:
+        maxc = int(c["context_lens_cpu"].max())
+        nw, _, wsb = P.decode_plan(c["batch"], c["hq"], c["hkv"], c["d"], maxc, c["k_cache"].dtype)
+        assert nw > 1 and wsb <= shared.numel()
+        run = lambda ws: P.paged_attention_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                                                  c["context_lens"], c["scale"], c.get("k_scale"), c.get("v_scale"),
+                                                  max_context_len=maxc, workspace=ws)
+        got = run(shared)
+        ref = run(P.new_workspace(DEV, wsb))
+        again = run(shared)
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref) and torch.equal(got, again)
+    assert P.device_status(clear=True) == 0
