@@ -621,57 +621,67 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
             const int idx = 2 * w + (stream_start(T, w, nw) >= gp0 ? 0 : 1);
             return p.slots + static_cast<long long>(idx) * p.slot_floats;
           };
-          // Two rounds of independent loads: lane g (< G) first finds
-          // M[g] = max_c m_c[g]; then, per contributor, lanes g compute
-          // w_c[g] = 2^(m_c[g] - M[g]) l_c[g] (l_c[g] sits at lane G + g) and
-          // every lane accumulates w_c[g] o_c[g][its kV columns] for all g.
-          constexpr int kV = kD / 32;  // output columns per lane
-          constexpr int kG = 8 * kNT;
-          float Mv = -INFINITY;
-          for (int c = 0; c < n_c; ++c) {
-            const float v = lane < G ? __ldcg(slot_of(c) + lane) : -INFINITY;
-            Mv = fmaxf(Mv, v);
-          }
-          float Lv = 0.0f;
-          float acc[kG][kV];
+          // One pass over the contributors per group of 8 heads, with a
+          // running max per head: every load of a contributor is independent
+          // of the others, and two contributors are in flight at once.  Each
+          // lane owns kD / 32 output columns of every head.
+          constexpr int kV = kD / 32;
+#pragma unroll 1
+          for (int g0 = 0; g0 < G; g0 += 8) {
+            float Mg[8], Lg[8], acc[8][kV];
 #pragma unroll
-          for (int g = 0; g < kG; ++g)
+            for (int gg = 0; gg < 8; ++gg) {
+              Mg[gg] = -INFINITY;
+              Lg[gg] = 0.0f;
 #pragma unroll
-            for (int e = 0; e < kV; ++e) acc[g][e] = 0.0f;
+              for (int e = 0; e < kV; ++e) acc[gg][e] = 0.0f;
+            }
 #pragma unroll 2
-          for (int c = 0; c < n_c; ++c) {
-            const float* sl = slot_of(c);
-            const float v = lane < 2 * G ? __ldcg(sl + lane) : 0.0f;
-            const float lc = __shfl_sync(0xffffffffu, v, (lane + G) & 31);
-            const float w = lane < G ? fast_exp2(v - Mv) * lc : 0.0f;
-            Lv += w;
+            for (int c = 0; c < n_c; ++c) {
+              const float* sl = slot_of(c);
+              float mc[8], lc[8], ov[8][kV];
 #pragma unroll
-            for (int g = 0; g < kG; ++g) {
-              if (g < G) {
-                const float wg = __shfl_sync(0xffffffffu, w, g);
-                const float* og = sl + ml + g * kD + lane * kV;
-                if constexpr (kV == 4) {
-                  const float4 ov = __ldcg(reinterpret_cast<const float4*>(og));
-                  acc[g][0] += wg * ov.x;
-                  acc[g][1] += wg * ov.y;
-                  acc[g][2] += wg * ov.z;
-                  acc[g][3] += wg * ov.w;
-                } else {
-                  const float2 ov = __ldcg(reinterpret_cast<const float2*>(og));
-                  acc[g][0] += wg * ov.x;
-                  acc[g][1] += wg * ov.y;
+              for (int gg = 0; gg < 8; ++gg) {
+                const int g = g0 + gg;
+                if (g < G) {
+                  mc[gg] = __ldcg(sl + g);
+                  lc[gg] = __ldcg(sl + G + g);
+                  const float* og = sl + ml + g * kD + lane * kV;
+                  if constexpr (kV == 4) {
+                    const float4 v = __ldcg(reinterpret_cast<const float4*>(og));
+                    ov[gg][0] = v.x;
+                    ov[gg][1] = v.y;
+                    ov[gg][2] = v.z;
+                    ov[gg][3] = v.w;
+                  } else {
+                    const float2 v = __ldcg(reinterpret_cast<const float2*>(og));
+                    ov[gg][0] = v.x;
+                    ov[gg][1] = v.y;
+                  }
+                }
+              }
+#pragma unroll
+              for (int gg = 0; gg < 8; ++gg) {
+                if (g0 + gg < G) {
+                  const float mn = fmaxf(Mg[gg], mc[gg]);
+                  const float a = fast_exp2(Mg[gg] - mn);  // 0 for the first contributor
+                  const float w = fast_exp2(mc[gg] - mn) * lc[gg];
+                  Lg[gg] = Lg[gg] * a + w;
+#pragma unroll
+                  for (int e = 0; e < kV; ++e) acc[gg][e] = acc[gg][e] * a + w * ov[gg][e];
+                  Mg[gg] = mn;
                 }
               }
             }
-          }
 #pragma unroll
-          for (int g = 0; g < kG; ++g) {
-            if (g < G) {
-              const float Lg = __shfl_sync(0xffffffffu, Lv, g);
-              const float inv = Lg > 0.0f ? 1.0f / Lg : 0.0f;
+            for (int gg = 0; gg < 8; ++gg) {
+              const int g = g0 + gg;
+              if (g < G) {
+                const float inv = Lg[gg] > 0.0f ? 1.0f / Lg[gg] : 0.0f;
 #pragma unroll
-              for (int e = 0; e < kV; ++e)
-                store_out<kOutBF16>(p.out, (head_row0 + g) * kD + lane * kV + e, acc[g][e] * inv);
+                for (int e = 0; e < kV; ++e)
+                  store_out<kOutBF16>(p.out, (head_row0 + g) * kD + lane * kV + e, acc[gg][e] * inv);
+              }
             }
           }
         }

@@ -339,19 +339,28 @@ class BlockAllocator:
                                     ctypes.byref(npairs)))
         return slots, pairs[:npairs.value].clone()
 
-    def batch_append(self, seq_ids):
-        """One token for each sequence; returns (slots [n], cow pairs [k, 2])."""
-        ids = torch.as_tensor(seq_ids, dtype=torch.int64).contiguous()
+    def batch_append(self, seq_ids, slots_out=None, pairs_out=None):
+        """One token for each sequence; returns (slots [n], cow pairs [k, 2]).
+        ``slots_out`` (int64 [n]) and ``pairs_out`` (int32 [>= n, 2]) may be
+        given (e.g. pinned host buffers); the pairs returned are then a view
+        of ``pairs_out``."""
+        ids = seq_ids if isinstance(seq_ids, torch.Tensor) and seq_ids.dtype == torch.int64 \
+            else torch.as_tensor(seq_ids, dtype=torch.int64)
+        ids = ids.contiguous()
         n = ids.numel()
-        slots = torch.empty(n, dtype=torch.int64)
-        pairs = torch.empty((max(n, 1), 2), dtype=torch.int32)
+        slots = torch.empty(n, dtype=torch.int64) if slots_out is None else slots_out
+        pairs = torch.empty((max(n, 1), 2), dtype=torch.int32) if pairs_out is None else pairs_out
         npairs = _I(0)
         _check(lib().pkv_batch_append(self._h, _ptr(ids), n, _ptr(slots), _ptr(pairs), pairs.shape[0],
                                       ctypes.byref(npairs)))
+        if pairs_out is not None:
+            return slots, pairs[:npairs.value]
         return slots, pairs[:npairs.value].clone()
 
     def batch_tables(self, seq_ids, max_blocks, out_tables=None, out_lens=None):
-        ids = torch.as_tensor(seq_ids, dtype=torch.int64).contiguous()
+        ids = seq_ids if isinstance(seq_ids, torch.Tensor) and seq_ids.dtype == torch.int64 \
+            else torch.as_tensor(seq_ids, dtype=torch.int64)
+        ids = ids.contiguous()
         n = ids.numel()
         bt = torch.empty((n, max_blocks), dtype=torch.int32) if out_tables is None else out_tables
         cl = torch.empty(n, dtype=torch.int32) if out_lens is None else out_lens
