@@ -82,9 +82,11 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload, cache):
-    """DRAM bytes per decode call from the committed ncu summary, or None
-    when absent or taken on a different kernel source."""
+def recorded_traffic(workload, cache, alg_bytes):
+    """DRAM bytes (read + write) per decode call from the committed ncu
+    record, or None when absent or taken on a different kernel source.  A
+    record captured on a smaller slice of the workload is scaled to this
+    call by its algorithmic bytes (traffic grows in proportion)."""
     p = os.path.join(ROOT, "profiles", "decode_traffic.json")
     if not os.path.exists(p):
         return None
@@ -94,7 +96,7 @@ def recorded_traffic(workload, cache):
     e = d.get(key)
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
-    return e.get("dram_bytes_per_call")
+    return int(e["dram_bytes_per_call"] * alg_bytes / e["alg_bytes_per_call"])
 
 
 # ---------------------------------------------------------------- clocks --
@@ -278,7 +280,7 @@ def run_ours(args, rank, world, device):
     from paged_kv_cache_438_b200 import pagedkv as P
     build.build()
     P.lib()
-    wl = DecodeWorkload(args.workload, args.cache, device, seed_offset=1000 * rank, batch=args.batch)
+    wl = DecodeWorkload(args.workload, args.cache, device, seed_offset=replica_seed_offset(rank), batch=args.batch)
     K, W = args.steps, args.warmup
     # host allocator outputs of every step, staged in HBM before timing
     staged = []
@@ -349,15 +351,7 @@ def run_ours(args, rank, world, device):
     if status:
         raise RuntimeError(f"device status {status} raised during the bench")
 
-    if world > 1:
-        t = torch.tensor([timed_ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        timed_ms = float(t.item())
-        tot = torch.tensor([float(kv_total), float(wl.B * K)], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(tot)
-        kv_all, seqsteps_all = float(tot[0]), float(tot[1])
-    else:
-        kv_all, seqsteps_all = float(kv_total), float(wl.B * K)
+    timed_ms, kv_all, seqsteps_all = aggregate_ranks(timed_ms, kv_total, wl.B * K, world, device)
 
     res = dict(wl=wl, K=K, W=W, timed_ms=timed_ms, dec_ms=dec_ms, kv_all=kv_all, kv_rank=kv_total,
                seqsteps_all=seqsteps_all, launches=launches, clocks=clocks, flush=flush, kv_step=kv_step,
@@ -365,6 +359,24 @@ def run_ours(args, rank, world, device):
     if not args.no_e2e:
         res["e2e"] = run_e2e(wl, K, W, device, world)
     return res
+
+
+def aggregate_ranks(ms, kv_bytes, seq_steps, world, device):
+    """Whole-job numbers of independent replicas: the time is the slowest
+    rank's, the bytes and sequence-steps are summed over ranks.  The only
+    collective of a multi-GPU run (no data moves between ranks)."""
+    if world <= 1:
+        return float(ms), float(kv_bytes), float(seq_steps)
+    t = torch.tensor([float(ms)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    tot = torch.tensor([float(kv_bytes), float(seq_steps)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(tot)
+    return float(t.item()), float(tot[0]), float(tot[1])
+
+
+def replica_seed_offset(rank):
+    """Each rank draws its own batch (weak scaling: per-GPU work is fixed)."""
+    return 1000 * rank
 
 
 def roll(wl, steps, out, ws, flush, scrub, device, seconds):
@@ -439,13 +451,7 @@ def run_e2e(wl, K, W, device, world):
         kv += c
     torch.cuda.synchronize(device)
     ms = (time.perf_counter() - t0) * 1e3
-    if world > 1:
-        t = torch.tensor([ms], device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
-        tot = torch.tensor([float(kv)], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(tot)
-        kv = float(tot[0])
+    ms, kv, _ = aggregate_ranks(ms, kv, 0, world, device)
     return {"value": round(kv / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms / K, 4),
             "h2d_bytes_per_step": h2d // K, "d2h_bytes_per_step": d2h,
             "timing": "host wall clock per step: allocator + H2D + kernels + D2H + stream sync"}
@@ -562,7 +568,7 @@ def main():
     small = wl.B * wl.hq * wl.d * 2 * 2 + (kv_call // (wl.hkv * wl.d * 2 * wl.elt * 16)) * 4
     alg_bytes = kv_call + small
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
-    traffic = recorded_traffic(args.workload, args.cache)
+    traffic = recorded_traffic(args.workload, args.cache, alg_bytes)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": r["K"],
         "warmup": r["W"], "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
