@@ -17,7 +17,9 @@ What it computes, and the passages it follows (pages are named by title):
   ("LLM 推理优化深度解析", §KV Cache 的本质 and §PagedAttention; the
   ascendai.csdn.net article, §二 核心突破 Fig. 2).
 * ``quant``      -- the per-token-per-head absmax INT8 / FP8-e4m3 quantising
-  rule with its own e4m3 encoder / decoder (OCP FP8 E4M3 definition).
+  rule with its own e4m3 encoder / decoder (OCP FP8 E4M3 definition), and
+  the asymmetric min/max uint8 rule with a zero point and its 128-token
+  grouped form ("大模型推理的KV Cache管理…优化实战", §四).
 * ``cache_ops``  -- the slot-mapped KV write (logical block = token // 16) and
   the block copy behind copy-on-write.
 * ``allocator``  -- a pure-Python free-list / refcount / fork / copy-on-write

@@ -10,7 +10,9 @@ result, so the oracle is the plain definition written out:
 
 1. gather: K_s[j] = k_cache[block_table[s][j // bs], :, j % bs, :] for j < ctx_s
    (and V likewise), converted to fp64; quantised caches are dequantised as
-   code * scale of that (block, head, slot);
+   code * scale of that (block, head, slot), or (code - zero_point) * scale
+   for the asymmetric uint8 format ("大模型推理的KV Cache管理…优化实战", §四
+   dequantize_key);
 2. attend: for query head i with KV head h = i // G (consecutive grouping,
    "LLM 推理优化深度解析", §MQA 与 GQA), logits = scale * K_s[:, h] @ q[s, i],
    p = softmax(logits), out[s, i] = p @ V_s[:, h].
@@ -20,17 +22,20 @@ A sequence with ctx = 0 yields a zero output row.
 import numpy as np
 
 
-def gather_sequence(cache, block_table, ctx, scale=None):
+def gather_sequence(cache, block_table, ctx, scale=None, zero=None):
     """Logically contiguous [ctx, H, D] fp64 copy of one sequence's K or V.
 
     cache: [NB, H, bs, D] array of values (fp64-convertible) or of codes when
-    ``scale`` ([NB, H, bs]) is given; block_table: 1-D int array.
+    ``scale`` ([NB, H, bs]) is given, with zero points ``zero`` ([NB, H, bs])
+    for the asymmetric format; block_table: 1-D int array.
     """
     bs = cache.shape[2]
     j = np.arange(ctx)
     blocks = np.asarray(block_table)[j // bs]
     offs = j % bs
     rows = cache[blocks, :, offs, :].astype(np.float64)          # [ctx, H, D]
+    if zero is not None:
+        rows = rows - zero[blocks, :, offs].astype(np.float64)[:, :, None]
     if scale is not None:
         rows = rows * scale[blocks, :, offs].astype(np.float64)[:, :, None]
     return rows
@@ -58,11 +63,13 @@ def contiguous_attention(q, K, V, scale):
 
 
 def paged_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale,
-                           k_scale=None, v_scale=None, seqs=None):
+                           k_scale=None, v_scale=None, seqs=None, k_zero=None, v_zero=None):
     """Decode attention for every (or the listed) sequence of a batch.
 
     q: [B, Hq, D]; k_cache, v_cache: [NB, Hkv, bs, D] (values, or codes with
-    k_scale / v_scale [NB, Hkv, bs]); block_tables: [B, MB]; context_lens: [B].
+    k_scale / v_scale [NB, Hkv, bs] and, for the asymmetric format, zero
+    points k_zero / v_zero [NB, Hkv, bs]); block_tables: [B, MB];
+    context_lens: [B].
     Returns [B, Hq, D] fp64 (rows of sequences not in ``seqs`` stay zero).
     """
     q = np.asarray(q, np.float64)
@@ -70,14 +77,14 @@ def paged_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scal
     out = np.zeros((B, Hq, D), np.float64)
     for s in (range(B) if seqs is None else seqs):
         ctx = int(context_lens[s])
-        K = gather_sequence(k_cache, block_tables[s], ctx, k_scale)
-        V = gather_sequence(v_cache, block_tables[s], ctx, v_scale)
+        K = gather_sequence(k_cache, block_tables[s], ctx, k_scale, k_zero)
+        V = gather_sequence(v_cache, block_tables[s], ctx, v_scale, v_zero)
         out[s] = contiguous_attention(q[s], K, V, scale)
     return out
 
 
 def paged_decode_attention_heads(q, k_cache, v_cache, block_tables, context_lens, scale,
-                                 pairs, k_scale=None, v_scale=None):
+                                 pairs, k_scale=None, v_scale=None, k_zero=None, v_zero=None):
     """Oracle output for a sample of (sequence, query head) pairs only.
 
     Used at full workload sizes where the whole batch would take too long;
@@ -99,9 +106,11 @@ def paged_decode_attention_heads(q, k_cache, v_cache, block_tables, context_lens
             cache.clear()
             bt = block_tables[s]
             K = gather_sequence(k_cache[:, h:h + 1], bt, ctx,
-                                None if k_scale is None else k_scale[:, h:h + 1])
+                                None if k_scale is None else k_scale[:, h:h + 1],
+                                None if k_zero is None else k_zero[:, h:h + 1])
             V = gather_sequence(v_cache[:, h:h + 1], bt, ctx,
-                                None if v_scale is None else v_scale[:, h:h + 1])
+                                None if v_scale is None else v_scale[:, h:h + 1],
+                                None if v_zero is None else v_zero[:, h:h + 1])
             cache[key] = (K[:, 0, :], V[:, 0, :])
         K, V = cache[key]
         logits = scale * (K @ q[s, i])

@@ -1,4 +1,9 @@
-"""Per-token-per-head absmax KV quantisation (oracle; test infrastructure only).
+"""KV quantisation rules (oracle; test infrastructure only).
+
+Two families: per-token-per-head symmetric absmax INT8 / FP8-e4m3 (this
+docstring), and the page's own asymmetric uint8 rule with a zero point
+(``quantize_u8_asym`` and ``quantize_grouped`` further down, with their
+readings).
 
 The pages store the KV cache at reduced precision to halve its size: INT8
 "几乎无精度损失" and FP8 as a 2x saving (ascendai.csdn.net article, §三 进阶优化
@@ -99,3 +104,74 @@ def dequantize_int8(codes, scales):
 
 def dequantize_fp8_e4m3(codes, scales):
     return e4m3_decode(codes) * np.asarray(scales, np.float64)[..., None]
+
+
+# --------------------------------------------------------------------------
+# Asymmetric uint8 quantisation with a zero point ("大模型推理的KV Cache管理…
+# 优化实战", §四, class KVQuantizationCache: quantize_key, dequantize_key,
+# quantize_grouped).  With the page's default per-channel setting the
+# statistics are the minimum and maximum over the last (head_dim) axis, so
+# every (token, head) row gets its own scale and zero point:
+#
+#   scale      = (max - min) / 255
+#   zero_point = round(-min / scale), clamped to [0, 255], stored as uint8
+#   code       = round((x - min) / scale), clamped to [0, 255], uint8
+#   x_hat      = (code - zero_point) * scale
+#
+# Readings where the page leaves a step open:
+# * arithmetic is IEEE fp32 from the fp32 value of each 16-bit input (the
+#   sketch applies torch ops in the tensor's own dtype; fp32 is the precision
+#   the absmax rule above uses too), every round half-to-even;
+# * a row with scale 0 (max == min, or a range too small for fp32 / 255) is
+#   stored as scale 0, zero point 0 and zero codes (the page's formula would
+#   divide by zero there);
+# * the page computes the code from (x - min) but dequantises through the
+#   rounded, clamped zero point, as written: a row that does not contain 0
+#   in [min, max] gets zero point 0 (all positive) or 255 (all negative) and
+#   dequantises to x - min or x - max.  This is kept as the page states it.
+# --------------------------------------------------------------------------
+
+U8_LEVELS = 255
+
+
+def quantize_u8_asym(x):
+    """x [..., D] -> (codes uint8 [..., D], scales fp32 [...], zero points
+    uint8 [...]), statistics over the last axis."""
+    x = np.asarray(x, np.float32)
+    lo = np.min(x, axis=-1)
+    hi = np.max(x, axis=-1)
+    s = ((hi - lo) / np.float32(U8_LEVELS)).astype(np.float32)
+    codes = np.zeros(x.shape, np.uint8)
+    zp = np.zeros(s.shape, np.uint8)
+    nz = s > 0
+    z = (-lo[nz] / s[nz]).astype(np.float32)
+    zp[nz] = np.clip(np.rint(z), 0, U8_LEVELS).astype(np.uint8)
+    y = ((x[nz] - lo[nz][..., None]) / s[nz][..., None]).astype(np.float32)
+    codes[nz] = np.clip(np.rint(y), 0, U8_LEVELS).astype(np.uint8)
+    return codes, s, zp
+
+
+def dequantize_u8_asym(codes, scales, zero_points):
+    """(code - zero_point) * scale in fp64."""
+    c = np.asarray(codes, np.float64)
+    z = np.asarray(zero_points, np.float64)[..., None]
+    return (c - z) * np.asarray(scales, np.float64)[..., None]
+
+
+def quantize_grouped(kv, group_size=128):
+    """kv [num_heads, seq_len, head_dim]: consecutive groups of ``group_size``
+    tokens (the last one may be shorter) are quantised independently with
+    ``quantize_u8_asym`` and the results concatenated along the token axis.
+    Returns (codes, scales, zero points); the page's sketch returns codes and
+    scales only, which leaves nothing to dequantise with, so the zero points
+    are kept as well."""
+    kv = np.asarray(kv, np.float32)
+    if kv.ndim != 3:
+        raise ValueError("kv must be [num_heads, seq_len, head_dim]")
+    n = kv.shape[1]
+    num_groups = (n + group_size - 1) // group_size
+    parts = [quantize_u8_asym(kv[:, g * group_size:min((g + 1) * group_size, n), :]) for g in range(num_groups)]
+    if not parts:
+        return (np.zeros(kv.shape, np.uint8), np.zeros(kv.shape[:2], np.float32),
+                np.zeros(kv.shape[:2], np.uint8))
+    return tuple(np.concatenate([p[i] for p in parts], axis=1) for i in range(3))

@@ -228,3 +228,30 @@ def test_head_sample_matches_full_oracle():
     part = A.paged_decode_attention_heads(q, kc, vc, bt, ctx, 0.4, pairs)
     for n, (s, i) in enumerate(pairs):
         np.testing.assert_allclose(part[n], full[s, i], rtol=0, atol=1e-14)
+
+
+def test_asymmetric_gather_subtracts_zero_point_then_scales():
+    # an integer-grid cache stored as (code, scale 2^-k, zero point) must give
+    # back the grid values, and paged attention over it must equal contiguous
+    # attention over those values (a sign or order slip in the zero point fails)
+    rng = np.random.default_rng(9)
+    ctx, hkv, hq, d = 37, 2, 4, 8
+    zp = rng.integers(20, 236, size=(ctx, hkv))
+    codes_log = rng.integers(0, 256, size=(ctx, hkv, d))
+    sc = np.exp2(-rng.integers(2, 6, size=(ctx, hkv))).astype(np.float32)
+    vals = (codes_log - zp[:, :, None]) * sc.astype(np.float64)[:, :, None]
+    nblk = (ctx + 15) // 16
+    perm = rng.permutation(nblk + 2)[:nblk]
+    nb = nblk + 2
+    kc = np.zeros((nb, hkv, 16, d), np.uint8)
+    kz = np.zeros((nb, hkv, 16), np.uint8)
+    ks = np.zeros((nb, hkv, 16), np.float32)
+    for j in range(ctx):
+        kc[perm[j // 16], :, j % 16] = codes_log[j]
+        kz[perm[j // 16], :, j % 16] = zp[j]
+        ks[perm[j // 16], :, j % 16] = sc[j]
+    got = A.gather_sequence(kc, perm, ctx, ks, kz)
+    assert np.array_equal(got, vals)
+    q = rng.standard_normal((1, hq, d))
+    paged = A.paged_decode_attention(q, kc, kc, np.array([perm]), [ctx], 0.5, ks, ks, k_zero=kz, v_zero=kz)
+    np.testing.assert_allclose(paged[0], _brute(q[0], vals, vals, 0.5), rtol=0, atol=1e-12)

@@ -104,3 +104,97 @@ def test_fp8_zero_row_and_dequant():
     c, s = Q.quantize_fp8_e4m3(x)
     assert s[0] == 1.0
     assert np.array_equal(Q.dequantize_fp8_e4m3(c, s)[0], x[0].astype(np.float64))
+
+
+# ---- asymmetric uint8 with zero point ("大模型推理的KV Cache管理…优化实战", §四) ----
+
+def test_u8_asym_exact_grid_row():
+    # min -51, max 204: scale (204 + 51) / 255 = 1, zero point 51, codes x + 51,
+    # and every value on the integer grid dequantises exactly
+    x = np.array([[-51.0, 0.0, 100.0, 204.0, -3.0]], np.float32)
+    c, s, z = Q.quantize_u8_asym(x)
+    assert s[0] == 1.0 and z[0] == 51
+    assert c[0].tolist() == [0, 51, 151, 255, 48]
+    assert np.array_equal(Q.dequantize_u8_asym(c, s, z)[0], x[0].astype(np.float64))
+
+
+def test_u8_asym_ties_round_half_to_even():
+    # scale 1, -min / scale = 0.5 -> zero point 0 (even); (x - min) = 0, 0.5,
+    # 1.5, 2.5, 255 -> codes 0, 0, 2, 2, 255
+    x = np.array([[-0.5, 0.0, 1.0, 2.0, 254.5]], np.float32)
+    c, s, z = Q.quantize_u8_asym(x)
+    assert s[0] == 1.0 and z[0] == 0
+    assert c[0].tolist() == [0, 0, 2, 2, 255]
+    # the two roundings can stack: x = 1 comes back as 2, one full step off
+    assert Q.dequantize_u8_asym(c, s, z)[0].tolist() == [0.0, 0.0, 2.0, 2.0, 255.0]
+
+
+def test_u8_asym_codes_are_nearest_of_all_256():
+    # brute force: every code is the nearest of all 256 levels to (x - min) / s
+    # (ties to the even level), with the division done in fp32 as stated
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal((64, 24)) * rng.uniform(0.01, 100, (64, 1))).astype(np.float32)
+    c, s, z = Q.quantize_u8_asym(x)
+    lo = x.min(-1)
+    levels = np.arange(256, dtype=np.float64)
+    for i in range(x.shape[0]):
+        y = ((x[i] - lo[i]) / s[i]).astype(np.float32).astype(np.float64)
+        for e in range(x.shape[1]):
+            d = np.abs(y[e] - levels)
+            ties = levels[d == d.min()]
+            pick = ties[0] if len(ties) == 1 else ties[np.mod(ties, 2) == 0][0]
+            assert c[i, e] == pick
+        zy = np.float32(-lo[i] / s[i])
+        assert z[i] == min(255, max(0, int(np.rint(zy))))
+
+
+def test_u8_asym_invariants_random():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((400, 4, 128)).astype(np.float32)
+    c, s, z = Q.quantize_u8_asym(x)
+    assert c.dtype == np.uint8 and z.dtype == np.uint8 and s.dtype == np.float32
+    lo, hi = x.min(-1), x.max(-1)
+    assert np.array_equal(s, ((hi - lo) / np.float32(255)).astype(np.float32))
+    # the minimum maps to code 0 and the maximum to 255; codes are monotone in x
+    assert np.all(np.take_along_axis(c, x.argmin(-1)[..., None], -1) == 0)
+    assert np.all(np.take_along_axis(c, x.argmax(-1)[..., None], -1) == 255)
+    order = np.argsort(x, axis=-1)
+    assert np.all(np.diff(np.take_along_axis(c.astype(np.int32), order, -1), axis=-1) >= 0)
+    # each code is within half a step of (x - min) / s; with the rounded zero
+    # point the reconstruction is within one step (rows here contain 0)
+    s64 = s.astype(np.float64)[..., None]
+    off = c.astype(np.float64) * s64 + lo.astype(np.float64)[..., None]
+    assert np.all(np.abs(off - x) <= s64 * (0.5 + 1e-5))
+    xh = Q.dequantize_u8_asym(c, s, z)
+    assert np.all(np.abs(xh - x) <= s64 * (1.0 + 1e-5))
+
+
+def test_u8_asym_rows_not_containing_zero_follow_the_page():
+    # all positive: -min / scale < 0 clamps the zero point to 0 and the row
+    # comes back shifted by -min; all negative: it clamps to 255, shift -max
+    x = np.array([[1.0, 256.0, 11.0], [-256.0, -1.0, -246.0]], np.float32)
+    c, s, z = Q.quantize_u8_asym(x)
+    assert s.tolist() == [1.0, 1.0] and z.tolist() == [0, 255]
+    assert c.tolist() == [[0, 255, 10], [0, 255, 10]]
+    xh = Q.dequantize_u8_asym(c, s, z)
+    assert xh.tolist() == [[0.0, 255.0, 10.0], [-255.0, 0.0, -245.0]]
+
+
+def test_u8_asym_constant_row():
+    c, s, z = Q.quantize_u8_asym(np.full((2, 16), 3.25, np.float32))
+    assert np.all(c == 0) and np.all(s == 0) and np.all(z == 0)
+
+
+def test_grouped_equals_per_row_for_any_group_size():
+    # the page's grouped form reduces over head_dim inside each token group,
+    # so grouping never changes a (token, head) row's scale, zero point or codes
+    rng = np.random.default_rng(5)
+    kv = rng.standard_normal((3, 300, 64)).astype(np.float32)
+    ref = Q.quantize_u8_asym(kv)
+    for gs in (128, 7, 1, 300, 512):
+        got = Q.quantize_grouped(kv, gs)
+        for a, b in zip(got, ref):
+            assert a.shape == b.shape and np.array_equal(a, b)
+    # a reduction over the wrong axis would break the per-row extremes
+    c, s, z = Q.quantize_grouped(kv, 128)
+    assert np.all(c.max(-1) == 255) and np.all(c.min(-1) == 0)
