@@ -55,7 +55,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama3_8b", choices=sorted(I.WORKLOADS))
-    ap.add_argument("--cache", default=None, choices=[None, "int8", "fp8"])
+    ap.add_argument("--cache", default=None, choices=[None, "int8", "fp8", "u8asym"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -166,6 +166,15 @@ class ClockSampler:
 
 # ------------------------------------------------------------- workload --
 
+def kv_bytes_per_token(hkv, d, cache):
+    """Algorithmic cache bytes one token of context costs a decode read: K
+    and V rows, plus per-(token, head) fp32 scales of quantised caches and
+    uint8 zero points of the asymmetric format."""
+    if cache is None:
+        return hkv * d * 2 * 2
+    return hkv * d * 2 + hkv * 2 * 4 + (hkv * 2 if cache == "u8asym" else 0)
+
+
 class DecodeWorkload:
     """A batch of sequences living in a paged cache on one GPU, advanced one
     decode step at a time through the library's public API."""
@@ -196,14 +205,18 @@ class DecodeWorkload:
         order = torch.randperm(nb, generator=gen).tolist()
         self.alloc = P.BlockAllocator(nb, initial_free_order=order)
         elt = 1 if cache else 2
-        cdt = {None: self.dtype, "int8": torch.int8, "fp8": torch.uint8}[cache]
+        cdt = {None: self.dtype, "int8": torch.int8, "fp8": torch.uint8, "u8asym": torch.uint8}[cache]
         self.k_cache = torch.empty((nb, self.hkv, 16, self.d), dtype=cdt, device=device)
         self.v_cache = torch.empty_like(self.k_cache)
-        self.k_scale = self.v_scale = None
+        self.k_scale = self.v_scale = self.k_zero = self.v_zero = None
         if cache:
             self.k_scale = torch.zeros((nb, self.hkv, 16), dtype=torch.float32, device=device)
             self.v_scale = torch.zeros_like(self.k_scale)
+        if cache == "u8asym":
+            self.k_zero = torch.zeros((nb, self.hkv, 16), dtype=torch.uint8, device=device)
+            self.v_zero = torch.zeros_like(self.k_zero)
         self.elt = elt
+        self.per_tok = kv_bytes_per_token(self.hkv, self.d, cache)
         self.dg = torch.Generator(device=device)
         self.dg.manual_seed(seed + 17)
         self.ids = list(range(self.B))
@@ -219,7 +232,8 @@ class DecodeWorkload:
             for s in range(self.B):
                 slots, pairs = self.alloc.append(s, lens[s])
                 if pairs.shape[0]:
-                    P.copy_blocks(self.k_cache, self.v_cache, pairs.to(device), self.k_scale, self.v_scale)
+                    P.copy_blocks(self.k_cache, self.v_cache, pairs.to(device), self.k_scale, self.v_scale,
+                                  k_zero=self.k_zero, v_zero=self.v_zero)
                 self._fill(slots)
         else:
             for s in range(self.B):
@@ -236,7 +250,8 @@ class DecodeWorkload:
             n = sl.numel()
             k = torch.randn((n, self.hkv, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
             v = torch.randn((n, self.hkv, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
-            self.P.kv_cache_write(k, v, self.k_cache, self.v_cache, sl, self.k_scale, self.v_scale)
+            self.P.kv_cache_write(k, v, self.k_cache, self.v_cache, sl, self.k_scale, self.v_scale,
+                                  k_zero=self.k_zero, v_zero=self.v_zero)
 
     def host_step(self):
         """Allocator work of one step: slots and CoW pairs for one new token per
@@ -246,8 +261,7 @@ class DecodeWorkload:
         return slots, pairs, bt, cl
 
     def kv_bytes(self, cl):
-        per_tok = self.hkv * self.d * 2 * self.elt + (self.hkv * 2 * 4 if self.cache_kind else 0)
-        return int(cl.sum()) * per_tok
+        return int(cl.sum()) * self.per_tok
 
     def new_rows(self):
         q = torch.randn((self.B, self.hq, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
@@ -262,15 +276,18 @@ class DecodeWorkload:
         P = self.P
         n = 0
         if pairs is not None and pairs.numel():
-            P.copy_blocks(self.k_cache, self.v_cache, pairs, self.k_scale, self.v_scale)
+            P.copy_blocks(self.k_cache, self.v_cache, pairs, self.k_scale, self.v_scale, k_zero=self.k_zero,
+                          v_zero=self.v_zero)
             n += 1
-        P.kv_cache_write(k, v, self.k_cache, self.v_cache, slots, self.k_scale, self.v_scale)
+        P.kv_cache_write(k, v, self.k_cache, self.v_cache, slots, self.k_scale, self.v_scale, k_zero=self.k_zero,
+                         v_zero=self.v_zero)
         self.decode(q, bt, cl, maxc, out, ws)
         return n + 2
 
     def decode(self, q, bt, cl, maxc, out, ws):
         self.P.paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.scale, self.k_scale,
-                                      self.v_scale, max_context_len=maxc, out=out, workspace=ws)
+                                      self.v_scale, max_context_len=maxc, out=out, workspace=ws,
+                                      k_zero=self.k_zero, v_zero=self.v_zero)
 
 
 # ------------------------------------------------------------------ ours --
@@ -470,8 +487,7 @@ def oracle_sample(name, cache, budget_s=10.0, seed_offset=0):
     gen = I.generator(spec["seed"] + seed_offset + 555)
     ctx = (I.context_lens(spec, gen) + spec.get("prefix", 0)).tolist()
     hq, hkv, d = spec["hq"], spec["hkv"], spec["d"]
-    elt = 1 if cache else 2
-    per_tok = hkv * d * 2 * elt + (hkv * 8 if cache else 0)
+    per_tok = kv_bytes_per_token(hkv, d, cache)
     spent, kvb, seqs = 0.0, 0, 0
     for c in ctx:
         nblk = I.blocks_for(c)
@@ -483,11 +499,11 @@ def oracle_sample(name, cache, budget_s=10.0, seed_offset=0):
         else:
             kc = case["k_cache"].to(torch.float64).numpy()
             vc = case["v_cache"].to(torch.float64).numpy()
-        ks = case["k_scale"].numpy() if cache else None
-        vs = case["v_scale"].numpy() if cache else None
+        side = {key: case[key].numpy() for key in ("k_scale", "v_scale", "k_zero", "v_zero") if key in case}
         q = case["q"].to(torch.float64).numpy()
         t0 = time.perf_counter()
-        OA.paged_decode_attention(q, kc, vc, case["block_tables"].numpy(), [c], case["scale"], ks, vs)
+        OA.paged_decode_attention(q, kc, vc, case["block_tables"].numpy(), [c], case["scale"], side.get("k_scale"),
+                                  side.get("v_scale"), k_zero=side.get("k_zero"), v_zero=side.get("v_zero"))
         spent += time.perf_counter() - t0
         kvb += c * per_tok
         seqs += 1
@@ -565,7 +581,7 @@ def main():
     nstreams, stream_tokens, ws_bytes = wl.P.decode_plan(wl.B, wl.hq, wl.hkv, wl.d, r["maxc"], wl.k_cache.dtype)
     kv_call = r["kv_rank"] / r["K"]
     # q read + out written + the block-table entries the step reads
-    small = wl.B * wl.hq * wl.d * 2 * 2 + (kv_call // (wl.hkv * wl.d * 2 * wl.elt * 16)) * 4
+    small = wl.B * wl.hq * wl.d * 2 * 2 + (kv_call // (wl.per_tok * 16)) * 4
     alg_bytes = kv_call + small
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
     traffic = recorded_traffic(args.workload, args.cache, alg_bytes)
@@ -573,7 +589,8 @@ def main():
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": r["K"],
         "warmup": r["W"], "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {None: "bf16" if wl.dtype == torch.bfloat16 else "f16",
-                                       "int8": "int8 KV / fp16 mma", "fp8": "fp8e4m3 KV / fp16 mma"}[args.cache],
+                                       "int8": "int8 KV / fp16 mma", "fp8": "fp8e4m3 KV / fp16 mma",
+                                       "u8asym": "u8 KV with zero point / fp16 mma"}[args.cache],
         "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload, "batch": wl.B,
                    "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.d, "block_size": 16,

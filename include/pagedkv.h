@@ -14,7 +14,7 @@
  *           §碎片问题, §三个直接推论 (KV 量化 FP8/INT8).
  *   [P-WMRH] "大模型推理的KV Cache管理从内存碎片到前缀缓存的优化实战" (wmrh.cn),
  *           §二 (KVCacheBlock, BlockTable, PagedKVCache.append_slot, copy_prefix),
- *           §四 (KV quantisation).
+ *           §四 (KVQuantizationCache: asymmetric uint8 with zero point).
  *   [P-LJT] "LLM 推理优化深度解析：KV Cache、Continuous Batching、PagedAttention
  *           与量化" (blog.longjiangtao.top), §KV Cache 的本质, §MQA 与 GQA,
  *           §PagedAttention：vLLM 的显存碎片治理.
@@ -35,6 +35,8 @@
  *   k_cache, v_cache : [num_blocks, num_kv_heads, 16, head_dim] of cache_dtype
  *   k_scale, v_scale : [num_blocks, num_kv_heads, 16] fp32 (quantised caches
  *                      only; one scale per token and KV head)
+ *   k_zero, v_zero   : [num_blocks, num_kv_heads, 16] uint8 (PKV_U8ASYM only;
+ *                      one zero point per token and KV head)
  * Token at flat slot `slot` of KV head h is row cache[slot / 16][h][slot % 16].
  *
  * Device-side checks never fault: an out-of-range slot, block id, copy pair or
@@ -65,6 +67,8 @@ extern "C" {
 #define PKV_BF16    1   /* bfloat16                                        */
 #define PKV_I8      2   /* int8 codes, symmetric absmax, range [-127, 127] */
 #define PKV_FP8E4M3 3   /* OCP FP8 E4M3 (e4m3fn) codes, absmax maps to 448 */
+#define PKV_U8ASYM  4   /* uint8 codes, min/max over head_dim, with a
+                           per-(token, head) scale and uint8 zero point     */
 
 /* ---- device status bits (pkv_device_status) ----------------------------- */
 #define PKV_DEV_BAD_SLOT     1u   /* slot >= num_blocks * 16 (write skipped)       */
@@ -89,7 +93,10 @@ int pkv_version(void);
  *                 (PKV_F16 or PKV_BF16).
  * k_cache, v_cache : device, cache layout above, cache_dtype.
  * k_scale, v_scale : device fp32 scale arrays; required (non-NULL) iff
- *                 cache_dtype is PKV_I8 or PKV_FP8E4M3, else ignored.
+ *                 cache_dtype is PKV_I8, PKV_FP8E4M3 or PKV_U8ASYM, else
+ *                 ignored.
+ * k_zero, v_zero : device uint8 zero-point arrays; required iff cache_dtype
+ *                 is PKV_U8ASYM, else ignored (may be NULL).
  * slot_mapping  : device int64 [num_tokens]; -1 skips the token.  Slots of
  *                 one call must be distinct (duplicates race).
  * For a 16-bit cache in_dtype must equal cache_dtype and the write is a bit
@@ -97,10 +104,18 @@ int pkv_version(void);
  *   a = max|x| (fp32), s = a / 127 (INT8) or a / 448 (FP8), code = round-to-
  *   nearest-even of x / s (IEEE fp32 division), clamped to +-127 / +-448
  *   before the e4m3 conversion; a = 0 stores s = 0 and zero codes.
+ * PKV_U8ASYM follows [P-WMRH] §四 quantize_key with its per-channel
+ * statistics (min and max over head_dim), in IEEE fp32 from the 16-bit
+ * inputs, rounding half to even:
+ *   s = (max - min) / 255, z = round(-min / s) clamped to [0, 255],
+ *   code = round((x - min) / s) clamped to [0, 255];
+ *   s = 0 (a constant row) stores s = 0, z = 0 and zero codes.
+ * The page's 128-token grouped form leaves every (token, head) row's
+ * statistics unchanged (they are taken over head_dim), so it stores the same.
  * Alignment: k, v, k_cache, v_cache 16 bytes; scales 4 bytes.
  */
 int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,
-                       float* k_scale, float* v_scale,
+                       float* k_scale, float* v_scale, uint8_t* k_zero, uint8_t* v_zero,
                        const int64_t* slot_mapping, int num_tokens,
                        int num_kv_heads, int head_dim, int block_size, int num_blocks,
                        int in_dtype, int cache_dtype, void* stream);
@@ -109,7 +124,7 @@ int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cach
  * pkv_decode_plan -- how pkv_paged_attention_decode will divide the work.
  *   The decode streams the ordered list of (sequence, KV head, block) items
  *   through warps that each own an equal contiguous share of it (a persistent
- *   grid of about two CTAs per SM by default).  A (sequence, head) pair whose
+ *   grid of one CTA of 4 or 8 warps per SM by default).  A (sequence, head) pair whose
  *   blocks span several warps is merged from per-warp partial softmax results
  *   by a log-sum-exp rule.  This split is the library's choice; the pages do
  *   not prescribe one.
@@ -143,14 +158,16 @@ int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, i
  * K_s[j], V_s[j] the rows of token j < context_lens[s] found through
  * block_tables[s][j / 16]:
  *   out[s][i] = sum_j softmax_j(scale * q[s][i] . K_s[j]) V_s[j]
- * (quantised caches are read as code * scale of that token and head).  A
- * context length of 0 gives a zero row.
+ * (quantised caches are read as code * scale of that token and head, and
+ * PKV_U8ASYM caches as (code - zero point) * scale, [P-WMRH] §四
+ * dequantize_key).  A context length of 0 gives a zero row.
  * out            : device, [num_seqs, num_q_heads, head_dim] of q_dtype.
  * q              : device, [num_seqs, num_q_heads, head_dim] of q_dtype
  *                  (PKV_F16 or PKV_BF16; equal to cache_dtype for 16-bit
  *                  caches; for quantised caches q is converted to fp16 and
  *                  must lie within fp16 range).
- * k_cache, v_cache, k_scale, v_scale : as for pkv_kv_cache_write.
+ * k_cache, v_cache, k_scale, v_scale, k_zero, v_zero : as for
+ *                  pkv_kv_cache_write.
  * block_tables   : device int32 [num_seqs, max_blocks_per_seq].
  * context_lens   : device int32 [num_seqs], each in [0, max_context_len] and
  *                  <= max_blocks_per_seq * 16.
@@ -171,11 +188,13 @@ int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, i
  * and waits for that kernel to complete before it reads q, the caches, or
  * writes out.  (This library's KV write kernel allows that early start; any
  * other preceding kernel completes first as usual.)
- * Alignment: k_cache, v_cache and scales 16 bytes; q, out 4 bytes.
+ * Alignment: k_cache, v_cache, scales and zero points 16 bytes; q, out 4
+ * bytes.
  */
 int pkv_paged_attention_decode(void* out, const void* q,
                                const void* k_cache, const void* v_cache,
                                const float* k_scale, const float* v_scale,
+                               const uint8_t* k_zero, const uint8_t* v_zero,
                                const int32_t* block_tables, const int32_t* context_lens,
                                int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int num_blocks, int max_blocks_per_seq,
@@ -212,6 +231,7 @@ int pkv_paged_attention_decode(void* out, const void* q,
 int pkv_paged_attention_decode_noalloc(void* out, const void* q,
                                        const void* k_cache, const void* v_cache,
                                        const float* k_scale, const float* v_scale,
+                                       const uint8_t* k_zero, const uint8_t* v_zero,
                                        const int32_t* block_tables, const int32_t* context_lens,
                                        int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                        int block_size, int num_blocks, int max_blocks_per_seq,
@@ -220,15 +240,18 @@ int pkv_paged_attention_decode_noalloc(void* out, const void* q,
 
 /*
  * pkv_copy_blocks -- copy whole physical blocks (K, V and, for quantised
- * caches, their scales): for each pair p, block src_dst_pairs[2p+1] becomes a
- * copy of block src_dst_pairs[2p].  This is the copy behind copy-on-write
- * prefix sharing ([P-ASC] §二 写时复制; [P-LJT] §意外的收获：prefix sharing).
+ * caches, their scales and zero points): for each pair p, block
+ * src_dst_pairs[2p+1] becomes a copy of block src_dst_pairs[2p].  This is
+ * the copy behind copy-on-write prefix sharing ([P-ASC] §二 写时复制; [P-LJT] §意外的收获：prefix sharing).
  * src_dst_pairs : device int32 [num_pairs, 2].  Destinations must be
  *                 distinct and no destination may also be a source in the
  *                 same call (then the result equals copying all pairs at once).
  * k_scale, v_scale : required iff cache_dtype is quantised.
+ * k_zero, v_zero   : required iff cache_dtype is PKV_U8ASYM.
+ * Alignment: caches, scales and zero points 16 bytes.
  */
 int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale,
+                    uint8_t* k_zero, uint8_t* v_zero,
                     const int32_t* src_dst_pairs, int num_pairs,
                     int num_kv_heads, int head_dim, int block_size, int num_blocks,
                     int cache_dtype, void* stream);

@@ -25,7 +25,8 @@ namespace {
 std::atomic<int> g_validate{0};
 
 bool is16(int dt) { return dt == PKV_F16 || dt == PKV_BF16; }
-bool is8(int dt) { return dt == PKV_I8 || dt == PKV_FP8E4M3; }
+bool is8(int dt) { return dt == PKV_I8 || dt == PKV_FP8E4M3 || dt == PKV_U8ASYM; }
+bool has_zero(int dt) { return dt == PKV_U8ASYM; }
 int elt_size(int dt) { return is16(dt) ? 2 : 1; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -210,7 +211,7 @@ template <int kD, int kCT>
 int dispatch_nt_q(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, bool q_bf16,
                   cudaStream_t st) {
   const bool nt2 = p.group > 8;
-  if constexpr (kCT == pkv::kI8 || kCT == pkv::kFP8) {
+  if constexpr (pkv::DecodeTraits<kD, kCT>::k8bit) {
     if (q_bf16)
       return nt2 ? launch_decode<kD, kCT, 2, true>(km, vm, p, st)
                  : launch_decode<kD, kCT, 1, true>(km, vm, p, st);
@@ -232,6 +233,7 @@ int dispatch_ct(int ct, const CUtensorMap& km, const CUtensorMap& vm, const pkv:
     case PKV_BF16: return dispatch_nt_q<kD, pkv::kBF16>(km, vm, p, q_bf16, st);
     case PKV_I8: return dispatch_nt_q<kD, pkv::kI8>(km, vm, p, q_bf16, st);
     case PKV_FP8E4M3: return dispatch_nt_q<kD, pkv::kFP8>(km, vm, p, q_bf16, st);
+    case PKV_U8ASYM: return dispatch_nt_q<kD, pkv::kU8>(km, vm, p, q_bf16, st);
   }
   return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", ct);
 }
@@ -266,7 +268,7 @@ int pkv_device_status(unsigned int* status_out, int clear) {
 }
 
 int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache, float* k_scale, float* v_scale,
-                       const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim, int block_size,
+                       uint8_t* k_zero, uint8_t* v_zero, const int64_t* slot_mapping, int num_tokens, int num_kv_heads, int head_dim, int block_size,
                        int num_blocks, int in_dtype, int cache_dtype, void* stream) {
   if (num_tokens < 0 || num_kv_heads <= 0 || num_blocks <= 0)
     return fail(PKV_ERR_INVALID_ARG, "bad sizes (num_tokens %d, num_kv_heads %d, num_blocks %d)", num_tokens,
@@ -283,6 +285,8 @@ int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cach
     return fail(PKV_ERR_INVALID_ARG, "k, v and caches must be 16-byte aligned");
   if (is8(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4)))
     return fail(PKV_ERR_INVALID_ARG, "quantised caches need k_scale and v_scale");
+  if (has_zero(cache_dtype) && (!k_zero || !v_zero))
+    return fail(PKV_ERR_INVALID_ARG, "PKV_U8ASYM caches need k_zero and v_zero");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (g_validate.load()) {
     std::vector<int64_t> sl;
@@ -310,19 +314,24 @@ int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cach
           static_cast<uint4*>(v_cache), slot_mapping, num_tokens, num_kv_heads, num_blocks);
   } else {
     const int grid = grid_for(rows, 8);  // 8 warps per CTA, one row per warp
-    const bool fp8 = cache_dtype == PKV_FP8E4M3;
     const bool bf = in_dtype == PKV_BF16;
     auto* kc = static_cast<uint8_t*>(k_cache);
     auto* vc = static_cast<uint8_t*>(v_cache);
-#define PKV_QW(D, F, B) \
-  pkv::kv_write_quant_kernel<D, F, B><<<grid, 256, 0, st>>>(k, v, kc, vc, k_scale, v_scale, slot_mapping, num_tokens, num_kv_heads, num_blocks)
-    if (head_dim == 128) {
-      if (fp8) { if (bf) PKV_QW(128, true, true); else PKV_QW(128, true, false); }
-      else { if (bf) PKV_QW(128, false, true); else PKV_QW(128, false, false); }
-    } else {
-      if (fp8) { if (bf) PKV_QW(64, true, true); else PKV_QW(64, true, false); }
-      else { if (bf) PKV_QW(64, false, true); else PKV_QW(64, false, false); }
-    }
+#define PKV_QW(D, F, B)                                                                                          \
+  pkv::kv_write_quant_kernel<D, F, B><<<grid, 256, 0, st>>>(k, v, kc, vc, k_scale, v_scale, k_zero, v_zero, \
+                                                             slot_mapping, num_tokens, num_kv_heads, num_blocks)
+#define PKV_QW_FMT(D, F) \
+  do { if (bf) PKV_QW(D, F, true); else PKV_QW(D, F, false); } while (0)
+#define PKV_QW_D(D)                                               \
+  do {                                                            \
+    if (cache_dtype == PKV_FP8E4M3) PKV_QW_FMT(D, PKV_FP8E4M3);   \
+    else if (cache_dtype == PKV_U8ASYM) PKV_QW_FMT(D, PKV_U8ASYM); \
+    else PKV_QW_FMT(D, PKV_I8);                                   \
+  } while (0)
+    if (head_dim == 128) PKV_QW_D(128);
+    else PKV_QW_D(64);
+#undef PKV_QW_D
+#undef PKV_QW_FMT
 #undef PKV_QW
   }
   cudaError_t e = cudaGetLastError();
@@ -354,7 +363,8 @@ int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, i
 }
 
 int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                               const float* k_scale, const float* v_scale, const int32_t* block_tables,
+                               const float* k_scale, const float* v_scale, const uint8_t* k_zero,
+                               const uint8_t* v_zero, const int32_t* block_tables,
                                const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
                                int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
                                int max_context_len, float scale, int q_dtype, int cache_dtype, int partition_tokens,
@@ -382,6 +392,8 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   if (!aligned(q, 4) || !aligned(out, 4)) return fail(PKV_ERR_INVALID_ARG, "q and out must be 4-byte aligned");
   if (is8(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 16) || !aligned(v_scale, 16)))
     return fail(PKV_ERR_INVALID_ARG, "quantised caches need 16-byte aligned k_scale and v_scale");
+  if (has_zero(cache_dtype) && (!k_zero || !v_zero || !aligned(k_zero, 16) || !aligned(v_zero, 16)))
+    return fail(PKV_ERR_INVALID_ARG, "PKV_U8ASYM caches need 16-byte aligned k_zero and v_zero");
   Plan pl{};
   int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens, &pl);
   if (rc != PKV_OK) return rc;
@@ -414,6 +426,8 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   p.q = q;
   p.k_scale = k_scale;
   p.v_scale = v_scale;
+  p.k_zero = k_zero;
+  p.v_zero = v_zero;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
   if (pl.num_streams > 1) {
@@ -440,7 +454,8 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   return ok();
 }
 
-int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale, const int32_t* src_dst_pairs,
+int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale, uint8_t* k_zero, uint8_t* v_zero,
+                    const int32_t* src_dst_pairs,
                     int num_pairs, int num_kv_heads, int head_dim, int block_size, int num_blocks, int cache_dtype,
                     void* stream) {
   if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "bad sizes");
@@ -453,6 +468,9 @@ int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale
   const bool q8 = is8(cache_dtype);
   if (q8 && (!k_scale || !v_scale || !aligned(k_scale, 16) || !aligned(v_scale, 16)))
     return fail(PKV_ERR_INVALID_ARG, "quantised caches need 16-byte aligned k_scale and v_scale");
+  const bool zp = has_zero(cache_dtype);
+  if (zp && (!k_zero || !v_zero || !aligned(k_zero, 16) || !aligned(v_zero, 16)))
+    return fail(PKV_ERR_INVALID_ARG, "PKV_U8ASYM caches need 16-byte aligned k_zero and v_zero");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (g_validate.load()) {
     std::vector<int32_t> pr;
@@ -471,10 +489,12 @@ int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale
   }
   const long long words = static_cast<long long>(num_kv_heads) * 16 * head_dim * elt_size(cache_dtype) / 16;
   const int swords = q8 ? num_kv_heads * 4 : 0;
+  const int zwords = zp ? num_kv_heads : 0;
   const int grid = std::min(num_pairs, 16 * sm_count());
   pkv::copy_blocks_kernel<<<grid, 256, 0, st>>>(static_cast<uint4*>(k_cache), static_cast<uint4*>(v_cache),
                                                 reinterpret_cast<uint4*>(k_scale), reinterpret_cast<uint4*>(v_scale),
-                                                src_dst_pairs, num_pairs, num_blocks, words, swords);
+                                                reinterpret_cast<uint4*>(k_zero), reinterpret_cast<uint4*>(v_zero),
+                                                src_dst_pairs, num_pairs, num_blocks, words, swords, zwords);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_fail(e, "copy_blocks launch");
   return ok();
@@ -526,6 +546,7 @@ int noalloc_scratch_address(void** out) {
 
 extern "C" int pkv_paged_attention_decode_noalloc(void* out, const void* q, const void* k_cache,
                                                   const void* v_cache, const float* k_scale, const float* v_scale,
+                                                  const uint8_t* k_zero, const uint8_t* v_zero,
                                                   const int32_t* block_tables, const int32_t* context_lens,
                                                   int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                                   int block_size, int num_blocks, int max_blocks_per_seq,
@@ -549,7 +570,8 @@ extern "C" int pkv_paged_attention_decode_noalloc(void* out, const void* q, cons
     rc = noalloc_scratch_address(&scratch);
     if (rc != PKV_OK) return rc;
   }
-  return pkv_paged_attention_decode(out, q, k_cache, v_cache, k_scale, v_scale, block_tables, context_lens,
+  return pkv_paged_attention_decode(out, q, k_cache, v_cache, k_scale, v_scale, k_zero, v_zero, block_tables,
+                                    context_lens,
                                     num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                     max_blocks_per_seq, max_context_len, scale, q_dtype, cache_dtype,
                                     partition_tokens, scratch, needs_scratch ? kNoAllocScratchBytes : 0, stream);

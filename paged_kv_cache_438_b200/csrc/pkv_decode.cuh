@@ -26,9 +26,11 @@
 //       S^T[16 tok x 8 g]  = K[16 x D] . Q^T[D x 8]         (mma.m16n8k16)
 //       O^T[D x 8 g]      += V^T[D x 16 tok] . P^T[16 x 8]
 //     P^T comes from the S^T accumulators through movmatrix.  8-bit codes
-//     are widened to fp16 in registers (int8 exactly through the 0x6400
-//     exponent trick, e4m3 with the hardware converter); per-token scales
-//     fold into S (keys) and P (values).  Online softmax in fp32, base 2.
+//     are widened to fp16 in registers (int8 and uint8 exactly through the
+//     0x6400 exponent trick, e4m3 with the hardware converter); a uint8
+//     code's zero point is subtracted in that same fp16 step (exact: the
+//     difference is an integer in [-255, 255]); per-token scales fold into
+//     S (keys) and P (values).  Online softmax in fp32, base 2.
 //   * Merge.  A warp that saw a whole (sequence, head) writes the output
 //     directly.  A pair split across warps gets one fp32 partial (m, l, o/l)
 //     per contributing warp; the last contributor to arrive (an epoch-tagged
@@ -46,13 +48,13 @@
 
 namespace pkv {
 
-enum CacheType : int { kF16 = PKV_F16, kBF16 = PKV_BF16, kI8 = PKV_I8, kFP8 = PKV_FP8E4M3 };
+enum CacheType : int { kF16 = PKV_F16, kBF16 = PKV_BF16, kI8 = PKV_I8, kFP8 = PKV_FP8E4M3, kU8 = PKV_U8ASYM };
 
 constexpr int round_up_c(int x, int m) { return (x + m - 1) / m * m; }
 
 template <int kD, int kCT>
 struct DecodeTraits {
-  static constexpr bool k8bit = (kCT == kI8 || kCT == kFP8);
+  static constexpr bool k8bit = (kCT == kI8 || kCT == kFP8 || kCT == kU8);
   static constexpr int kElt = k8bit ? 1 : 2;
   static constexpr int kRowBytes = kD * kElt;                       // one token's K (or V) row
   static constexpr int kTileBytes = kRowBytes < 128 ? kRowBytes : 128;  // TMA box width == swizzle span
@@ -61,7 +63,9 @@ struct DecodeTraits {
   static constexpr int kChunksPerTileRow = kTileBytes / 16;
   static constexpr int kKVBytes = 16 * kRowBytes;                   // one block of one head, K or V
   static constexpr int kScaleBytes = k8bit ? 64 : 0;                // 16 fp32 scales
-  static constexpr int kStageTx = 2 * kKVBytes + 2 * kScaleBytes;   // bytes landing per stage
+  static constexpr int kZeroBytes = kCT == kU8 ? 16 : 0;            // 16 uint8 zero points
+  // stage layout: K tile, V tile, K scales, V scales, K zero points, V zero points
+  static constexpr int kStageTx = 2 * kKVBytes + 2 * kScaleBytes + 2 * kZeroBytes;  // bytes landing per stage
   static constexpr int kStageBytes = round_up_c(kStageTx, 1024);    // keeps every tile 1024-aligned
   static constexpr int kMaxWarps = 8;
   // One CTA per SM.  Its warps (4 or 8, chosen per call) share this many
@@ -84,6 +88,8 @@ struct DecodeParams {
   const void* q;
   const float* k_scale;
   const float* v_scale;
+  const uint8_t* k_zero;
+  const uint8_t* v_zero;
   const int32_t* block_tables;
   const int32_t* context_lens;
   unsigned long long* counters;  // [B * Hkv] arrival counters (workspace)
@@ -143,7 +149,7 @@ __device__ __forceinline__ void store_out(void* out, long long idx, float v) {
 template <int kCT, bool kQBF16>
 __device__ __forceinline__ uint32_t load_q_pair(const void* q, long long idx) {
   const uint32_t raw = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(q) + idx);
-  if constexpr (kCT == kI8 || kCT == kFP8) {
+  if constexpr (DecodeTraits<64, kCT>::k8bit) {
     if constexpr (kQBF16) {
       const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&raw);
       const __half2 h = __float22half2_rn(__bfloat1622float2(b));
@@ -314,6 +320,10 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       bulk_load(st + 2 * Tr::kKVBytes, p.k_scale + row0, 64, bar);
       bulk_load(st + 2 * Tr::kKVBytes + 64, p.v_scale + row0, 64, bar);
     }
+    if constexpr (Tr::kZeroBytes > 0) {
+      bulk_load(st + 2 * Tr::kKVBytes + 128, p.k_zero + row0, 16, bar);
+      bulk_load(st + 2 * Tr::kKVBytes + 144, p.v_zero + row0, 16, bar);
+    }
   };
 
   // the caches may still be being written by the preceding kernel
@@ -399,6 +409,13 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       }
     } else {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
+      // uint8: fp16 pairs (1024 + z) of this lane's two tokens r and r + 8
+      uint32_t zk_r = 0, zk_r8 = 0;
+      if constexpr (kCT == kU8) {
+        const uint8_t* zk = base_ptr + (st - base) + 2 * Tr::kKVBytes + 128;
+        zk_r = (0x6400u + zk[r]) * 0x10001u;
+        zk_r8 = (0x6400u + zk[r + 8]) * 0x10001u;
+      }
 #pragma unroll
       for (int jj = 0; jj < kKS; jj += 2) {
         uint32_t w[4];
@@ -412,6 +429,11 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
             hi_r = i8pair_to_h2(u0, 0x4342u);
             lo_r8 = i8pair_to_h2(u1, 0x4140u);
             hi_r8 = i8pair_to_h2(u1, 0x4342u);
+          } else if constexpr (kCT == kU8) {
+            lo_r = u8pair_minus_zero(w[2 * j2], 0x4140u, zk_r);
+            hi_r = u8pair_minus_zero(w[2 * j2], 0x4342u, zk_r);
+            lo_r8 = u8pair_minus_zero(w[2 * j2 + 1], 0x4140u, zk_r8);
+            hi_r8 = u8pair_minus_zero(w[2 * j2 + 1], 0x4342u, zk_r8);
           } else {
             e4m3x4_to_h2x2(w[2 * j2], lo_r, hi_r);
             e4m3x4_to_h2x2(w[2 * j2 + 1], lo_r8, hi_r8);
@@ -495,6 +517,14 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       }
     } else {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
+      // uint8: fp16 pairs (1024 + z) of this lane's tokens (2q, 2q + 1) and
+      // (2q + 8, 2q + 9)
+      uint32_t zv_x = 0, zv_y = 0;
+      if constexpr (kCT == kU8) {
+        const uint8_t* zv = base_ptr + (st - base) + 2 * Tr::kKVBytes + 144;
+        zv_x = (0x6400u + zv[2 * q4]) | ((0x6400u + zv[2 * q4 + 1]) << 16);
+        zv_y = (0x6400u + zv[2 * q4 + 8]) | ((0x6400u + zv[2 * q4 + 9]) << 16);
+      }
 #pragma unroll
       for (int i = 0; i < kMT; i += 2) {
         uint32_t w[4];
@@ -509,6 +539,11 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
             x1 = i8pair_to_h2(u0, 0x4341u);
             y0 = i8pair_to_h2(u1, 0x4240u);
             y1 = i8pair_to_h2(u1, 0x4341u);
+          } else if constexpr (kCT == kU8) {
+            x0 = u8pair_minus_zero(w[2 * ii], 0x4240u, zv_x);
+            x1 = u8pair_minus_zero(w[2 * ii], 0x4341u, zv_x);
+            y0 = u8pair_minus_zero(w[2 * ii + 1], 0x4240u, zv_y);
+            y1 = u8pair_minus_zero(w[2 * ii + 1], 0x4341u, zv_y);
           } else {
             e4m3x4_to_h2x2(prmt(w[2 * ii], w[2 * ii], 0x3120u), x0, x1);
             e4m3x4_to_h2x2(prmt(w[2 * ii + 1], w[2 * ii + 1], 0x3120u), y0, y1);

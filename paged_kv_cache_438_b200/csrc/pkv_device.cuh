@@ -174,6 +174,16 @@ __device__ __forceinline__ uint32_t i8pair_to_h2(uint32_t u, uint32_t sel) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Two uint8 codes in bytes (i, j) of w, minus their zero points, -> fp16x2
+// (byte i in the low half), exactly.  Placing code c under the fp16 pattern
+// 0x64 gives 1024 + c; `zz` holds the fp16 pair (1024 + z_i, 1024 + z_j), so
+// the difference is c - z, an integer in [-255, 255].
+__device__ __forceinline__ uint32_t u8pair_minus_zero(uint32_t w, uint32_t sel, uint32_t zz) {
+  uint32_t t = prmt(w, 0x64646464u, sel);
+  __half2 h = __hsub2(*reinterpret_cast<__half2*>(&t), *reinterpret_cast<__half2*>(&zz));
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 // Four E4M3 codes [b0 b1 b2 b3] of v -> fp16x2 (b0, b1) and (b2, b3), low
 // byte in the low half, with the hardware converter (exact: e4m3 values are
 // all representable in fp16).

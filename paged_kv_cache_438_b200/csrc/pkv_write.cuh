@@ -7,9 +7,13 @@
 // article §三 1. KV Cache量化; "KV Cache 与 PagedAttention" §三个直接推论):
 // a = max|x|, s = a / 127 or a / 448, code = RNE(x / s) clamped, with IEEE
 // fp32 divisions (this translation unit is compiled without fast-math).
+// The asymmetric uint8 format ("大模型推理的KV Cache管理…优化实战" §四
+// quantize_key, per-channel statistics over head_dim) stores, per (token,
+// head), s = (max - min) / 255, z = RNE(-min / s) and code = RNE((x - min) / s),
+// both clamped to [0, 255]; s = 0 stores zeros.
 //
 // Copy (ascendai.csdn.net article §二 写时复制): block dst := block src for K,
-// V and scales.
+// V, scales and zero points.
 #pragma once
 
 #include "pkv_device.cuh"
@@ -67,6 +71,18 @@ __device__ __forceinline__ float warp_max(float x) {
   return x;
 }
 
+__device__ __forceinline__ float warp_min(float x) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
+  return x;
+}
+
+// RNE of y clamped to [0, 255] (y >= 0 or +inf for codes; any sign for the
+// zero point).
+__device__ __forceinline__ uint32_t round_u8(float y) {
+  return static_cast<uint32_t>(fminf(fmaxf(rintf(y), 0.0f), 255.0f));
+}
+
 // One quantised code from x given scale s (s > 0).
 template <bool kFP8>
 __device__ __forceinline__ uint32_t quantize_one(float x, float s) {
@@ -82,13 +98,18 @@ __device__ __forceinline__ uint32_t quantize_one(float x, float s) {
 }
 
 // Quantising write: one warp per (token, head) row, D / 32 elements per lane.
-template <int kD, bool kFP8, bool kInBF16>
+// kFmt: PKV_I8 or PKV_FP8E4M3 (symmetric absmax) or PKV_U8ASYM (min/max with
+// a zero point; kz / vz receive the zero points).
+template <int kD, int kFmt, bool kInBF16>
 __global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restrict__ k, const void* __restrict__ v,
                                                              uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
                                                              float* __restrict__ ks, float* __restrict__ vs,
+                                                             uint8_t* __restrict__ kz, uint8_t* __restrict__ vz,
                                                              const int64_t* __restrict__ slots, int num_tokens,
                                                              int num_kv_heads, int num_blocks) {
   constexpr int kE = kD / 32;
+  constexpr bool kFP8 = kFmt == PKV_FP8E4M3;
+  constexpr bool kAsym = kFmt == PKV_U8ASYM;
   asm volatile("griddepcontrol.launch_dependents;");  // see kv_write_copy_kernel
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(num_tokens) * num_kv_heads;
@@ -113,18 +134,37 @@ __global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restr
       uint8_t* cache = which == 0 ? kc : vc;
       float* scales = which == 0 ? ks : vs;
       float x[kE];
-      float a = 0.0f;
 #pragma unroll
-      for (int e = 0; e < kE; ++e) {
-        x[e] = load_in<kInBF16>(src, row * kD + lane * kE + e);
-        a = fmaxf(a, fabsf(x[e]));
-      }
-      a = warp_max(a);
-      const float s = __fdiv_rn(a, kFP8 ? 448.0f : 127.0f);
+      for (int e = 0; e < kE; ++e) x[e] = load_in<kInBF16>(src, row * kD + lane * kE + e);
+      float s;
       uint32_t packed = 0;
-      if (a > 0.0f) {
+      if constexpr (kAsym) {
+        float lo = x[0], hi = x[0];
 #pragma unroll
-        for (int e = 0; e < kE; ++e) packed |= quantize_one<kFP8>(x[e], s) << (8 * e);
+        for (int e = 1; e < kE; ++e) {
+          lo = fminf(lo, x[e]);
+          hi = fmaxf(hi, x[e]);
+        }
+        lo = warp_min(lo);
+        hi = warp_max(hi);
+        s = __fdiv_rn(__fsub_rn(hi, lo), 255.0f);
+        uint32_t z = 0;
+        if (s > 0.0f) {
+          z = round_u8(__fdiv_rn(-lo, s));
+#pragma unroll
+          for (int e = 0; e < kE; ++e) packed |= round_u8(__fdiv_rn(__fsub_rn(x[e], lo), s)) << (8 * e);
+        }
+        if (lane == 0) (which == 0 ? kz : vz)[dst_row] = static_cast<uint8_t>(z);
+      } else {
+        float a = 0.0f;
+#pragma unroll
+        for (int e = 0; e < kE; ++e) a = fmaxf(a, fabsf(x[e]));
+        a = warp_max(a);
+        s = __fdiv_rn(a, kFP8 ? 448.0f : 127.0f);
+        if (a > 0.0f) {
+#pragma unroll
+          for (int e = 0; e < kE; ++e) packed |= quantize_one<kFP8>(x[e], s) << (8 * e);
+        }
       }
       if constexpr (kE == 4) {
         reinterpret_cast<uint32_t*>(cache + dst_row * kD)[lane] = packed;
@@ -138,11 +178,13 @@ __global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restr
 
 // Block copy: grid.x walks pairs, each CTA copies whole blocks with 16-byte
 // vectors.  `words` = 16-byte units per block of one cache; `swords` = 16-byte
-// units of one block's scales (0 for 16-bit caches).
+// units of one block's scales (0 for 16-bit caches); `zwords` those of its
+// zero points (0 unless the format has them).
 __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ kc, uint4* __restrict__ vc,
                                                           uint4* __restrict__ ks, uint4* __restrict__ vs,
+                                                          uint4* __restrict__ kz, uint4* __restrict__ vz,
                                                           const int32_t* __restrict__ pairs, int num_pairs,
-                                                          int num_blocks, long long words, int swords) {
+                                                          int num_blocks, long long words, int swords, int zwords) {
   for (int p = blockIdx.x; p < num_pairs; p += gridDim.x) {
     const int src = pairs[2 * p];
     const int dst = pairs[2 * p + 1];
@@ -163,6 +205,10 @@ __global__ void __launch_bounds__(256) copy_blocks_kernel(uint4* __restrict__ kc
     for (int i = threadIdx.x; i < swords; i += blockDim.x) {
       ks[static_cast<long long>(dst) * swords + i] = ks[static_cast<long long>(src) * swords + i];
       vs[static_cast<long long>(dst) * swords + i] = vs[static_cast<long long>(src) * swords + i];
+    }
+    for (int i = threadIdx.x; i < zwords; i += blockDim.x) {
+      kz[static_cast<long long>(dst) * zwords + i] = kz[static_cast<long long>(src) * zwords + i];
+      vz[static_cast<long long>(dst) * zwords + i] = vz[static_cast<long long>(src) * zwords + i];
     }
   }
 }

@@ -17,7 +17,8 @@ Workloads (shapes of the Llama families the pages discuss; values N(0, 1)):
                   blocks of one 2048-token prefix plus own suffixes U[64, 1024].
 * ``quant_mha``   Llama-2-7B heads (32 q / 32 KV), batch 256, context
                   log-uniform[128, 8192], INT8 or FP8-e4m3 codes with fp32
-                  per-(token, head) scales.
+                  per-(token, head) scales, or uint8 codes with a scale and
+                  a uint8 zero point per (token, head).
 """
 import math
 
@@ -35,7 +36,7 @@ WORKLOADS = {
     "prefix_shared": dict(batch=128, hq=32, hkv=8, d=128, dtype="bf16", ctx=("uniform", 64, 1024),
                           prefix=2048, pool=("need", 1.1), seed=1003),
     "quant_mha": dict(batch=256, hq=32, hkv=32, d=128, dtype="bf16", ctx=("loguniform", 128, 8192),
-                      pool=("need", 1.1), cache=("int8", "fp8"), seed=1004),
+                      pool=("need", 1.1), cache=("int8", "fp8", "u8asym"), seed=1004),
 }
 
 TORCH_DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16}
@@ -106,8 +107,11 @@ def randn(shape, gen, dtype):
 def random_codes(shape, gen, kind):
     """Random cache codes with a bell-shaped value mix: N(0, 1) values spread
     over the code range and converted by torch's own casts (int8: rounded and
-    clamped to +-127; fp8: torch.float8_e4m3fn, raw bytes returned as uint8)."""
+    clamped to +-127; fp8: torch.float8_e4m3fn, raw bytes returned as uint8;
+    u8asym: centred on 127.5, rounded and clamped to [0, 255])."""
     x = torch.randn(shape, generator=gen, dtype=torch.float32)
+    if kind == "u8asym":
+        return (x * (255.0 / 6.0) + 127.5).round().clamp(0, 255).to(torch.uint8)
     if kind == "int8":
         return (x * (127.0 / 3.0)).round().clamp(-127, 127).to(torch.int8)
     if kind == "fp8":
@@ -117,10 +121,18 @@ def random_codes(shape, gen, kind):
 
 
 def random_scales(shape, gen, kind):
-    """Positive fp32 scales of the size an absmax rule gives N(0, 1) data."""
-    qmax = 127.0 if kind == "int8" else 448.0
+    """Positive fp32 scales of the size an absmax rule (or, for u8asym, a
+    min/max rule over 128 values) gives N(0, 1) data."""
+    qmax = {"int8": 127.0, "fp8": 448.0, "u8asym": 255.0}[kind]
     u = torch.rand(shape, generator=gen, dtype=torch.float32)
+    if kind == "u8asym":
+        return (4.0 + 2.0 * u) / qmax
     return (2.0 + 2.0 * u) / qmax
+
+
+def random_zero_points(shape, gen):
+    """uint8 zero points around the middle of the code range."""
+    return torch.randint(96, 161, shape, generator=gen, dtype=torch.int64).to(torch.uint8)
 
 
 def decode_case(name, seed=None, batch=None, ctx_override=None, cache_kind=None, num_blocks=None,
@@ -166,6 +178,9 @@ def decode_case(name, seed=None, batch=None, ctx_override=None, cache_kind=None,
         out["v_cache"] = random_codes((nb, hkv, BLOCK_SIZE, d), gen, kind)
         out["k_scale"] = random_scales((nb, hkv, BLOCK_SIZE), gen, kind)
         out["v_scale"] = random_scales((nb, hkv, BLOCK_SIZE), gen, kind)
+        if kind == "u8asym":
+            out["k_zero"] = random_zero_points((nb, hkv, BLOCK_SIZE), gen)
+            out["v_zero"] = random_zero_points((nb, hkv, BLOCK_SIZE), gen)
     return out
 
 
@@ -227,11 +242,18 @@ def device_decode_case(name, device, seed=None, batch=None, cache_kind=None, ctx
             x = torch.randn(shape, generator=dg, device=device, dtype=torch.float16)
             if kind == "int8":
                 out[key] = (x * (127.0 / 3.0)).round().clamp(-127, 127).to(torch.int8)
+            elif kind == "u8asym":
+                out[key] = (x.float() * (255.0 / 6.0) + 127.5).round().clamp(0, 255).to(torch.uint8)
             else:
                 out[key] = (x.float() * (448.0 / 3.0)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
             del x
-        qmax = 127.0 if kind == "int8" else 448.0
+        qmax = {"int8": 127.0, "fp8": 448.0, "u8asym": 255.0}[kind]
+        span = 4.0 if kind == "u8asym" else 2.0
         for key in ("k_scale", "v_scale"):
             u = torch.rand((nb, hkv, BLOCK_SIZE), generator=dg, device=device, dtype=torch.float32)
-            out[key] = (2.0 + 2.0 * u) / qmax
+            out[key] = (span + 2.0 * u) / qmax
+        if kind == "u8asym":
+            for key in ("k_zero", "v_zero"):
+                out[key] = torch.randint(96, 161, (nb, hkv, BLOCK_SIZE), generator=dg, device=device,
+                                         dtype=torch.int64).to(torch.uint8)
     return out

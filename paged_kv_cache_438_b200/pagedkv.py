@@ -20,7 +20,8 @@ PKV_ERR_CUDA = -4
 PKV_ERR_NOT_FOUND = -5
 PKV_ERR_EXISTS = -6
 
-PKV_F16, PKV_BF16, PKV_I8, PKV_FP8E4M3 = 0, 1, 2, 3
+PKV_F16, PKV_BF16, PKV_I8, PKV_FP8E4M3, PKV_U8ASYM = 0, 1, 2, 3, 4
+QUANTISED = (PKV_I8, PKV_FP8E4M3, PKV_U8ASYM)
 
 DEV_BAD_SLOT, DEV_BAD_BLOCK, DEV_BAD_CONTEXT, DEV_TIMEOUT, DEV_BAD_PAIR = 1, 2, 4, 8, 16
 
@@ -56,15 +57,15 @@ def _signatures(lib):
     sig = {
         "pkv_last_error": ([], ctypes.c_char_p),
         "pkv_version": ([], _I),
-        "pkv_kv_cache_write": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
+        "pkv_kv_cache_write": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _P], _I),
         "pkv_decode_plan": ([_I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
                              ctypes.POINTER(_SZ)], _I),
         "pkv_decode_workspace_size": ([_I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
-        "pkv_paged_attention_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F,
-                                        _I, _I, _I, _P, _SZ, _P], _I),
-        "pkv_paged_attention_decode_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
-                                                _F, _I, _I, _I, _P], _I),
-        "pkv_copy_blocks": ([_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P], _I),
+        "pkv_paged_attention_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                                        _F, _I, _I, _I, _P, _SZ, _P], _I),
+        "pkv_paged_attention_decode_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                                _I, _I, _F, _I, _I, _I, _P], _I),
+        "pkv_copy_blocks": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P], _I),
         "pkv_device_status": ([ctypes.POINTER(ctypes.c_uint), _I], _I),
         "pkv_set_validation": ([_I], _I),
         "pkv_alloc_create": ([_I, _I, _P, ctypes.POINTER(_P)], _I),
@@ -121,6 +122,16 @@ def dtype_code(t):
     raise TypeError(f"unsupported dtype {d}")
 
 
+def cache_code(cache, k_zero=None):
+    """Cache format code: the asymmetric uint8 format when zero points are
+    given, else the cache tensor's dtype (uint8 alone means FP8-e4m3)."""
+    if k_zero is not None:
+        if cache.dtype != torch.uint8:
+            raise TypeError("a cache with zero points must be uint8")
+        return PKV_U8ASYM
+    return dtype_code(cache)
+
+
 def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
@@ -159,10 +170,21 @@ def device_status(clear=True):
     return v.value
 
 
-def kv_cache_write(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=None, stream=None):
+def _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero):
+    if ct in QUANTISED:
+        _need(k_scale, "k_scale", device=dev, dtype=torch.float32)
+        _need(v_scale, "v_scale", device=dev, dtype=torch.float32)
+    if ct == PKV_U8ASYM:
+        _need(k_zero, "k_zero", device=dev, dtype=torch.uint8)
+        _need(v_zero, "v_zero", device=dev, dtype=torch.uint8)
+
+
+def kv_cache_write(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=None, stream=None,
+                   k_zero=None, v_zero=None):
     """Writes rows k, v [T, Hkv, D] into the paged caches at slot_mapping [T]
-    (int64, -1 skips).  Quantised caches (int8 / float8_e4m3fn) need the
-    fp32 scale arrays [NB, Hkv, 16]."""
+    (int64, -1 skips).  Quantised caches (int8 / float8_e4m3fn, or uint8 with
+    zero points) need the fp32 scale arrays [NB, Hkv, 16]; the asymmetric
+    uint8 format also the uint8 zero-point arrays k_zero, v_zero [NB, Hkv, 16]."""
     for n, t in (("k", k), ("v", v), ("k_cache", k_cache), ("v_cache", v_cache)):
         _need(t, n, device=k.device)
     _need(slot_mapping, "slot_mapping", device=k.device, dtype=torch.int64)
@@ -172,13 +194,11 @@ def kv_cache_write(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=N
     nb = k_cache.shape[0]
     if k_cache.shape[1] != hkv or k_cache.shape[3] != d or slot_mapping.numel() != T:
         raise ValueError("shape mismatch between k and the caches")
-    ct = dtype_code(k_cache)
-    if ct in (PKV_I8, PKV_FP8E4M3):
-        _need(k_scale, "k_scale", device=k.device, dtype=torch.float32)
-        _need(v_scale, "v_scale", device=k.device, dtype=torch.float32)
+    ct = cache_code(k_cache, k_zero)
+    _need_quant(ct, k.device, k_scale, v_scale, k_zero, v_zero)
     _check(lib().pkv_kv_cache_write(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
-                                    _ptr(slot_mapping), T, hkv, d, k_cache.shape[2], nb, dtype_code(k), ct,
-                                    _stream(stream)))
+                                    _ptr(k_zero), _ptr(v_zero), _ptr(slot_mapping), T, hkv, d, k_cache.shape[2], nb,
+                                    dtype_code(k), ct, _stream(stream)))
 
 
 def decode_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens=0):
@@ -214,7 +234,8 @@ def new_workspace(device, nbytes):
 
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale=None, v_scale=None,
-                           max_context_len=None, out=None, workspace=None, partition_tokens=0, stream=None):
+                           max_context_len=None, out=None, workspace=None, partition_tokens=0, stream=None,
+                           k_zero=None, v_zero=None):
     """out[s, i] = softmax(scale * q[s, i] . K_s) V_s through block tables.
 
     q [B, Hq, D] fp16/bf16; caches [NB, Hkv, 16, D]; block_tables [B, MB]
@@ -222,8 +243,9 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     bound on context_lens (if None it is read from the device, which
     synchronises).  ``workspace`` (uint8, from ``new_workspace``) must be
     zero-filled before its first use and serve one call at a time; when None
-    a cached per-stream workspace is used.  Returns ``out`` [B, Hq, D] in q's
-    dtype."""
+    a cached per-stream workspace is used.  A uint8 cache with ``k_zero`` /
+    ``v_zero`` is the asymmetric format, read as (code - zero) * scale.
+    Returns ``out`` [B, Hq, D] in q's dtype."""
     dev = q.device
     for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
         _need(t, n, device=dev)
@@ -235,10 +257,8 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     nb, hkv, bs, dk = k_cache.shape
     if dk != d or block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.numel() != B:
         raise ValueError("shape mismatch")
-    ct = dtype_code(k_cache)
-    if ct in (PKV_I8, PKV_FP8E4M3):
-        _need(k_scale, "k_scale", device=dev, dtype=torch.float32)
-        _need(v_scale, "v_scale", device=dev, dtype=torch.float32)
+    ct = cache_code(k_cache, k_zero)
+    _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero)
     if max_context_len is None:
         max_context_len = int(context_lens.max().item()) if B else 0
     if out is None:
@@ -250,9 +270,9 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         workspace = _cached_workspace(dev, stream, ws_bytes)
     ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check(lib().pkv_paged_attention_decode(
-        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
-        _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], max_context_len, float(scale),
-        dtype_code(q), ct, partition_tokens, _ptr(workspace), ws_len, _stream(stream)))
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero), _ptr(v_zero),
+        _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], max_context_len,
+        float(scale), dtype_code(q), ct, partition_tokens, _ptr(workspace), ws_len, _stream(stream)))
     return out
 
 
@@ -260,7 +280,8 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 
 def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
-                                   out, k_scale=None, v_scale=None, partition_tokens=0, stream=None):
+                                   out, k_scale=None, v_scale=None, partition_tokens=0, stream=None,
+                                   k_zero=None, v_zero=None):
     """paged_attention_decode for callers that cannot allocate device memory
     (for instance a plugin whose host framework owns every allocation and
     hands it only input and output buffers): ``out`` must be given, no
@@ -276,25 +297,30 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
     _need(context_lens, "context_lens", device=dev, dtype=torch.int32)
     B, hq, d = q.shape
     nb, hkv, bs, _ = k_cache.shape
+    ct = cache_code(k_cache, k_zero)
+    _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero)
     _check(lib().pkv_paged_attention_decode_noalloc(
-        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(block_tables),
-        _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], int(max_context_len), float(scale),
-        dtype_code(q), dtype_code(k_cache), partition_tokens, _stream(stream)))
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero), _ptr(v_zero),
+        _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], int(max_context_len),
+        float(scale), dtype_code(q), ct, partition_tokens, _stream(stream)))
     return out
 
 
-def copy_blocks(k_cache, v_cache, src_dst_pairs, k_scale=None, v_scale=None, stream=None):
+def copy_blocks(k_cache, v_cache, src_dst_pairs, k_scale=None, v_scale=None, stream=None, k_zero=None,
+                v_zero=None):
     """Block dst := block src for every row (src, dst) of src_dst_pairs
-    [N, 2] int32 (device), for K, V and the scales of quantised caches."""
+    [N, 2] int32 (device), for K, V and the scales (and zero points) of
+    quantised caches."""
     dev = k_cache.device
     _need(k_cache, "k_cache", device=dev)
     _need(v_cache, "v_cache", device=dev)
     _need(src_dst_pairs, "src_dst_pairs", device=dev, dtype=torch.int32)
     nb, hkv, bs, d = k_cache.shape
-    ct = dtype_code(k_cache)
+    ct = cache_code(k_cache, k_zero)
+    _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero)
     n = src_dst_pairs.numel() // 2
-    _check(lib().pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(src_dst_pairs),
-                                 n, hkv, d, bs, nb, ct, _stream(stream)))
+    _check(lib().pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero),
+                                 _ptr(v_zero), _ptr(src_dst_pairs), n, hkv, d, bs, nb, ct, _stream(stream)))
 
 
 # --------------------------------------------------------- block allocator --

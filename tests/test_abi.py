@@ -45,38 +45,44 @@ def _err(rc, code):
 
 def test_write_rejects_bad_block_size_and_dtypes(lib):
     n = ctypes.c_void_p(16)
-    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, n, 4, 2, 64, 8, 10, P.PKV_F16, P.PKV_F16, None),
+    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, None, None, n, 4, 2, 64, 8, 10, P.PKV_F16, P.PKV_F16, None),
          P.PKV_ERR_UNSUPPORTED)
-    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, n, 4, 2, 96, 16, 10, P.PKV_F16, P.PKV_F16, None),
+    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, None, None, n, 4, 2, 96, 16, 10, P.PKV_F16, P.PKV_F16, None),
          P.PKV_ERR_UNSUPPORTED)
-    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, n, 4, 2, 64, 16, 10, P.PKV_BF16, P.PKV_F16, None),
+    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, None, None, n, 4, 2, 64, 16, 10, P.PKV_BF16, P.PKV_F16, None),
          P.PKV_ERR_UNSUPPORTED)
     # quantised cache without scale arrays
-    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, n, 4, 2, 64, 16, 10, P.PKV_BF16, P.PKV_I8, None),
+    _err(lib.pkv_kv_cache_write(n, n, n, n, None, None, None, None, n, 4, 2, 64, 16, 10, P.PKV_BF16, P.PKV_I8, None),
          P.PKV_ERR_INVALID_ARG)
+    # asymmetric uint8 cache with scales but no zero points
+    _err(lib.pkv_kv_cache_write(n, n, n, n, n, n, None, None, n, 4, 2, 64, 16, 10, P.PKV_BF16, P.PKV_U8ASYM, None),
+         P.PKV_ERR_INVALID_ARG)
+    assert b"k_zero" in lib.pkv_last_error()
     # misaligned cache pointer
     m = ctypes.c_void_p(18)
-    _err(lib.pkv_kv_cache_write(n, n, m, n, None, None, n, 4, 2, 64, 16, 10, P.PKV_F16, P.PKV_F16, None),
+    _err(lib.pkv_kv_cache_write(n, n, m, n, None, None, None, None, n, 4, 2, 64, 16, 10, P.PKV_F16, P.PKV_F16, None),
          P.PKV_ERR_INVALID_ARG)
     assert b"aligned" in lib.pkv_last_error()
 
 
 def test_write_zero_tokens_is_a_noop(lib):
-    _err(lib.pkv_kv_cache_write(None, None, None, None, None, None, None, 0, 2, 64, 16, 10, P.PKV_F16, P.PKV_F16,
+    _err(lib.pkv_kv_cache_write(None, None, None, None, None, None, None, None, None, 0, 2, 64, 16, 10, P.PKV_F16, P.PKV_F16,
                                 None), P.PKV_OK)
 
 
 def _decode(lib, **kw):
     n = ctypes.c_void_p(256)
-    a = dict(out=n, q=n, kc=n, vc=n, ks=None, vs=None, bt=n, cl=n, B=2, hq=8, hkv=2, d=128, bs=16, nb=100, mb=4,
+    a = dict(out=n, q=n, kc=n, vc=n, ks=None, vs=None, kz=None, vz=None, bt=n, cl=n, B=2, hq=8, hkv=2, d=128, bs=16, nb=100, mb=4,
              maxc=64, scale=0.1, qd=P.PKV_BF16, cd=P.PKV_BF16, pt=0, ws=None, wsb=0)
     a.update(kw)
-    return lib.pkv_paged_attention_decode(a["out"], a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["bt"], a["cl"],
+    return lib.pkv_paged_attention_decode(a["out"], a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["kz"], a["vz"],
+                                          a["bt"], a["cl"],
                                           a["B"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["mb"], a["maxc"],
                                           a["scale"], a["qd"], a["cd"], a["pt"], a["ws"], a["wsb"], None)
 
 
 def test_decode_host_rejections(lib):
+    n = ctypes.c_void_p(256)
     _err(_decode(lib, hq=7), P.PKV_ERR_INVALID_ARG)              # Hq % Hkv != 0
     _err(_decode(lib, hq=64, hkv=2), P.PKV_ERR_UNSUPPORTED)       # G = 32 > 16
     _err(_decode(lib, d=80), P.PKV_ERR_UNSUPPORTED)
@@ -85,6 +91,10 @@ def test_decode_host_rejections(lib):
     _err(_decode(lib, maxc=65), P.PKV_ERR_INVALID_ARG)            # > max_blocks * 16
     _err(_decode(lib, scale=float("nan")), P.PKV_ERR_INVALID_ARG)
     _err(_decode(lib, cd=P.PKV_I8), P.PKV_ERR_INVALID_ARG)        # quantised without scales
+    _err(_decode(lib, cd=P.PKV_U8ASYM, ks=n, vs=n), P.PKV_ERR_INVALID_ARG)   # without zero points
+    _err(_decode(lib, cd=P.PKV_U8ASYM, ks=n, vs=n, kz=n, vz=ctypes.c_void_p(264)),
+         P.PKV_ERR_INVALID_ARG)                                    # misaligned zero points
+    _err(_decode(lib, cd=5, ks=n, vs=n), P.PKV_ERR_UNSUPPORTED)   # unknown format
     _err(_decode(lib, pt=24), P.PKV_ERR_INVALID_ARG)              # partition not a multiple of 16
     # split plan needs a workspace
     _err(_decode(lib, maxc=64, pt=16), P.PKV_ERR_INVALID_ARG)
@@ -107,6 +117,8 @@ def test_plan_is_consistent(lib):
 
 def test_copy_rejections(lib):
     n = ctypes.c_void_p(256)
-    _err(lib.pkv_copy_blocks(n, n, None, None, n, 3, 2, 128, 16, 10, P.PKV_FP8E4M3, None), P.PKV_ERR_INVALID_ARG)
-    _err(lib.pkv_copy_blocks(n, n, None, None, n, 3, 2, 128, 12, 10, P.PKV_BF16, None), P.PKV_ERR_UNSUPPORTED)
-    _err(lib.pkv_copy_blocks(n, n, None, None, n, 0, 2, 128, 16, 10, P.PKV_BF16, None), P.PKV_OK)
+    _err(lib.pkv_copy_blocks(n, n, None, None, None, None, n, 3, 2, 128, 16, 10, P.PKV_FP8E4M3, None), P.PKV_ERR_INVALID_ARG)
+    _err(lib.pkv_copy_blocks(n, n, None, None, None, None, n, 3, 2, 128, 12, 10, P.PKV_BF16, None), P.PKV_ERR_UNSUPPORTED)
+    _err(lib.pkv_copy_blocks(n, n, None, None, None, None, n, 0, 2, 128, 16, 10, P.PKV_BF16, None), P.PKV_OK)
+    _err(lib.pkv_copy_blocks(n, n, n, n, None, None, n, 3, 2, 128, 16, 10, P.PKV_U8ASYM, None),
+         P.PKV_ERR_INVALID_ARG)

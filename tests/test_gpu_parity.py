@@ -3,7 +3,7 @@
 Bars: writes, block copies and quantisation are bit-exact; attention is within
 max-abs 2e-2 and mean-rel 1e-2 (sum |gpu - ref| / sum |ref|) for fp16 / bf16
 caches, and within 6e-2 max-abs of the oracle on the unquantised values for
-INT8 / FP8 caches.  Inputs come from the seeded generators in
+INT8 / FP8 / asymmetric uint8 caches.  Inputs come from the seeded generators in
 paged_kv_cache_438_b200.inputs; nothing the oracle sees is produced by the
 library's kernels.
 """
@@ -58,9 +58,14 @@ def cache_values(t, kind):
     (decoded by the oracle's own e4m3 decoder for FP8)."""
     if kind == "fp8":
         return OQ.e4m3_decode(t.detach().cpu().contiguous().view(torch.uint8).numpy())
-    if kind == "int8":
+    if kind in ("int8", "u8asym"):
         return t.detach().cpu().numpy().astype(np.float64)
     return np64(t)
+
+
+def cpu_or_none(case, key):
+    t = case.get(key)
+    return None if t is None else t.detach().cpu().numpy()
 
 
 def check_attn(got, ref, atol=ATOL, meanrel=MEANREL):
@@ -90,7 +95,8 @@ def run_decode(g, partition_tokens=0, max_context_len=None):
     P.device_status(clear=True)
     out = P.paged_attention_decode(g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"],
                                    g["scale"], k_scale=g.get("k_scale"), v_scale=g.get("v_scale"),
-                                   max_context_len=max_context_len, partition_tokens=partition_tokens)
+                                   max_context_len=max_context_len, partition_tokens=partition_tokens,
+                                   k_zero=g.get("k_zero"), v_zero=g.get("v_zero"))
     torch.cuda.synchronize()
     assert P.device_status(clear=True) == 0
     return out
@@ -98,12 +104,11 @@ def run_decode(g, partition_tokens=0, max_context_len=None):
 
 def oracle_full(case):
     kind = case["cache_kind"]
-    ks = case.get("k_scale")
-    vs = case.get("v_scale")
     return OA.paged_decode_attention(np64(case["q"]), cache_values(case["k_cache"], kind),
                                      cache_values(case["v_cache"], kind), case["block_tables"].numpy(),
                                      case["context_lens"].numpy(), case["scale"],
-                                     None if ks is None else ks.numpy(), None if vs is None else vs.numpy())
+                                     cpu_or_none(case, "k_scale"), cpu_or_none(case, "v_scale"),
+                                     k_zero=cpu_or_none(case, "k_zero"), v_zero=cpu_or_none(case, "v_zero"))
 
 
 def oracle_sampled(g, pairs, seed=0):
@@ -131,13 +136,14 @@ def oracle_sampled(g, pairs, seed=0):
         pool_idx = torch.as_tensor(np.argsort(perm), device=DEV)  # logical j stored at pool row perm[j]
         kc = g["k_cache"][blocks][:, h:h + 1][pool_idx]
         vc = g["v_cache"][blocks][:, h:h + 1][pool_idx]
-        ks = vs = None
-        if kind != "float":
-            ks = g["k_scale"][blocks][:, h:h + 1][pool_idx].cpu().numpy()
-            vs = g["v_scale"][blocks][:, h:h + 1][pool_idx].cpu().numpy()
+        side = {}
+        for key in ("k_scale", "v_scale", "k_zero", "v_zero"):
+            if key in g:
+                side[key] = g[key][blocks][:, h:h + 1][pool_idx].cpu().numpy()
         q = np64(g["q"][s, heads])[None]
         ref = OA.paged_decode_attention(q, cache_values(kc, kind), cache_values(vc, kind), perm[None],
-                                        [ctx], g["scale"], ks, vs)[0]
+                                        [ctx], g["scale"], side.get("k_scale"), side.get("v_scale"),
+                                        k_zero=side.get("k_zero"), v_zero=side.get("v_zero"))[0]
         for n, i in enumerate(heads):
             res[(s, i)] = ref[n]
     return np.stack([res[p] for p in pairs])
@@ -162,43 +168,64 @@ def test_write_16bit_bit_exact(dtype, d, T, nb):
 
 
 def _special_rows(k):
-    """Rows that exercise the quantiser's edge cases: all zero, exact ties at
-    scale 1 (INT8), and signed zeros."""
+    """Rows that exercise the quantisers' edge cases: all zero, exact ties at
+    scale 1 (INT8), signed zeros; for the asymmetric rule also a constant
+    row, rows that do not contain 0 (zero point clamped to 0 or 255) and a
+    scale-1 grid with ties in both the zero point and the codes."""
+    d = k.shape[-1]
     k[0, 0].zero_()
-    row = torch.zeros(k.shape[-1])
+    row = torch.zeros(d)
     row[:9] = torch.tensor([127.0, 2.5, 3.5, -2.5, -3.5, 0.5, -0.5, 1.5, 126.5])
     k[1, 0] = row.to(k.dtype)
     k[2, 0, 1::2] = -0.0
+    k[3, 0] = torch.full((d,), 3.25).to(k.dtype)
+    k[4, 0] = (1.0 + torch.arange(d) % 7).to(k.dtype)
+    k[5, 0] = (-2.0 - torch.arange(d) % 5).to(k.dtype)
+    row = torch.zeros(d)
+    row[:5] = torch.tensor([-0.5, 0.0, 1.0, 2.0, 254.5])
+    k[6, 0] = row.to(k.dtype)
     return k
 
 
-@pytest.mark.parametrize("kind", ["int8", "fp8"])
+QUANT = {"int8": (torch.int8, np.int8, lambda x: OQ.quantize_int8(x) + (None,)),
+         "fp8": (torch.uint8, np.uint8, lambda x: OQ.quantize_fp8_e4m3(x) + (None,)),
+         "u8asym": (torch.uint8, np.uint8, OQ.quantize_u8_asym)}
+
+
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym"])
 @pytest.mark.parametrize("in_dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("d,T", [(64, 50), (128, 600)])
 def test_write_quantised_bit_exact(kind, in_dtype, d, T):
     hkv, nb = 4, 64
     k, v = I.new_tokens(T, hkv, d, in_dtype, seed=3 * T + d)
     k = _special_rows(k)
-    slots = I.distinct_slots(T, nb, seed=T + 1, skip_every=9)
-    cdt = torch.int8 if kind == "int8" else torch.uint8
+    slots = I.distinct_slots(T, nb, seed=T + 1)
+    slots[9::9] = -1                                    # skip some tokens, keep the special rows
+    cdt, ndt, quant = QUANT[kind]
     gk = torch.zeros((nb, hkv, 16, d), dtype=cdt, device=DEV)
     gv = torch.zeros_like(gk)
     gks = torch.zeros((nb, hkv, 16), dtype=torch.float32, device=DEV)
     gvs = torch.zeros_like(gks)
-    P.kv_cache_write(k.to(DEV), v.to(DEV), gk, gv, slots.to(DEV), gks, gvs)
+    gkz = gvz = None
+    if kind == "u8asym":
+        gkz = torch.full((nb, hkv, 16), 7, dtype=torch.uint8, device=DEV)
+        gvz = torch.full_like(gkz, 7)
+    P.kv_cache_write(k.to(DEV), v.to(DEV), gk, gv, slots.to(DEV), gks, gvs, k_zero=gkz, v_zero=gvz)
     torch.cuda.synchronize()
-    quant = OQ.quantize_int8 if kind == "int8" else OQ.quantize_fp8_e4m3
-    zero_codes = np.zeros((nb, hkv, 16, d), np.int8 if kind == "int8" else np.uint8)
+    zero_codes = np.zeros((nb, hkv, 16, d), ndt)
     zero_sc = np.zeros((nb, hkv, 16), np.float32)
-    for x, gc, gs in ((k, gk, gks), (v, gv, gvs)):
-        codes, sc = quant(x.float().numpy())
+    for x, gc, gs, gz in ((k, gk, gks, gkz), (v, gv, gvs, gvz)):
+        codes, sc, zp = quant(x.float().numpy())
         assert np.array_equal(bits(gc), OC.kv_write(zero_codes, codes, slots.numpy()))
         assert np.array_equal(bits(gs), OC.scale_write(zero_sc, sc, slots.numpy()).view(np.int32))
+        if gz is not None:
+            assert np.array_equal(bits(gz), OC.scale_write(np.full((nb, hkv, 16), 7, np.uint8), zp,
+                                                           slots.numpy()))
 
 
 # ------------------------------------------------------------ block copy --
 
-@pytest.mark.parametrize("kind", ["float", "int8", "fp8"])
+@pytest.mark.parametrize("kind", ["float", "int8", "fp8", "u8asym"])
 def test_copy_blocks_bit_exact(kind):
     case = I.decode_case("llama3_8b", batch=4, cache_kind=None if kind == "float" else kind, num_blocks=200,
                          ctx_override=[300, 500, 17, 1])
@@ -207,13 +234,14 @@ def test_copy_blocks_bit_exact(kind):
     perm = rng.permutation(200)
     pairs = np.stack([perm[:40], perm[40:80]], 1).astype(np.int32)   # sources and destinations disjoint
     P.copy_blocks(g["k_cache"], g["v_cache"], torch.as_tensor(pairs, device=DEV), g.get("k_scale"),
-                  g.get("v_scale"))
+                  g.get("v_scale"), k_zero=g.get("k_zero"), v_zero=g.get("v_zero"))
     torch.cuda.synchronize()
     arrays = [bits(case["k_cache"]), bits(case["v_cache"])]
     got = [bits(g["k_cache"]), bits(g["v_cache"])]
-    if kind != "float":
-        arrays += [bits(case["k_scale"]), bits(case["v_scale"])]
-        got += [bits(g["k_scale"]), bits(g["v_scale"])]
+    for key in ("k_scale", "v_scale", "k_zero", "v_zero"):
+        if key in case:
+            arrays.append(bits(case[key]))
+            got.append(bits(g[key]))
     for ref, out in zip(OC.copy_blocks(arrays, pairs), got):
         assert np.array_equal(ref, out)
 
@@ -250,7 +278,7 @@ def test_decode_sweep_16bit(dtype, d, group, ptok):
     np.testing.assert_allclose(got[1], np.repeat(v0, group, axis=0), atol=1e-2)
 
 
-@pytest.mark.parametrize("kind", ["int8", "fp8"])
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym"])
 @pytest.mark.parametrize("qdtype", ["bf16", "f16"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("group", [1, 8, 16])
@@ -285,7 +313,7 @@ def _sample_pairs(B, hq, n, seed):
 
 @pytest.mark.parametrize("name,kind,n", [("llama3_8b", None, 48), ("llama3_70b_32k", None, 16),
                                          ("prefix_shared", None, 40), ("quant_mha", "int8", 40),
-                                         ("quant_mha", "fp8", 40)])
+                                         ("quant_mha", "fp8", 40), ("quant_mha", "u8asym", 40)])
 def test_decode_full_workload_sampled(name, kind, n):
     g = I.device_decode_case(name, DEV, cache_kind=kind)
     maxc = int(g["context_lens_cpu"].max())
@@ -367,7 +395,7 @@ def test_prefix_sharing_copy_on_write_end_to_end():
     check_attn(np64(out)[sample], ref[sample])
 
 
-@pytest.mark.parametrize("kind", ["int8", "fp8"])
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym"])
 def test_quantised_write_then_decode_end_to_end(kind):
     """bf16 token rows are quantised by the write kernel and attended by the
     decode kernel; against the oracle on the unquantised rows (6e-2) and on
@@ -382,31 +410,37 @@ def test_quantised_write_then_decode_end_to_end(kind):
                        for s, c in enumerate(ctx.tolist())])
     T = slots.numel()
     k, v = I.new_tokens(T, hkv, d, "bf16", seed=92)
-    cdt = torch.int8 if kind == "int8" else torch.uint8
+    cdt, _, quant = QUANT[kind]
     gk = torch.zeros((nb, hkv, 16, d), dtype=cdt, device=DEV)
     gv = torch.zeros_like(gk)
     gks = torch.zeros((nb, hkv, 16), dtype=torch.float32, device=DEV)
     gvs = torch.zeros_like(gks)
-    P.kv_cache_write(k.to(DEV), v.to(DEV), gk, gv, slots.to(DEV), gks, gvs)
+    gkz = gvz = None
+    if kind == "u8asym":
+        gkz = torch.zeros((nb, hkv, 16), dtype=torch.uint8, device=DEV)
+        gvz = torch.zeros_like(gkz)
+    P.kv_cache_write(k.to(DEV), v.to(DEV), gk, gv, slots.to(DEV), gks, gvs, k_zero=gkz, v_zero=gvz)
     q = I.randn((B, hq, d), gen, "bf16")
     out = np64(P.paged_attention_decode(q.to(DEV), gk, gv, bt.to(DEV), ctx.to(DEV), 1 / math.sqrt(d), gks, gvs,
-                                        max_context_len=int(ctx.max())))
+                                        max_context_len=int(ctx.max()), k_zero=gkz, v_zero=gvz))
     # (i) against attention over the unquantised bf16 rows
     raw_k = OC.kv_write(np.zeros((nb, hkv, 16, d)), k.double().numpy(), slots.numpy())
     raw_v = OC.kv_write(np.zeros((nb, hkv, 16, d)), v.double().numpy(), slots.numpy())
     ref_raw = OA.paged_decode_attention(np64(q), raw_k, raw_v, bt.numpy(), ctx.numpy(), 1 / math.sqrt(d))
     check_attn(out, ref_raw, atol=QATOL, meanrel=None)
     # (ii) against the oracle's own quantisation of the same rows
-    quant = OQ.quantize_int8 if kind == "int8" else OQ.quantize_fp8_e4m3
-    dec = (lambda c: c.astype(np.float64)) if kind == "int8" else OQ.e4m3_decode
-    ck, sk = quant(k.float().numpy())
-    cv, sv = quant(v.float().numpy())
+    dec = OQ.e4m3_decode if kind == "fp8" else (lambda c: c.astype(np.float64))
+    ck, sk, zk = quant(k.float().numpy())
+    cv, sv, zv = quant(v.float().numpy())
     zc = np.zeros((nb, hkv, 16, d))
     zs = np.zeros((nb, hkv, 16), np.float32)
-    ref_q = OA.paged_decode_attention(np64(q), OC.kv_write(zc, dec(ck), slots.numpy()),
-                                      OC.kv_write(zc, dec(cv), slots.numpy()), bt.numpy(), ctx.numpy(),
-                                      1 / math.sqrt(d), OC.scale_write(zs, sk, slots.numpy()),
-                                      OC.scale_write(zs, sv, slots.numpy()))
+    zz = np.zeros((nb, hkv, 16), np.uint8)
+    sl = slots.numpy()
+    ref_q = OA.paged_decode_attention(np64(q), OC.kv_write(zc, dec(ck), sl), OC.kv_write(zc, dec(cv), sl),
+                                      bt.numpy(), ctx.numpy(), 1 / math.sqrt(d), OC.scale_write(zs, sk, sl),
+                                      OC.scale_write(zs, sv, sl),
+                                      k_zero=None if zk is None else OC.scale_write(zz, zk, sl),
+                                      v_zero=None if zv is None else OC.scale_write(zz, zv, sl))
     check_attn(out, ref_q)
 
 
@@ -436,10 +470,10 @@ def test_validation_mode_rejects_bad_indices_before_launch():
 # ------------------------------------------------- workspace reuse, determinism --
 
 def test_workspace_reused_across_shapes_matches_fresh_workspaces():
-    """One workspace serving calls of different shapes (the arrival counters,
-    the claim counter and the partial slots of one call overlap different
-    fields of the next) must give exactly what a fresh zero-filled workspace
-    gives.  The shapes are large enough for dynamically claimed tail chunks."""
+    """One workspace serving calls of different shapes (the arrival counters
+    and the partial slots of one call overlap different fields of the next)
+    must give exactly what a fresh zero-filled workspace gives, and repeated
+    calls must give identical bits."""
     cases = [I.device_decode_case("llama3_8b", DEV, batch=32, seed=5),
              I.device_decode_case("prefix_shared", DEV, batch=48, seed=6),
              I.device_decode_case("quant_mha", DEV, batch=64, cache_kind="int8", seed=7)]
