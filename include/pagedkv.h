@@ -203,6 +203,53 @@ int pkv_paged_attention_decode(void* out, const void* q,
                                void* stream);
 
 /*
+ * pkv_multi_query_plan -- the work division pkv_paged_attention_multi_query
+ *   will use (as pkv_decode_plan; the (token, head) columns of one KV head
+ *   are cut into tiles of 8 or 16, each tile a pair of its own in the work
+ *   list).  max_query_len bounds the new tokens of any sequence.
+ */
+int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
+                         int max_context_len, int max_query_len, int cache_dtype,
+                         int partition_tokens, int* num_streams_out,
+                         int* partition_tokens_out, size_t* workspace_bytes_out);
+
+/*
+ * pkv_paged_attention_multi_query -- attention of several new tokens per
+ * sequence over the paged cache, for chunked prefill (a long prompt cut into
+ * chunks interleaved with decode steps, [P-LJT] §Continuous Batching and
+ * §调优心法) and the verify pass of speculative decoding (the large model
+ * scores all drafted positions in one pass, [P-LJT] §投机解码).
+ * The n_s = query_start_loc[s+1] - query_start_loc[s] new tokens of sequence
+ * s are the last n_s of its context_lens[s] tokens (their K/V already written
+ * with pkv_kv_cache_write); new token t (0-based) attends keys
+ * 0 .. context_lens[s] - n_s + t, i.e. causally among the new tokens and to
+ * every earlier token:
+ *   out[r][i] = sum_{j <= ctx - n + t} softmax_j(scale * q[r][i] . K_s[j]) V_s[j]
+ * for r = query_start_loc[s] + t, KV head i / G as in decode.
+ * out, q          : device, [num_q_tokens, num_q_heads, head_dim] of q_dtype,
+ *                   rows grouped by sequence.
+ * query_start_loc : device int32 [num_seqs + 1], non-decreasing, from 0 to
+ *                   num_q_tokens; each n_s <= max_query_len and <= context.
+ * max_query_len   : host-side bound of n_s (sizes the work list).
+ * Everything else as for pkv_paged_attention_decode (with
+ * pkv_multi_query_plan's workspace size).  Rows of new tokens beyond a
+ * sequence's context (an invalid input) are written as zeros and raise
+ * PKV_DEV_BAD_CONTEXT.  With every n_s = 1 the result equals decode.
+ */
+int pkv_paged_attention_multi_query(void* out, const void* q,
+                                    const void* k_cache, const void* v_cache,
+                                    const float* k_scale, const float* v_scale,
+                                    const uint8_t* k_zero, const uint8_t* v_zero,
+                                    const int32_t* block_tables, const int32_t* context_lens,
+                                    const int32_t* query_start_loc, int num_seqs,
+                                    int num_q_tokens, int max_query_len,
+                                    int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int num_blocks, int max_blocks_per_seq,
+                                    int max_context_len, float scale, int q_dtype, int cache_dtype,
+                                    int partition_tokens, void* workspace, size_t workspace_bytes,
+                                    void* stream);
+
+/*
  * pkv_paged_attention_decode_noalloc -- pkv_paged_attention_decode for
  * callers that cannot allocate device memory (no counterpart on the pages;
  * this is a library convenience).  Typical such callers: a plugin inside a

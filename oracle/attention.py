@@ -118,3 +118,40 @@ def paged_decode_attention_heads(q, k_cache, v_cache, block_tables, context_lens
         p /= p.sum()
         out[n] = p @ V
     return out
+
+
+def paged_multi_query_attention(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
+                                k_scale=None, v_scale=None, k_zero=None, v_zero=None):
+    """Attention of several new tokens per sequence over the paged cache.
+
+    Several query tokens of one sequence in one pass serve chunked prefill
+    (a long prompt cut into chunks interleaved with decode steps, "LLM 推理
+    优化深度解析", §Continuous Batching and §调优心法) and the verify pass of
+    speculative decoding (one forward of the large model scores the k drafted
+    positions at once, same page, §投机解码).  Reading taken: the n_s new
+    tokens of sequence s are the last n_s of its context_lens[s] tokens, their
+    K/V already in the cache; new token t (0-based) sits at position
+    ctx_s - n_s + t and attends keys 0 .. ctx_s - n_s + t (causal among the
+    new tokens, everything before them visible).
+
+    q: [T, Hq, D] packed by sequence, rows query_start_loc[s] ..
+    query_start_loc[s + 1] - 1 belonging to sequence s (query_start_loc
+    [B + 1], non-decreasing, starting at 0); returns [T, Hq, D] fp64.
+    """
+    q = np.asarray(q, np.float64)
+    T, Hq, D = q.shape
+    out = np.zeros((T, Hq, D), np.float64)
+    qsl = np.asarray(query_start_loc).tolist()
+    for s in range(len(qsl) - 1):
+        n = qsl[s + 1] - qsl[s]
+        if n == 0:
+            continue
+        ctx = int(context_lens[s])
+        if n > ctx:
+            raise ValueError("a sequence has more new tokens than context")
+        K = gather_sequence(k_cache, block_tables[s], ctx, k_scale, k_zero)
+        V = gather_sequence(v_cache, block_tables[s], ctx, v_scale, v_zero)
+        for t in range(n):
+            vis = ctx - n + t + 1
+            out[qsl[s] + t] = contiguous_attention(q[qsl[s] + t], K[:vis], V[:vis], scale)
+    return out

@@ -96,6 +96,8 @@ struct Plan {
   size_t workspace;    // arrival counters + partial slots
   size_t counter_bytes;
   int slot_floats;
+  int tile_cols;       // columns per pair: G (decode) or 8 / 16 (multi-query)
+  int max_tiles;       // pairs per KV head of the longest sequence (1 for decode)
 };
 
 // One partial: m[G] and l[G] padded to a multiple of 4 floats, then o[G][D];
@@ -104,14 +106,23 @@ int slot_floats(int G, int D) { return (2 * G + 3) / 4 * 4 + G * D; }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-// The work list has at most B * Hkv * ceil(max_ctx / 16) items.  By default
-// it is spread over the warps of the resident CTAs (one per SM for 16-bit
-// caches, two for 8-bit: a persistent grid)
-// but never thinner than 16 blocks per warp; partition_tokens > 0 instead caps
-// the items per warp at partition_tokens / 16.
-int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int req_tokens, Plan* out) {
+// The work list has at most B * Hkv * tiles * ceil(max_ctx / 16) items
+// (tiles = 1 for decode; multi-query mode (max_q > 0) cuts the max_q * G
+// (token, head) columns of a KV head into tiles of 8 or 16).  By default it
+// is spread over the warps of the resident CTAs (one CTA per SM: a
+// persistent grid) but never thinner than 16 blocks per warp;
+// partition_tokens > 0 instead caps the items per warp at partition_tokens / 16.
+int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int req_tokens, Plan* out,
+              int max_q = 0) {
+  const int G = Hq / Hkv;
+  int tile_cols = G, max_tiles = 1;
+  if (max_q > 0) {
+    const long long cols = static_cast<long long>(max_q) * G;
+    tile_cols = cols > 8 ? 16 : 8;
+    max_tiles = static_cast<int>((cols + tile_cols - 1) / tile_cols);
+  }
   const long long blocks_max = std::max(1, (max_ctx + 15) / 16);
-  const long long t_max = static_cast<long long>(std::max(B, 1)) * Hkv * blocks_max;
+  const long long t_max = static_cast<long long>(std::max(B, 1)) * Hkv * max_tiles * blocks_max;
   if (t_max >= (1LL << 31)) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31 (sequence, head, block) items");
   // One CTA per SM.  8-bit caches always use 8 warps (more conversion work per
   // byte); 16-bit caches use 4 warps with twice the ring depth when each of 8
@@ -127,15 +138,23 @@ int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int r
     nw = (t_max + per - 1) / per;
   } else {
     nw = std::min(static_cast<long long>(warps) * sms, (t_max + 15) / 16);
+    if (max_tiles > 1) {
+      // Several column tiles per KV head re-read the same K/V blocks: one
+      // stream per (sequence, head, tile) bound makes the warps of a CTA (and
+      // neighbouring CTAs) walk the same blocks of one head at the same time,
+      // so the re-reads hit L2 instead of HBM.  The grid then runs in waves.
+      nw = static_cast<long long>(std::max(B, 1)) * Hkv * max_tiles;
+    }
   }
   nw = std::max(1LL, std::min(nw, t_max));
   if (nw > (1LL << 24)) return fail(PKV_ERR_UNSUPPORTED, "more than 2^24 decode streams");
-  const int G = Hq / Hkv;
   out->warps = warps;
   out->num_streams = static_cast<int>(nw);
   out->stream_tokens = static_cast<int>((t_max + nw - 1) / nw * 16);
-  out->counter_bytes = align_up(static_cast<size_t>(std::max(B, 1)) * Hkv * 8, 256);
-  out->slot_floats = slot_floats(G, D);
+  out->counter_bytes = align_up(static_cast<size_t>(std::max(B, 1)) * Hkv * max_tiles * 8, 256);
+  out->slot_floats = slot_floats(tile_cols, D);
+  out->tile_cols = tile_cols;
+  out->max_tiles = max_tiles;
   out->workspace = out->counter_bytes + 2 * static_cast<size_t>(nw) * out->slot_floats * 4;
   return PKV_OK;
 }
@@ -177,10 +196,10 @@ size_t decode_smem_bytes(int num_seqs, int warps) {
          (static_cast<size_t>(num_seqs) + 1) * 4;
 }
 
-template <int kD, int kCT, int kNT, bool kQBF16>
+template <int kD, int kCT, int kNT, bool kQBF16, bool kMQ>
 int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, cudaStream_t st) {
   using Tr = pkv::DecodeTraits<kD, kCT>;
-  auto kernel = pkv::paged_decode_kernel<kD, kCT, kNT, kQBF16>;
+  auto kernel = pkv::paged_decode_kernel<kD, kCT, kNT, kQBF16, kMQ>;
   const int warps = p.ring_warps;
   if (warps < 1 || warps > Tr::kMaxWarps) return fail(PKV_ERR_INVALID_ARG, "bad warp count %d", warps);
   pkv::DecodeParams q = p;
@@ -207,33 +226,35 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::Decod
   return PKV_OK;
 }
 
-template <int kD, int kCT>
+// kNT = 2 (16 columns per pair) when the group (decode) or the tile
+// (multi-query) is wider than 8.
+template <int kD, int kCT, bool kMQ>
 int dispatch_nt_q(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, bool q_bf16,
                   cudaStream_t st) {
-  const bool nt2 = p.group > 8;
+  const bool nt2 = (kMQ ? p.tile_cols : p.group) > 8;
   if constexpr (pkv::DecodeTraits<kD, kCT>::k8bit) {
     if (q_bf16)
-      return nt2 ? launch_decode<kD, kCT, 2, true>(km, vm, p, st)
-                 : launch_decode<kD, kCT, 1, true>(km, vm, p, st);
-    return nt2 ? launch_decode<kD, kCT, 2, false>(km, vm, p, st)
-               : launch_decode<kD, kCT, 1, false>(km, vm, p, st);
+      return nt2 ? launch_decode<kD, kCT, 2, true, kMQ>(km, vm, p, st)
+                 : launch_decode<kD, kCT, 1, true, kMQ>(km, vm, p, st);
+    return nt2 ? launch_decode<kD, kCT, 2, false, kMQ>(km, vm, p, st)
+               : launch_decode<kD, kCT, 1, false, kMQ>(km, vm, p, st);
   } else {
     (void)q_bf16;
     constexpr bool kQ = (kCT == pkv::kBF16);
-    return nt2 ? launch_decode<kD, kCT, 2, kQ>(km, vm, p, st)
-               : launch_decode<kD, kCT, 1, kQ>(km, vm, p, st);
+    return nt2 ? launch_decode<kD, kCT, 2, kQ, kMQ>(km, vm, p, st)
+               : launch_decode<kD, kCT, 1, kQ, kMQ>(km, vm, p, st);
   }
 }
 
-template <int kD>
+template <int kD, bool kMQ>
 int dispatch_ct(int ct, const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, bool q_bf16,
                 cudaStream_t st) {
   switch (ct) {
-    case PKV_F16: return dispatch_nt_q<kD, pkv::kF16>(km, vm, p, q_bf16, st);
-    case PKV_BF16: return dispatch_nt_q<kD, pkv::kBF16>(km, vm, p, q_bf16, st);
-    case PKV_I8: return dispatch_nt_q<kD, pkv::kI8>(km, vm, p, q_bf16, st);
-    case PKV_FP8E4M3: return dispatch_nt_q<kD, pkv::kFP8>(km, vm, p, q_bf16, st);
-    case PKV_U8ASYM: return dispatch_nt_q<kD, pkv::kU8>(km, vm, p, q_bf16, st);
+    case PKV_F16: return dispatch_nt_q<kD, pkv::kF16, kMQ>(km, vm, p, q_bf16, st);
+    case PKV_BF16: return dispatch_nt_q<kD, pkv::kBF16, kMQ>(km, vm, p, q_bf16, st);
+    case PKV_I8: return dispatch_nt_q<kD, pkv::kI8, kMQ>(km, vm, p, q_bf16, st);
+    case PKV_FP8E4M3: return dispatch_nt_q<kD, pkv::kFP8, kMQ>(km, vm, p, q_bf16, st);
+    case PKV_U8ASYM: return dispatch_nt_q<kD, pkv::kU8, kMQ>(km, vm, p, q_bf16, st);
   }
   return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", ct);
 }
@@ -362,16 +383,24 @@ int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, i
                          nullptr, bytes);
 }
 
-int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
-                               const float* k_scale, const float* v_scale, const uint8_t* k_zero,
-                               const uint8_t* v_zero, const int32_t* block_tables,
-                               const int32_t* context_lens, int num_seqs, int num_q_heads, int num_kv_heads,
-                               int head_dim, int block_size, int num_blocks, int max_blocks_per_seq,
-                               int max_context_len, float scale, int q_dtype, int cache_dtype, int partition_tokens,
-                               void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Shared body of the decode and multi-query entry points (mq: query_start_loc
+// and the packed query rows are used; otherwise one query row per sequence).
+int attention_call(void* out, const void* q, const void* k_cache, const void* v_cache, const float* k_scale,
+                   const float* v_scale, const uint8_t* k_zero, const uint8_t* v_zero, const int32_t* block_tables,
+                   const int32_t* context_lens, const int32_t* query_start_loc, int num_q_tokens, int max_query_len,
+                   bool mq, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                   int num_blocks, int max_blocks_per_seq, int max_context_len, float scale, int q_dtype,
+                   int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0)
     return fail(PKV_ERR_INVALID_ARG, "bad sizes");
+  if (mq && (num_q_tokens < 0 || max_query_len < 0))
+    return fail(PKV_ERR_INVALID_ARG, "bad query sizes (num_q_tokens %d, max_query_len %d)", num_q_tokens,
+                max_query_len);
   if (block_size != 16) return fail(PKV_ERR_UNSUPPORTED, "block_size must be 16 (got %d)", block_size);
   if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
   if (num_q_heads % num_kv_heads != 0) return fail(PKV_ERR_INVALID_ARG, "num_q_heads %% num_kv_heads != 0");
@@ -385,8 +414,8 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
     return fail(PKV_ERR_UNSUPPORTED, "pool too large for 32-bit copy coordinates");
   if (static_cast<long long>(max_context_len) > static_cast<long long>(max_blocks_per_seq) * 16)
     return fail(PKV_ERR_INVALID_ARG, "max_context_len %d exceeds max_blocks_per_seq * 16", max_context_len);
-  if (num_seqs == 0) return ok();
-  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens)
+  if (num_seqs == 0 || (mq && (num_q_tokens == 0 || max_query_len == 0))) return ok();
+  if (!out || !q || !k_cache || !v_cache || !block_tables || !context_lens || (mq && !query_start_loc))
     return fail(PKV_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(PKV_ERR_INVALID_ARG, "caches must be 16-byte aligned");
   if (!aligned(q, 4) || !aligned(out, 4)) return fail(PKV_ERR_INVALID_ARG, "q and out must be 4-byte aligned");
@@ -395,16 +424,18 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   if (has_zero(cache_dtype) && (!k_zero || !v_zero || !aligned(k_zero, 16) || !aligned(v_zero, 16)))
     return fail(PKV_ERR_INVALID_ARG, "PKV_U8ASYM caches need 16-byte aligned k_zero and v_zero");
   Plan pl{};
-  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens, &pl);
+  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens,
+                     &pl, mq ? max_query_len : 0);
   if (rc != PKV_OK) return rc;
   if (pl.num_streams > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned(workspace, 256)))
     return fail(PKV_ERR_INVALID_ARG, "workspace of %zu bytes (256-byte aligned) required, got %zu", pl.workspace,
                 workspace ? workspace_bytes : 0);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   if (g_validate.load()) {
-    std::vector<int32_t> ctx, bt;
+    std::vector<int32_t> ctx, bt, qsl;
     rc = fetch(&ctx, context_lens, static_cast<size_t>(num_seqs), st);
     if (rc == PKV_OK) rc = fetch(&bt, block_tables, static_cast<size_t>(num_seqs) * max_blocks_per_seq, st);
+    if (rc == PKV_OK && mq) rc = fetch(&qsl, query_start_loc, static_cast<size_t>(num_seqs) + 1, st);
     if (rc != PKV_OK) return rc;
     for (int s = 0; s < num_seqs; ++s) {
       if (ctx[s] < 0 || ctx[s] > max_context_len)
@@ -412,6 +443,16 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
       for (int j = 0; j < (ctx[s] + 15) / 16; ++j) {
         const int32_t b = bt[static_cast<size_t>(s) * max_blocks_per_seq + j];
         if (b < 0 || b >= num_blocks) return fail(PKV_ERR_INVALID_ARG, "block_tables[%d][%d] = %d out of range", s, j, b);
+      }
+    }
+    if (mq) {
+      if (qsl[0] != 0 || qsl[num_seqs] != num_q_tokens)
+        return fail(PKV_ERR_INVALID_ARG, "query_start_loc must run from 0 to num_q_tokens (%d)", num_q_tokens);
+      for (int s = 0; s < num_seqs; ++s) {
+        const int n = qsl[s + 1] - qsl[s];
+        if (n < 0 || n > max_query_len || n > ctx[s])
+          return fail(PKV_ERR_INVALID_ARG, "sequence %d has %d new tokens (max_query_len %d, context %d)", s, n,
+                      max_query_len, ctx[s]);
       }
     }
   }
@@ -430,6 +471,7 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   p.v_zero = v_zero;
   p.block_tables = block_tables;
   p.context_lens = context_lens;
+  p.query_start_loc = mq ? query_start_loc : nullptr;
   if (pl.num_streams > 1) {
     auto* ws = static_cast<uint8_t*>(workspace);
     p.counters = reinterpret_cast<unsigned long long*>(ws);
@@ -445,13 +487,69 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
   p.num_streams = pl.num_streams;
   p.ring_warps = pl.warps;
   p.slot_floats = pl.slot_floats;
+  p.tile_cols = pl.tile_cols;
+  p.max_tiles = pl.max_tiles;
+  p.num_q_tokens = mq ? num_q_tokens : num_seqs;
   p.epoch = next_epoch();
   p.qk_scale_log2 = scale * 1.4426950408889634f;
   const bool q_bf16 = q_dtype == PKV_BF16;
-  rc = head_dim == 128 ? dispatch_ct<128>(cache_dtype, km, vm, p, q_bf16, st)
-                       : dispatch_ct<64>(cache_dtype, km, vm, p, q_bf16, st);
+  if (mq)
+    rc = head_dim == 128 ? dispatch_ct<128, true>(cache_dtype, km, vm, p, q_bf16, st)
+                         : dispatch_ct<64, true>(cache_dtype, km, vm, p, q_bf16, st);
+  else
+    rc = head_dim == 128 ? dispatch_ct<128, false>(cache_dtype, km, vm, p, q_bf16, st)
+                         : dispatch_ct<64, false>(cache_dtype, km, vm, p, q_bf16, st);
   if (rc != PKV_OK) return rc;
   return ok();
+}
+
+}  // namespace
+
+extern "C" {
+
+int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, const void* v_cache,
+                               const float* k_scale, const float* v_scale, const uint8_t* k_zero,
+                               const uint8_t* v_zero, const int32_t* block_tables, const int32_t* context_lens,
+                               int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
+                               int num_blocks, int max_blocks_per_seq, int max_context_len, float scale, int q_dtype,
+                               int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  return attention_call(out, q, k_cache, v_cache, k_scale, v_scale, k_zero, v_zero, block_tables, context_lens,
+                        nullptr, num_seqs, 1, false, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
+                        num_blocks, max_blocks_per_seq, max_context_len, scale, q_dtype, cache_dtype,
+                        partition_tokens, workspace, workspace_bytes, stream);
+}
+
+int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
+                         int max_query_len, int cache_dtype, int partition_tokens, int* num_streams_out,
+                         int* partition_tokens_out, size_t* workspace_bytes_out) {
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0 || max_query_len < 0)
+    return fail(PKV_ERR_INVALID_ARG, "bad sizes");
+  if (num_q_heads % num_kv_heads != 0) return fail(PKV_ERR_INVALID_ARG, "num_q_heads %% num_kv_heads != 0");
+  if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  Plan pl{};
+  int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens,
+                     &pl, std::max(max_query_len, 1));
+  if (rc != PKV_OK) return rc;
+  if (num_streams_out) *num_streams_out = pl.num_streams;
+  if (partition_tokens_out) *partition_tokens_out = pl.stream_tokens;
+  if (workspace_bytes_out) *workspace_bytes_out = pl.workspace;
+  return ok();
+}
+
+int pkv_paged_attention_multi_query(void* out, const void* q, const void* k_cache, const void* v_cache,
+                                    const float* k_scale, const float* v_scale, const uint8_t* k_zero,
+                                    const uint8_t* v_zero, const int32_t* block_tables, const int32_t* context_lens,
+                                    const int32_t* query_start_loc, int num_seqs, int num_q_tokens,
+                                    int max_query_len, int num_q_heads, int num_kv_heads, int head_dim,
+                                    int block_size, int num_blocks, int max_blocks_per_seq, int max_context_len,
+                                    float scale, int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
+                                    size_t workspace_bytes, void* stream) {
+  return attention_call(out, q, k_cache, v_cache, k_scale, v_scale, k_zero, v_zero, block_tables, context_lens,
+                        query_start_loc, num_q_tokens, max_query_len, true, num_seqs, num_q_heads, num_kv_heads,
+                        head_dim, block_size, num_blocks, max_blocks_per_seq, max_context_len, scale, q_dtype,
+                        cache_dtype, partition_tokens, workspace, workspace_bytes, stream);
 }
 
 int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale, uint8_t* k_zero, uint8_t* v_zero,

@@ -42,6 +42,15 @@
 //     (programmatic dependent launch): it scans the context lengths, reads the
 //     block tables and q, and waits for the write only before its first copy
 //     from the cache.
+//   * Multi-query mode (kMQ: several new tokens per sequence, for chunked
+//     prefill and speculative verification, "LLM 推理优化深度解析"
+//     §Continuous Batching and §投机解码): the N columns of a pair are
+//     (new token, query head) pairs of one KV head, up to 8 * kNT of them per
+//     "tile"; a sequence with n new tokens has ceil(n * G / (8 * kNT)) tiles
+//     per KV head, each a pair of its own in the work list.  New token t of n
+//     sees keys up to position ctx - n + t, so the mask is per column; a
+//     column can meet a block that is wholly masked for it, so its running
+//     max may still be -inf and the exponentials use a finite base.
 #pragma once
 
 #include "pkv_device.cuh"
@@ -92,7 +101,8 @@ struct DecodeParams {
   const uint8_t* v_zero;
   const int32_t* block_tables;
   const int32_t* context_lens;
-  unsigned long long* counters;  // [B * Hkv] arrival counters (workspace)
+  const int32_t* query_start_loc;  // [B + 1] (multi-query mode only)
+  unsigned long long* counters;  // [B * Hkv * max_tiles] arrival counters (workspace)
   float* slots;                  // [2 * num_streams][slot_floats] partials (workspace)
   int num_seqs;
   int num_q_heads;
@@ -104,7 +114,11 @@ struct DecodeParams {
   int num_streams;   // warps sharing the work list
   int ring;          // copy stages per warp (set at launch from ring_warps)
   int ring_warps;    // warps per CTA
-  int slot_floats;   // ml + G * D: m[G], l[G] padded to ml = round_up(2G, 4), then o[G][D]
+  int slot_floats;   // ml + C * D: m[C], l[C] padded to ml = round_up(2C, 4), then o[C][D];
+                     // C = G (decode) or tile_cols (multi-query)
+  int tile_cols;     // multi-query: columns per tile (8 * kNT)
+  int max_tiles;     // multi-query: tiles per KV head of the longest query run (1 for decode)
+  int num_q_tokens;  // multi-query: rows of q and out
   unsigned long long epoch;  // this call's epoch, nonzero, < 2^40
   float qk_scale_log2;       // softmax scale * log2(e)
 };
@@ -163,8 +177,42 @@ __device__ __forceinline__ int blocks_of(const DecodeParams& p, int s, bool repo
   return (clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, report) + 15) >> 4;
 }
 
-// cum[s] = sum over sequences s' < s of blocks(s') * Hkv, for s = 0..B; one
-// entry per (sequence, KV head, block) work item before sequence s.
+__device__ __forceinline__ void query_range(const DecodeParams& p, int s, int ctx, int& q0, int& q1, int& n,
+                                            bool report);
+
+// New tokens of sequence s in multi-query mode (see query_range).
+__device__ __forceinline__ int new_tokens_of(const DecodeParams& p, int s, int ctx) {
+  int q0, q1, n;
+  query_range(p, s, ctx, q0, q1, n, false);
+  return n;
+}
+
+// Pairs per KV head of sequence s: 1 for decode, the column tiles of its new
+// tokens in multi-query mode.
+template <bool kMQ>
+__device__ __forceinline__ int tiles_of(const DecodeParams& p, int s, int ctx) {
+  if constexpr (kMQ) {
+    const int n = new_tokens_of(p, s, ctx);
+    return (n * p.group + p.tile_cols - 1) / p.tile_cols;
+  } else {
+    return 1;
+  }
+}
+
+// Work items of sequence s: blocks * Hkv * tiles.
+template <bool kMQ>
+__device__ __forceinline__ int items_of(const DecodeParams& p, int s, bool report) {
+  if constexpr (kMQ) {
+    const int ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, report);
+    return ((ctx + 15) >> 4) * p.num_kv_heads * tiles_of<true>(p, s, ctx);
+  } else {
+    return blocks_of(p, s, report) * p.num_kv_heads;
+  }
+}
+
+// cum[s] = sum over sequences s' < s of their work items, for s = 0..B; one
+// entry per (sequence, KV head[, tile], block) work item before sequence s.
+template <bool kMQ>
 __device__ __forceinline__ void scan_work(const DecodeParams& p, int32_t* cum) {
   __shared__ int warp_sums[32];
   const int B = p.num_seqs;
@@ -177,7 +225,7 @@ __device__ __forceinline__ void scan_work(const DecodeParams& p, int32_t* cum) {
   const int s1 = min(s0 + per, B);
   const bool report = blockIdx.x == 0;
   int local = 0;
-  for (int s = s0; s < s1; ++s) local += blocks_of(p, s, report) * p.num_kv_heads;
+  for (int s = s0; s < s1; ++s) local += items_of<kMQ>(p, s, report);
   int x = local;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -190,7 +238,7 @@ __device__ __forceinline__ void scan_work(const DecodeParams& p, int32_t* cum) {
   for (int w = 0; w < warp; ++w) run += warp_sums[w];
   if (tid == 0) cum[0] = 0;
   for (int s = s0; s < s1; ++s) {
-    run += blocks_of(p, s, false) * p.num_kv_heads;
+    run += items_of<kMQ>(p, s, false);
     cum[s + 1] = run;
   }
   __syncthreads();
@@ -206,19 +254,44 @@ __device__ __forceinline__ int find_seq(const int32_t* cum, int B, int g) {
   return lo;
 }
 
+// Blocks per pair of sequence s (a sequence with work has at least one).
+template <bool kMQ>
+__device__ __forceinline__ int pair_blocks(const DecodeParams& p, const int32_t* cum, int s) {
+  if constexpr (kMQ) {
+    return blocks_of(p, s, false);
+  } else {
+    return (cum[s + 1] - cum[s]) / p.num_kv_heads;
+  }
+}
+
 // TMA row coordinate (block * Hkv + head) * 16 of work item g.
+template <bool kMQ>
 __device__ __forceinline__ int item_row(const DecodeParams& p, const int32_t* cum, int g) {
   const int s = find_seq(cum, p.num_seqs, g);
-  const int nb = (cum[s + 1] - cum[s]) / p.num_kv_heads;
+  const int nb = pair_blocks<kMQ>(p, cum, s);
   const int off = g - cum[s];
-  const int h = off / nb;
-  const int j = off - h * nb;
+  const int pr = off / nb;
+  const int j = off - pr * nb;
+  // pairs of a sequence run KV head by KV head, tiles innermost
+  const int h = kMQ ? pr / ((cum[s + 1] - cum[s]) / (nb * p.num_kv_heads)) : pr;
   int id = p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + j];
   if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
     raise_status(PKV_DEV_BAD_BLOCK);
     id = 0;
   }
   return (id * p.num_kv_heads + h) * 16;
+}
+
+// Rows [q0, q0 + n) of q / out hold the new tokens of sequence s in
+// multi-query mode: query_start_loc clamped to [0, num_q_tokens] and n to
+// the context (an inconsistent entry raises a status bit when `report`).
+__device__ __forceinline__ void query_range(const DecodeParams& p, int s, int ctx, int& q0, int& q1, int& n,
+                                            bool report) {
+  const int a = p.query_start_loc[s], b = p.query_start_loc[s + 1];
+  q0 = min(max(a, 0), p.num_q_tokens);
+  q1 = min(max(b, q0), p.num_q_tokens);
+  n = min(q1 - q0, ctx);
+  if (report && (a != q0 || b != q1 || q1 - q0 != n)) raise_status(PKV_DEV_BAD_CONTEXT);
 }
 
 // First work item of stream w among T items split over nw streams.
@@ -231,7 +304,7 @@ __device__ __forceinline__ int stream_of(long long T, long long g, long long nw)
   return static_cast<int>(((g + 1) * nw - 1) / T);
 }
 
-template <int kD, int kCT, int kNT, bool kQBF16>
+template <int kD, int kCT, int kNT, bool kQBF16, bool kMQ>
 __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                         const DecodeParams p) {
@@ -264,15 +337,24 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     for (int j = 0; j < kR; ++j) mbar_init(bar_base + (warp * kR + j) * 8, 1);
     fence_barrier_init();
   }
-  scan_work(p, cum);  // ends with __syncthreads (barrier init visible too)
+  scan_work<kMQ>(p, cum);  // ends with __syncthreads (barrier init visible too)
 
-  // Sequences without context get zero rows.  (Only the caches and scales can
-  // still be in flight from a KV write launched just before this kernel; the
-  // wait for it comes right before the first copy is issued.)
+  // Sequences without context get zero rows (multi-query: rows of new tokens
+  // beyond the context).  (Only the caches and scales can still be in flight
+  // from a KV write launched just before this kernel; the wait for it comes
+  // right before the first copy is issued.)
   for (int s = blockIdx.x; s < B; s += gridDim.x) {
-    if (cum[s + 1] == cum[s]) {
-      for (int idx = threadIdx.x; idx < Hq * kD; idx += blockDim.x)
-        store_out<kOutBF16>(p.out, static_cast<long long>(s) * Hq * kD + idx, 0.0f);
+    if constexpr (kMQ) {
+      int q0, q1, n;
+      query_range(p, s, clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false), q0, q1,
+                  n, false);
+      for (long long idx = threadIdx.x; idx < static_cast<long long>(q1 - q0 - n) * Hq * kD; idx += blockDim.x)
+        store_out<kOutBF16>(p.out, static_cast<long long>(q0 + n) * Hq * kD + idx, 0.0f);
+    } else {
+      if (cum[s + 1] == cum[s]) {
+        for (int idx = threadIdx.x; idx < Hq * kD; idx += blockDim.x)
+          store_out<kOutBF16>(p.out, static_cast<long long>(s) * Hq * kD + idx, 0.0f);
+      }
     }
   }
 
@@ -290,7 +372,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
   int offset;
   {
     const int sl = find_seq(cum, B, g1 - 1);
-    const int nbl = (cum[sl + 1] - cum[sl]) / Hkv;
+    const int nbl = pair_blocks<kMQ>(p, cum, sl);
     const int gpl = cum[sl] + ((g1 - 1 - cum[sl]) / nbl) * nbl;
     offset = gpl > g0 ? gpl - g0 : 0;
   }
@@ -300,8 +382,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
   const uint32_t bars = bar_base + warp * kR * 8;
 
   // Copy coordinates of this warp's items, 32 at a time, two chunks ahead.
-  int pre0 = lane < count ? item_row(p, cum, item_of(lane)) : 0;
-  int pre1 = 32 + lane < count ? item_row(p, cum, item_of(32 + lane)) : 0;
+  int pre0 = lane < count ? item_row<kMQ>(p, cum, item_of(lane)) : 0;
+  int pre1 = 32 + lane < count ? item_row<kMQ>(p, cum, item_of(32 + lane)) : 0;
 
   int istage = 0;  // ring stage of the next item to issue (only lane 0 issues)
   auto issue = [&](int row0) {
@@ -334,28 +416,66 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     if (lane == 0) issue(row0);
   }
 
-  // ---- cursor over (sequence, head, block), in processing order ----
-  int s, nb, h, j, ctx;
+  // ---- cursor over (sequence, pair, block), in processing order; a pair is
+  // a KV head (decode) or a (KV head, column tile) (multi-query) ----
+  int s, nb, pr, h, j, ctx;
+  int ntile = 1, tile = 0, q0 = 0, n_new = 1;  // multi-query only
+  auto set_pair = [&]() {
+    if constexpr (kMQ) {
+      h = pr / ntile;
+      tile = pr - h * ntile;
+    } else {
+      h = pr;
+    }
+  };
+  auto enter_seq = [&]() {
+    nb = pair_blocks<kMQ>(p, cum, s);
+    ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false);
+    if constexpr (kMQ) {
+      int q1;
+      query_range(p, s, ctx, q0, q1, n_new, false);
+      ntile = (cum[s + 1] - cum[s]) / (nb * Hkv);
+    }
+  };
   auto locate = [&](int g) {
     s = find_seq(cum, B, g);
-    nb = (cum[s + 1] - cum[s]) / Hkv;
-    h = (g - cum[s]) / nb;
-    j = (g - cum[s]) - h * nb;
-    ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false);
+    enter_seq();
+    pr = (g - cum[s]) / nb;
+    j = (g - cum[s]) - pr * nb;
+    set_pair();
   };
   locate(item_of(0));
+
+  // Multi-query: column c of tile `tile` is (new token t, head g) with
+  // tile * C + c = t * G + g; its keys are positions < ctx - n_new + t + 1.
+  auto col_token = [&](int c) { return (tile * p.tile_cols + c) / G; };
+  auto col_head = [&](int c) { return (tile * p.tile_cols + c) % G; };
 
   uint32_t qf[kNT][kKS][2];
   float o[kMT][kNT][4];
   float m_run[kNT][2], l_run[kNT][2];
+  int colv[kNT][2];  // multi-query: visible keys of the lane's accumulator columns
 
   auto begin_pair = [&]() {
     const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
       const int g = nt * 8 + r;
-      const bool valid = g < G;
-      const long long qrow = (head_row0 + (valid ? g : 0)) * kD;
+      bool valid;
+      long long qrow;
+      if constexpr (kMQ) {
+        const int t = col_token(g);
+        valid = t < n_new;
+        qrow = valid ? (static_cast<long long>(q0 + t) * Hq + static_cast<long long>(h) * G + col_head(g)) * kD : 0;
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+          const int tc = col_token(nt * 8 + 2 * q4 + c);
+          colv[nt][c] = tc < n_new ? ctx - n_new + tc + 1 : ctx;
+        }
+      } else {
+        valid = g < G;
+        qrow = (head_row0 + (valid ? g : 0)) * kD;
+      }
 #pragma unroll
       for (int jj = 0; jj < kKS; ++jj) {
         // 16-bit K: k-index 2q,2q+1 -> d 16jj+2q.. ; 2q+8.. -> d 16jj+8+2q..
@@ -467,10 +587,18 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     float alpha[kNT][2];
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
-      const float s0 = ok_r ? sacc[nt][0] * f_r : -INFINITY;
-      const float s1 = ok_r ? sacc[nt][1] * f_r : -INFINITY;
-      const float s2 = ok_r8 ? sacc[nt][2] * f_r8 : -INFINITY;
-      const float s3 = ok_r8 ? sacc[nt][3] * f_r8 : -INFINITY;
+      bool ok0 = ok_r, ok1 = ok_r, ok2 = ok_r8, ok3 = ok_r8;
+      if constexpr (kMQ) {
+        const int va = colv[nt][0] - j * 16, vb = colv[nt][1] - j * 16;
+        ok0 = r < va;
+        ok1 = r < vb;
+        ok2 = r + 8 < va;
+        ok3 = r + 8 < vb;
+      }
+      const float s0 = ok0 ? sacc[nt][0] * f_r : -INFINITY;
+      const float s1 = ok1 ? sacc[nt][1] * f_r : -INFINITY;
+      const float s2 = ok2 ? sacc[nt][2] * f_r8 : -INFINITY;
+      const float s3 = ok3 ? sacc[nt][3] * f_r8 : -INFINITY;
       float mx_a = fmaxf(s0, s2), mx_b = fmaxf(s1, s3);
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
@@ -484,8 +612,12 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       alpha[nt][1] = mn_b == m_run[nt][1] ? 1.0f : fast_exp2(m_run[nt][1] - mn_b);
       m_run[nt][0] = mn_a;
       m_run[nt][1] = mn_b;
-      const float p0 = fast_exp2(s0 - mn_a), p1 = fast_exp2(s1 - mn_b);
-      const float p2 = fast_exp2(s2 - mn_a), p3 = fast_exp2(s3 - mn_b);
+      // a column with no visible key yet keeps m = -inf: exponentiate
+      // against 0 instead, which gives p = 0 for its masked entries
+      const float b_a = (kMQ && mn_a == -INFINITY) ? 0.0f : mn_a;
+      const float b_b = (kMQ && mn_b == -INFINITY) ? 0.0f : mn_b;
+      const float p0 = fast_exp2(s0 - b_a), p1 = fast_exp2(s1 - b_b);
+      const float p2 = fast_exp2(s2 - b_a), p3 = fast_exp2(s3 - b_b);
       l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (p0 + p2);
       l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (p1 + p3);
       // P^T operand: rows = tokens of the block, columns = query heads
@@ -563,7 +695,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
         // entering chunk `chunk` (held in pre[chunk & 1]); chunk - 1 is spent,
         // so its register takes chunk + 1
         const int ki = (chunk + 1) * 32 + lane;
-        const int nxt = ki < count ? item_row(p, cum, item_of(ki)) : 0;
+        const int nxt = ki < count ? item_row<kMQ>(p, cum, item_of(ki)) : 0;
         if (chunk & 1) pre0 = nxt; else pre1 = nxt;
       }
       const int row0 = __shfl_sync(0xffffffffu, (chunk & 1) ? pre1 : pre0, kn & 31);
@@ -587,7 +719,17 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
         lsum[nt][1] = lb;
       }
       const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
-      const int gp0 = cum[s] + h * nb;  // the pair's first and last items
+      // columns of this pair: G heads (decode) or a tile of (token, head)
+      const int C = kMQ ? p.tile_cols : G;
+      const int ncols = kMQ ? min(p.tile_cols, n_new * G - tile * p.tile_cols) : G;
+      auto out_row = [&](int c) -> long long {
+        if constexpr (kMQ) {
+          return static_cast<long long>(q0 + col_token(c)) * Hq + static_cast<long long>(h) * G + col_head(c);
+        } else {
+          return head_row0 + c;
+        }
+      };
+      const int gp0 = cum[s] + pr * nb;  // the pair's first and last items
       const int gpe = gp0 + nb - 1;
       if (gp0 >= g0 && gpe < g1) {
         // the whole pair went through this warp: write the output
@@ -596,30 +738,32 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int g = nt * 8 + 2 * q4 + c;
-            if (g >= G) continue;
+            if (g >= ncols) continue;
             const float inv = 1.0f / lsum[nt][c];
+            const long long row = out_row(g);
 #pragma unroll
             for (int i = 0; i < kMT; ++i) {
               const int d0 = k8 ? 16 * i + 2 * r : 16 * i + r;
               const int d1 = k8 ? d0 + 1 : d0 + 8;
-              store_out<kOutBF16>(p.out, (head_row0 + g) * kD + d0, o[i][nt][c] * inv);
-              store_out<kOutBF16>(p.out, (head_row0 + g) * kD + d1, o[i][nt][2 + c] * inv);
+              store_out<kOutBF16>(p.out, row * kD + d0, o[i][nt][c] * inv);
+              store_out<kOutBF16>(p.out, row * kD + d1, o[i][nt][2 + c] * inv);
             }
           }
       } else {
         // a share of a split pair: publish (m, l, o / l), then count arrivals
-        const int ml = p.slot_floats - G * kD;
+        const int ml = p.slot_floats - C * kD;
         float* slot = p.slots + static_cast<long long>(2 * gw + (gp0 <= g0 && g0 <= gpe ? 0 : 1)) * p.slot_floats;
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
           for (int c = 0; c < 2; ++c) {
             const int g = nt * 8 + 2 * q4 + c;
-            if (g >= G) continue;
-            const float inv = 1.0f / lsum[nt][c];
+            if (g >= ncols) continue;
+            // multi-query: a share may hold no visible key of a column (l = 0)
+            const float inv = (kMQ && lsum[nt][c] == 0.0f) ? 0.0f : 1.0f / lsum[nt][c];
             if (r == 0) {
               slot[g] = m_run[nt][c];
-              slot[G + g] = lsum[nt][c];
+              slot[C + g] = lsum[nt][c];
             }
             float* og = slot + ml + g * kD;
 #pragma unroll
@@ -636,7 +780,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
         const int n_c = stream_of(T, gpe, nw) - w_first + 1;
         int last = 0;
         if (lane == 0) {
-          unsigned long long* ctr = p.counters + static_cast<long long>(s) * Hkv + h;
+          unsigned long long* ctr =
+              p.counters + (static_cast<long long>(s) * Hkv + h) * (kMQ ? p.max_tiles : 1) + (kMQ ? tile : 0);
           const unsigned long long E = p.epoch;
           unsigned long long old = atomicAdd(ctr, 0ull), assumed, next;
           do {
@@ -662,7 +807,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
           // lane owns kD / 32 output columns of every head.
           constexpr int kV = kD / 32;
 #pragma unroll 1
-          for (int g0 = 0; g0 < G; g0 += 8) {
+          for (int g0 = 0; g0 < ncols; g0 += 8) {
             float Mg[8], Lg[8], acc[8][kV];
 #pragma unroll
             for (int gg = 0; gg < 8; ++gg) {
@@ -678,9 +823,9 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 #pragma unroll
               for (int gg = 0; gg < 8; ++gg) {
                 const int g = g0 + gg;
-                if (g < G) {
+                if (g < ncols) {
                   mc[gg] = __ldcg(sl + g);
-                  lc[gg] = __ldcg(sl + G + g);
+                  lc[gg] = __ldcg(sl + C + g);
                   const float* og = sl + ml + g * kD + lane * kV;
                   if constexpr (kV == 4) {
                     const float4 v = __ldcg(reinterpret_cast<const float4*>(og));
@@ -697,7 +842,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
               }
 #pragma unroll
               for (int gg = 0; gg < 8; ++gg) {
-                if (g0 + gg < G) {
+                // multi-query: skip a share that saw no visible key of the column
+                if (g0 + gg < ncols && (!kMQ || mc[gg] != -INFINITY)) {
                   const float mn = fmaxf(Mg[gg], mc[gg]);
                   const float a = fast_exp2(Mg[gg] - mn);  // 0 for the first contributor
                   const float w = fast_exp2(mc[gg] - mn) * lc[gg];
@@ -711,11 +857,12 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 #pragma unroll
             for (int gg = 0; gg < 8; ++gg) {
               const int g = g0 + gg;
-              if (g < G) {
+              if (g < ncols) {
                 const float inv = Lg[gg] > 0.0f ? 1.0f / Lg[gg] : 0.0f;
+                const long long row = out_row(g);
 #pragma unroll
                 for (int e = 0; e < kV; ++e)
-                  store_out<kOutBF16>(p.out, (head_row0 + g) * kD + lane * kV + e, acc[gg][e] * inv);
+                  store_out<kOutBF16>(p.out, row * kD + lane * kV + e, acc[gg][e] * inv);
               }
             }
           }
@@ -726,14 +873,14 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
           locate(g0);
         } else {
           j = 0;
-          if (++h == Hkv) {
-            h = 0;
+          if (++pr == Hkv * ntile) {
+            pr = 0;
             do {
               ++s;
             } while (cum[s + 1] == cum[s]);
-            nb = (cum[s + 1] - cum[s]) / Hkv;
-            ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false);
+            enter_seq();
           }
+          set_pair();
         }
         begin_pair();
       }

@@ -19,6 +19,14 @@ Workloads (shapes of the Llama families the pages discuss; values N(0, 1)):
                   log-uniform[128, 8192], INT8 or FP8-e4m3 codes with fp32
                   per-(token, head) scales, or uint8 codes with a scale and
                   a uint8 zero point per (token, head).
+
+Multi-query workloads (several new tokens per sequence; context includes
+them):
+
+* ``spec_verify``      Llama-3-8B heads, batch 64, context U[512, 4096],
+                       4 new tokens per sequence (verifying 4 drafted tokens).
+* ``chunked_prefill``  Llama-3-8B heads, batch 8, context U[1024, 4096], the
+                       last 512 tokens new (one prefill chunk per sequence).
 """
 import math
 
@@ -37,6 +45,10 @@ WORKLOADS = {
                           prefix=2048, pool=("need", 1.1), seed=1003),
     "quant_mha": dict(batch=256, hq=32, hkv=32, d=128, dtype="bf16", ctx=("loguniform", 128, 8192),
                       pool=("need", 1.1), cache=("int8", "fp8", "u8asym"), seed=1004),
+    "spec_verify": dict(batch=64, hq=32, hkv=8, d=128, dtype="bf16", ctx=("uniform", 512, 4096),
+                        q_len=4, pool=("need", 1.1), seed=1005),
+    "chunked_prefill": dict(batch=8, hq=32, hkv=8, d=128, dtype="bf16", ctx=("uniform", 1024, 4096),
+                            q_len=512, pool=("need", 1.1), seed=1006),
 }
 
 TORCH_DTYPES = {"f16": torch.float16, "bf16": torch.bfloat16}
@@ -257,3 +269,46 @@ def device_decode_case(name, device, seed=None, batch=None, cache_kind=None, ctx
                 out[key] = torch.randint(96, 161, (nb, hkv, BLOCK_SIZE), generator=dg, device=device,
                                          dtype=torch.int64).to(torch.uint8)
     return out
+
+
+def multi_query_case(name, seed=None, batch=None, ctx_override=None, q_lens=None, cache_kind=None,
+                     num_blocks=None, **shape):
+    """A random multi-query problem on the CPU: ``decode_case`` plus
+    query_start_loc [B + 1] int32 and q [T, Hq, D] packed by sequence.  The
+    new-token counts are the workload's q_len (clamped to each context) unless
+    ``q_lens`` gives them."""
+    case = decode_case(name, seed=seed, batch=batch, ctx_override=ctx_override, cache_kind=cache_kind,
+                       num_blocks=num_blocks, **shape)
+    spec = WORKLOADS[name]
+    ctx = case["context_lens"]
+    if q_lens is None:
+        n = torch.clamp(torch.full_like(ctx, spec.get("q_len", 1)), max=ctx)
+    else:
+        n = torch.as_tensor(q_lens, dtype=torch.int32).reshape(-1)
+    qsl = torch.zeros(ctx.numel() + 1, dtype=torch.int32)
+    qsl[1:] = torch.cumsum(n, 0)
+    gen = generator((spec["seed"] if seed is None else seed) + 31)
+    case["query_start_loc"] = qsl
+    case["max_query_len"] = int(n.max()) if n.numel() else 0
+    case["q"] = randn((int(qsl[-1]), case["hq"], case["d"]), gen, shape.get("dtype", spec["dtype"]))
+    return case
+
+
+def device_multi_query_case(name, device, seed=None, batch=None, cache_kind=None):
+    """``device_decode_case`` plus query_start_loc (on the device, and a CPU
+    copy) and q [T, Hq, D] drawn on the device; each sequence gets the
+    workload's q_len new tokens (clamped to its context)."""
+    case = device_decode_case(name, device, seed=seed, batch=batch, cache_kind=cache_kind)
+    spec = WORKLOADS[name]
+    ctx = case["context_lens_cpu"]
+    n = torch.clamp(torch.full_like(ctx, spec.get("q_len", 1)), max=ctx)
+    qsl = torch.zeros(ctx.numel() + 1, dtype=torch.int32)
+    qsl[1:] = torch.cumsum(n, 0)
+    dg = torch.Generator(device=device)
+    dg.manual_seed((spec["seed"] if seed is None else seed) + 104729)
+    case["query_start_loc_cpu"] = qsl
+    case["query_start_loc"] = qsl.to(device)
+    case["max_query_len"] = int(n.max()) if n.numel() else 0
+    case["q"] = torch.randn((int(qsl[-1]), case["hq"], case["d"]), generator=dg, device=device,
+                            dtype=TORCH_DTYPES[spec["dtype"]])
+    return case

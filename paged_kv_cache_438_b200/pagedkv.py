@@ -27,7 +27,8 @@ DEV_BAD_SLOT, DEV_BAD_BLOCK, DEV_BAD_CONTEXT, DEV_TIMEOUT, DEV_BAD_PAIR = 1, 2, 
 
 EXPORTS = [
     "pkv_last_error", "pkv_version", "pkv_kv_cache_write", "pkv_decode_plan", "pkv_decode_workspace_size",
-    "pkv_paged_attention_decode", "pkv_paged_attention_decode_noalloc", "pkv_copy_blocks", "pkv_device_status", "pkv_set_validation",
+    "pkv_paged_attention_decode", "pkv_paged_attention_decode_noalloc", "pkv_multi_query_plan",
+    "pkv_paged_attention_multi_query", "pkv_copy_blocks", "pkv_device_status", "pkv_set_validation",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_fork", "pkv_seq_append",
     "pkv_batch_append", "pkv_batch_tables", "pkv_seq_free", "pkv_seq_block_table", "pkv_seq_len",
     "pkv_block_refcount", "pkv_alloc_stats",
@@ -65,6 +66,10 @@ def _signatures(lib):
                                         _F, _I, _I, _I, _P, _SZ, _P], _I),
         "pkv_paged_attention_decode_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
                                                 _I, _I, _F, _I, _I, _I, _P], _I),
+        "pkv_multi_query_plan": ([_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
+                                  ctypes.POINTER(_SZ)], _I),
+        "pkv_paged_attention_multi_query": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                             _I, _I, _I, _I, _F, _I, _I, _I, _P, _SZ, _P], _I),
         "pkv_copy_blocks": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P], _I),
         "pkv_device_status": ([ctypes.POINTER(ctypes.c_uint), _I], _I),
         "pkv_set_validation": ([_I], _I),
@@ -273,6 +278,57 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero), _ptr(v_zero),
         _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], max_context_len,
         float(scale), dtype_code(q), ct, partition_tokens, _ptr(workspace), ws_len, _stream(stream)))
+    return out
+
+
+def multi_query_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, max_query_len, cache_dtype,
+                     partition_tokens=0):
+    """(num_streams, tokens_per_stream_bound, workspace_bytes) of a
+    multi-query call (see decode_plan)."""
+    nst, ptok, ws = _I(0), _I(0), _SZ(0)
+    ct = cache_dtype if isinstance(cache_dtype, int) else dtype_code(cache_dtype)
+    _check(lib().pkv_multi_query_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len,
+                                      max_query_len, ct, partition_tokens, ctypes.byref(nst), ctypes.byref(ptok),
+                                      ctypes.byref(ws)))
+    return nst.value, ptok.value, ws.value
+
+
+def paged_attention_multi_query(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
+                                max_query_len, max_context_len, k_scale=None, v_scale=None, k_zero=None,
+                                v_zero=None, out=None, workspace=None, partition_tokens=0, stream=None):
+    """Several new tokens per sequence (chunked prefill, speculative verify):
+    q [T, Hq, D] packed by sequence with query_start_loc [B + 1] int32; the
+    n_s new tokens of sequence s are the last n_s of its context_lens[s]
+    tokens and attend causally.  max_query_len and max_context_len are
+    host-side bounds.  Returns out [T, Hq, D] in q's dtype."""
+    dev = q.device
+    for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
+        _need(t, n, device=dev)
+    _need(block_tables, "block_tables", device=dev, dtype=torch.int32)
+    _need(context_lens, "context_lens", device=dev, dtype=torch.int32)
+    _need(query_start_loc, "query_start_loc", device=dev, dtype=torch.int32)
+    if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
+        raise ValueError("q must be [T, Hq, D]; caches [NB, Hkv, 16, D]")
+    T, hq, d = q.shape
+    nb, hkv, bs, dk = k_cache.shape
+    B = context_lens.numel()
+    if dk != d or block_tables.dim() != 2 or block_tables.shape[0] != B or query_start_loc.numel() != B + 1:
+        raise ValueError("shape mismatch")
+    ct = cache_code(k_cache, k_zero)
+    _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _need(out, "out", device=dev, dtype=q.dtype)
+    nstreams, _, ws_bytes = multi_query_plan(B, hq, hkv, d, max_context_len, max_query_len, ct, partition_tokens)
+    if nstreams > 1 and workspace is None:
+        workspace = _cached_workspace(dev, stream, ws_bytes)
+    ws_len = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(lib().pkv_paged_attention_multi_query(
+        _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero), _ptr(v_zero),
+        _ptr(block_tables), _ptr(context_lens), _ptr(query_start_loc), B, T, int(max_query_len), hq, hkv, d, bs, nb,
+        block_tables.shape[1], int(max_context_len), float(scale), dtype_code(q), ct, partition_tokens,
+        _ptr(workspace), ws_len, _stream(stream)))
     return out
 
 

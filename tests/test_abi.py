@@ -122,3 +122,37 @@ def test_copy_rejections(lib):
     _err(lib.pkv_copy_blocks(n, n, None, None, None, None, n, 0, 2, 128, 16, 10, P.PKV_BF16, None), P.PKV_OK)
     _err(lib.pkv_copy_blocks(n, n, n, n, None, None, n, 3, 2, 128, 16, 10, P.PKV_U8ASYM, None),
          P.PKV_ERR_INVALID_ARG)
+
+
+def _mq(lib, **kw):
+    n = ctypes.c_void_p(256)
+    a = dict(out=n, q=n, kc=n, vc=n, ks=None, vs=None, kz=None, vz=None, bt=n, cl=n, qsl=n, B=2, T=8, mq=4, hq=8,
+             hkv=2, d=128, bs=16, nb=100, mb=4, maxc=64, scale=0.1, qd=P.PKV_BF16, cd=P.PKV_BF16, pt=0, ws=None,
+             wsb=0)
+    a.update(kw)
+    return lib.pkv_paged_attention_multi_query(a["out"], a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["kz"],
+                                               a["vz"], a["bt"], a["cl"], a["qsl"], a["B"], a["T"], a["mq"],
+                                               a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["mb"], a["maxc"],
+                                               a["scale"], a["qd"], a["cd"], a["pt"], a["ws"], a["wsb"], None)
+
+
+def test_multi_query_host_rejections(lib):
+    _err(_mq(lib, qsl=None), P.PKV_ERR_INVALID_ARG)               # no query_start_loc
+    _err(_mq(lib, T=-1), P.PKV_ERR_INVALID_ARG)
+    _err(_mq(lib, hq=7), P.PKV_ERR_INVALID_ARG)
+    _err(_mq(lib, d=96), P.PKV_ERR_UNSUPPORTED)
+    _err(_mq(lib, pt=16), P.PKV_ERR_INVALID_ARG)                  # split plan needs a workspace
+    assert b"workspace" in lib.pkv_last_error()
+    _err(_mq(lib, T=0), P.PKV_OK)                                # nothing to do
+    _err(_mq(lib, mq=0), P.PKV_OK)
+
+
+def test_multi_query_plan_tiles(lib):
+    # 4 new tokens x G 4 = 16 columns: one tile per KV head, the decode-style plan
+    nw, per, ws = P.multi_query_plan(64, 32, 8, 128, 4096, 4, P.PKV_BF16)
+    nwd, _, _ = P.decode_plan(64, 32, 8, 128, 4096, P.PKV_BF16)
+    assert nw == nwd
+    # 512 new tokens x G 4 = 2048 columns = 128 tiles: one stream per (sequence, head, tile)
+    nw, per, ws = P.multi_query_plan(8, 32, 8, 128, 4096, 512, P.PKV_BF16)
+    assert nw == 8 * 8 * 128 and per == 4096
+    assert ws >= 8 * 8 * 128 * 8 + 2 * nw * (32 + 16 * 128) * 4

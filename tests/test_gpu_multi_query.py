@@ -1,0 +1,170 @@
+"""GPU parity of multi-query paged attention (several new tokens per
+sequence: chunked prefill, speculative verification) against the fp64
+oracle, through the C ABI.
+
+Bars as for decode: max-abs 2e-2 and mean-rel 1e-2 for fp16 / bf16 caches,
+the same against the oracle on the stored codes for 8-bit caches.  With one
+new token per sequence the result must equal the decode entry point's bit
+for bit (same arithmetic in the same order).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as OA
+from paged_kv_cache_438_b200 import inputs as I
+from paged_kv_cache_438_b200 import pagedkv as P
+from test_gpu_parity import DEV, check_attn, cache_values, cpu_or_none, gpu_case, np64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    from paged_kv_cache_438_b200 import build
+    build.build()
+    P.lib()
+    P.device_status(clear=True)
+    yield
+    assert P.device_status(clear=True) == 0, "a kernel raised a device status bit"
+
+
+def run_mq(g, partition_tokens=0, max_query_len=None):
+    out = P.paged_attention_multi_query(
+        g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"], g["query_start_loc"], g["scale"],
+        max_query_len=g["max_query_len"] if max_query_len is None else max_query_len,
+        max_context_len=int(g["context_lens"].max()), k_scale=g.get("k_scale"), v_scale=g.get("v_scale"),
+        k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), partition_tokens=partition_tokens)
+    torch.cuda.synchronize()
+    assert P.device_status(clear=True) == 0
+    return out
+
+
+def oracle_mq(case, seqs=None):
+    """Oracle rows for all sequences, or only for ``seqs`` (others zero)."""
+    kind = case["cache_kind"]
+    qsl = case["query_start_loc"].numpy()
+    ctx = case["context_lens"].numpy()
+    bt = case["block_tables"].numpy()
+    if seqs is not None:
+        keep = np.zeros(len(ctx), bool)
+        keep[list(seqs)] = True
+        ctx = np.where(keep, ctx, 0)
+        n = np.where(keep, np.diff(qsl), 0)
+        q = np64(case["q"])
+        sub_qsl = np.concatenate([[0], np.cumsum(n)])
+        rows = np.concatenate([np.arange(qsl[s], qsl[s + 1]) for s in range(len(n)) if keep[s]] or [[]]).astype(int)
+        sub = OA.paged_multi_query_attention(q[rows], cache_values(case["k_cache"], kind),
+                                             cache_values(case["v_cache"], kind), bt, ctx, sub_qsl, case["scale"],
+                                             cpu_or_none(case, "k_scale"), cpu_or_none(case, "v_scale"),
+                                             cpu_or_none(case, "k_zero"), cpu_or_none(case, "v_zero"))
+        return rows, sub
+    return OA.paged_multi_query_attention(np64(case["q"]), cache_values(case["k_cache"], kind),
+                                          cache_values(case["v_cache"], kind), bt, ctx, qsl, case["scale"],
+                                          cpu_or_none(case, "k_scale"), cpu_or_none(case, "v_scale"),
+                                          cpu_or_none(case, "k_zero"), cpu_or_none(case, "v_zero"))
+
+
+CTX = [1, 15, 16, 17, 40, 257, 1000, 33, 0, 300]
+NQ = [1, 15, 3, 17, 40, 5, 24, 1, 0, 9]
+
+
+@pytest.mark.parametrize("dtype", ["f16", "bf16"])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("group", [1, 4, 8, 16])
+@pytest.mark.parametrize("ptok", [0, 16])
+def test_multi_query_sweep_16bit(dtype, d, group, ptok):
+    hkv = 2
+    case = I.multi_query_case("spec_verify", seed=d * 10 + group, ctx_override=CTX, q_lens=NQ, hq=hkv * group,
+                              hkv=hkv, d=d, dtype=dtype)
+    got = np64(run_mq(gpu_case(case), partition_tokens=ptok))
+    check_attn(got, oracle_mq(case))
+
+
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym"])
+@pytest.mark.parametrize("group", [1, 4])
+def test_multi_query_quantised(kind, group):
+    hkv = 4
+    case = I.multi_query_case("spec_verify", seed=group + 70, ctx_override=CTX, q_lens=NQ, hq=hkv * group, hkv=hkv,
+                              d=128, cache_kind=kind)
+    check_attn(np64(run_mq(gpu_case(case))), oracle_mq(case))
+
+
+@pytest.mark.parametrize("group", [4, 16])
+def test_one_new_token_equals_decode_bitwise(group):
+    hkv = 2
+    ctx = [1, 17, 300, 1000, 0, 64]
+    case = I.multi_query_case("spec_verify", seed=5, ctx_override=ctx, q_lens=[min(c, 1) for c in ctx],
+                              hq=hkv * group, hkv=hkv, d=128)
+    g = gpu_case(case)
+    mq = run_mq(g)
+    # decode reads one query row per sequence: scatter the packed rows
+    qd = torch.zeros((len(ctx), hkv * group, 128), dtype=g["q"].dtype, device=DEV)
+    has = torch.tensor([c > 0 for c in ctx], device=DEV)
+    qd[has] = g["q"]
+    dec = P.paged_attention_decode(qd, g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"],
+                                   g["scale"], max_context_len=max(ctx))
+    torch.cuda.synchronize()
+    assert torch.equal(mq, dec[has])
+
+
+def test_chunking_does_not_change_results():
+    """Twelve new tokens in one pass against three passes of 5, 4 and 3
+    tokens over the context up to each pass's last token."""
+    hkv, group = 2, 4
+    ctx, n = 500, 12
+    case = I.multi_query_case("spec_verify", seed=8, ctx_override=[ctx], q_lens=[n], hq=hkv * group, hkv=hkv, d=128)
+    g = gpu_case(case)
+    one = np64(run_mq(g))
+    parts, start = [], 0
+    for m in (5, 4, 3):
+        c = ctx - n + start + m
+        sub = dict(g)
+        sub["q"] = g["q"][start:start + m]
+        sub["context_lens"] = torch.tensor([c], dtype=torch.int32, device=DEV)
+        sub["query_start_loc"] = torch.tensor([0, m], dtype=torch.int32, device=DEV)
+        sub["max_query_len"] = m
+        parts.append(np64(run_mq(sub)))
+        start += m
+    check_attn(np.concatenate(parts), one, atol=4e-3, meanrel=1e-3)
+
+
+@pytest.mark.parametrize("name,nseq", [("spec_verify", 6), ("chunked_prefill", 2)])
+def test_multi_query_full_workload_sampled(name, nseq):
+    g = I.device_multi_query_case(name, DEV)
+    out = P.paged_attention_multi_query(g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"],
+                                        g["query_start_loc"], g["scale"], max_query_len=g["max_query_len"],
+                                        max_context_len=int(g["context_lens_cpu"].max()))
+    torch.cuda.synchronize()
+    assert P.device_status(clear=True) == 0
+    assert torch.isfinite(out.float()).all()
+    rng = np.random.default_rng(len(name))
+    seqs = sorted(rng.choice(g["batch"], size=nseq, replace=False).tolist())
+    # oracle on the sampled sequences only: move just their blocks to the host
+    qsl = g["query_start_loc_cpu"]
+    for s in seqs:
+        ctx = int(g["context_lens_cpu"][s])
+        nblk = (ctx + 15) // 16
+        blocks = g["block_tables_cpu"][s, :nblk].long()
+        kc = g["k_cache"][blocks.to(DEV)].cpu()
+        vc = g["v_cache"][blocks.to(DEV)].cpu()
+        rows = np.arange(int(qsl[s]), int(qsl[s + 1]))
+        ref = OA.paged_multi_query_attention(np64(g["q"][rows[0]:rows[-1] + 1]), np64(kc), np64(vc),
+                                             np.arange(nblk)[None], [ctx], [0, len(rows)], g["scale"])
+        check_attn(np64(out[rows[0]:rows[-1] + 1]), ref)
+
+
+def test_validation_rejects_inconsistent_query_runs():
+    case = I.multi_query_case("spec_verify", seed=3, ctx_override=[20, 40], q_lens=[4, 4], hq=8, hkv=2, d=64)
+    g = gpu_case(case)
+    P.set_validation(True)
+    try:
+        bad = dict(g)
+        bad["query_start_loc"] = torch.tensor([0, 25, 8], dtype=torch.int32, device=DEV)
+        with pytest.raises(P.PagedKVError, match="new tokens"):
+            run_mq(bad, max_query_len=30)
+        bad["query_start_loc"] = torch.tensor([0, 4, 7], dtype=torch.int32, device=DEV)
+        with pytest.raises(P.PagedKVError, match="num_q_tokens"):
+            run_mq(bad)
+    finally:
+        P.set_validation(False)

@@ -255,3 +255,79 @@ def test_asymmetric_gather_subtracts_zero_point_then_scales():
     q = rng.standard_normal((1, hq, d))
     paged = A.paged_decode_attention(q, kc, kc, np.array([perm]), [ctx], 0.5, ks, ks, k_zero=kz, v_zero=kz)
     np.testing.assert_allclose(paged[0], _brute(q[0], vals, vals, 0.5), rtol=0, atol=1e-12)
+
+
+# ---------------------------------------------------------- multi-query --
+
+def _mq_case(rng, ctxs, nq, hq, hkv, d, spare=3):
+    nblk = [(c + 15) // 16 for c in ctxs]
+    nb = sum(nblk) + spare
+    perm = rng.permutation(nb)
+    bt = np.zeros((len(ctxs), max(nblk)), np.int64)
+    cur = 0
+    for s, k in enumerate(nblk):
+        bt[s, :k] = perm[cur:cur + k]
+        cur += k
+    kc = rng.standard_normal((nb, hkv, 16, d))
+    vc = rng.standard_normal((nb, hkv, 16, d))
+    qsl = np.concatenate([[0], np.cumsum(nq)])
+    q = rng.standard_normal((int(qsl[-1]), hq, d))
+    return q, kc, vc, bt, qsl
+
+
+def test_multi_query_with_one_token_is_decode_bitwise():
+    rng = np.random.default_rng(21)
+    ctxs = [1, 17, 40, 33]
+    q, kc, vc, bt, qsl = _mq_case(rng, ctxs, [1, 1, 1, 1], 8, 2, 8)
+    mq = A.paged_multi_query_attention(q, kc, vc, bt, ctxs, qsl, 0.37)
+    dec = A.paged_decode_attention(q, kc, vc, bt, ctxs, 0.37)
+    assert np.array_equal(mq, dec)
+
+
+def test_multi_query_full_prefill_matches_sdpa_causal():
+    # all of a sequence's tokens new at once: plain causal self-attention
+    rng = np.random.default_rng(22)
+    ctx, hq, hkv, d = 45, 8, 2, 16
+    q, kc, vc, bt, qsl = _mq_case(rng, [ctx], [ctx], hq, hkv, d)
+    got = A.paged_multi_query_attention(q, kc, vc, bt, [ctx], qsl, 0.25)
+    K = torch.from_numpy(np.stack([kc[bt[0, j // 16], :, j % 16] for j in range(ctx)]))   # [ctx, hkv, d]
+    V = torch.from_numpy(np.stack([vc[bt[0, j // 16], :, j % 16] for j in range(ctx)]))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q).transpose(0, 1), K.transpose(0, 1), V.transpose(0, 1), is_causal=True, scale=0.25,
+        enable_gqa=True).transpose(0, 1).numpy()
+    np.testing.assert_allclose(got, ref, rtol=0, atol=1e-12)
+
+
+def test_multi_query_is_independent_of_chunking():
+    # the output for a token does not depend on how the new tokens are split
+    # into passes: one pass of 12 tokens == three passes of 5, 4 and 3 tokens
+    # (each pass seeing the context up to its own last token), == 12 decodes
+    rng = np.random.default_rng(23)
+    ctx, n, hq, hkv, d = 70, 12, 4, 4, 8
+    q, kc, vc, bt, _ = _mq_case(rng, [ctx], [n], hq, hkv, d)
+    one = A.paged_multi_query_attention(q, kc, vc, bt, [ctx], [0, n], 0.5)
+    parts, start = [], 0
+    for m in (5, 4, 3):
+        c = ctx - n + start + m
+        parts.append(A.paged_multi_query_attention(q[start:start + m], kc, vc, bt, [c], [0, m], 0.5))
+        start += m
+    assert np.array_equal(np.concatenate(parts), one)
+    for t in range(n):
+        dec = A.paged_decode_attention(q[t:t + 1], kc, vc, bt, [ctx - n + t + 1], 0.5)[0]
+        assert np.array_equal(dec, one[t])
+
+
+def test_multi_query_brute_force_and_empty_sequences():
+    rng = np.random.default_rng(24)
+    ctxs = [20, 0, 9, 33]
+    nq = [3, 0, 9, 2]
+    hq, hkv, d = 4, 2, 4
+    q, kc, vc, bt, qsl = _mq_case(rng, [max(c, 1) for c in ctxs], nq, hq, hkv, d)
+    got = A.paged_multi_query_attention(q, kc, vc, bt, ctxs, qsl, 0.6)
+    for s, (c, n) in enumerate(zip(ctxs, nq)):
+        K_log = [[kc[bt[s, j // 16], h, j % 16] for h in range(hkv)] for j in range(c)]
+        V_log = [[vc[bt[s, j // 16], h, j % 16] for h in range(hkv)] for j in range(c)]
+        for t in range(n):
+            vis = c - n + t + 1
+            ref = _brute(q[qsl[s] + t], K_log[:vis], V_log[:vis], 0.6)
+            np.testing.assert_allclose(got[qsl[s] + t], ref, rtol=0, atol=1e-12)
