@@ -36,6 +36,7 @@ from paged_kv_cache_438_b200 import inputs as I  # noqa: E402
 METRIC = "paged decode attention: effective KV-read GB/s (% of HBM peak), seq-steps/s"
 NOMINAL_HBM_GBS = 8000.0
 FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
 L2_BYTES = 126 * 2 ** 20
 
 WORKLOAD_TEXT = {
@@ -46,6 +47,10 @@ WORKLOAD_TEXT = {
     "prefix_shared": "prefix-shared: Llama-3-8B heads, 128 seqs sharing one 2048-token prefix + suffix U[64,1024], bf16",
     "quant_mha": "quantised KV: Llama-2-7B MHA 32/32 heads, head_dim 128, batch 256, context log-uniform[128,8192]",
     "tiny": "tiny: batch 4, 8 q / 2 KV heads, head_dim 64, context U[1,256], fp16",
+    "spec_verify": "speculative verify: Llama-3-8B heads (32 q / 8 KV), head_dim 128, batch 64, context U[512,4096] "
+                   "incl. 4 new tokens per sequence, causal among them, bf16",
+    "chunked_prefill": "chunked prefill: Llama-3-8B heads (32 q / 8 KV), head_dim 128, batch 8, context "
+                       "U[1024,4096] whose last 512 tokens are one new chunk, causal, bf16",
 }
 
 
@@ -72,6 +77,18 @@ def peaks():
             d = json.load(f)
         return float(d["hbm_gbs"]), "measured"
     return FALLBACK_HBM_GBS, "fallback"
+
+
+def tensor_peak():
+    """Dense bf16 tensor TFLOP/s (burst) of MEASURED_PEAKS.json, else the
+    fallback figure."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops" in d:
+            return float(d["bf16_tflops"]), "measured"
+    return FALLBACK_BF16_TFLOPS, "fallback"
 
 
 def kernel_source_hash():
@@ -289,6 +306,115 @@ class DecodeWorkload:
                                       self.v_scale, max_context_len=maxc, out=out, workspace=ws,
                                       k_zero=self.k_zero, v_zero=self.v_zero)
 
+    # shapes and plan of one step (the multi-query workload overrides these)
+    q_rows = property(lambda self: self.B)
+    mq = False
+
+    def plan(self, maxc):
+        return self.P.decode_plan(self.B, self.hq, self.hkv, self.d, maxc, self.k_cache.dtype)
+
+    def flops(self, cl):
+        """Tensor-core FLOPs of the step's attention (2 per multiply-add, QK
+        and PV) for each (query, key) pair a query head sees."""
+        return 4 * self.d * self.hq * int(cl.sum())
+
+
+class MultiQueryWorkload(DecodeWorkload):
+    """Sequences whose last n tokens are new (speculative verify, one prefill
+    chunk).  The cache holds every sequence's full context; a step writes the
+    n new K/V rows of every sequence into their slots and runs multi-query
+    attention over the whole context.  The state does not advance between
+    steps (each step re-scores the same new tokens), so every step does the
+    same work."""
+
+    mq = True
+
+    def __init__(self, name, cache, device, seed_offset=0, batch=None):
+        from paged_kv_cache_438_b200 import pagedkv as P
+        self.P = P
+        self.name = name
+        spec = dict(I.WORKLOADS[name])
+        if batch is not None:
+            spec["batch"] = batch
+        self.spec = spec
+        self.dev = device
+        seed = spec["seed"] + seed_offset
+        gen = I.generator(seed)
+        self.B, self.hq, self.hkv, self.d = spec["batch"], spec["hq"], spec["hkv"], spec["d"]
+        self.dtype = I.TORCH_DTYPES[spec["dtype"]]
+        self.cache_kind = cache
+        ctx = I.context_lens(spec, gen)
+        self.n = torch.clamp(torch.full_like(ctx, spec["q_len"]), max=ctx)
+        need = sum(I.blocks_for(c) for c in ctx.tolist())
+        nb = I.pool_size(spec, need)
+        self.nb = nb
+        order = torch.randperm(nb, generator=gen).tolist()
+        self.alloc = P.BlockAllocator(nb, initial_free_order=order)
+        cdt = {None: self.dtype, "int8": torch.int8, "fp8": torch.uint8, "u8asym": torch.uint8}[cache]
+        self.k_cache = torch.empty((nb, self.hkv, 16, self.d), dtype=cdt, device=device)
+        self.v_cache = torch.empty_like(self.k_cache)
+        self.k_scale = self.v_scale = self.k_zero = self.v_zero = None
+        if cache:
+            self.k_scale = torch.zeros((nb, self.hkv, 16), dtype=torch.float32, device=device)
+            self.v_scale = torch.zeros_like(self.k_scale)
+        if cache == "u8asym":
+            self.k_zero = torch.zeros((nb, self.hkv, 16), dtype=torch.uint8, device=device)
+            self.v_zero = torch.zeros_like(self.k_zero)
+        self.elt = 1 if cache else 2
+        self.per_tok = kv_bytes_per_token(self.hkv, self.d, cache)
+        self.dg = torch.Generator(device=device)
+        self.dg.manual_seed(seed + 17)
+        self.ids = list(range(self.B))
+        new_slots = []
+        for s in range(self.B):
+            self.alloc.add(s)
+            slots, _ = self.alloc.append(s, int(ctx[s] - self.n[s]))
+            self._fill(slots)
+            slots, _ = self.alloc.append(s, int(self.n[s]))
+            self._fill(slots)
+            new_slots.append(slots)
+        self.new_slots = torch.cat(new_slots)
+        self.max_blocks = max(I.blocks_for(c) for c in ctx.tolist())
+        self.qsl = torch.zeros(self.B + 1, dtype=torch.int32)
+        self.qsl[1:] = torch.cumsum(self.n, 0)
+        self.max_q = int(self.n.max())
+        self.qsl_dev = self.qsl.to(device)
+        torch.cuda.synchronize(device)
+        self.scale = 1.0 / math.sqrt(self.d)
+
+    q_rows = property(lambda self: int(self.qsl[-1]))
+
+    def host_step(self):
+        bt, cl = self.alloc.batch_tables(self.ids, self.max_blocks)
+        return self.new_slots, torch.empty((0, 2), dtype=torch.int32), bt, cl
+
+    def new_rows(self):
+        T = self.q_rows
+        q = torch.randn((T, self.hq, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
+        k = torch.randn((T, self.hkv, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
+        v = torch.randn((T, self.hkv, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
+        return q, k, v
+
+    def decode(self, q, bt, cl, maxc, out, ws):
+        self.P.paged_attention_multi_query(q, self.k_cache, self.v_cache, bt, cl, self.qsl_dev, self.scale,
+                                           max_query_len=self.max_q, max_context_len=maxc, k_scale=self.k_scale,
+                                           v_scale=self.v_scale, k_zero=self.k_zero, v_zero=self.v_zero, out=out,
+                                           workspace=ws)
+
+    def plan(self, maxc):
+        return self.P.multi_query_plan(self.B, self.hq, self.hkv, self.d, maxc, self.max_q, self.k_cache.dtype)
+
+    def flops(self, cl):
+        # new token t of n sees ctx - n + t + 1 keys
+        n = self.n.long()
+        seen = (cl.long() - n) * n + n * (n + 1) // 2
+        return 4 * self.d * self.hq * int(seen.sum())
+
+
+def make_workload(name, cache, device, seed_offset=0, batch=None):
+    cls = MultiQueryWorkload if "q_len" in I.WORKLOADS[name] else DecodeWorkload
+    return cls(name, cache, device, seed_offset=seed_offset, batch=batch)
+
 
 # ------------------------------------------------------------------ ours --
 
@@ -297,7 +423,7 @@ def run_ours(args, rank, world, device):
     from paged_kv_cache_438_b200 import pagedkv as P
     build.build()
     P.lib()
-    wl = DecodeWorkload(args.workload, args.cache, device, seed_offset=replica_seed_offset(rank), batch=args.batch)
+    wl = make_workload(args.workload, args.cache, device, seed_offset=replica_seed_offset(rank), batch=args.batch)
     K, W = args.steps, args.warmup
     # host allocator outputs of every step, staged in HBM before timing
     staged = []
@@ -306,11 +432,11 @@ def run_ours(args, rank, world, device):
         q, k, v = wl.new_rows()
         staged.append(dict(slots=slots.to(device), pairs=pairs.to(device) if pairs.numel() else None,
                            bt=bt.to(device), cl=cl.to(device), maxc=int(cl.max()), q=q, k=k, v=v,
-                           kv=wl.kv_bytes(cl)))
+                           kv=wl.kv_bytes(cl), flops=wl.flops(cl)))
     maxc_all = max(s["maxc"] for s in staged)
-    _, _, ws_bytes = P.decode_plan(wl.B, wl.hq, wl.hkv, wl.d, maxc_all, wl.k_cache.dtype)
+    _, _, ws_bytes = wl.plan(maxc_all)
     ws = P.new_workspace(device, ws_bytes)
-    out = torch.empty((wl.B, wl.hq, wl.d), dtype=wl.dtype, device=device)
+    out = torch.empty((wl.q_rows, wl.hq, wl.d), dtype=wl.dtype, device=device)
     kv_step = staged[0]["kv"]
     flush = kv_step < 4 * L2_BYTES
     scrub = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device) if flush else None
@@ -371,6 +497,7 @@ def run_ours(args, rank, world, device):
     timed_ms, kv_all, seqsteps_all = aggregate_ranks(timed_ms, kv_total, wl.B * K, world, device)
 
     res = dict(wl=wl, K=K, W=W, timed_ms=timed_ms, dec_ms=dec_ms, kv_all=kv_all, kv_rank=kv_total,
+               flops_call=staged[W]["flops"],
                seqsteps_all=seqsteps_all, launches=launches, clocks=clocks, flush=flush, kv_step=kv_step,
                maxc=maxc_all, staged=staged)
     if not args.no_e2e:
@@ -418,38 +545,49 @@ def run_e2e(wl, K, W, device, world):
     host-to-device, the kernels run, and the output is copied back and waited
     for."""
     P = wl.P
-    B, MB = wl.B, wl.max_blocks
-    pin = dict(q=torch.empty((B, wl.hq, wl.d), dtype=wl.dtype).pin_memory(),
-               k=torch.empty((B, wl.hkv, wl.d), dtype=wl.dtype).pin_memory(),
-               v=torch.empty((B, wl.hkv, wl.d), dtype=wl.dtype).pin_memory(),
-               out=torch.empty((B, wl.hq, wl.d), dtype=wl.dtype).pin_memory(),
-               slots=torch.empty(B, dtype=torch.int64).pin_memory(),
+    B, MB, T = wl.B, wl.max_blocks, wl.q_rows
+    pin = dict(q=torch.empty((T, wl.hq, wl.d), dtype=wl.dtype).pin_memory(),
+               k=torch.empty((T, wl.hkv, wl.d), dtype=wl.dtype).pin_memory(),
+               v=torch.empty((T, wl.hkv, wl.d), dtype=wl.dtype).pin_memory(),
+               out=torch.empty((T, wl.hq, wl.d), dtype=wl.dtype).pin_memory(),
+               slots=torch.empty(T, dtype=torch.int64).pin_memory(),
                pairs=torch.empty((B, 2), dtype=torch.int32).pin_memory(),
                bt=torch.empty((B, MB), dtype=torch.int32).pin_memory(),
                cl=torch.empty(B, dtype=torch.int32).pin_memory())
     dev = {k: torch.empty_like(v, device=device) for k, v in pin.items() if k != "out"}
-    out = torch.empty((B, wl.hq, wl.d), dtype=wl.dtype, device=device)
+    out = torch.empty((T, wl.hq, wl.d), dtype=wl.dtype, device=device)
     ids = torch.arange(B, dtype=torch.int64)
     g = I.generator(4242)
     for key in ("q", "k", "v"):
         pin[key].copy_(torch.randn(pin[key].shape, generator=g).to(wl.dtype))
-    _, _, wsb = P.decode_plan(B, wl.hq, wl.hkv, wl.d, MB * 16, wl.k_cache.dtype)
+    _, _, wsb = wl.plan(MB * 16)
     ws = P.new_workspace(device, wsb)
+    if wl.mq:
+        # the new tokens' slots are fixed; the query layout travels every step
+        pin["qsl"] = wl.qsl.clone().pin_memory()
+        dev["qsl"] = torch.empty_like(pin["qsl"], device=device)
+        pin["slots"].copy_(wl.new_slots)
     stream = torch.cuda.current_stream(device)
-    fixed = sum(pin[k].numel() * pin[k].element_size() for k in ("q", "k", "v", "slots", "bt", "cl"))
+    keys = ("q", "k", "v", "slots", "bt", "cl") + (("qsl",) if wl.mq else ())
+    fixed = sum(pin[k].numel() * pin[k].element_size() for k in keys)
     d2h = pin["out"].numel() * pin["out"].element_size()
 
     def one():
-        slots, pairs = wl.alloc.batch_append(ids, slots_out=pin["slots"], pairs_out=pin["pairs"])
+        if wl.mq:
+            pairs = pin["pairs"][:0]
+        else:
+            slots, pairs = wl.alloc.batch_append(ids, slots_out=pin["slots"], pairs_out=pin["pairs"])
         wl.alloc.batch_tables(ids, MB, out_tables=pin["bt"], out_lens=pin["cl"])
         npairs = pairs.shape[0]
-        for key in ("q", "k", "v", "slots", "bt", "cl"):
+        for key in keys:
             dev[key].copy_(pin[key], non_blocking=True)
         gp = None
         if npairs:
             gp = dev["pairs"][:npairs]
             gp.copy_(pin["pairs"][:npairs], non_blocking=True)
         maxc = int(pin["cl"].max())
+        if wl.mq:
+            wl.qsl_dev = dev["qsl"]
         wl.device_step(dev["q"], dev["k"], dev["v"], dev["slots"], gp, dev["bt"], dev["cl"], maxc, out, ws)
         pin["out"].copy_(out, non_blocking=True)
         stream.synchronize()
@@ -491,8 +629,12 @@ def oracle_sample(name, cache, budget_s=10.0, seed_offset=0):
     spent, kvb, seqs = 0.0, 0, 0
     for c in ctx:
         nblk = I.blocks_for(c)
-        case = I.decode_case(name, seed=int(gen.initial_seed()) + seqs, ctx_override=[c], cache_kind=cache,
-                             num_blocks=nblk)
+        if "q_len" in spec:
+            case = I.multi_query_case(name, seed=int(gen.initial_seed()) + seqs, ctx_override=[c],
+                                      q_lens=[min(spec["q_len"], c)], cache_kind=cache, num_blocks=nblk)
+        else:
+            case = I.decode_case(name, seed=int(gen.initial_seed()) + seqs, ctx_override=[c], cache_kind=cache,
+                                 num_blocks=nblk)
         kind = case["cache_kind"]
         if kind == "fp8":
             kc, vc = OQ.e4m3_decode(case["k_cache"].numpy()), OQ.e4m3_decode(case["v_cache"].numpy())
@@ -502,8 +644,14 @@ def oracle_sample(name, cache, budget_s=10.0, seed_offset=0):
         side = {key: case[key].numpy() for key in ("k_scale", "v_scale", "k_zero", "v_zero") if key in case}
         q = case["q"].to(torch.float64).numpy()
         t0 = time.perf_counter()
-        OA.paged_decode_attention(q, kc, vc, case["block_tables"].numpy(), [c], case["scale"], side.get("k_scale"),
-                                  side.get("v_scale"), k_zero=side.get("k_zero"), v_zero=side.get("v_zero"))
+        if "q_len" in spec:
+            OA.paged_multi_query_attention(q, kc, vc, case["block_tables"].numpy(), [c],
+                                           case["query_start_loc"].numpy(), case["scale"], side.get("k_scale"),
+                                           side.get("v_scale"), side.get("k_zero"), side.get("v_zero"))
+        else:
+            OA.paged_decode_attention(q, kc, vc, case["block_tables"].numpy(), [c], case["scale"],
+                                      side.get("k_scale"), side.get("v_scale"), k_zero=side.get("k_zero"),
+                                      v_zero=side.get("v_zero"))
         spent += time.perf_counter() - t0
         kvb += c * per_tok
         seqs += 1
@@ -578,13 +726,18 @@ def main():
     seqsteps = r["seqsteps_all"] / (r["timed_ms"] * 1e-3)
     # roofline of the decode call (decode kernel + reduce when split) on this rank
     dec_ms = r["dec_ms"] / r["K"]
-    nstreams, stream_tokens, ws_bytes = wl.P.decode_plan(wl.B, wl.hq, wl.hkv, wl.d, r["maxc"], wl.k_cache.dtype)
+    nstreams, stream_tokens, ws_bytes = wl.plan(r["maxc"])
     kv_call = r["kv_rank"] / r["K"]
     # q read + out written + the block-table entries the step reads
-    small = wl.B * wl.hq * wl.d * 2 * 2 + (kv_call // (wl.per_tok * 16)) * 4
+    small = wl.q_rows * wl.hq * wl.d * 2 * 2 + (kv_call // (wl.per_tok * 16)) * 4
     alg_bytes = kv_call + small
     achieved = alg_bytes / (dec_ms * 1e-3) / 1e9
     traffic = recorded_traffic(args.workload, args.cache, alg_bytes)
+    tflops_peak, tflops_kind = tensor_peak()
+    flops_call = r["flops_call"]
+    # the bound is whichever floor is higher: bytes at the copy bandwidth or
+    # FLOPs at the dense bf16 tensor rate
+    tensor_bound = flops_call / (tflops_peak * 1e12) > alg_bytes / (peak * 1e9)
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world, "steps": r["K"],
         "warmup": r["W"], "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
@@ -602,15 +755,25 @@ def main():
         "seq_steps_per_s": round(seqsteps, 1),
         "pct_of_hbm_measured": round(100 * value / (peak * world), 2),
         "pct_of_hbm_nominal_8tbs": round(100 * value / (NOMINAL_HBM_GBS * world), 2),
-        "roofline": {"kernel": "paged_decode_kernel (one launch per decode call)", "bound": "hbm",
-                     "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
-                     "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
-                     "timing": "decode-only launches of the timed steps' inputs, CUDA events on the launching stream",
-                     "traffic": traffic, "algorithmic_bytes_per_call": int(alg_bytes),
-                     "ms_per_call": round(dec_ms, 4)},
+        "roofline": ({"kernel": "paged_decode_kernel (one launch per decode call)", "bound": "hbm",
+                      "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
+                      "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy, burst)"}
+                     if not tensor_bound else
+                     {"kernel": "paged_decode_kernel, multi-query mode (one launch per call)", "bound": "tensor",
+                      "achieved": round(flops_call / (dec_ms * 1e-3) / 1e12, 2), "peak": tflops_peak,
+                      "unit": "TFLOP/s", "frac": round(flops_call / (dec_ms * 1e-3) / 1e12 / tflops_peak, 4),
+                      "peak_source": f"{tflops_kind} bf16_tflops (cuBLAS, burst)",
+                      "hbm_achieved_gbs": round(achieved, 1)}),
         "gpu_launches": r["launches"],
         "clocks": r["clocks"],
     }
+    line["roofline"].update({
+        "timing": "decode-only launches of the timed steps' inputs, CUDA events on the launching stream",
+        "traffic": traffic, "algorithmic_bytes_per_call": int(alg_bytes), "flops_per_call": int(flops_call),
+        "ms_per_call": round(dec_ms, 4)})
+    if wl.mq:
+        line["query_tokens_per_s"] = round(wl.q_rows * r["K"] * world / (r["timed_ms"] * 1e-3), 1)
+        line["config"]["new_tokens_per_sequence"] = wl.spec["q_len"]
     if "e2e" in r:
         line["e2e"] = r["e2e"]
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

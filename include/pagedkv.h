@@ -233,8 +233,10 @@ int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int he
  * max_query_len   : host-side bound of n_s (sizes the work list).
  * Everything else as for pkv_paged_attention_decode (with
  * pkv_multi_query_plan's workspace size).  Rows of new tokens beyond a
- * sequence's context (an invalid input) are written as zeros and raise
- * PKV_DEV_BAD_CONTEXT.  With every n_s = 1 the result equals decode.
+ * sequence's context or beyond max_query_len (invalid inputs) are written as
+ * zeros and raise PKV_DEV_BAD_CONTEXT; query_start_loc entries outside
+ * [0, num_q_tokens] are clamped to it.  With every n_s = 1 the result equals
+ * decode.
  */
 int pkv_paged_attention_multi_query(void* out, const void* q,
                                     const void* k_cache, const void* v_cache,

@@ -490,6 +490,7 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
   p.tile_cols = pl.tile_cols;
   p.max_tiles = pl.max_tiles;
   p.num_q_tokens = mq ? num_q_tokens : num_seqs;
+  p.max_query_len = mq ? max_query_len : 1;
   p.epoch = next_epoch();
   p.qk_scale_log2 = scale * 1.4426950408889634f;
   const bool q_bf16 = q_dtype == PKV_BF16;

@@ -119,6 +119,7 @@ struct DecodeParams {
   int tile_cols;     // multi-query: columns per tile (8 * kNT)
   int max_tiles;     // multi-query: tiles per KV head of the longest query run (1 for decode)
   int num_q_tokens;  // multi-query: rows of q and out
+  int max_query_len; // multi-query: host bound of new tokens per sequence (sizes the counters)
   unsigned long long epoch;  // this call's epoch, nonzero, < 2^40
   float qk_scale_log2;       // softmax scale * log2(e)
 };
@@ -180,31 +181,16 @@ __device__ __forceinline__ int blocks_of(const DecodeParams& p, int s, bool repo
 __device__ __forceinline__ void query_range(const DecodeParams& p, int s, int ctx, int& q0, int& q1, int& n,
                                             bool report);
 
-// New tokens of sequence s in multi-query mode (see query_range).
-__device__ __forceinline__ int new_tokens_of(const DecodeParams& p, int s, int ctx) {
-  int q0, q1, n;
-  query_range(p, s, ctx, q0, q1, n, false);
-  return n;
-}
-
-// Pairs per KV head of sequence s: 1 for decode, the column tiles of its new
-// tokens in multi-query mode.
-template <bool kMQ>
-__device__ __forceinline__ int tiles_of(const DecodeParams& p, int s, int ctx) {
-  if constexpr (kMQ) {
-    const int n = new_tokens_of(p, s, ctx);
-    return (n * p.group + p.tile_cols - 1) / p.tile_cols;
-  } else {
-    return 1;
-  }
-}
-
-// Work items of sequence s: blocks * Hkv * tiles.
+// Work items of sequence s: blocks * Hkv (decode), times the column tiles
+// of its new tokens in multi-query mode.
 template <bool kMQ>
 __device__ __forceinline__ int items_of(const DecodeParams& p, int s, bool report) {
   if constexpr (kMQ) {
     const int ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, report);
-    return ((ctx + 15) >> 4) * p.num_kv_heads * tiles_of<true>(p, s, ctx);
+    int q0, q1, n;
+    query_range(p, s, ctx, q0, q1, n, report);
+    const int tiles = (n * p.group + p.tile_cols - 1) / p.tile_cols;
+    return ((ctx + 15) >> 4) * p.num_kv_heads * tiles;
   } else {
     return blocks_of(p, s, report) * p.num_kv_heads;
   }
@@ -284,13 +270,14 @@ __device__ __forceinline__ int item_row(const DecodeParams& p, const int32_t* cu
 
 // Rows [q0, q0 + n) of q / out hold the new tokens of sequence s in
 // multi-query mode: query_start_loc clamped to [0, num_q_tokens] and n to
-// the context (an inconsistent entry raises a status bit when `report`).
+// the context and to max_query_len (an inconsistent entry raises a status
+// bit when `report`; rows [q0 + n, q1) are then written as zeros).
 __device__ __forceinline__ void query_range(const DecodeParams& p, int s, int ctx, int& q0, int& q1, int& n,
                                             bool report) {
   const int a = p.query_start_loc[s], b = p.query_start_loc[s + 1];
   q0 = min(max(a, 0), p.num_q_tokens);
   q1 = min(max(b, q0), p.num_q_tokens);
-  n = min(q1 - q0, ctx);
+  n = min(min(q1 - q0, ctx), p.max_query_len);
   if (report && (a != q0 || b != q1 || q1 - q0 != n)) raise_status(PKV_DEV_BAD_CONTEXT);
 }
 
