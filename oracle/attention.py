@@ -18,6 +18,10 @@ result, so the oracle is the plain definition written out:
    p = softmax(logits), out[s, i] = p @ V_s[:, h].
 
 A sequence with ctx = 0 yields a zero output row.
+
+Sliding window ("KV Cache 与 PagedAttention", §三个直接推论, the KV-saving
+table: keep only the most recent window): with window W > 0 a query at
+position P sees keys max(0, P - W + 1) .. P only (W = 0: no window).
 """
 import numpy as np
 
@@ -62,8 +66,13 @@ def contiguous_attention(q, K, V, scale):
     return out
 
 
+def _window_start(vis, window):
+    """First visible key of a query that sees keys < vis, under window W."""
+    return max(0, vis - window) if window > 0 else 0
+
+
 def paged_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scale,
-                           k_scale=None, v_scale=None, seqs=None, k_zero=None, v_zero=None):
+                           k_scale=None, v_scale=None, seqs=None, k_zero=None, v_zero=None, window=0):
     """Decode attention for every (or the listed) sequence of a batch.
 
     q: [B, Hq, D]; k_cache, v_cache: [NB, Hkv, bs, D] (values, or codes with
@@ -79,7 +88,8 @@ def paged_decode_attention(q, k_cache, v_cache, block_tables, context_lens, scal
         ctx = int(context_lens[s])
         K = gather_sequence(k_cache, block_tables[s], ctx, k_scale, k_zero)
         V = gather_sequence(v_cache, block_tables[s], ctx, v_scale, v_zero)
-        out[s] = contiguous_attention(q[s], K, V, scale)
+        lo = _window_start(ctx, window)
+        out[s] = contiguous_attention(q[s], K[lo:], V[lo:], scale)
     return out
 
 
@@ -121,7 +131,7 @@ def paged_decode_attention_heads(q, k_cache, v_cache, block_tables, context_lens
 
 
 def paged_multi_query_attention(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
-                                k_scale=None, v_scale=None, k_zero=None, v_zero=None):
+                                k_scale=None, v_scale=None, k_zero=None, v_zero=None, window=0):
     """Attention of several new tokens per sequence over the paged cache.
 
     Several query tokens of one sequence in one pass serve chunked prefill
@@ -153,5 +163,6 @@ def paged_multi_query_attention(q, k_cache, v_cache, block_tables, context_lens,
         V = gather_sequence(v_cache, block_tables[s], ctx, v_scale, v_zero)
         for t in range(n):
             vis = ctx - n + t + 1
-            out[qsl[s] + t] = contiguous_attention(q[qsl[s] + t], K[:vis], V[:vis], scale)
+            lo = _window_start(vis, window)
+            out[qsl[s] + t] = contiguous_attention(q[qsl[s] + t], K[lo:vis], V[lo:vis], scale)
     return out

@@ -331,3 +331,45 @@ def test_multi_query_brute_force_and_empty_sequences():
             vis = c - n + t + 1
             ref = _brute(q[qsl[s] + t], K_log[:vis], V_log[:vis], 0.6)
             np.testing.assert_allclose(got[qsl[s] + t], ref, rtol=0, atol=1e-12)
+
+
+# ------------------------------------------------------- sliding window --
+
+def test_window_covering_the_context_changes_nothing():
+    rng = np.random.default_rng(31)
+    ctxs = [5, 40, 17]
+    q, kc, vc, bt, qsl = _mq_case(rng, ctxs, [2, 7, 1], 4, 2, 8)
+    full = A.paged_multi_query_attention(q, kc, vc, bt, ctxs, qsl, 0.4)
+    assert np.array_equal(A.paged_multi_query_attention(q, kc, vc, bt, ctxs, qsl, 0.4, window=40), full)
+    dq = rng.standard_normal((3, 4, 8))
+    assert np.array_equal(A.paged_decode_attention(dq, kc, vc, bt, ctxs, 0.4, window=10 ** 6),
+                          A.paged_decode_attention(dq, kc, vc, bt, ctxs, 0.4))
+
+
+def test_window_of_one_returns_the_own_value_row():
+    rng = np.random.default_rng(32)
+    ctxs = [33, 18]
+    q, kc, vc, bt, qsl = _mq_case(rng, ctxs, [3, 18], 4, 2, 8)
+    got = A.paged_multi_query_attention(q, kc, vc, bt, ctxs, qsl, 0.4, window=1)
+    for s, (c, n) in enumerate(zip(ctxs, [3, 18])):
+        for t in range(n):
+            pos = c - n + t
+            v = vc[bt[s, pos // 16], :, pos % 16]                 # [hkv, d]
+            assert np.array_equal(got[qsl[s] + t], np.repeat(v, 2, axis=0))
+
+
+def test_window_brute_force():
+    rng = np.random.default_rng(33)
+    ctxs = [50, 9]
+    nq = [6, 9]
+    q, kc, vc, bt, qsl = _mq_case(rng, ctxs, nq, 4, 2, 4)
+    W = 13
+    got = A.paged_multi_query_attention(q, kc, vc, bt, ctxs, qsl, 0.7, window=W)
+    for s, (c, n) in enumerate(zip(ctxs, nq)):
+        K_log = [[kc[bt[s, j // 16], h, j % 16] for h in range(2)] for j in range(c)]
+        V_log = [[vc[bt[s, j // 16], h, j % 16] for h in range(2)] for j in range(c)]
+        for t in range(n):
+            pos = c - n + t
+            keep = [j for j in range(c) if pos - W < j <= pos]
+            ref = _brute(q[qsl[s] + t], [K_log[j] for j in keep], [V_log[j] for j in keep], 0.7)
+            np.testing.assert_allclose(got[qsl[s] + t], ref, rtol=0, atol=1e-12)
