@@ -174,6 +174,11 @@ int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, i
  * num_blocks     : physical blocks in the pool (entries of block_tables must
  *                  lie in [0, num_blocks)).
  * max_context_len: host-side upper bound of context_lens (sizes the grid).
+ * sliding_window : 0 = attend the whole context; W > 0 = a query at position
+ *                  P attends keys max(0, P - W + 1) .. P only ([P-WIKI]
+ *                  §三个直接推论: keep only the most recent window).  Blocks
+ *                  wholly before every query's window are not read, so their
+ *                  block-table entries may be stale (e.g. already freed).
  * num_q_heads / num_kv_heads = G must be an integer in [1, 16].
  * partition_tokens: as for pkv_decode_plan.
  * workspace      : device scratch of at least the planned bytes, 256-byte
@@ -198,7 +203,7 @@ int pkv_paged_attention_decode(void* out, const void* q,
                                const int32_t* block_tables, const int32_t* context_lens,
                                int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                int block_size, int num_blocks, int max_blocks_per_seq,
-                               int max_context_len, float scale, int q_dtype, int cache_dtype,
+                               int max_context_len, float scale, int sliding_window, int q_dtype, int cache_dtype,
                                int partition_tokens, void* workspace, size_t workspace_bytes,
                                void* stream);
 
@@ -247,7 +252,7 @@ int pkv_paged_attention_multi_query(void* out, const void* q,
                                     int num_q_tokens, int max_query_len,
                                     int num_q_heads, int num_kv_heads, int head_dim,
                                     int block_size, int num_blocks, int max_blocks_per_seq,
-                                    int max_context_len, float scale, int q_dtype, int cache_dtype,
+                                    int max_context_len, float scale, int sliding_window, int q_dtype, int cache_dtype,
                                     int partition_tokens, void* workspace, size_t workspace_bytes,
                                     void* stream);
 
@@ -284,7 +289,7 @@ int pkv_paged_attention_decode_noalloc(void* out, const void* q,
                                        const int32_t* block_tables, const int32_t* context_lens,
                                        int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                        int block_size, int num_blocks, int max_blocks_per_seq,
-                                       int max_context_len, float scale, int q_dtype, int cache_dtype,
+                                       int max_context_len, float scale, int sliding_window, int q_dtype, int cache_dtype,
                                        int partition_tokens, void* stream);
 
 /*

@@ -393,8 +393,9 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
                    const float* v_scale, const uint8_t* k_zero, const uint8_t* v_zero, const int32_t* block_tables,
                    const int32_t* context_lens, const int32_t* query_start_loc, int num_q_tokens, int max_query_len,
                    bool mq, int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                   int num_blocks, int max_blocks_per_seq, int max_context_len, float scale, int q_dtype,
-                   int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
+                   int num_blocks, int max_blocks_per_seq, int max_context_len, float scale, int sliding_window,
+                   int q_dtype, int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
+                   void* stream) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_blocks <= 0 || max_blocks_per_seq <= 0 ||
       max_context_len < 0)
     return fail(PKV_ERR_INVALID_ARG, "bad sizes");
@@ -410,6 +411,7 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
   if (is16(cache_dtype) && q_dtype != cache_dtype) return fail(PKV_ERR_UNSUPPORTED, "q dtype must match a 16-bit cache");
   if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
   if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "scale is not finite");
+  if (sliding_window < 0) return fail(PKV_ERR_INVALID_ARG, "sliding_window %d < 0", sliding_window);
   if (static_cast<long long>(num_blocks) * num_kv_heads * 16 >= (1LL << 31))
     return fail(PKV_ERR_UNSUPPORTED, "pool too large for 32-bit copy coordinates");
   if (static_cast<long long>(max_context_len) > static_cast<long long>(max_blocks_per_seq) * 16)
@@ -491,6 +493,7 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
   p.max_tiles = pl.max_tiles;
   p.num_q_tokens = mq ? num_q_tokens : num_seqs;
   p.max_query_len = mq ? max_query_len : 1;
+  p.window = sliding_window;
   p.epoch = next_epoch();
   p.qk_scale_log2 = scale * 1.4426950408889634f;
   const bool q_bf16 = q_dtype == PKV_BF16;
@@ -512,13 +515,13 @@ int pkv_paged_attention_decode(void* out, const void* q, const void* k_cache, co
                                const float* k_scale, const float* v_scale, const uint8_t* k_zero,
                                const uint8_t* v_zero, const int32_t* block_tables, const int32_t* context_lens,
                                int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int block_size,
-                               int num_blocks, int max_blocks_per_seq, int max_context_len, float scale, int q_dtype,
-                               int cache_dtype, int partition_tokens, void* workspace, size_t workspace_bytes,
-                               void* stream) {
+                               int num_blocks, int max_blocks_per_seq, int max_context_len, float scale,
+                               int sliding_window, int q_dtype, int cache_dtype, int partition_tokens,
+                               void* workspace, size_t workspace_bytes, void* stream) {
   return attention_call(out, q, k_cache, v_cache, k_scale, v_scale, k_zero, v_zero, block_tables, context_lens,
                         nullptr, num_seqs, 1, false, num_seqs, num_q_heads, num_kv_heads, head_dim, block_size,
-                        num_blocks, max_blocks_per_seq, max_context_len, scale, q_dtype, cache_dtype,
-                        partition_tokens, workspace, workspace_bytes, stream);
+                        num_blocks, max_blocks_per_seq, max_context_len, scale, sliding_window, q_dtype,
+                        cache_dtype, partition_tokens, workspace, workspace_bytes, stream);
 }
 
 int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim, int max_context_len,
@@ -545,12 +548,12 @@ int pkv_paged_attention_multi_query(void* out, const void* q, const void* k_cach
                                     const int32_t* query_start_loc, int num_seqs, int num_q_tokens,
                                     int max_query_len, int num_q_heads, int num_kv_heads, int head_dim,
                                     int block_size, int num_blocks, int max_blocks_per_seq, int max_context_len,
-                                    float scale, int q_dtype, int cache_dtype, int partition_tokens, void* workspace,
-                                    size_t workspace_bytes, void* stream) {
+                                    float scale, int sliding_window, int q_dtype, int cache_dtype,
+                                    int partition_tokens, void* workspace, size_t workspace_bytes, void* stream) {
   return attention_call(out, q, k_cache, v_cache, k_scale, v_scale, k_zero, v_zero, block_tables, context_lens,
                         query_start_loc, num_q_tokens, max_query_len, true, num_seqs, num_q_heads, num_kv_heads,
-                        head_dim, block_size, num_blocks, max_blocks_per_seq, max_context_len, scale, q_dtype,
-                        cache_dtype, partition_tokens, workspace, workspace_bytes, stream);
+                        head_dim, block_size, num_blocks, max_blocks_per_seq, max_context_len, scale,
+                        sliding_window, q_dtype, cache_dtype, partition_tokens, workspace, workspace_bytes, stream);
 }
 
 int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale, uint8_t* k_zero, uint8_t* v_zero,
@@ -649,8 +652,8 @@ extern "C" int pkv_paged_attention_decode_noalloc(void* out, const void* q, cons
                                                   const int32_t* block_tables, const int32_t* context_lens,
                                                   int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                                                   int block_size, int num_blocks, int max_blocks_per_seq,
-                                                  int max_context_len, float scale, int q_dtype, int cache_dtype,
-                                                  int partition_tokens, void* stream) {
+                                                  int max_context_len, float scale, int sliding_window,
+                                                  int q_dtype, int cache_dtype, int partition_tokens, void* stream) {
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0)
     return fail(PKV_ERR_INVALID_ARG, "bad sizes");
   if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128 (got %d)", head_dim);
@@ -672,6 +675,6 @@ extern "C" int pkv_paged_attention_decode_noalloc(void* out, const void* q, cons
   return pkv_paged_attention_decode(out, q, k_cache, v_cache, k_scale, v_scale, k_zero, v_zero, block_tables,
                                     context_lens,
                                     num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
-                                    max_blocks_per_seq, max_context_len, scale, q_dtype, cache_dtype,
+                                    max_blocks_per_seq, max_context_len, scale, sliding_window, q_dtype, cache_dtype,
                                     partition_tokens, scratch, needs_scratch ? kNoAllocScratchBytes : 0, stream);
 }

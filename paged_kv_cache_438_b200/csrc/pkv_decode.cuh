@@ -119,6 +119,7 @@ struct DecodeParams {
   int tile_cols;     // multi-query: columns per tile (8 * kNT)
   int max_tiles;     // multi-query: tiles per KV head of the longest query run (1 for decode)
   int num_q_tokens;  // multi-query: rows of q and out
+  int window;        // sliding window: a query at position P sees keys P - window + 1 .. P (0: all)
   int max_query_len; // multi-query: host bound of new tokens per sequence (sizes the counters)
   unsigned long long epoch;  // this call's epoch, nonzero, < 2^40
   float qk_scale_log2;       // softmax scale * log2(e)
@@ -174,25 +175,30 @@ __device__ __forceinline__ uint32_t load_q_pair(const void* q, long long idx) {
   return raw;
 }
 
-__device__ __forceinline__ int blocks_of(const DecodeParams& p, int s, bool report) {
-  return (clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, report) + 15) >> 4;
-}
-
 __device__ __forceinline__ void query_range(const DecodeParams& p, int s, int ctx, int& q0, int& q1, int& n,
                                             bool report);
 
-// Work items of sequence s: blocks * Hkv (decode), times the column tiles
-// of its new tokens in multi-query mode.
+// First block any query of a sequence can see under the sliding window: its
+// earliest new token (position ctx - n) sees keys from ctx - n + 1 - window.
+// Blocks before it are never read (their table entries may be stale).
+__device__ __forceinline__ int window_first_block(const DecodeParams& p, int ctx, int n) {
+  if (p.window <= 0) return 0;
+  const int lo = ctx - n + 1 - p.window;
+  return lo > 0 ? (lo >> 4) : 0;
+}
+
+// Work items of sequence s: its blocks from the window's first block on,
+// times Hkv, times (multi-query mode) the column tiles of its new tokens.
 template <bool kMQ>
 __device__ __forceinline__ int items_of(const DecodeParams& p, int s, bool report) {
+  const int ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, report);
   if constexpr (kMQ) {
-    const int ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, report);
     int q0, q1, n;
     query_range(p, s, ctx, q0, q1, n, report);
     const int tiles = (n * p.group + p.tile_cols - 1) / p.tile_cols;
-    return ((ctx + 15) >> 4) * p.num_kv_heads * tiles;
+    return (((ctx + 15) >> 4) - window_first_block(p, ctx, n)) * p.num_kv_heads * tiles;
   } else {
-    return blocks_of(p, s, report) * p.num_kv_heads;
+    return (((ctx + 15) >> 4) - window_first_block(p, ctx, 1)) * p.num_kv_heads;
   }
 }
 
@@ -240,12 +246,21 @@ __device__ __forceinline__ int find_seq(const int32_t* cum, int B, int g) {
   return lo;
 }
 
-// Blocks per pair of sequence s (a sequence with work has at least one).
+// Blocks per pair of sequence s (a sequence with work has at least one) and
+// the first of them (nonzero only under a sliding window).
 template <bool kMQ>
-__device__ __forceinline__ int pair_blocks(const DecodeParams& p, const int32_t* cum, int s) {
+__device__ __forceinline__ int pair_blocks(const DecodeParams& p, const int32_t* cum, int s, int& jb) {
   if constexpr (kMQ) {
-    return blocks_of(p, s, false);
+    const int ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false);
+    int q0, q1, n;
+    query_range(p, s, ctx, q0, q1, n, false);
+    jb = window_first_block(p, ctx, n);
+    return ((ctx + 15) >> 4) - jb;
   } else {
+    jb = p.window > 0
+             ? window_first_block(p, clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq,
+                                                   false), 1)
+             : 0;
     return (cum[s + 1] - cum[s]) / p.num_kv_heads;
   }
 }
@@ -254,13 +269,14 @@ __device__ __forceinline__ int pair_blocks(const DecodeParams& p, const int32_t*
 template <bool kMQ>
 __device__ __forceinline__ int item_row(const DecodeParams& p, const int32_t* cum, int g) {
   const int s = find_seq(cum, p.num_seqs, g);
-  const int nb = pair_blocks<kMQ>(p, cum, s);
+  int jb;
+  const int nb = pair_blocks<kMQ>(p, cum, s, jb);
   const int off = g - cum[s];
   const int pr = off / nb;
   const int j = off - pr * nb;
   // pairs of a sequence run KV head by KV head, tiles innermost
   const int h = kMQ ? pr / ((cum[s + 1] - cum[s]) / (nb * p.num_kv_heads)) : pr;
-  int id = p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + j];
+  int id = p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + jb + j];
   if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
     raise_status(PKV_DEV_BAD_BLOCK);
     id = 0;
@@ -359,7 +375,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
   int offset;
   {
     const int sl = find_seq(cum, B, g1 - 1);
-    const int nbl = pair_blocks<kMQ>(p, cum, sl);
+    int jbl;
+    const int nbl = pair_blocks<kMQ>(p, cum, sl, jbl);
     const int gpl = cum[sl] + ((g1 - 1 - cum[sl]) / nbl) * nbl;
     offset = gpl > g0 ? gpl - g0 : 0;
   }
@@ -406,6 +423,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
   // ---- cursor over (sequence, pair, block), in processing order; a pair is
   // a KV head (decode) or a (KV head, column tile) (multi-query) ----
   int s, nb, pr, h, j, ctx;
+  int jb = 0;  // first block read (sliding window)
   int ntile = 1, tile = 0, q0 = 0, n_new = 1;  // multi-query only
   auto set_pair = [&]() {
     if constexpr (kMQ) {
@@ -416,7 +434,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     }
   };
   auto enter_seq = [&]() {
-    nb = pair_blocks<kMQ>(p, cum, s);
+    nb = pair_blocks<kMQ>(p, cum, s, jb);
     ctx = clamp_context(p.context_lens[s], p.max_context_len, p.max_blocks_per_seq, false);
     if constexpr (kMQ) {
       int q1;
@@ -496,7 +514,10 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       for (int kk = k + 1; kk < count && kk < k + kR; ++kk) mbar_wait(bars + (kk % kR) * 8, (kk / kR) & 1);
       return;
     }
-    const int valid = ctx - j * 16;  // >= 1 tokens of this block count
+    const int base = (jb + j) * 16;  // position of the block's first token
+    const int valid = ctx - base;    // >= 1 tokens of this block count
+    // sliding window: tokens before position ctx - window are not seen
+    const int lowv = p.window > 0 ? ctx - p.window - base : -32;
 
     // ---- S^T = K . Q^T (two independent accumulation chains, summed) ----
     float sacc[kNT][4], sacc2[kNT][4];
@@ -567,8 +588,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       vs_r = sc[16 + r];
       vs_r8 = sc[16 + r + 8];
     }
-    const bool ok_r = r < valid;
-    const bool ok_r8 = r + 8 < valid;
+    const bool ok_r = r < valid && r >= lowv;
+    const bool ok_r8 = r + 8 < valid && r + 8 >= lowv;
     uint32_t pb[kNT][2];
     bool grow = false;
     float alpha[kNT][2];
@@ -576,11 +597,12 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     for (int nt = 0; nt < kNT; ++nt) {
       bool ok0 = ok_r, ok1 = ok_r, ok2 = ok_r8, ok3 = ok_r8;
       if constexpr (kMQ) {
-        const int va = colv[nt][0] - j * 16, vb = colv[nt][1] - j * 16;
-        ok0 = r < va;
-        ok1 = r < vb;
-        ok2 = r + 8 < va;
-        ok3 = r + 8 < vb;
+        const int va = colv[nt][0] - base, vb = colv[nt][1] - base;
+        const int la = p.window > 0 ? va - p.window : -32, lb = p.window > 0 ? vb - p.window : -32;
+        ok0 = r < va && r >= la;
+        ok1 = r < vb && r >= lb;
+        ok2 = r + 8 < va && r + 8 >= la;
+        ok3 = r + 8 < vb && r + 8 >= lb;
       }
       const float s0 = ok0 ? sacc[nt][0] * f_r : -INFINITY;
       const float s1 = ok1 ? sacc[nt][1] * f_r : -INFINITY;

@@ -63,13 +63,13 @@ def _signatures(lib):
                              ctypes.POINTER(_SZ)], _I),
         "pkv_decode_workspace_size": ([_I, _I, _I, _I, _I, _I, ctypes.POINTER(_SZ)], _I),
         "pkv_paged_attention_decode": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
-                                        _F, _I, _I, _I, _P, _SZ, _P], _I),
+                                        _F, _I, _I, _I, _I, _P, _SZ, _P], _I),
         "pkv_paged_attention_decode_noalloc": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
-                                                _I, _I, _F, _I, _I, _I, _P], _I),
+                                                _I, _I, _F, _I, _I, _I, _I, _P], _I),
         "pkv_multi_query_plan": ([_I, _I, _I, _I, _I, _I, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I),
                                   ctypes.POINTER(_SZ)], _I),
         "pkv_paged_attention_multi_query": ([_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
-                                             _I, _I, _I, _I, _F, _I, _I, _I, _P, _SZ, _P], _I),
+                                             _I, _I, _I, _I, _F, _I, _I, _I, _I, _P, _SZ, _P], _I),
         "pkv_copy_blocks": ([_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P], _I),
         "pkv_device_status": ([ctypes.POINTER(ctypes.c_uint), _I], _I),
         "pkv_set_validation": ([_I], _I),
@@ -240,7 +240,7 @@ def new_workspace(device, nbytes):
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale=None, v_scale=None,
                            max_context_len=None, out=None, workspace=None, partition_tokens=0, stream=None,
-                           k_zero=None, v_zero=None):
+                           k_zero=None, v_zero=None, sliding_window=0):
     """out[s, i] = softmax(scale * q[s, i] . K_s) V_s through block tables.
 
     q [B, Hq, D] fp16/bf16; caches [NB, Hkv, 16, D]; block_tables [B, MB]
@@ -250,6 +250,7 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     zero-filled before its first use and serve one call at a time; when None
     a cached per-stream workspace is used.  A uint8 cache with ``k_zero`` /
     ``v_zero`` is the asymmetric format, read as (code - zero) * scale.
+    ``sliding_window`` W > 0 limits each query to its W most recent keys.
     Returns ``out`` [B, Hq, D] in q's dtype."""
     dev = q.device
     for n, t in (("q", q), ("k_cache", k_cache), ("v_cache", v_cache)):
@@ -277,7 +278,8 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     _check(lib().pkv_paged_attention_decode(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero), _ptr(v_zero),
         _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], max_context_len,
-        float(scale), dtype_code(q), ct, partition_tokens, _ptr(workspace), ws_len, _stream(stream)))
+        float(scale), int(sliding_window), dtype_code(q), ct, partition_tokens, _ptr(workspace), ws_len,
+        _stream(stream)))
     return out
 
 
@@ -295,7 +297,8 @@ def multi_query_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_
 
 def paged_attention_multi_query(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
                                 max_query_len, max_context_len, k_scale=None, v_scale=None, k_zero=None,
-                                v_zero=None, out=None, workspace=None, partition_tokens=0, stream=None):
+                                v_zero=None, out=None, workspace=None, partition_tokens=0, stream=None,
+                                sliding_window=0):
     """Several new tokens per sequence (chunked prefill, speculative verify):
     q [T, Hq, D] packed by sequence with query_start_loc [B + 1] int32; the
     n_s new tokens of sequence s are the last n_s of its context_lens[s]
@@ -327,8 +330,8 @@ def paged_attention_multi_query(q, k_cache, v_cache, block_tables, context_lens,
     _check(lib().pkv_paged_attention_multi_query(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero), _ptr(v_zero),
         _ptr(block_tables), _ptr(context_lens), _ptr(query_start_loc), B, T, int(max_query_len), hq, hkv, d, bs, nb,
-        block_tables.shape[1], int(max_context_len), float(scale), dtype_code(q), ct, partition_tokens,
-        _ptr(workspace), ws_len, _stream(stream)))
+        block_tables.shape[1], int(max_context_len), float(scale), int(sliding_window), dtype_code(q), ct,
+        partition_tokens, _ptr(workspace), ws_len, _stream(stream)))
     return out
 
 
@@ -337,7 +340,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
                                    out, k_scale=None, v_scale=None, partition_tokens=0, stream=None,
-                                   k_zero=None, v_zero=None):
+                                   k_zero=None, v_zero=None, sliding_window=0):
     """paged_attention_decode for callers that cannot allocate device memory
     (for instance a plugin whose host framework owns every allocation and
     hands it only input and output buffers): ``out`` must be given, no
@@ -358,7 +361,7 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
     _check(lib().pkv_paged_attention_decode_noalloc(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero), _ptr(v_zero),
         _ptr(block_tables), _ptr(context_lens), B, hq, hkv, d, bs, nb, block_tables.shape[1], int(max_context_len),
-        float(scale), dtype_code(q), ct, partition_tokens, _stream(stream)))
+        float(scale), int(sliding_window), dtype_code(q), ct, partition_tokens, _stream(stream)))
     return out
 
 

@@ -73,12 +73,12 @@ def test_write_zero_tokens_is_a_noop(lib):
 def _decode(lib, **kw):
     n = ctypes.c_void_p(256)
     a = dict(out=n, q=n, kc=n, vc=n, ks=None, vs=None, kz=None, vz=None, bt=n, cl=n, B=2, hq=8, hkv=2, d=128, bs=16, nb=100, mb=4,
-             maxc=64, scale=0.1, qd=P.PKV_BF16, cd=P.PKV_BF16, pt=0, ws=None, wsb=0)
+             maxc=64, scale=0.1, win=0, qd=P.PKV_BF16, cd=P.PKV_BF16, pt=0, ws=None, wsb=0)
     a.update(kw)
     return lib.pkv_paged_attention_decode(a["out"], a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["kz"], a["vz"],
                                           a["bt"], a["cl"],
                                           a["B"], a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["mb"], a["maxc"],
-                                          a["scale"], a["qd"], a["cd"], a["pt"], a["ws"], a["wsb"], None)
+                                          a["scale"], a["win"], a["qd"], a["cd"], a["pt"], a["ws"], a["wsb"], None)
 
 
 def test_decode_host_rejections(lib):
@@ -90,6 +90,7 @@ def test_decode_host_rejections(lib):
     _err(_decode(lib, qd=P.PKV_F16), P.PKV_ERR_UNSUPPORTED)       # q dtype must match a 16-bit cache
     _err(_decode(lib, maxc=65), P.PKV_ERR_INVALID_ARG)            # > max_blocks * 16
     _err(_decode(lib, scale=float("nan")), P.PKV_ERR_INVALID_ARG)
+    _err(_decode(lib, win=-1), P.PKV_ERR_INVALID_ARG)
     _err(_decode(lib, cd=P.PKV_I8), P.PKV_ERR_INVALID_ARG)        # quantised without scales
     _err(_decode(lib, cd=P.PKV_U8ASYM, ks=n, vs=n), P.PKV_ERR_INVALID_ARG)   # without zero points
     _err(_decode(lib, cd=P.PKV_U8ASYM, ks=n, vs=n, kz=n, vz=ctypes.c_void_p(264)),
@@ -127,13 +128,14 @@ def test_copy_rejections(lib):
 def _mq(lib, **kw):
     n = ctypes.c_void_p(256)
     a = dict(out=n, q=n, kc=n, vc=n, ks=None, vs=None, kz=None, vz=None, bt=n, cl=n, qsl=n, B=2, T=8, mq=4, hq=8,
-             hkv=2, d=128, bs=16, nb=100, mb=4, maxc=64, scale=0.1, qd=P.PKV_BF16, cd=P.PKV_BF16, pt=0, ws=None,
-             wsb=0)
+             hkv=2, d=128, bs=16, nb=100, mb=4, maxc=64, scale=0.1, win=0, qd=P.PKV_BF16, cd=P.PKV_BF16, pt=0,
+             ws=None, wsb=0)
     a.update(kw)
     return lib.pkv_paged_attention_multi_query(a["out"], a["q"], a["kc"], a["vc"], a["ks"], a["vs"], a["kz"],
                                                a["vz"], a["bt"], a["cl"], a["qsl"], a["B"], a["T"], a["mq"],
                                                a["hq"], a["hkv"], a["d"], a["bs"], a["nb"], a["mb"], a["maxc"],
-                                               a["scale"], a["qd"], a["cd"], a["pt"], a["ws"], a["wsb"], None)
+                                               a["scale"], a["win"], a["qd"], a["cd"], a["pt"], a["ws"], a["wsb"],
+                                               None)
 
 
 def test_multi_query_host_rejections(lib):

@@ -29,18 +29,18 @@ def _lib():
     assert P.device_status(clear=True) == 0, "a kernel raised a device status bit"
 
 
-def run_mq(g, partition_tokens=0, max_query_len=None):
+def run_mq(g, partition_tokens=0, max_query_len=None, window=0):
     out = P.paged_attention_multi_query(
         g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"], g["query_start_loc"], g["scale"],
         max_query_len=g["max_query_len"] if max_query_len is None else max_query_len,
         max_context_len=int(g["context_lens"].max()), k_scale=g.get("k_scale"), v_scale=g.get("v_scale"),
-        k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), partition_tokens=partition_tokens)
+        k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), partition_tokens=partition_tokens, sliding_window=window)
     torch.cuda.synchronize()
     assert P.device_status(clear=True) == 0
     return out
 
 
-def oracle_mq(case, seqs=None):
+def oracle_mq(case, seqs=None, window=0):
     """Oracle rows for all sequences, or only for ``seqs`` (others zero)."""
     kind = case["cache_kind"]
     qsl = case["query_start_loc"].numpy()
@@ -57,12 +57,12 @@ def oracle_mq(case, seqs=None):
         sub = OA.paged_multi_query_attention(q[rows], cache_values(case["k_cache"], kind),
                                              cache_values(case["v_cache"], kind), bt, ctx, sub_qsl, case["scale"],
                                              cpu_or_none(case, "k_scale"), cpu_or_none(case, "v_scale"),
-                                             cpu_or_none(case, "k_zero"), cpu_or_none(case, "v_zero"))
+                                             cpu_or_none(case, "k_zero"), cpu_or_none(case, "v_zero"), window)
         return rows, sub
     return OA.paged_multi_query_attention(np64(case["q"]), cache_values(case["k_cache"], kind),
                                           cache_values(case["v_cache"], kind), bt, ctx, qsl, case["scale"],
                                           cpu_or_none(case, "k_scale"), cpu_or_none(case, "v_scale"),
-                                          cpu_or_none(case, "k_zero"), cpu_or_none(case, "v_zero"))
+                                          cpu_or_none(case, "k_zero"), cpu_or_none(case, "v_zero"), window)
 
 
 CTX = [1, 15, 16, 17, 40, 257, 1000, 33, 0, 300]
@@ -88,6 +88,22 @@ def test_multi_query_quantised(kind, group):
     case = I.multi_query_case("spec_verify", seed=group + 70, ctx_override=CTX, q_lens=NQ, hq=hkv * group, hkv=hkv,
                               d=128, cache_kind=kind)
     check_attn(np64(run_mq(gpu_case(case))), oracle_mq(case))
+
+
+@pytest.mark.parametrize("window", [1, 7, 33, 200])
+@pytest.mark.parametrize("group", [1, 4])
+@pytest.mark.parametrize("ptok", [0, 16])
+def test_multi_query_sliding_window(window, group, ptok):
+    hkv = 2
+    case = I.multi_query_case("spec_verify", seed=window * 3 + group, ctx_override=CTX, q_lens=NQ, hq=hkv * group,
+                              hkv=hkv, d=128)
+    g = gpu_case(case)
+    bt = g["block_tables"].clone()
+    for s, (c, n) in enumerate(zip(CTX, NQ)):
+        if n:
+            bt[s, :max(0, c - n + 1 - window) // 16] = case["num_blocks"] + 3   # never read
+    g["block_tables"] = bt
+    check_attn(np64(run_mq(g, partition_tokens=ptok, window=window)), oracle_mq(case, window=window))
 
 
 @pytest.mark.parametrize("group", [4, 16])

@@ -91,24 +91,25 @@ def gpu_case(case):
     return out
 
 
-def run_decode(g, partition_tokens=0, max_context_len=None):
+def run_decode(g, partition_tokens=0, max_context_len=None, window=0):
     P.device_status(clear=True)
     out = P.paged_attention_decode(g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"],
                                    g["scale"], k_scale=g.get("k_scale"), v_scale=g.get("v_scale"),
                                    max_context_len=max_context_len, partition_tokens=partition_tokens,
-                                   k_zero=g.get("k_zero"), v_zero=g.get("v_zero"))
+                                   k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), sliding_window=window)
     torch.cuda.synchronize()
     assert P.device_status(clear=True) == 0
     return out
 
 
-def oracle_full(case):
+def oracle_full(case, window=0):
     kind = case["cache_kind"]
     return OA.paged_decode_attention(np64(case["q"]), cache_values(case["k_cache"], kind),
                                      cache_values(case["v_cache"], kind), case["block_tables"].numpy(),
                                      case["context_lens"].numpy(), case["scale"],
                                      cpu_or_none(case, "k_scale"), cpu_or_none(case, "v_scale"),
-                                     k_zero=cpu_or_none(case, "k_zero"), v_zero=cpu_or_none(case, "v_zero"))
+                                     k_zero=cpu_or_none(case, "k_zero"), v_zero=cpu_or_none(case, "v_zero"),
+                                     window=window)
 
 
 def oracle_sampled(g, pairs, seed=0):
@@ -290,6 +291,28 @@ def test_decode_sweep_quantised(kind, qdtype, d, group, ptok):
     g = gpu_case(case)
     got = np64(run_decode(g, partition_tokens=ptok))
     check_attn(got, oracle_full(case))
+
+
+@pytest.mark.parametrize("window", [1, 16, 40, 300])
+@pytest.mark.parametrize("group,d", [(4, 128), (16, 128), (8, 64)])
+@pytest.mark.parametrize("ptok", [0, 16])
+def test_decode_sliding_window(window, group, d, ptok):
+    hkv = 2
+    case = I.decode_case("llama3_8b", seed=window + group, ctx_override=CTX_MIX, hq=hkv * group, hkv=hkv, d=d)
+    g = gpu_case(case)
+    # blocks wholly before the window are never read: poison their table entries
+    bt = g["block_tables"].clone()
+    for s, c in enumerate(CTX_MIX):
+        first = max(0, c - window) // 16
+        bt[s, :first] = case["num_blocks"] + 7
+    g["block_tables"] = bt
+    got = np64(run_decode(g, partition_tokens=ptok, window=window))
+    check_attn(got, oracle_full(case, window=window))
+
+
+def test_decode_sliding_window_quantised():
+    case = I.decode_case("quant_mha", seed=41, ctx_override=CTX_MIX, hq=8, hkv=2, d=128, cache_kind="u8asym")
+    check_attn(np64(run_decode(gpu_case(case), window=100)), oracle_full(case, window=100))
 
 
 def test_max_context_len_above_actual_is_fine():
