@@ -382,6 +382,60 @@ int pkv_block_refcount(void* handle, int32_t block, int* rc_out);
  * total free / largest contiguous free run). */
 int pkv_alloc_stats(void* handle, int* num_free, int* num_shared, int* largest_free_run);
 
+/* ======================================================================= *
+ * Automatic prefix caching in the allocator ([P-WMRH] §三
+ * AutomaticPrefixCache / PrefixRadixTree): the longest cached prefix of a
+ * request's token ids is found in a radix tree and rounded down to whole
+ * blocks; the cache key is the 16-byte BLAKE2b digest of the token ids as
+ * little-endian int32; least recently used entries are evicted.
+ *   - Every full block of a cached sequence is one tree node whose edge is
+ *     that block's 16 token ids (the KV of a sequence covers each of its
+ *     prefixes), so a hit is the longest run of whole leading blocks that
+ *     some cached sequence shares with the request.
+ *   - The cache holds one reference on each cached block.  A cached block is
+ *     evictable when no sequence holds it and no cached block lies below it
+ *     in the tree; eviction takes the least recently used evictable block (a
+ *     logical clock ticks once per insert / match / add-cached call; ties go
+ *     to the older node) and returns it to the free list.
+ *   - An append that finds the free list empty evicts one block that way
+ *     before failing with PKV_ERR_NO_BLOCKS (a failed append restores the
+ *     cache too).
+ * ======================================================================= */
+
+/* BLAKE2b-128 (RFC 7693, no key) of n token ids as little-endian int32;
+ * key_out: 16 bytes. */
+int pkv_prefix_key(const int32_t* token_ids, int n_tokens, uint8_t* key_out);
+
+/* Cache the first floor(min(n_tokens, length) / 16) blocks of a sequence
+ * whose first tokens are token_ids (host int32 [n_tokens]).  A block whose
+ * prefix is already cached is left as it is (its last use is refreshed);
+ * newly_cached_out (nullable) counts blocks that became cached. */
+int pkv_prefix_cache_insert(void* handle, int64_t seq_id, const int32_t* token_ids, int n_tokens,
+                            int* newly_cached_out);
+
+/* Longest cached whole-block prefix of token_ids: hit_tokens_out (a multiple
+ * of 16), key_out (nullable; 16 bytes: the key of the hit prefix, zeros on a
+ * miss).  Counts one lookup, and one hit when hit_tokens > 0. */
+int pkv_prefix_cache_match(void* handle, const int32_t* token_ids, int n_tokens, int* hit_tokens_out,
+                           uint8_t* key_out);
+
+/* Register a sequence whose block table starts with the blocks of the
+ * longest cached prefix of token_ids (their counts + 1) and whose length is
+ * the hit (hit_tokens_out); the caller then appends and computes the rest.
+ * A fully cached request gets all its tokens; pass one token fewer to have
+ * the last one recomputed. */
+int pkv_seq_add_cached(void* handle, int64_t seq_id, const int32_t* token_ids, int n_tokens,
+                       int* hit_tokens_out);
+
+/* Evict until at most max_cached_blocks blocks are cached or nothing more is
+ * evictable ([P-WMRH] §三 evict_lru, with the budget in blocks). */
+int pkv_prefix_cache_evict(void* handle, int max_cached_blocks, int* evicted_out);
+
+/* Cached blocks, evictable blocks now, lookups, hits (hit rate = hits /
+ * lookups, [P-WMRH] §三 metrics table), evictions so far.  Outputs nullable. */
+int pkv_prefix_cache_stats(void* handle, int* cached_blocks, int* evictable_blocks, int64_t* lookups,
+                           int64_t* hits, int64_t* evictions);
+
 #ifdef __cplusplus
 }
 #endif

@@ -15,13 +15,29 @@
 //
 // Every mutating call is transactional: an undo log restores the exact prior
 // state (free-list order included) when a block allocation fails.
+//
+// Automatic prefix caching (same page, §三 AutomaticPrefixCache and
+// PrefixRadixTree): the longest cached prefix of a request's token ids is
+// found in a radix tree and rounded down to whole blocks; the key is a
+// 16-byte BLAKE2b digest of the token ids as little-endian int32; least
+// recently used entries are evicted.  Here every full block of a cached
+// sequence is one tree node (its edge: that block's 16 token ids), since the
+// KV of a sequence covers all of its prefixes.  The cache holds a reference
+// on each cached block; only blocks no sequence holds, with no cached block
+// below them, can be evicted (least recently used first, by a logical clock
+// that ticks once per cache call, ties to the older node).  An allocation
+// that finds the free list empty evicts one such block.
 #include <algorithm>
+#include <array>
 #include <cstdint>
 #include <cstring>
 #include <new>
+#include <set>
+#include <tuple>
 #include <unordered_map>
 #include <vector>
 
+#include "pkv_blake2b.h"
 #include "pkv_error.h"
 
 namespace pkv {
@@ -38,6 +54,34 @@ struct Sequence {
   int64_t len = 0;
 };
 
+using Chunk = std::array<int32_t, 16>;
+
+struct ChildKey {
+  int parent;
+  Chunk chunk;
+  bool operator==(const ChildKey& o) const { return parent == o.parent && chunk == o.chunk; }
+};
+
+struct ChildKeyHash {
+  size_t operator()(const ChildKey& k) const {
+    uint64_t h = 1469598103934665603ull ^ static_cast<uint64_t>(k.parent);
+    for (int32_t t : k.chunk) h = (h ^ static_cast<uint32_t>(t)) * 1099511628211ull;
+    return static_cast<size_t>(h);
+  }
+};
+
+// One cached block of the prefix tree (node 0 is the root, which has none).
+struct Node {
+  int parent = -1;
+  Chunk chunk{};
+  int32_t block = -1;
+  uint8_t key[16] = {};
+  int64_t last = 0;   // logical time of the last use
+  int64_t order = 0;  // creation order (LRU tie-break)
+  int children = 0;
+  bool alive = false;
+};
+
 class BlockManager {
  public:
   BlockManager(int num_blocks, int block_size, const int32_t* order)
@@ -48,6 +92,120 @@ class BlockManager {
     } else {
       for (int b = 0; b < num_blocks; ++b) free_.push_back(b);
     }
+    nodes_.emplace_back();  // root
+    nodes_[0].alive = true;
+  }
+
+  // ---- prefix cache --------------------------------------------------------
+  // Nodes of the longest cached whole-block prefix of tokens[0, n).
+  void walk(const int32_t* tokens, int n, std::vector<int>* path) const {
+    path->clear();
+    int cur = 0;
+    for (int i = 0; i + 16 <= n; i += 16) {
+      ChildKey k{cur, {}};
+      std::copy(tokens + i, tokens + i + 16, k.chunk.begin());
+      auto it = children_.find(k);
+      if (it == children_.end()) break;
+      cur = it->second;
+      path->push_back(cur);
+    }
+  }
+
+  void touch(int id) {
+    Node& nd = nodes_[id];
+    lru_.erase(std::make_tuple(nd.last, nd.order, id));
+    nd.last = clock_;
+    lru_.insert(std::make_tuple(nd.last, nd.order, id));
+  }
+
+  int match(const int32_t* tokens, int n, int* hit, uint8_t* key) {
+    ++clock_;
+    walk(tokens, n, &path_);
+    for (int id : path_) touch(id);
+    ++lookups_;
+    if (!path_.empty()) ++hits_;
+    if (hit) *hit = static_cast<int>(path_.size()) * block_size_;
+    if (key) {
+      if (path_.empty()) std::memset(key, 0, 16);
+      else std::memcpy(key, nodes_[path_.back()].key, 16);
+    }
+    return ok();
+  }
+
+  int add_cached(int64_t id, const int32_t* tokens, int n, int* hit_out) {
+    if (seqs_.count(id)) return fail(PKV_ERR_EXISTS, "sequence %lld already exists", (long long)id);
+    int hit = 0;
+    match(tokens, n, &hit, nullptr);
+    Sequence s;
+    for (int nd : path_) {
+      s.table.push_back(nodes_[nd].block);
+      ++rc_[nodes_[nd].block];
+    }
+    s.len = hit;
+    seqs_.emplace(id, std::move(s));
+    if (hit_out) *hit_out = hit;
+    return ok();
+  }
+
+  int insert(int64_t id, const int32_t* tokens, int n, int* newly) {
+    auto it = seqs_.find(id);
+    if (it == seqs_.end()) return fail(PKV_ERR_NOT_FOUND, "sequence %lld not found", (long long)id);
+    const Sequence& s = it->second;
+    const int nblk = static_cast<int>(std::min<int64_t>(n, s.len) / block_size_);
+    ++clock_;
+    Blake2b128 st;
+    int cur = 0, added = 0;
+    for (int i = 0; i < nblk; ++i) {
+      const int32_t* c = tokens + static_cast<size_t>(i) * 16;
+      blake2b_tokens(&st, c, 16);
+      ChildKey k{cur, {}};
+      std::copy(c, c + 16, k.chunk.begin());
+      auto f = children_.find(k);
+      if (f != children_.end()) {
+        cur = f->second;
+        touch(cur);
+        continue;
+      }
+      const int nid = new_node();
+      Node& nd = nodes_[nid];
+      nd.parent = cur;
+      nd.chunk = k.chunk;
+      nd.block = s.table[static_cast<size_t>(i)];
+      st.digest(nd.key);
+      nd.last = clock_;
+      nd.order = next_order_++;
+      nd.children = 0;
+      nd.alive = true;
+      children_.emplace(k, nid);
+      ++nodes_[cur].children;
+      lru_.insert(std::make_tuple(nd.last, nd.order, nid));
+      ++rc_[nd.block];
+      ++cached_;
+      ++added;
+      cur = nid;
+    }
+    if (newly) *newly = added;
+    return ok();
+  }
+
+  int evict_to(int max_cached, int* evicted) {
+    int k = 0;
+    while (cached_ > max_cached && evict_one(false)) ++k;
+    if (evicted) *evicted = k;
+    return ok();
+  }
+
+  void cache_stats(int* cached, int* evictable, int64_t* lookups, int64_t* hits, int64_t* evictions) const {
+    int ev = 0;
+    for (size_t i = 1; i < nodes_.size(); ++i) {
+      const Node& nd = nodes_[i];
+      if (nd.alive && nd.children == 0 && rc_[nd.block] == 1) ++ev;
+    }
+    if (cached) *cached = cached_;
+    if (evictable) *evictable = ev;
+    if (lookups) *lookups = lookups_;
+    if (hits) *hits = hits_;
+    if (evictions) *evictions = evictions_;
   }
 
   int num_blocks() const { return static_cast<int>(rc_.size()); }
@@ -113,6 +271,9 @@ class BlockManager {
       }
     }
     if (n_pairs) *n_pairs = np;
+    for (const Undo& u : undo_)  // committed: evicted nodes' slots can be reused
+      if (u.op == Op::kEvict) dead_.push_back(static_cast<int>(u.aux));
+    undo_.clear();
     return ok();
   }
 
@@ -148,17 +309,52 @@ class BlockManager {
   }
 
  private:
-  enum class Op { kPush, kCow, kLen };
+  enum class Op { kPush, kCow, kLen, kEvict };
   struct Undo {
     Op op;
     int64_t seq;
     int32_t block;   // block taken from the free list
     int32_t old;     // kCow: the shared block that was replaced
-    int64_t aux = 0; // kCow: logical index; kLen: previous length
+    int64_t aux = 0; // kCow: logical index; kLen: previous length; kEvict: node id
   };
 
+  int new_node() {
+    if (!dead_.empty()) {
+      const int id = dead_.back();
+      dead_.pop_back();
+      return id;
+    }
+    nodes_.emplace_back();
+    return static_cast<int>(nodes_.size()) - 1;
+  }
+
+  // Evicts the least recently used cached block that no sequence holds and
+  // that has no cached child; its block returns to the free list.
+  bool evict_one(bool log) {
+    for (auto it = lru_.begin(); it != lru_.end(); ++it) {
+      const int id = std::get<2>(*it);
+      Node& nd = nodes_[id];
+      if (nd.children != 0 || rc_[nd.block] != 1) continue;
+      lru_.erase(it);
+      children_.erase(ChildKey{nd.parent, nd.chunk});
+      --nodes_[nd.parent].children;
+      nd.alive = false;
+      rc_[nd.block] = 0;
+      free_.push_back(nd.block);
+      --cached_;
+      ++evictions_;
+      if (log) {
+        undo_.push_back({Op::kEvict, 0, nd.block, 0, id});
+      } else {
+        dead_.push_back(id);
+      }
+      return true;
+    }
+    return false;
+  }
+
   bool pop(int32_t* b) {
-    if (free_.empty()) return false;
+    if (free_.empty() && !evict_one(true)) return false;
     *b = free_.back();
     free_.pop_back();
     rc_[*b] = 1;
@@ -167,6 +363,20 @@ class BlockManager {
 
   int rollback(int code, const char* fmt, ...) {
     for (auto it = undo_.rbegin(); it != undo_.rend(); ++it) {
+      if (it->op == Op::kEvict) {
+        // the evicted block went to the back of the free list; take it back
+        const int id = static_cast<int>(it->aux);
+        Node& nd = nodes_[id];
+        free_.pop_back();
+        rc_[nd.block] = 1;
+        nd.alive = true;
+        children_.emplace(ChildKey{nd.parent, nd.chunk}, id);
+        ++nodes_[nd.parent].children;
+        lru_.insert(std::make_tuple(nd.last, nd.order, id));
+        ++cached_;
+        --evictions_;
+        continue;
+      }
       Sequence& s = seqs_[it->seq];
       switch (it->op) {
         case Op::kLen:
@@ -183,6 +393,8 @@ class BlockManager {
           rc_[it->block] = 0;
           free_.push_back(it->block);
           break;
+        case Op::kEvict:
+          break;
       }
     }
     undo_.clear();
@@ -198,6 +410,16 @@ class BlockManager {
   std::vector<int32_t> rc_;
   std::unordered_map<int64_t, Sequence> seqs_;
   std::vector<Undo> undo_;
+  // prefix cache
+  std::vector<Node> nodes_;
+  std::vector<int> dead_;  // reusable node slots
+  std::unordered_map<ChildKey, int, ChildKeyHash> children_;
+  std::set<std::tuple<int64_t, int64_t, int>> lru_;
+  std::vector<int> path_;
+  int64_t clock_ = 0;
+  int64_t next_order_ = 1;
+  int cached_ = 0;
+  int64_t lookups_ = 0, hits_ = 0, evictions_ = 0;
 };
 
 BlockManager* as_mgr(void* h) { return static_cast<BlockManager*>(h); }
@@ -326,6 +548,45 @@ int pkv_block_refcount(void* h, int32_t block, int* rc_out) {
 int pkv_alloc_stats(void* h, int* num_free, int* num_shared, int* largest_free_run) {
   if (!h) return fail(PKV_ERR_INVALID_ARG, "NULL handle");
   pkv::as_mgr(h)->stats(num_free, num_shared, largest_free_run);
+  return ok();
+}
+
+int pkv_prefix_key(const int32_t* token_ids, int n_tokens, uint8_t* key_out) {
+  if (n_tokens < 0 || (n_tokens > 0 && !token_ids) || !key_out) return fail(PKV_ERR_INVALID_ARG, "bad arguments");
+  pkv::Blake2b128 st;
+  pkv::blake2b_tokens(&st, token_ids, n_tokens);
+  st.digest(key_out);
+  return ok();
+}
+
+int pkv_prefix_cache_insert(void* h, int64_t seq_id, const int32_t* token_ids, int n_tokens, int* newly_cached_out) {
+  if (!h) return fail(PKV_ERR_INVALID_ARG, "NULL handle");
+  if (n_tokens < 0 || (n_tokens > 0 && !token_ids)) return fail(PKV_ERR_INVALID_ARG, "bad token arguments");
+  return pkv::as_mgr(h)->insert(seq_id, token_ids, n_tokens, newly_cached_out);
+}
+
+int pkv_prefix_cache_match(void* h, const int32_t* token_ids, int n_tokens, int* hit_tokens_out, uint8_t* key_out) {
+  if (!h) return fail(PKV_ERR_INVALID_ARG, "NULL handle");
+  if (n_tokens < 0 || (n_tokens > 0 && !token_ids)) return fail(PKV_ERR_INVALID_ARG, "bad token arguments");
+  return pkv::as_mgr(h)->match(token_ids, n_tokens, hit_tokens_out, key_out);
+}
+
+int pkv_seq_add_cached(void* h, int64_t seq_id, const int32_t* token_ids, int n_tokens, int* hit_tokens_out) {
+  if (!h) return fail(PKV_ERR_INVALID_ARG, "NULL handle");
+  if (n_tokens < 0 || (n_tokens > 0 && !token_ids)) return fail(PKV_ERR_INVALID_ARG, "bad token arguments");
+  return pkv::as_mgr(h)->add_cached(seq_id, token_ids, n_tokens, hit_tokens_out);
+}
+
+int pkv_prefix_cache_evict(void* h, int max_cached_blocks, int* evicted_out) {
+  if (!h) return fail(PKV_ERR_INVALID_ARG, "NULL handle");
+  if (max_cached_blocks < 0) return fail(PKV_ERR_INVALID_ARG, "max_cached_blocks < 0");
+  return pkv::as_mgr(h)->evict_to(max_cached_blocks, evicted_out);
+}
+
+int pkv_prefix_cache_stats(void* h, int* cached_blocks, int* evictable_blocks, int64_t* lookups, int64_t* hits,
+                           int64_t* evictions) {
+  if (!h) return fail(PKV_ERR_INVALID_ARG, "NULL handle");
+  pkv::as_mgr(h)->cache_stats(cached_blocks, evictable_blocks, lookups, hits, evictions);
   return ok();
 }
 

@@ -31,7 +31,8 @@ EXPORTS = [
     "pkv_paged_attention_multi_query", "pkv_copy_blocks", "pkv_device_status", "pkv_set_validation",
     "pkv_alloc_create", "pkv_alloc_destroy", "pkv_seq_add", "pkv_seq_fork", "pkv_seq_append",
     "pkv_batch_append", "pkv_batch_tables", "pkv_seq_free", "pkv_seq_block_table", "pkv_seq_len",
-    "pkv_block_refcount", "pkv_alloc_stats",
+    "pkv_block_refcount", "pkv_alloc_stats", "pkv_prefix_key", "pkv_prefix_cache_insert", "pkv_prefix_cache_match",
+    "pkv_seq_add_cached", "pkv_prefix_cache_evict", "pkv_prefix_cache_stats",
 ]
 
 
@@ -85,6 +86,13 @@ def _signatures(lib):
         "pkv_seq_len": ([_P, _I64, ctypes.POINTER(_I)], _I),
         "pkv_block_refcount": ([_P, ctypes.c_int32, ctypes.POINTER(_I)], _I),
         "pkv_alloc_stats": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
+        "pkv_prefix_key": ([_P, _I, _P], _I),
+        "pkv_prefix_cache_insert": ([_P, _I64, _P, _I, ctypes.POINTER(_I)], _I),
+        "pkv_prefix_cache_match": ([_P, _P, _I, ctypes.POINTER(_I), _P], _I),
+        "pkv_seq_add_cached": ([_P, _I64, _P, _I, ctypes.POINTER(_I)], _I),
+        "pkv_prefix_cache_evict": ([_P, _I, ctypes.POINTER(_I)], _I),
+        "pkv_prefix_cache_stats": ([_P, ctypes.POINTER(_I), ctypes.POINTER(_I), ctypes.POINTER(_I64),
+                                    ctypes.POINTER(_I64), ctypes.POINTER(_I64)], _I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -477,3 +485,54 @@ class BlockAllocator:
         a, b, c = _I(0), _I(0), _I(0)
         _check(lib().pkv_alloc_stats(self._h, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
         return a.value, b.value, c.value
+
+    # -- automatic prefix caching --------------------------------------------
+    def prefix_insert(self, seq_id, token_ids):
+        """Cache the sequence's full blocks under their token prefix; returns
+        how many blocks became newly cached."""
+        t = _tokens(token_ids)
+        n = _I(0)
+        _check(lib().pkv_prefix_cache_insert(self._h, seq_id, _ptr(t), t.numel(), ctypes.byref(n)))
+        return n.value
+
+    def prefix_match(self, token_ids):
+        """(hit tokens, 16-byte key of the hit prefix)."""
+        t = _tokens(token_ids)
+        hit = _I(0)
+        key = (ctypes.c_uint8 * 16)()
+        _check(lib().pkv_prefix_cache_match(self._h, _ptr(t), t.numel(), ctypes.byref(hit), key))
+        return hit.value, bytes(key)
+
+    def add_cached(self, seq_id, token_ids):
+        """New sequence starting with its longest cached prefix; returns the hit."""
+        t = _tokens(token_ids)
+        hit = _I(0)
+        _check(lib().pkv_seq_add_cached(self._h, seq_id, _ptr(t), t.numel(), ctypes.byref(hit)))
+        return hit.value
+
+    def prefix_evict(self, max_cached_blocks):
+        n = _I(0)
+        _check(lib().pkv_prefix_cache_evict(self._h, max_cached_blocks, ctypes.byref(n)))
+        return n.value
+
+    def prefix_stats(self):
+        """(cached blocks, evictable now, lookups, hits, evictions)."""
+        a, b = _I(0), _I(0)
+        c, d, e = _I64(0), _I64(0), _I64(0)
+        _check(lib().pkv_prefix_cache_stats(self._h, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c),
+                                            ctypes.byref(d), ctypes.byref(e)))
+        return a.value, b.value, c.value, d.value, e.value
+
+
+def _tokens(token_ids):
+    t = token_ids if isinstance(token_ids, torch.Tensor) and token_ids.dtype == torch.int32 \
+        else torch.as_tensor(list(token_ids), dtype=torch.int32)
+    return t.contiguous()
+
+
+def prefix_key(token_ids):
+    """BLAKE2b-128 of token ids as little-endian int32 (the prefix cache key)."""
+    t = _tokens(token_ids)
+    key = (ctypes.c_uint8 * 16)()
+    _check(lib().pkv_prefix_key(_ptr(t) if t.numel() else None, t.numel(), key))
+    return bytes(key)
