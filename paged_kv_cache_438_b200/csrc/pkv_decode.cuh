@@ -322,9 +322,9 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw_addr = smem_addr(smem_raw);
-  const uint32_t base = (raw_addr + 1023u) & ~1023u;
-  uint8_t* const base_ptr = smem_raw + (base - raw_addr);
-  const uint32_t bar_base = base + kW * kR * Tr::kStageBytes;
+  const uint32_t smem_base = (raw_addr + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (smem_base - raw_addr);
+  const uint32_t bar_base = smem_base + kW * kR * Tr::kStageBytes;
   int32_t* const cum = reinterpret_cast<int32_t*>(base_ptr + kW * kR * Tr::kStageBytes + kW * kR * 8);
 
   const int warp = threadIdx.x >> 5;
@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
   }
   auto item_of = [&](int k) { return g0 + (k + offset < count ? k + offset : k + offset - count); };
 
-  const uint32_t ring = base + warp * kR * Tr::kStageBytes;
+  const uint32_t ring = smem_base + warp * kR * Tr::kStageBytes;
   const uint32_t bars = bar_base + warp * kR * 8;
 
   // Copy coordinates of this warp's items, 32 at a time, two chunks ahead.
@@ -514,10 +514,10 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       for (int kk = k + 1; kk < count && kk < k + kR; ++kk) mbar_wait(bars + (kk % kR) * 8, (kk / kR) & 1);
       return;
     }
-    const int base = (jb + j) * 16;  // position of the block's first token
-    const int valid = ctx - base;    // >= 1 tokens of this block count
+    const int kpos0 = (jb + j) * 16;  // position of the block's first token
+    const int valid = ctx - kpos0;    // >= 1 tokens of this block count
     // sliding window: tokens before position ctx - window are not seen
-    const int lowv = p.window > 0 ? ctx - p.window - base : -32;
+    const int lowv = p.window > 0 ? ctx - p.window - kpos0 : -32;
 
     // ---- S^T = K . Q^T (two independent accumulation chains, summed) ----
     float sacc[kNT][4], sacc2[kNT][4];
@@ -540,7 +540,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       // uint8: fp16 pairs (1024 + z) of this lane's two tokens r and r + 8
       uint32_t zk_r = 0, zk_r8 = 0;
       if constexpr (kCT == kU8) {
-        const uint8_t* zk = base_ptr + (st - base) + 2 * Tr::kKVBytes + 128;
+        const uint8_t* zk = base_ptr + (st - smem_base) + 2 * Tr::kKVBytes + 128;
         zk_r = (0x6400u + zk[r]) * 0x10001u;
         zk_r8 = (0x6400u + zk[r + 8]) * 0x10001u;
       }
@@ -582,7 +582,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     float f_r = p.qk_scale_log2, f_r8 = p.qk_scale_log2;
     float vs_r = 1.0f, vs_r8 = 1.0f;
     if constexpr (k8) {
-      const float* sc = reinterpret_cast<const float*>(base_ptr + (st - base) + 2 * Tr::kKVBytes);
+      const float* sc = reinterpret_cast<const float*>(base_ptr + (st - smem_base) + 2 * Tr::kKVBytes);
       f_r *= sc[r];
       f_r8 *= sc[r + 8];
       vs_r = sc[16 + r];
@@ -597,7 +597,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     for (int nt = 0; nt < kNT; ++nt) {
       bool ok0 = ok_r, ok1 = ok_r, ok2 = ok_r8, ok3 = ok_r8;
       if constexpr (kMQ) {
-        const int va = colv[nt][0] - base, vb = colv[nt][1] - base;
+        const int va = colv[nt][0] - kpos0, vb = colv[nt][1] - kpos0;
         const int la = p.window > 0 ? va - p.window : -32, lb = p.window > 0 ? vb - p.window : -32;
         ok0 = r < va && r >= la;
         ok1 = r < vb && r >= lb;
@@ -662,7 +662,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       // (2q + 8, 2q + 9)
       uint32_t zv_x = 0, zv_y = 0;
       if constexpr (kCT == kU8) {
-        const uint8_t* zv = base_ptr + (st - base) + 2 * Tr::kKVBytes + 144;
+        const uint8_t* zv = base_ptr + (st - smem_base) + 2 * Tr::kKVBytes + 144;
         zv_x = (0x6400u + zv[2 * q4]) | ((0x6400u + zv[2 * q4 + 1]) << 16);
         zv_y = (0x6400u + zv[2 * q4 + 8]) | ((0x6400u + zv[2 * q4 + 9]) << 16);
       }
@@ -816,7 +816,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
           // lane owns kD / 32 output columns of every head.
           constexpr int kV = kD / 32;
 #pragma unroll 1
-          for (int g0 = 0; g0 < ncols; g0 += 8) {
+          for (int c0 = 0; c0 < ncols; c0 += 8) {
             float Mg[8], Lg[8], acc[8][kV];
 #pragma unroll
             for (int gg = 0; gg < 8; ++gg) {
@@ -831,7 +831,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
               float mc[8], lc[8], ov[8][kV];
 #pragma unroll
               for (int gg = 0; gg < 8; ++gg) {
-                const int g = g0 + gg;
+                const int g = c0 + gg;
                 if (g < ncols) {
                   mc[gg] = __ldcg(sl + g);
                   lc[gg] = __ldcg(sl + C + g);
@@ -852,7 +852,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 #pragma unroll
               for (int gg = 0; gg < 8; ++gg) {
                 // multi-query: skip a share that saw no visible key of the column
-                if (g0 + gg < ncols && (!kMQ || mc[gg] != -INFINITY)) {
+                if (c0 + gg < ncols && (!kMQ || mc[gg] != -INFINITY)) {
                   const float mn = fmaxf(Mg[gg], mc[gg]);
                   const float a = fast_exp2(Mg[gg] - mn);  // 0 for the first contributor
                   const float w = fast_exp2(mc[gg] - mn) * lc[gg];
@@ -865,7 +865,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
             }
 #pragma unroll
             for (int gg = 0; gg < 8; ++gg) {
-              const int g = g0 + gg;
+              const int g = c0 + gg;
               if (g < ncols) {
                 const float inv = Lg[gg] > 0.0f ? 1.0f / Lg[gg] : 0.0f;
                 const long long row = out_row(g);
