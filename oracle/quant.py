@@ -175,3 +175,104 @@ def quantize_grouped(kv, group_size=128):
         return (np.zeros(kv.shape, np.uint8), np.zeros(kv.shape[:2], np.float32),
                 np.zeros(kv.shape[:2], np.uint8))
     return tuple(np.concatenate([p[i] for p in parts], axis=1) for i in range(3))
+
+
+# --------------------------------------------------------------------------
+# 4-bit KV: INT4 and FP4 (E2M1).  The pages list FP4 KV at a quarter of the
+# fp16 size ("ascendai.csdn.net" article, §三 1. KV Cache量化, the precision
+# table) and INT4 as the more aggressive step after INT8 ("大模型推理的KV
+# Cache管理…优化实战", §四).  They fix no scheme; the reading taken is the
+# same per-(token, head) symmetric absmax rule as INT8 / FP8:
+#
+# * INT4: s = a / 7, code = clamp(rint(x / s), -7, 7) (two's complement
+#   nibble; -8 unused);
+# * FP4 E2M1: s = a / 6, y = clamp(x / s, -6, 6), code = e2m1(y) rounded to
+#   nearest, ties to even.  E2M1 (OCP microscaling formats): 1 sign bit, 2
+#   exponent bits with bias 1, 1 mantissa bit; exponent field 0 is
+#   subnormal (0 or 0.5); magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6.
+# * a = 0 gives s = 0 and zero codes; arithmetic in IEEE fp32.
+# * Two codes per byte along head_dim: element 2k in the low nibble of byte
+#   k, element 2k + 1 in the high nibble.
+# --------------------------------------------------------------------------
+
+INT4_QMAX = 7
+FP4_E2M1_MAX = 6.0
+
+
+def e2m1_decode(codes):
+    """4-bit E2M1 codes (0..15) -> fp64 values."""
+    c = np.asarray(codes).astype(np.int64) & 0xF
+    sign = np.where(c & 0x8, -1.0, 1.0)
+    e = (c >> 1) & 0x3
+    m = c & 0x1
+    mag = np.where(e == 0, 0.5 * m, (1.0 + 0.5 * m) * np.exp2(e.astype(np.float64) - 1))
+    return sign * mag
+
+
+def e2m1_encode(y):
+    """Values with |y| <= 6 -> 4-bit E2M1 codes, round to nearest, ties to
+    even (the code with mantissa bit 0).  The sign of zero is kept."""
+    y = np.asarray(y, np.float64)
+    if np.any(np.abs(y) > FP4_E2M1_MAX) or np.any(np.isnan(y)):
+        raise ValueError("e2m1_encode expects finite |y| <= 6")
+    a = np.abs(y)
+    _, ex = np.frexp(a)                       # a in [2^(ex-1), 2^ex)
+    E = np.maximum(ex - 1, 0)                 # binade; below 1 the spacing is 0.5
+    quantum = np.ldexp(0.5, E)                # 1 mantissa bit
+    v = np.rint(a / quantum) * quantum        # exact scaling, half-to-even on the quantum grid
+    # encode v: 0 -> 0, 0.5 -> 1, 1 -> 2, 1.5 -> 3, 2 -> 4, 3 -> 5, 4 -> 6, 6 -> 7
+    lut = {0.0: 0, 0.5: 1, 1.0: 2, 1.5: 3, 2.0: 4, 3.0: 5, 4.0: 6, 6.0: 7}
+    mag = np.vectorize(lambda t: lut[float(t)], otypes=[np.int64])(v) if v.size else v.astype(np.int64)
+    code = np.where(np.signbit(y), mag | 0x8, mag)
+    return code.astype(np.uint8)
+
+
+def pack_nibbles(codes):
+    """[..., D] codes (0..15) -> [..., D / 2] uint8, element 2k in the low nibble."""
+    c = np.asarray(codes).astype(np.uint8) & 0xF
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack_nibbles(packed):
+    """[..., D / 2] uint8 -> [..., D] codes 0..15."""
+    p = np.asarray(packed, np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), np.uint8)
+    out[..., 0::2] = p & 0xF
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def quantize_int4(x):
+    """x [..., D] -> (packed codes uint8 [..., D / 2], scales fp32 [...])."""
+    x = np.asarray(x, np.float32)
+    a = absmax_rows(x)
+    s = (a / np.float32(INT4_QMAX)).astype(np.float32)
+    q = np.zeros(x.shape, np.int64)
+    nz = a > 0
+    y = (x[nz] / s[nz][..., None]).astype(np.float32)
+    q[nz] = np.clip(np.rint(y), -INT4_QMAX, INT4_QMAX).astype(np.int64)
+    return pack_nibbles(q & 0xF), s
+
+
+def quantize_fp4_e2m1(x):
+    """x [..., D] -> (packed codes uint8 [..., D / 2], scales fp32 [...])."""
+    x = np.asarray(x, np.float32)
+    a = absmax_rows(x)
+    s = (a / np.float32(FP4_E2M1_MAX)).astype(np.float32)
+    codes = np.zeros(x.shape, np.uint8)
+    nz = a > 0
+    y = (x[nz] / s[nz][..., None]).astype(np.float32)
+    y = np.clip(y, np.float32(-FP4_E2M1_MAX), np.float32(FP4_E2M1_MAX))
+    codes[nz] = e2m1_encode(y)
+    return pack_nibbles(codes), s
+
+
+def int4_values(packed):
+    """Packed INT4 codes -> fp64 code values (-7..7) [..., D]."""
+    c = unpack_nibbles(packed).astype(np.int64)
+    return np.where(c >= 8, c - 16, c).astype(np.float64)
+
+
+def fp4_values(packed):
+    """Packed E2M1 codes -> fp64 values [..., D]."""
+    return e2m1_decode(unpack_nibbles(packed))

@@ -198,3 +198,70 @@ def test_grouped_equals_per_row_for_any_group_size():
     # a reduction over the wrong axis would break the per-row extremes
     c, s, z = Q.quantize_grouped(kv, 128)
     assert np.all(c.max(-1) == 255) and np.all(c.min(-1) == 0)
+
+
+# ---- 4-bit: INT4 and FP4 E2M1 ----
+
+def test_e2m1_decode_table():
+    vals = Q.e2m1_decode(np.arange(16))
+    assert vals[:8].tolist() == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert vals[8:].tolist() == [-0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+
+
+def test_e2m1_encode_is_nearest_with_ties_to_even_by_brute_force():
+    grid = Q.e2m1_decode(np.arange(8))          # non-negative magnitudes, codes 0..7
+    rng = np.random.default_rng(7)
+    mids = (grid[:-1] + grid[1:]) / 2
+    y = np.concatenate([rng.uniform(-6, 6, 20000), grid, -grid, mids, -mids,
+                        np.nextafter(mids, 7), np.nextafter(mids, -1)])
+    codes = Q.e2m1_encode(y)
+    for v, c in zip(y.tolist(), codes.tolist()):
+        d = np.abs(abs(v) - grid)
+        best = np.flatnonzero(d == d.min())
+        want = best[0] if len(best) == 1 else best[best % 2 == 0][0]   # even mantissa bit
+        assert (c & 0x7) == want, (v, c)
+        if abs(v) > 0 or np.signbit(v):
+            assert (c >> 3) == int(np.signbit(v))
+
+
+def test_nibble_packing_layout():
+    c = np.array([[1, 2, 3, 4, 15, 0]], np.uint8)
+    p = Q.pack_nibbles(c)
+    assert p.tolist() == [[0x21, 0x43, 0x0F]]
+    assert np.array_equal(Q.unpack_nibbles(p), c)
+
+
+def test_int4_invariants_and_ties():
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal((300, 4, 128)).astype(np.float32)
+    p, s = Q.quantize_int4(x)
+    v = Q.int4_values(p)
+    assert p.shape == (300, 4, 64) and np.all(np.abs(v) <= 7)
+    top = np.take_along_axis(v, np.abs(x).argmax(-1)[..., None], -1)[..., 0]
+    assert np.all(np.abs(top) == 7)
+    err = np.abs(x - v * s[..., None])
+    assert np.all(err <= s[..., None] * (0.5 + 1e-5))
+    # scale 1: ties to even, negative codes as two's complement nibbles
+    p, s = Q.quantize_int4(np.array([[7.0, 2.5, 3.5, -2.5, -3.5, 0.5, -0.5, -7.0]], np.float32))
+    assert s[0] == 1.0
+    assert Q.int4_values(p)[0].tolist() == [7, 2, 4, -2, -4, 0, 0, -7]
+    assert Q.unpack_nibbles(p)[0].tolist() == [7, 2, 4, 14, 12, 0, 0, 9]
+
+
+def test_fp4_invariants_and_zero_rows():
+    rng = np.random.default_rng(9)
+    x = rng.standard_normal((300, 4, 64)).astype(np.float32)
+    p, s = Q.quantize_fp4_e2m1(x)
+    v = Q.fp4_values(p)
+    top = np.take_along_axis(v, np.abs(x).argmax(-1)[..., None], -1)[..., 0]
+    assert np.all(np.abs(top) == 6.0)
+    y = x.astype(np.float64) / s[..., None]
+    # within half a grid step of the nearest representable value
+    grid = np.array([0, 0.5, 1, 1.5, 2, 3, 4, 6])
+    step = np.where(np.abs(y) < 2, 0.5, np.where(np.abs(y) < 4, 1.0, 2.0))
+    assert np.all(np.abs(np.abs(v) - np.abs(y)) <= step / 2 + 1e-6)
+    p0, s0 = Q.quantize_fp4_e2m1(np.zeros((1, 8), np.float32))
+    assert np.all(p0 == 0) and s0[0] == 0
+    p, s = Q.quantize_fp4_e2m1(np.array([[6.0, 5.0, -5.0, 2.5, 0.25, 0.75, 1.25, 0.0]], np.float32))
+    assert s[0] == 1.0
+    assert Q.fp4_values(p)[0][:7].tolist() == [6.0, 4.0, -4.0, 2.0, 0.0, 1.0, 1.0]
