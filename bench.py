@@ -60,7 +60,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama3_8b", choices=sorted(I.WORKLOADS))
-    ap.add_argument("--cache", default=None, choices=[None, "int8", "fp8", "u8asym"])
+    ap.add_argument("--cache", default=None, choices=[None, "int8", "fp8", "u8asym", "int4", "fp4"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -189,7 +189,8 @@ def kv_bytes_per_token(hkv, d, cache):
     uint8 zero points of the asymmetric format."""
     if cache is None:
         return hkv * d * 2 * 2
-    return hkv * d * 2 + hkv * 2 * 4 + (hkv * 2 if cache == "u8asym" else 0)
+    codes = hkv * d * 2 // (2 if cache in ("int4", "fp4") else 1)
+    return codes + hkv * 2 * 4 + (hkv * 2 if cache == "u8asym" else 0)
 
 
 class DecodeWorkload:
@@ -222,8 +223,11 @@ class DecodeWorkload:
         order = torch.randperm(nb, generator=gen).tolist()
         self.alloc = P.BlockAllocator(nb, initial_free_order=order)
         elt = 1 if cache else 2
-        cdt = {None: self.dtype, "int8": torch.int8, "fp8": torch.uint8, "u8asym": torch.uint8}[cache]
-        self.k_cache = torch.empty((nb, self.hkv, 16, self.d), dtype=cdt, device=device)
+        cdt = {None: self.dtype, "int8": torch.int8, "fp8": torch.uint8, "u8asym": torch.uint8, "int4": torch.uint8,
+               "fp4": torch.uint8}[cache]
+        self.kv_format = cache if cache in ("int4", "fp4") else None
+        dc = self.d // 2 if self.kv_format else self.d
+        self.k_cache = torch.empty((nb, self.hkv, 16, dc), dtype=cdt, device=device)
         self.v_cache = torch.empty_like(self.k_cache)
         self.k_scale = self.v_scale = self.k_zero = self.v_zero = None
         if cache:
@@ -250,7 +254,7 @@ class DecodeWorkload:
                 slots, pairs = self.alloc.append(s, lens[s])
                 if pairs.shape[0]:
                     P.copy_blocks(self.k_cache, self.v_cache, pairs.to(device), self.k_scale, self.v_scale,
-                                  k_zero=self.k_zero, v_zero=self.v_zero)
+                                  k_zero=self.k_zero, v_zero=self.v_zero, kv_format=self.kv_format)
                 self._fill(slots)
         else:
             for s in range(self.B):
@@ -268,7 +272,7 @@ class DecodeWorkload:
             k = torch.randn((n, self.hkv, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
             v = torch.randn((n, self.hkv, self.d), generator=self.dg, device=self.dev, dtype=self.dtype)
             self.P.kv_cache_write(k, v, self.k_cache, self.v_cache, sl, self.k_scale, self.v_scale,
-                                  k_zero=self.k_zero, v_zero=self.v_zero)
+                                  k_zero=self.k_zero, v_zero=self.v_zero, kv_format=self.kv_format)
 
     def host_step(self):
         """Allocator work of one step: slots and CoW pairs for one new token per
@@ -294,24 +298,27 @@ class DecodeWorkload:
         n = 0
         if pairs is not None and pairs.numel():
             P.copy_blocks(self.k_cache, self.v_cache, pairs, self.k_scale, self.v_scale, k_zero=self.k_zero,
-                          v_zero=self.v_zero)
+                          v_zero=self.v_zero, kv_format=self.kv_format)
             n += 1
         P.kv_cache_write(k, v, self.k_cache, self.v_cache, slots, self.k_scale, self.v_scale, k_zero=self.k_zero,
-                         v_zero=self.v_zero)
+                         v_zero=self.v_zero, kv_format=self.kv_format)
         self.decode(q, bt, cl, maxc, out, ws)
         return n + 2
 
     def decode(self, q, bt, cl, maxc, out, ws):
         self.P.paged_attention_decode(q, self.k_cache, self.v_cache, bt, cl, self.scale, self.k_scale,
                                       self.v_scale, max_context_len=maxc, out=out, workspace=ws,
-                                      k_zero=self.k_zero, v_zero=self.v_zero)
+                                      k_zero=self.k_zero, v_zero=self.v_zero, kv_format=self.kv_format)
+
+    def cache_code(self):
+        return self.P.cache_code(self.k_cache, self.k_zero, self.kv_format)
 
     # shapes and plan of one step (the multi-query workload overrides these)
     q_rows = property(lambda self: self.B)
     mq = False
 
     def plan(self, maxc):
-        return self.P.decode_plan(self.B, self.hq, self.hkv, self.d, maxc, self.k_cache.dtype)
+        return self.P.decode_plan(self.B, self.hq, self.hkv, self.d, maxc, self.cache_code())
 
     def flops(self, cl):
         """Tensor-core FLOPs of the step's attention (2 per multiply-add, QK
@@ -350,8 +357,11 @@ class MultiQueryWorkload(DecodeWorkload):
         self.nb = nb
         order = torch.randperm(nb, generator=gen).tolist()
         self.alloc = P.BlockAllocator(nb, initial_free_order=order)
-        cdt = {None: self.dtype, "int8": torch.int8, "fp8": torch.uint8, "u8asym": torch.uint8}[cache]
-        self.k_cache = torch.empty((nb, self.hkv, 16, self.d), dtype=cdt, device=device)
+        cdt = {None: self.dtype, "int8": torch.int8, "fp8": torch.uint8, "u8asym": torch.uint8, "int4": torch.uint8,
+               "fp4": torch.uint8}[cache]
+        self.kv_format = cache if cache in ("int4", "fp4") else None
+        dc = self.d // 2 if self.kv_format else self.d
+        self.k_cache = torch.empty((nb, self.hkv, 16, dc), dtype=cdt, device=device)
         self.v_cache = torch.empty_like(self.k_cache)
         self.k_scale = self.v_scale = self.k_zero = self.v_zero = None
         if cache:
@@ -399,10 +409,10 @@ class MultiQueryWorkload(DecodeWorkload):
         self.P.paged_attention_multi_query(q, self.k_cache, self.v_cache, bt, cl, self.qsl_dev, self.scale,
                                            max_query_len=self.max_q, max_context_len=maxc, k_scale=self.k_scale,
                                            v_scale=self.v_scale, k_zero=self.k_zero, v_zero=self.v_zero, out=out,
-                                           workspace=ws)
+                                           workspace=ws, kv_format=self.kv_format)
 
     def plan(self, maxc):
-        return self.P.multi_query_plan(self.B, self.hq, self.hkv, self.d, maxc, self.max_q, self.k_cache.dtype)
+        return self.P.multi_query_plan(self.B, self.hq, self.hkv, self.d, maxc, self.max_q, self.cache_code())
 
     def flops(self, cl):
         # new token t of n sees ctx - n + t + 1 keys
@@ -638,6 +648,9 @@ def oracle_sample(name, cache, budget_s=10.0, seed_offset=0):
         kind = case["cache_kind"]
         if kind == "fp8":
             kc, vc = OQ.e4m3_decode(case["k_cache"].numpy()), OQ.e4m3_decode(case["v_cache"].numpy())
+        elif kind in ("int4", "fp4"):
+            dec = OQ.int4_values if kind == "int4" else OQ.fp4_values
+            kc, vc = dec(case["k_cache"].numpy()), dec(case["v_cache"].numpy())
         else:
             kc = case["k_cache"].to(torch.float64).numpy()
             vc = case["v_cache"].to(torch.float64).numpy()
@@ -743,7 +756,8 @@ def main():
         "warmup": r["W"], "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": {None: "bf16" if wl.dtype == torch.bfloat16 else "f16",
                                        "int8": "int8 KV / fp16 mma", "fp8": "fp8e4m3 KV / fp16 mma",
-                                       "u8asym": "u8 KV with zero point / fp16 mma"}[args.cache],
+                                       "u8asym": "u8 KV with zero point / fp16 mma",
+                                       "int4": "int4 KV / fp16 mma", "fp4": "fp4e2m1 KV / fp16 mma"}[args.cache],
         "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[args.workload], "name": args.workload, "batch": wl.B,
                    "q_heads": wl.hq, "kv_heads": wl.hkv, "head_dim": wl.d, "block_size": 16,

@@ -33,6 +33,7 @@
  * Cache layout (per [P-WMRH] §二 KVCacheBlock: one block stores
  * [num_heads, block_size, head_dim]):
  *   k_cache, v_cache : [num_blocks, num_kv_heads, 16, head_dim] of cache_dtype
+ *                      ([..., head_dim / 2] bytes for the 4-bit formats)
  *   k_scale, v_scale : [num_blocks, num_kv_heads, 16] fp32 (quantised caches
  *                      only; one scale per token and KV head)
  *   k_zero, v_zero   : [num_blocks, num_kv_heads, 16] uint8 (PKV_U8ASYM only;
@@ -69,6 +70,10 @@ extern "C" {
 #define PKV_FP8E4M3 3   /* OCP FP8 E4M3 (e4m3fn) codes, absmax maps to 448 */
 #define PKV_U8ASYM  4   /* uint8 codes, min/max over head_dim, with a
                            per-(token, head) scale and uint8 zero point     */
+#define PKV_I4      5   /* int4 codes, symmetric absmax, range [-7, 7],
+                           two per byte (element 2k in the low nibble)      */
+#define PKV_FP4E2M1 6   /* OCP FP4 E2M1 codes, absmax maps to 6, two per
+                           byte (element 2k in the low nibble)              */
 
 /* ---- device status bits (pkv_device_status) ----------------------------- */
 #define PKV_DEV_BAD_SLOT     1u   /* slot >= num_blocks * 16 (write skipped)       */
@@ -93,8 +98,8 @@ int pkv_version(void);
  *                 (PKV_F16 or PKV_BF16).
  * k_cache, v_cache : device, cache layout above, cache_dtype.
  * k_scale, v_scale : device fp32 scale arrays; required (non-NULL) iff
- *                 cache_dtype is PKV_I8, PKV_FP8E4M3 or PKV_U8ASYM, else
- *                 ignored.
+ *                 cache_dtype is quantised (PKV_I8, PKV_FP8E4M3, PKV_U8ASYM,
+ *                 PKV_I4, PKV_FP4E2M1), else ignored.
  * k_zero, v_zero : device uint8 zero-point arrays; required iff cache_dtype
  *                 is PKV_U8ASYM, else ignored (may be NULL).
  * slot_mapping  : device int64 [num_tokens]; -1 skips the token.  Slots of
@@ -112,6 +117,9 @@ int pkv_version(void);
  *   s = 0 (a constant row) stores s = 0, z = 0 and zero codes.
  * The page's 128-token grouped form leaves every (token, head) row's
  * statistics unchanged (they are taken over head_dim), so it stores the same.
+ * PKV_I4 / PKV_FP4E2M1 ([P-ASC] §三 FP4 KV at a quarter of fp16; [P-WMRH] §四
+ * INT4): the absmax rule with s = a / 7 (INT4, codes clamped to [-7, 7]) or
+ * s = a / 6 (E2M1, x / s clamped to [-6, 6], round to nearest even).
  * Alignment: k, v, k_cache, v_cache 16 bytes; scales 4 bytes.
  */
 int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cache,

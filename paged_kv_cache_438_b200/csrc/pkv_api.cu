@@ -25,8 +25,12 @@ namespace {
 std::atomic<int> g_validate{0};
 
 bool is16(int dt) { return dt == PKV_F16 || dt == PKV_BF16; }
-bool is8(int dt) { return dt == PKV_I8 || dt == PKV_FP8E4M3 || dt == PKV_U8ASYM; }
+bool is4(int dt) { return dt == PKV_I4 || dt == PKV_FP4E2M1; }
+// quantised formats: per-token scales, 8 or 4 bits per element
+bool isq(int dt) { return dt == PKV_I8 || dt == PKV_FP8E4M3 || dt == PKV_U8ASYM || is4(dt); }
 bool has_zero(int dt) { return dt == PKV_U8ASYM; }
+// bytes of one token's K (or V) row in the cache
+int row_bytes(int dt, int head_dim) { return is16(dt) ? 2 * head_dim : (is4(dt) ? head_dim / 2 : head_dim); }
 int elt_size(int dt) { return is16(dt) ? 2 : 1; }
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
@@ -65,19 +69,20 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 2-D view of a cache: rows of head_dim elements, one row per (block, head,
-// token); box = one 16-token block x (128 bytes or the whole row) with the
-// matching swizzle.
-int make_cache_map(CUtensorMap* map, const void* cache, int head_dim, int elt, long long rows) {
+// 2-D view of a cache: one row of row_bytes per (block, head, token), in
+// elements of elt bytes (2 for 16-bit caches, else bytes); box = one 16-token
+// block x (128 bytes or the whole row) with the matching swizzle.
+int make_cache_map(CUtensorMap* map, const void* cache, int row_bytes, int elt, long long rows) {
   auto fn = encode_fn();
   if (!fn) return fail(PKV_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
-  const int row_bytes = head_dim * elt;
   const int tile_bytes = row_bytes < 128 ? row_bytes : 128;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(head_dim), static_cast<cuuint64_t>(rows)};
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(row_bytes / elt), static_cast<cuuint64_t>(rows)};
   cuuint64_t strides[1] = {static_cast<cuuint64_t>(row_bytes)};
   cuuint32_t box[2] = {static_cast<cuuint32_t>(tile_bytes / elt), 16u};
   cuuint32_t estr[2] = {1u, 1u};
-  const CUtensorMapSwizzle swz = tile_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  const CUtensorMapSwizzle swz = tile_bytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                 : tile_bytes == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                                    : CU_TENSOR_MAP_SWIZZLE_32B;
   CUresult r = fn(map, elt == 2 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                   const_cast<void*>(cache), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -130,7 +135,7 @@ int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int r
   // long contexts keep HBM busiest that way, short or L2-resident work wants
   // the extra warps).
   const long long sms = sm_count();
-  const int warps = (!is8(cache_dtype) && t_max / (8 * sms) >= kLongStreamBlocks) ? 4 : 8;
+  const int warps = (!isq(cache_dtype) && t_max / (8 * sms) >= kLongStreamBlocks) ? 4 : 8;
   long long nw;
   if (req_tokens > 0) {
     if (req_tokens % 16 != 0) return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d is not a multiple of 16", req_tokens);
@@ -232,7 +237,7 @@ template <int kD, int kCT, bool kMQ>
 int dispatch_nt_q(const CUtensorMap& km, const CUtensorMap& vm, const pkv::DecodeParams& p, bool q_bf16,
                   cudaStream_t st) {
   const bool nt2 = (kMQ ? p.tile_cols : p.group) > 8;
-  if constexpr (pkv::DecodeTraits<kD, kCT>::k8bit) {
+  if constexpr (pkv::DecodeTraits<kD, kCT>::kQuant) {
     if (q_bf16)
       return nt2 ? launch_decode<kD, kCT, 2, true, kMQ>(km, vm, p, st)
                  : launch_decode<kD, kCT, 1, true, kMQ>(km, vm, p, st);
@@ -255,6 +260,8 @@ int dispatch_ct(int ct, const CUtensorMap& km, const CUtensorMap& vm, const pkv:
     case PKV_I8: return dispatch_nt_q<kD, pkv::kI8, kMQ>(km, vm, p, q_bf16, st);
     case PKV_FP8E4M3: return dispatch_nt_q<kD, pkv::kFP8, kMQ>(km, vm, p, q_bf16, st);
     case PKV_U8ASYM: return dispatch_nt_q<kD, pkv::kU8, kMQ>(km, vm, p, q_bf16, st);
+    case PKV_I4: return dispatch_nt_q<kD, pkv::kI4, kMQ>(km, vm, p, q_bf16, st);
+    case PKV_FP4E2M1: return dispatch_nt_q<kD, pkv::kFP4, kMQ>(km, vm, p, q_bf16, st);
   }
   return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", ct);
 }
@@ -299,12 +306,12 @@ int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cach
   if (!is16(in_dtype)) return fail(PKV_ERR_UNSUPPORTED, "input dtype %d (need PKV_F16 or PKV_BF16)", in_dtype);
   if (is16(cache_dtype) && cache_dtype != in_dtype)
     return fail(PKV_ERR_UNSUPPORTED, "a 16-bit cache must have the input's dtype");
-  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  if (!is16(cache_dtype) && !isq(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
   if (num_tokens == 0) return ok();
   if (!k || !v || !k_cache || !v_cache || !slot_mapping) return fail(PKV_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(k, 16) || !aligned(v, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16))
     return fail(PKV_ERR_INVALID_ARG, "k, v and caches must be 16-byte aligned");
-  if (is8(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4)))
+  if (isq(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 4) || !aligned(v_scale, 4)))
     return fail(PKV_ERR_INVALID_ARG, "quantised caches need k_scale and v_scale");
   if (has_zero(cache_dtype) && (!k_zero || !v_zero))
     return fail(PKV_ERR_INVALID_ARG, "PKV_U8ASYM caches need k_zero and v_zero");
@@ -343,11 +350,13 @@ int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cach
                                                              slot_mapping, num_tokens, num_kv_heads, num_blocks)
 #define PKV_QW_FMT(D, F) \
   do { if (bf) PKV_QW(D, F, true); else PKV_QW(D, F, false); } while (0)
-#define PKV_QW_D(D)                                               \
-  do {                                                            \
-    if (cache_dtype == PKV_FP8E4M3) PKV_QW_FMT(D, PKV_FP8E4M3);   \
-    else if (cache_dtype == PKV_U8ASYM) PKV_QW_FMT(D, PKV_U8ASYM); \
-    else PKV_QW_FMT(D, PKV_I8);                                   \
+#define PKV_QW_D(D)                                                 \
+  do {                                                              \
+    if (cache_dtype == PKV_FP8E4M3) PKV_QW_FMT(D, PKV_FP8E4M3);     \
+    else if (cache_dtype == PKV_U8ASYM) PKV_QW_FMT(D, PKV_U8ASYM);   \
+    else if (cache_dtype == PKV_I4) PKV_QW_FMT(D, PKV_I4);           \
+    else if (cache_dtype == PKV_FP4E2M1) PKV_QW_FMT(D, PKV_FP4E2M1); \
+    else PKV_QW_FMT(D, PKV_I8);                                     \
   } while (0)
     if (head_dim == 128) PKV_QW_D(128);
     else PKV_QW_D(64);
@@ -366,7 +375,7 @@ int pkv_decode_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_di
   if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || max_context_len < 0)
     return fail(PKV_ERR_INVALID_ARG, "bad sizes");
   if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
-  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  if (!is16(cache_dtype) && !isq(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
   Plan pl{};
   int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens, &pl);
   if (rc != PKV_OK) return rc;
@@ -409,7 +418,7 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
   if (G > 16) return fail(PKV_ERR_UNSUPPORTED, "query group %d > 16", G);
   if (!is16(q_dtype)) return fail(PKV_ERR_UNSUPPORTED, "q dtype %d", q_dtype);
   if (is16(cache_dtype) && q_dtype != cache_dtype) return fail(PKV_ERR_UNSUPPORTED, "q dtype must match a 16-bit cache");
-  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  if (!is16(cache_dtype) && !isq(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
   if (!std::isfinite(scale)) return fail(PKV_ERR_INVALID_ARG, "scale is not finite");
   if (sliding_window < 0) return fail(PKV_ERR_INVALID_ARG, "sliding_window %d < 0", sliding_window);
   if (static_cast<long long>(num_blocks) * num_kv_heads * 16 >= (1LL << 31))
@@ -421,7 +430,7 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
     return fail(PKV_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(PKV_ERR_INVALID_ARG, "caches must be 16-byte aligned");
   if (!aligned(q, 4) || !aligned(out, 4)) return fail(PKV_ERR_INVALID_ARG, "q and out must be 4-byte aligned");
-  if (is8(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 16) || !aligned(v_scale, 16)))
+  if (isq(cache_dtype) && (!k_scale || !v_scale || !aligned(k_scale, 16) || !aligned(v_scale, 16)))
     return fail(PKV_ERR_INVALID_ARG, "quantised caches need 16-byte aligned k_scale and v_scale");
   if (has_zero(cache_dtype) && (!k_zero || !v_zero || !aligned(k_zero, 16) || !aligned(v_zero, 16)))
     return fail(PKV_ERR_INVALID_ARG, "PKV_U8ASYM caches need 16-byte aligned k_zero and v_zero");
@@ -460,8 +469,8 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
   }
   CUtensorMap km, vm;
   const long long rows = static_cast<long long>(num_blocks) * num_kv_heads * 16;
-  rc = make_cache_map(&km, k_cache, head_dim, elt_size(cache_dtype), rows);
-  if (rc == PKV_OK) rc = make_cache_map(&vm, v_cache, head_dim, elt_size(cache_dtype), rows);
+  rc = make_cache_map(&km, k_cache, row_bytes(cache_dtype, head_dim), elt_size(cache_dtype), rows);
+  if (rc == PKV_OK) rc = make_cache_map(&vm, v_cache, row_bytes(cache_dtype, head_dim), elt_size(cache_dtype), rows);
   if (rc != PKV_OK) return rc;
 
   pkv::DecodeParams p{};
@@ -531,7 +540,7 @@ int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int he
     return fail(PKV_ERR_INVALID_ARG, "bad sizes");
   if (num_q_heads % num_kv_heads != 0) return fail(PKV_ERR_INVALID_ARG, "num_q_heads %% num_kv_heads != 0");
   if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
-  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  if (!is16(cache_dtype) && !isq(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
   Plan pl{};
   int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens,
                      &pl, std::max(max_query_len, 1));
@@ -563,11 +572,11 @@ int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale
   if (num_pairs < 0 || num_kv_heads <= 0 || num_blocks <= 0) return fail(PKV_ERR_INVALID_ARG, "bad sizes");
   if (block_size != 16) return fail(PKV_ERR_UNSUPPORTED, "block_size must be 16 (got %d)", block_size);
   if (head_dim != 64 && head_dim != 128) return fail(PKV_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
-  if (!is16(cache_dtype) && !is8(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
+  if (!is16(cache_dtype) && !isq(cache_dtype)) return fail(PKV_ERR_UNSUPPORTED, "cache dtype %d", cache_dtype);
   if (num_pairs == 0) return ok();
   if (!k_cache || !v_cache || !src_dst_pairs) return fail(PKV_ERR_INVALID_ARG, "NULL pointer");
   if (!aligned(k_cache, 16) || !aligned(v_cache, 16)) return fail(PKV_ERR_INVALID_ARG, "caches must be 16-byte aligned");
-  const bool q8 = is8(cache_dtype);
+  const bool q8 = isq(cache_dtype);
   if (q8 && (!k_scale || !v_scale || !aligned(k_scale, 16) || !aligned(v_scale, 16)))
     return fail(PKV_ERR_INVALID_ARG, "quantised caches need 16-byte aligned k_scale and v_scale");
   const bool zp = has_zero(cache_dtype);
@@ -589,7 +598,7 @@ int pkv_copy_blocks(void* k_cache, void* v_cache, float* k_scale, float* v_scale
     for (int32_t b : dsts)
       if (srcs.count(b)) return fail(PKV_ERR_INVALID_ARG, "block %d is both a source and a destination", b);
   }
-  const long long words = static_cast<long long>(num_kv_heads) * 16 * head_dim * elt_size(cache_dtype) / 16;
+  const long long words = static_cast<long long>(num_kv_heads) * 16 * row_bytes(cache_dtype, head_dim) / 16;
   const int swords = q8 ? num_kv_heads * 4 : 0;
   const int zwords = zp ? num_kv_heads : 0;
   const int grid = std::min(num_pairs, 16 * sm_count());

@@ -57,21 +57,25 @@
 
 namespace pkv {
 
-enum CacheType : int { kF16 = PKV_F16, kBF16 = PKV_BF16, kI8 = PKV_I8, kFP8 = PKV_FP8E4M3, kU8 = PKV_U8ASYM };
+enum CacheType : int {
+  kF16 = PKV_F16, kBF16 = PKV_BF16, kI8 = PKV_I8, kFP8 = PKV_FP8E4M3, kU8 = PKV_U8ASYM, kI4 = PKV_I4, kFP4 = PKV_FP4E2M1
+};
 
 constexpr int round_up_c(int x, int m) { return (x + m - 1) / m * m; }
 
 template <int kD, int kCT>
 struct DecodeTraits {
   static constexpr bool k8bit = (kCT == kI8 || kCT == kFP8 || kCT == kU8);
-  static constexpr int kElt = k8bit ? 1 : 2;
-  static constexpr int kRowBytes = kD * kElt;                       // one token's K (or V) row
+  static constexpr bool k4bit = (kCT == kI4 || kCT == kFP4);
+  static constexpr bool kQuant = k8bit || k4bit;                    // per-token scales, fp16 math
+  static constexpr int kElt = kQuant ? 1 : 2;                       // bytes per tensor-map element
+  static constexpr int kRowBytes = k4bit ? kD / 2 : kD * kElt;      // one token's K (or V) row
   static constexpr int kTileBytes = kRowBytes < 128 ? kRowBytes : 128;  // TMA box width == swizzle span
   static constexpr int kNumColTiles = kRowBytes / kTileBytes;
   static constexpr int kColTileBytes = 16 * kTileBytes;             // 16 tokens x one column tile
   static constexpr int kChunksPerTileRow = kTileBytes / 16;
   static constexpr int kKVBytes = 16 * kRowBytes;                   // one block of one head, K or V
-  static constexpr int kScaleBytes = k8bit ? 64 : 0;                // 16 fp32 scales
+  static constexpr int kScaleBytes = kQuant ? 64 : 0;               // 16 fp32 scales
   static constexpr int kZeroBytes = kCT == kU8 ? 16 : 0;            // 16 uint8 zero points
   // stage layout: K tile, V tile, K scales, V scales, K zero points, V zero points
   static constexpr int kStageTx = 2 * kKVBytes + 2 * kScaleBytes + 2 * kZeroBytes;  // bytes landing per stage
@@ -80,7 +84,7 @@ struct DecodeTraits {
   // One CTA per SM.  Its warps (4 or 8, chosen per call) share this many
   // bytes of copy ring: 4 warps x 4 stages or 8 warps x 2 stages of 8 KiB for
   // bf16 / fp16 at head_dim 128; 8-bit caches keep 8 warps and more stages.
-  static constexpr int kRingBudget = k8bit ? 160 * 1024 : 128 * 1024;
+  static constexpr int kRingBudget = kQuant ? 160 * 1024 : 128 * 1024;
   static int ring_depth(int warps) {
     const int r = kRingBudget / (warps * kStageBytes);
     return r < 2 ? 2 : (r > 8 ? 8 : r);
@@ -146,8 +150,10 @@ __device__ __forceinline__ uint32_t swz(int t, int c) {
   int x;
   if constexpr (Tr::kTileBytes == 128) {
     x = cc ^ (t & 7);
-  } else {
+  } else if constexpr (Tr::kTileBytes == 64) {
     x = cc ^ ((t >> 1) & 3);
+  } else {  // 32-byte rows, 32-byte swizzle
+    x = cc ^ ((t >> 2) & 1);
   }
   return static_cast<uint32_t>(ct * Tr::kColTileBytes + t * Tr::kTileBytes + (x << 4));
 }
@@ -165,7 +171,7 @@ __device__ __forceinline__ void store_out(void* out, long long idx, float v) {
 template <int kCT, bool kQBF16>
 __device__ __forceinline__ uint32_t load_q_pair(const void* q, long long idx) {
   const uint32_t raw = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(q) + idx);
-  if constexpr (DecodeTraits<64, kCT>::k8bit) {
+  if constexpr (DecodeTraits<64, kCT>::kQuant) {
     if constexpr (kQBF16) {
       const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&raw);
       const __half2 h = __float22half2_rn(__bfloat1622float2(b));
@@ -173,6 +179,21 @@ __device__ __forceinline__ uint32_t load_q_pair(const void* q, long long idx) {
     }
   }
   return raw;
+}
+
+// Two query elements (d0, d1), not adjacent, as an fp16x2 B operand pair
+// (4-bit caches; the mma runs in fp16).
+template <bool kQBF16>
+__device__ __forceinline__ uint32_t load_q_two(const void* q, long long i0, long long i1) {
+  const uint16_t* p = reinterpret_cast<const uint16_t*>(q);
+  const uint16_t a = p[i0], b = p[i1];
+  __half2 h;
+  if constexpr (kQBF16) {
+    h = __floats2half2_rn(__bfloat162float(__ushort_as_bfloat16(a)), __bfloat162float(__ushort_as_bfloat16(b)));
+  } else {
+    h = __halves2half2(__ushort_as_half(a), __ushort_as_half(b));
+  }
+  return *reinterpret_cast<uint32_t*>(&h);
 }
 
 __device__ __forceinline__ void query_range(const DecodeParams& p, int s, int ctx, int& q0, int& q1, int& n,
@@ -313,8 +334,10 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
                         const DecodeParams p) {
   using Tr = DecodeTraits<kD, kCT>;
   constexpr bool k8 = Tr::k8bit;
+  constexpr bool k4 = Tr::k4bit;
+  constexpr bool kQt = Tr::kQuant;
   constexpr bool kMmaBF16 = (kCT == kBF16);
-  constexpr bool kOutBF16 = k8 ? kQBF16 : (kCT == kBF16);
+  constexpr bool kOutBF16 = kQt ? kQBF16 : (kCT == kBF16);
   const int kW = blockDim.x >> 5;  // warps of this CTA
   const int kR = p.ring;           // stages per warp (<= 8)
   constexpr int kKS = kD / 16;  // k-steps of S^T = K Q^T
@@ -402,7 +425,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       tma_load_2d(st + ct * Tr::kColTileBytes, &kmap, x, row0, bar);
       tma_load_2d(st + Tr::kKVBytes + ct * Tr::kColTileBytes, &vmap, x, row0, bar);
     }
-    if constexpr (k8) {
+    if constexpr (kQt) {
       bulk_load(st + 2 * Tr::kKVBytes, p.k_scale + row0, 64, bar);
       bulk_load(st + 2 * Tr::kKVBytes + 64, p.v_scale + row0, 64, bar);
     }
@@ -483,12 +506,29 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       }
 #pragma unroll
       for (int jj = 0; jj < kKS; ++jj) {
-        // 16-bit K: k-index 2q,2q+1 -> d 16jj+2q.. ; 2q+8.. -> d 16jj+8+2q..
-        // 8-bit K:  k-index 2q,2q+1 -> d 16jj+4q.. ; 2q+8.. -> d 16jj+4q+2..
-        const int da = k8 ? 16 * jj + 4 * q4 : 16 * jj + 2 * q4;
-        const int db = k8 ? da + 2 : da + 8;
-        qf[nt][jj][0] = valid ? load_q_pair<kCT, kQBF16>(p.q, qrow + da) : 0u;
-        qf[nt][jj][1] = valid ? load_q_pair<kCT, kQBF16>(p.q, qrow + db) : 0u;
+        if constexpr (k4) {
+          // 4-bit K: k-step jj is half (jj & 1) of 32-code chunk jj / 2; a
+          // lane's word holds d = 32(jj/2) + 8q .. + 7 and the widening
+          // pairs them as (0,4)(1,5)(2,6)(3,7) for INT4, (0,1)(2,3)(4,5)(6,7)
+          // for E2M1; k-slots 2q,2q+1 take the first pair of the step,
+          // 2q+8,2q+9 the second
+          const long long b8 = qrow + 32 * (jj >> 1) + 8 * q4;
+          int e0, e1, e2, e3;  // d offsets of slots 2q, 2q+1, 2q+8, 2q+9
+          if constexpr (kCT == kI4) {
+            e0 = 2 * (jj & 1); e1 = e0 + 4; e2 = e0 + 1; e3 = e0 + 5;
+          } else {
+            e0 = 4 * (jj & 1); e1 = e0 + 1; e2 = e0 + 2; e3 = e0 + 3;
+          }
+          qf[nt][jj][0] = valid ? load_q_two<kQBF16>(p.q, b8 + e0, b8 + e1) : 0u;
+          qf[nt][jj][1] = valid ? load_q_two<kQBF16>(p.q, b8 + e2, b8 + e3) : 0u;
+        } else {
+          // 16-bit K: k-index 2q,2q+1 -> d 16jj+2q.. ; 2q+8.. -> d 16jj+8+2q..
+          // 8-bit K:  k-index 2q,2q+1 -> d 16jj+4q.. ; 2q+8.. -> d 16jj+4q+2..
+          const int da = k8 ? 16 * jj + 4 * q4 : 16 * jj + 2 * q4;
+          const int db = k8 ? da + 2 : da + 8;
+          qf[nt][jj][0] = valid ? load_q_pair<kCT, kQBF16>(p.q, qrow + da) : 0u;
+          qf[nt][jj][1] = valid ? load_q_pair<kCT, kQBF16>(p.q, qrow + db) : 0u;
+        }
       }
       m_run[nt][0] = m_run[nt][1] = -INFINITY;
       l_run[nt][0] = l_run[nt][1] = 0.0f;
@@ -525,7 +565,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0.0f;
-    if constexpr (!k8) {
+    if constexpr (!kQt) {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
       for (int jj = 0; jj < kKS; ++jj) {
@@ -534,6 +574,31 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt)
           mma_16816<kMmaBF16>((jj & 1) ? sacc2[nt] : sacc[nt], a0, a1, a2, a3, qf[nt][jj][0], qf[nt][jj][1]);
+      }
+    } else if constexpr (k4) {
+      // one ldmatrix.x4 = tokens 0-7 / 8-15 of two 32-code chunks (4 k-steps)
+      const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int c = 0; c < kD / 32; c += 2) {
+        uint32_t w[4];
+        ldsm_x4(st + swz<Tr>(t, c + (lane >> 4)), w[0], w[1], w[2], w[3]);
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t x[4], y[4];  // fp16 pairs of token r (x) and token r + 8 (y)
+          if constexpr (kCT == kI4) {
+            i4x8_to_h2x4(w[2 * c2], x);
+            i4x8_to_h2x4(w[2 * c2 + 1], y);
+          } else {
+            e2m1x8_to_h2x4(w[2 * c2], x);
+            e2m1x8_to_h2x4(w[2 * c2 + 1], y);
+          }
+          const int jj = 2 * (c + c2);
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            mma_16816<false>(sacc[nt], x[0], y[0], x[1], y[1], qf[nt][jj][0], qf[nt][jj][1]);
+            mma_16816<false>(sacc2[nt], x[2], y[2], x[3], y[3], qf[nt][jj + 1][0], qf[nt][jj + 1][1]);
+          }
+        }
       }
     } else {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -581,7 +646,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     // ---- scale, mask, online softmax (base 2) ----
     float f_r = p.qk_scale_log2, f_r8 = p.qk_scale_log2;
     float vs_r = 1.0f, vs_r8 = 1.0f;
-    if constexpr (k8) {
+    if constexpr (kQt) {
       const float* sc = reinterpret_cast<const float*>(base_ptr + (st - smem_base) + 2 * Tr::kKVBytes);
       f_r *= sc[r];
       f_r8 *= sc[r + 8];
@@ -647,7 +712,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 
     // ---- O^T += V^T . P^T ----
     const uint32_t vt = st + Tr::kKVBytes;
-    if constexpr (!k8) {
+    if constexpr (!kQt) {
       const int t = (lane & 7) + (lane >> 4) * 8;
 #pragma unroll
       for (int i = 0; i < kMT; ++i) {
@@ -655,6 +720,43 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
         ldsm_x4_t(vt + swz<Tr>(t, 2 * i + ((lane >> 3) & 1)), a0, a1, a2, a3);
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) mma_16816<kMmaBF16>(o[i][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+      }
+    } else if constexpr (k4) {
+      // transposed load: a lane's word holds tokens 2q (bytes 0-1) and 2q+1
+      // (bytes 2-3) at d = 32c + 4r .. + 3; pairs (token 2q, token 2q+1) at
+      // one d are (n0,n4) (n1,n5) (n2,n6) (n3,n7): m-tile 2c takes d offsets
+      // 0 / 1 as rows r / r + 8, m-tile 2c + 1 offsets 2 / 3
+      const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+      for (int c = 0; c < kD / 32; c += 2) {
+        uint32_t w[4];
+        ldsm_x4_t(vt + swz<Tr>(t, c + (lane >> 4)), w[0], w[1], w[2], w[3]);
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {
+          uint32_t x[4], y[4];  // x: tokens 0-7 of the block, y: tokens 8-15
+          if constexpr (kCT == kI4) {
+            i4x8_to_h2x4(w[2 * c2], x);
+            i4x8_to_h2x4(w[2 * c2 + 1], y);
+          } else {
+            uint32_t a[4], b[4];
+            e2m1x8_to_h2x4(w[2 * c2], a);
+            e2m1x8_to_h2x4(w[2 * c2 + 1], b);
+            x[0] = prmt(a[0], a[2], 0x5410u);
+            x[1] = prmt(a[0], a[2], 0x7632u);
+            x[2] = prmt(a[1], a[3], 0x5410u);
+            x[3] = prmt(a[1], a[3], 0x7632u);
+            y[0] = prmt(b[0], b[2], 0x5410u);
+            y[1] = prmt(b[0], b[2], 0x7632u);
+            y[2] = prmt(b[1], b[3], 0x5410u);
+            y[3] = prmt(b[1], b[3], 0x7632u);
+          }
+          const int i = 2 * (c + c2);
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            mma_16816<false>(o[i][nt], x[0], x[1], y[0], y[1], pb[nt][0], pb[nt][1]);
+            mma_16816<false>(o[i + 1][nt], x[2], x[3], y[2], y[3], pb[nt][0], pb[nt][1]);
+          }
+        }
       }
     } else {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
@@ -752,8 +854,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
             const long long row = out_row(g);
 #pragma unroll
             for (int i = 0; i < kMT; ++i) {
-              const int d0 = k8 ? 16 * i + 2 * r : 16 * i + r;
-              const int d1 = k8 ? d0 + 1 : d0 + 8;
+              const int d0 = k4 ? 32 * (i >> 1) + 4 * r + 2 * (i & 1) : (k8 ? 16 * i + 2 * r : 16 * i + r);
+              const int d1 = kQt ? d0 + 1 : d0 + 8;
               store_out<kOutBF16>(p.out, row * kD + d0, o[i][nt][c] * inv);
               store_out<kOutBF16>(p.out, row * kD + d1, o[i][nt][2 + c] * inv);
             }
@@ -777,8 +879,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
             float* og = slot + ml + g * kD;
 #pragma unroll
             for (int i = 0; i < kMT; ++i) {
-              const int d0 = k8 ? 16 * i + 2 * r : 16 * i + r;
-              const int d1 = k8 ? d0 + 1 : d0 + 8;
+              const int d0 = k4 ? 32 * (i >> 1) + 4 * r + 2 * (i & 1) : (k8 ? 16 * i + 2 * r : 16 * i + r);
+              const int d1 = kQt ? d0 + 1 : d0 + 8;
               og[d0] = o[i][nt][c] * inv;
               og[d1] = o[i][nt][2 + c] * inv;
             }

@@ -184,6 +184,42 @@ __device__ __forceinline__ uint32_t u8pair_minus_zero(uint32_t w, uint32_t sel, 
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// (a & b) | c in one instruction.
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// Eight signed INT4 codes n0..n7 of w (n0 in the lowest nibble) -> four
+// fp16x2 pairs x[k] = (n_k, n_{k+4}), exactly.  u = w ^ 0x88888888 turns
+// code x into x + 8; a nibble placed under the fp16 pattern 0x6400 reads as
+// 1024 + (x + 8); subtracting 1032 leaves x.
+__device__ __forceinline__ void i4x8_to_h2x4(uint32_t w, uint32_t (&x)[4]) {
+  const uint32_t u = w ^ 0x88888888u;
+  const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    uint32_t t = and_or(u >> (4 * k), 0x000F000Fu, 0x64006400u);
+    __half2 h = __hsub2(*reinterpret_cast<__half2*>(&t), bias);
+    x[k] = *reinterpret_cast<uint32_t*>(&h);
+  }
+}
+
+// Eight E2M1 codes of w (two per byte, low nibble first) -> four fp16x2
+// pairs q[k] = (n_2k, n_2k+1) with the hardware converter (exact: every
+// E2M1 value is an fp16 value).
+__device__ __forceinline__ void e2m1x8_to_h2x4(uint32_t w, uint32_t (&q)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(q[0]), "=r"(q[1]), "=r"(q[2]), "=r"(q[3])
+      : "r"(w));
+}
+
 // Four E4M3 codes [b0 b1 b2 b3] of v -> fp16x2 (b0, b1) and (b2, b3), low
 // byte in the low half, with the hardware converter (exact: e4m3 values are
 // all representable in fp16).

@@ -83,6 +83,17 @@ __device__ __forceinline__ uint32_t round_u8(float y) {
   return static_cast<uint32_t>(fminf(fmaxf(rintf(y), 0.0f), 255.0f));
 }
 
+// E2M1 code of y (|y| <= 6), round to nearest, ties to the even code
+// (mantissa bit 0), sign of zero kept.  Magnitude codes 0..7 stand for
+// 0, 0.5, 1, 1.5, 2, 3, 4, 6; the code is the number of decision points
+// below |y|, where a tie counts when the upper neighbour is the even code.
+__device__ __forceinline__ uint32_t e2m1_code(float y) {
+  const float a = fabsf(y);
+  const uint32_t m = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) +
+                     (a > 5.0f);
+  return m | (signbit(y) ? 8u : 0u);
+}
+
 // One quantised code from x given scale s (s > 0).
 template <bool kFP8>
 __device__ __forceinline__ uint32_t quantize_one(float x, float s) {
@@ -99,7 +110,8 @@ __device__ __forceinline__ uint32_t quantize_one(float x, float s) {
 
 // Quantising write: one warp per (token, head) row, D / 32 elements per lane.
 // kFmt: PKV_I8 or PKV_FP8E4M3 (symmetric absmax) or PKV_U8ASYM (min/max with
-// a zero point; kz / vz receive the zero points).
+// a zero point; kz / vz receive the zero points) or PKV_I4 / PKV_FP4E2M1
+// (symmetric absmax, two codes per byte, element 2k in the low nibble).
 template <int kD, int kFmt, bool kInBF16>
 __global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restrict__ k, const void* __restrict__ v,
                                                              uint8_t* __restrict__ kc, uint8_t* __restrict__ vc,
@@ -110,6 +122,8 @@ __global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restr
   constexpr int kE = kD / 32;
   constexpr bool kFP8 = kFmt == PKV_FP8E4M3;
   constexpr bool kAsym = kFmt == PKV_U8ASYM;
+  constexpr bool k4 = kFmt == PKV_I4 || kFmt == PKV_FP4E2M1;
+  constexpr int kRowBytes = k4 ? kD / 2 : kD;
   asm volatile("griddepcontrol.launch_dependents;");  // see kv_write_copy_kernel
   const int lane = threadIdx.x & 31;
   const long long rows = static_cast<long long>(num_tokens) * num_kv_heads;
@@ -155,6 +169,26 @@ __global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restr
           for (int e = 0; e < kE; ++e) packed |= round_u8(__fdiv_rn(__fsub_rn(x[e], lo), s)) << (8 * e);
         }
         if (lane == 0) (which == 0 ? kz : vz)[dst_row] = static_cast<uint8_t>(z);
+      } else if constexpr (k4) {
+        float a = 0.0f;
+#pragma unroll
+        for (int e = 0; e < kE; ++e) a = fmaxf(a, fabsf(x[e]));
+        a = warp_max(a);
+        constexpr bool kF4 = kFmt == PKV_FP4E2M1;
+        s = __fdiv_rn(a, kF4 ? 6.0f : 7.0f);
+        if (a > 0.0f) {
+#pragma unroll
+          for (int e = 0; e < kE; ++e) {
+            const float y = __fdiv_rn(x[e], s);
+            uint32_t c;
+            if constexpr (kF4) {
+              c = e2m1_code(fminf(fmaxf(y, -6.0f), 6.0f));
+            } else {
+              c = static_cast<uint32_t>(max(-7, min(7, __float2int_rn(y)))) & 0xFu;
+            }
+            packed |= c << (4 * e);
+          }
+        }
       } else {
         float a = 0.0f;
 #pragma unroll
@@ -166,10 +200,13 @@ __global__ void __launch_bounds__(256) kv_write_quant_kernel(const void* __restr
           for (int e = 0; e < kE; ++e) packed |= quantize_one<kFP8>(x[e], s) << (8 * e);
         }
       }
-      if constexpr (kE == 4) {
-        reinterpret_cast<uint32_t*>(cache + dst_row * kD)[lane] = packed;
+      // a lane's kE codes are contiguous: kE bytes, or kE / 2 bytes of nibbles
+      if constexpr (k4 && kE == 2) {
+        (cache + dst_row * kRowBytes)[lane] = static_cast<uint8_t>(packed);
+      } else if constexpr ((k4 && kE == 4) || (!k4 && kE == 2)) {
+        reinterpret_cast<uint16_t*>(cache + dst_row * kRowBytes)[lane] = static_cast<uint16_t>(packed);
       } else {
-        reinterpret_cast<uint16_t*>(cache + dst_row * kD)[lane] = static_cast<uint16_t>(packed);
+        reinterpret_cast<uint32_t*>(cache + dst_row * kRowBytes)[lane] = packed;
       }
       if (lane == 0) scales[dst_row] = s;
     }

@@ -44,7 +44,7 @@ WORKLOADS = {
     "prefix_shared": dict(batch=128, hq=32, hkv=8, d=128, dtype="bf16", ctx=("uniform", 64, 1024),
                           prefix=2048, pool=("need", 1.1), seed=1003),
     "quant_mha": dict(batch=256, hq=32, hkv=32, d=128, dtype="bf16", ctx=("loguniform", 128, 8192),
-                      pool=("need", 1.1), cache=("int8", "fp8", "u8asym"), seed=1004),
+                      pool=("need", 1.1), cache=("int8", "fp8", "u8asym", "int4", "fp4"), seed=1004),
     "spec_verify": dict(batch=64, hq=32, hkv=8, d=128, dtype="bf16", ctx=("uniform", 512, 4096),
                         q_len=4, pool=("need", 1.1), seed=1005),
     "chunked_prefill": dict(batch=8, hq=32, hkv=8, d=128, dtype="bf16", ctx=("uniform", 1024, 4096),
@@ -120,7 +120,11 @@ def random_codes(shape, gen, kind):
     """Random cache codes with a bell-shaped value mix: N(0, 1) values spread
     over the code range and converted by torch's own casts (int8: rounded and
     clamped to +-127; fp8: torch.float8_e4m3fn, raw bytes returned as uint8;
-    u8asym: centred on 127.5, rounded and clamped to [0, 255])."""
+    u8asym: centred on 127.5, rounded and clamped to [0, 255]).  The 4-bit
+    kinds (int4, fp4) are uniformly random bytes, two codes each, over the
+    last axis halved."""
+    if kind in ("int4", "fp4"):
+        return torch.randint(0, 256, shape[:-1] + (shape[-1] // 2,), generator=gen, dtype=torch.int64).to(torch.uint8)
     x = torch.randn(shape, generator=gen, dtype=torch.float32)
     if kind == "u8asym":
         return (x * (255.0 / 6.0) + 127.5).round().clamp(0, 255).to(torch.uint8)
@@ -135,7 +139,7 @@ def random_codes(shape, gen, kind):
 def random_scales(shape, gen, kind):
     """Positive fp32 scales of the size an absmax rule (or, for u8asym, a
     min/max rule over 128 values) gives N(0, 1) data."""
-    qmax = {"int8": 127.0, "fp8": 448.0, "u8asym": 255.0}[kind]
+    qmax = {"int8": 127.0, "fp8": 448.0, "u8asym": 255.0, "int4": 7.0, "fp4": 6.0}[kind]
     u = torch.rand(shape, generator=gen, dtype=torch.float32)
     if kind == "u8asym":
         return (4.0 + 2.0 * u) / qmax
@@ -252,14 +256,17 @@ def device_decode_case(name, device, seed=None, batch=None, cache_kind=None, ctx
     else:
         for key in ("k_cache", "v_cache"):
             x = torch.randn(shape, generator=dg, device=device, dtype=torch.float16)
-            if kind == "int8":
+            if kind in ("int4", "fp4"):
+                out[key] = torch.randint(0, 256, shape[:-1] + (shape[-1] // 2,), generator=dg, device=device,
+                                         dtype=torch.int64).to(torch.uint8)
+            elif kind == "int8":
                 out[key] = (x * (127.0 / 3.0)).round().clamp(-127, 127).to(torch.int8)
             elif kind == "u8asym":
                 out[key] = (x.float() * (255.0 / 6.0) + 127.5).round().clamp(0, 255).to(torch.uint8)
             else:
                 out[key] = (x.float() * (448.0 / 3.0)).clamp(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
             del x
-        qmax = {"int8": 127.0, "fp8": 448.0, "u8asym": 255.0}[kind]
+        qmax = {"int8": 127.0, "fp8": 448.0, "u8asym": 255.0, "int4": 7.0, "fp4": 6.0}[kind]
         span = 4.0 if kind == "u8asym" else 2.0
         for key in ("k_scale", "v_scale"):
             u = torch.rand((nb, hkv, BLOCK_SIZE), generator=dg, device=device, dtype=torch.float32)

@@ -20,8 +20,10 @@ PKV_ERR_CUDA = -4
 PKV_ERR_NOT_FOUND = -5
 PKV_ERR_EXISTS = -6
 
-PKV_F16, PKV_BF16, PKV_I8, PKV_FP8E4M3, PKV_U8ASYM = 0, 1, 2, 3, 4
-QUANTISED = (PKV_I8, PKV_FP8E4M3, PKV_U8ASYM)
+PKV_F16, PKV_BF16, PKV_I8, PKV_FP8E4M3, PKV_U8ASYM, PKV_I4, PKV_FP4E2M1 = 0, 1, 2, 3, 4, 5, 6
+QUANTISED = (PKV_I8, PKV_FP8E4M3, PKV_U8ASYM, PKV_I4, PKV_FP4E2M1)
+FOUR_BIT = (PKV_I4, PKV_FP4E2M1)
+KV_FORMATS = {"int8": PKV_I8, "fp8": PKV_FP8E4M3, "u8asym": PKV_U8ASYM, "int4": PKV_I4, "fp4": PKV_FP4E2M1}
 
 DEV_BAD_SLOT, DEV_BAD_BLOCK, DEV_BAD_CONTEXT, DEV_TIMEOUT, DEV_BAD_PAIR = 1, 2, 4, 8, 16
 
@@ -135,9 +137,16 @@ def dtype_code(t):
     raise TypeError(f"unsupported dtype {d}")
 
 
-def cache_code(cache, k_zero=None):
-    """Cache format code: the asymmetric uint8 format when zero points are
-    given, else the cache tensor's dtype (uint8 alone means FP8-e4m3)."""
+def cache_code(cache, k_zero=None, kv_format=None):
+    """Cache format code: ``kv_format`` when given ("int8", "fp8", "u8asym",
+    "int4", "fp4"; the 4-bit caches are uint8 [NB, Hkv, 16, D / 2]), else the
+    asymmetric uint8 format when zero points are given, else the cache
+    tensor's dtype (uint8 alone means FP8-e4m3)."""
+    if kv_format is not None:
+        ct = KV_FORMATS[kv_format]
+        if ct != PKV_I8 and cache.dtype != torch.uint8:
+            raise TypeError(f"a {kv_format} cache must be uint8")
+        return ct
     if k_zero is not None:
         if cache.dtype != torch.uint8:
             raise TypeError("a cache with zero points must be uint8")
@@ -192,8 +201,12 @@ def _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero):
         _need(v_zero, "v_zero", device=dev, dtype=torch.uint8)
 
 
+def _head_dim_of_cache(cache, ct):
+    return cache.shape[3] * (2 if ct in FOUR_BIT else 1)
+
+
 def kv_cache_write(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=None, stream=None,
-                   k_zero=None, v_zero=None):
+                   k_zero=None, v_zero=None, kv_format=None):
     """Writes rows k, v [T, Hkv, D] into the paged caches at slot_mapping [T]
     (int64, -1 skips).  Quantised caches (int8 / float8_e4m3fn, or uint8 with
     zero points) need the fp32 scale arrays [NB, Hkv, 16]; the asymmetric
@@ -205,9 +218,9 @@ def kv_cache_write(k, v, k_cache, v_cache, slot_mapping, k_scale=None, v_scale=N
         raise ValueError("k, v must be [T, Hkv, D]; caches [NB, Hkv, 16, D]")
     T, hkv, d = k.shape
     nb = k_cache.shape[0]
-    if k_cache.shape[1] != hkv or k_cache.shape[3] != d or slot_mapping.numel() != T:
+    ct = cache_code(k_cache, k_zero, kv_format)
+    if k_cache.shape[1] != hkv or _head_dim_of_cache(k_cache, ct) != d or slot_mapping.numel() != T:
         raise ValueError("shape mismatch between k and the caches")
-    ct = cache_code(k_cache, k_zero)
     _need_quant(ct, k.device, k_scale, v_scale, k_zero, v_zero)
     _check(lib().pkv_kv_cache_write(_ptr(k), _ptr(v), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale),
                                     _ptr(k_zero), _ptr(v_zero), _ptr(slot_mapping), T, hkv, d, k_cache.shape[2], nb,
@@ -248,7 +261,7 @@ def new_workspace(device, nbytes):
 
 def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scale, k_scale=None, v_scale=None,
                            max_context_len=None, out=None, workspace=None, partition_tokens=0, stream=None,
-                           k_zero=None, v_zero=None, sliding_window=0):
+                           k_zero=None, v_zero=None, sliding_window=0, kv_format=None):
     """out[s, i] = softmax(scale * q[s, i] . K_s) V_s through block tables.
 
     q [B, Hq, D] fp16/bf16; caches [NB, Hkv, 16, D]; block_tables [B, MB]
@@ -268,10 +281,11 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
         raise ValueError("q must be [B, Hq, D]; caches [NB, Hkv, 16, D]")
     B, hq, d = q.shape
-    nb, hkv, bs, dk = k_cache.shape
-    if dk != d or block_tables.dim() != 2 or block_tables.shape[0] != B or context_lens.numel() != B:
+    nb, hkv, bs, _ = k_cache.shape
+    ct = cache_code(k_cache, k_zero, kv_format)
+    if _head_dim_of_cache(k_cache, ct) != d or block_tables.dim() != 2 or block_tables.shape[0] != B or \
+            context_lens.numel() != B:
         raise ValueError("shape mismatch")
-    ct = cache_code(k_cache, k_zero)
     _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero)
     if max_context_len is None:
         max_context_len = int(context_lens.max().item()) if B else 0
@@ -306,7 +320,7 @@ def multi_query_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_
 def paged_attention_multi_query(q, k_cache, v_cache, block_tables, context_lens, query_start_loc, scale,
                                 max_query_len, max_context_len, k_scale=None, v_scale=None, k_zero=None,
                                 v_zero=None, out=None, workspace=None, partition_tokens=0, stream=None,
-                                sliding_window=0):
+                                sliding_window=0, kv_format=None):
     """Several new tokens per sequence (chunked prefill, speculative verify):
     q [T, Hq, D] packed by sequence with query_start_loc [B + 1] int32; the
     n_s new tokens of sequence s are the last n_s of its context_lens[s]
@@ -321,11 +335,12 @@ def paged_attention_multi_query(q, k_cache, v_cache, block_tables, context_lens,
     if q.dim() != 3 or k_cache.dim() != 4 or v_cache.shape != k_cache.shape:
         raise ValueError("q must be [T, Hq, D]; caches [NB, Hkv, 16, D]")
     T, hq, d = q.shape
-    nb, hkv, bs, dk = k_cache.shape
+    nb, hkv, bs, _ = k_cache.shape
     B = context_lens.numel()
-    if dk != d or block_tables.dim() != 2 or block_tables.shape[0] != B or query_start_loc.numel() != B + 1:
+    ct = cache_code(k_cache, k_zero, kv_format)
+    if _head_dim_of_cache(k_cache, ct) != d or block_tables.dim() != 2 or block_tables.shape[0] != B or \
+            query_start_loc.numel() != B + 1:
         raise ValueError("shape mismatch")
-    ct = cache_code(k_cache, k_zero)
     _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero)
     if out is None:
         out = torch.empty_like(q)
@@ -348,7 +363,7 @@ NOALLOC_SCRATCH_BYTES = 16 << 20
 
 def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_lens, scale, max_context_len,
                                    out, k_scale=None, v_scale=None, partition_tokens=0, stream=None,
-                                   k_zero=None, v_zero=None, sliding_window=0):
+                                   k_zero=None, v_zero=None, sliding_window=0, kv_format=None):
     """paged_attention_decode for callers that cannot allocate device memory
     (for instance a plugin whose host framework owns every allocation and
     hands it only input and output buffers): ``out`` must be given, no
@@ -364,7 +379,7 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
     _need(context_lens, "context_lens", device=dev, dtype=torch.int32)
     B, hq, d = q.shape
     nb, hkv, bs, _ = k_cache.shape
-    ct = cache_code(k_cache, k_zero)
+    ct = cache_code(k_cache, k_zero, kv_format)
     _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero)
     _check(lib().pkv_paged_attention_decode_noalloc(
         _ptr(out), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero), _ptr(v_zero),
@@ -374,7 +389,7 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
 
 
 def copy_blocks(k_cache, v_cache, src_dst_pairs, k_scale=None, v_scale=None, stream=None, k_zero=None,
-                v_zero=None):
+                v_zero=None, kv_format=None):
     """Block dst := block src for every row (src, dst) of src_dst_pairs
     [N, 2] int32 (device), for K, V and the scales (and zero points) of
     quantised caches."""
@@ -382,8 +397,9 @@ def copy_blocks(k_cache, v_cache, src_dst_pairs, k_scale=None, v_scale=None, str
     _need(k_cache, "k_cache", device=dev)
     _need(v_cache, "v_cache", device=dev)
     _need(src_dst_pairs, "src_dst_pairs", device=dev, dtype=torch.int32)
-    nb, hkv, bs, d = k_cache.shape
-    ct = cache_code(k_cache, k_zero)
+    nb, hkv, bs, _ = k_cache.shape
+    ct = cache_code(k_cache, k_zero, kv_format)
+    d = _head_dim_of_cache(k_cache, ct)
     _need_quant(ct, dev, k_scale, v_scale, k_zero, v_zero)
     n = src_dst_pairs.numel() // 2
     _check(lib().pkv_copy_blocks(_ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), _ptr(k_zero),

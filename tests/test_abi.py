@@ -95,7 +95,7 @@ def test_decode_host_rejections(lib):
     _err(_decode(lib, cd=P.PKV_U8ASYM, ks=n, vs=n), P.PKV_ERR_INVALID_ARG)   # without zero points
     _err(_decode(lib, cd=P.PKV_U8ASYM, ks=n, vs=n, kz=n, vz=ctypes.c_void_p(264)),
          P.PKV_ERR_INVALID_ARG)                                    # misaligned zero points
-    _err(_decode(lib, cd=5, ks=n, vs=n), P.PKV_ERR_UNSUPPORTED)   # unknown format
+    _err(_decode(lib, cd=9, ks=n, vs=n), P.PKV_ERR_UNSUPPORTED)   # unknown format
     _err(_decode(lib, pt=24), P.PKV_ERR_INVALID_ARG)              # partition not a multiple of 16
     # split plan needs a workspace
     _err(_decode(lib, maxc=64, pt=16), P.PKV_ERR_INVALID_ARG)

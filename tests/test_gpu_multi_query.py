@@ -34,7 +34,8 @@ def run_mq(g, partition_tokens=0, max_query_len=None, window=0):
         g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"], g["query_start_loc"], g["scale"],
         max_query_len=g["max_query_len"] if max_query_len is None else max_query_len,
         max_context_len=int(g["context_lens"].max()), k_scale=g.get("k_scale"), v_scale=g.get("v_scale"),
-        k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), partition_tokens=partition_tokens, sliding_window=window)
+        k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), partition_tokens=partition_tokens, sliding_window=window,
+        kv_format=g.get("cache_kind") if g.get("cache_kind") in ("int4", "fp4") else None)
     torch.cuda.synchronize()
     assert P.device_status(clear=True) == 0
     return out
@@ -81,7 +82,7 @@ def test_multi_query_sweep_16bit(dtype, d, group, ptok):
     check_attn(got, oracle_mq(case))
 
 
-@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym"])
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym", "int4", "fp4"])
 @pytest.mark.parametrize("group", [1, 4])
 def test_multi_query_quantised(kind, group):
     hkv = 4

@@ -3,7 +3,10 @@
 Bars: writes, block copies and quantisation are bit-exact; attention is within
 max-abs 2e-2 and mean-rel 1e-2 (sum |gpu - ref| / sum |ref|) for fp16 / bf16
 caches, and within 6e-2 max-abs of the oracle on the unquantised values for
-INT8 / FP8 / asymmetric uint8 caches.  Inputs come from the seeded generators in
+INT8 / FP8 / asymmetric uint8 caches (2.5e-1 for the 4-bit formats, whose own
+rounding error against unquantised attention reaches about 0.1 on these
+mixes); every quantised format is also held to the 16-bit bars against the
+oracle on its stored codes.  Inputs come from the seeded generators in
 paged_kv_cache_438_b200.inputs; nothing the oracle sees is produced by the
 library's kernels.
 """
@@ -22,7 +25,8 @@ from paged_kv_cache_438_b200 import pagedkv as P
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda:0")
-ATOL, MEANREL, QATOL = 2e-2, 1e-2, 6e-2
+ATOL, MEANREL, QATOL, Q4ATOL = 2e-2, 1e-2, 6e-2, 2.5e-1
+FOUR_BIT = ("int4", "fp4")
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -60,6 +64,10 @@ def cache_values(t, kind):
         return OQ.e4m3_decode(t.detach().cpu().contiguous().view(torch.uint8).numpy())
     if kind in ("int8", "u8asym"):
         return t.detach().cpu().numpy().astype(np.float64)
+    if kind == "int4":
+        return OQ.int4_values(t.detach().cpu().numpy())
+    if kind == "fp4":
+        return OQ.fp4_values(t.detach().cpu().numpy())
     return np64(t)
 
 
@@ -96,7 +104,8 @@ def run_decode(g, partition_tokens=0, max_context_len=None, window=0):
     out = P.paged_attention_decode(g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"],
                                    g["scale"], k_scale=g.get("k_scale"), v_scale=g.get("v_scale"),
                                    max_context_len=max_context_len, partition_tokens=partition_tokens,
-                                   k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), sliding_window=window)
+                                   k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), sliding_window=window,
+                                   kv_format=g.get("cache_kind") if g.get("cache_kind") in FOUR_BIT else None)
     torch.cuda.synchronize()
     assert P.device_status(clear=True) == 0
     return out
@@ -190,10 +199,17 @@ def _special_rows(k):
 
 QUANT = {"int8": (torch.int8, np.int8, lambda x: OQ.quantize_int8(x) + (None,)),
          "fp8": (torch.uint8, np.uint8, lambda x: OQ.quantize_fp8_e4m3(x) + (None,)),
-         "u8asym": (torch.uint8, np.uint8, OQ.quantize_u8_asym)}
+         "u8asym": (torch.uint8, np.uint8, OQ.quantize_u8_asym),
+         "int4": (torch.uint8, np.uint8, lambda x: OQ.quantize_int4(x) + (None,)),
+         "fp4": (torch.uint8, np.uint8, lambda x: OQ.quantize_fp4_e2m1(x) + (None,))}
 
 
-@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym"])
+def fmt(kind):
+    """kv_format argument of the binding for a cache kind."""
+    return kind if kind in FOUR_BIT else None
+
+
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym", "int4", "fp4"])
 @pytest.mark.parametrize("in_dtype", ["bf16", "f16"])
 @pytest.mark.parametrize("d,T", [(64, 50), (128, 600)])
 def test_write_quantised_bit_exact(kind, in_dtype, d, T):
@@ -203,7 +219,8 @@ def test_write_quantised_bit_exact(kind, in_dtype, d, T):
     slots = I.distinct_slots(T, nb, seed=T + 1)
     slots[9::9] = -1                                    # skip some tokens, keep the special rows
     cdt, ndt, quant = QUANT[kind]
-    gk = torch.zeros((nb, hkv, 16, d), dtype=cdt, device=DEV)
+    dc = d // 2 if kind in FOUR_BIT else d
+    gk = torch.zeros((nb, hkv, 16, dc), dtype=cdt, device=DEV)
     gv = torch.zeros_like(gk)
     gks = torch.zeros((nb, hkv, 16), dtype=torch.float32, device=DEV)
     gvs = torch.zeros_like(gks)
@@ -211,9 +228,10 @@ def test_write_quantised_bit_exact(kind, in_dtype, d, T):
     if kind == "u8asym":
         gkz = torch.full((nb, hkv, 16), 7, dtype=torch.uint8, device=DEV)
         gvz = torch.full_like(gkz, 7)
-    P.kv_cache_write(k.to(DEV), v.to(DEV), gk, gv, slots.to(DEV), gks, gvs, k_zero=gkz, v_zero=gvz)
+    P.kv_cache_write(k.to(DEV), v.to(DEV), gk, gv, slots.to(DEV), gks, gvs, k_zero=gkz, v_zero=gvz,
+                     kv_format=fmt(kind))
     torch.cuda.synchronize()
-    zero_codes = np.zeros((nb, hkv, 16, d), ndt)
+    zero_codes = np.zeros((nb, hkv, 16, dc), ndt)
     zero_sc = np.zeros((nb, hkv, 16), np.float32)
     for x, gc, gs, gz in ((k, gk, gks, gkz), (v, gv, gvs, gvz)):
         codes, sc, zp = quant(x.float().numpy())
@@ -226,7 +244,7 @@ def test_write_quantised_bit_exact(kind, in_dtype, d, T):
 
 # ------------------------------------------------------------ block copy --
 
-@pytest.mark.parametrize("kind", ["float", "int8", "fp8", "u8asym"])
+@pytest.mark.parametrize("kind", ["float", "int8", "fp8", "u8asym", "int4"])
 def test_copy_blocks_bit_exact(kind):
     case = I.decode_case("llama3_8b", batch=4, cache_kind=None if kind == "float" else kind, num_blocks=200,
                          ctx_override=[300, 500, 17, 1])
@@ -235,7 +253,7 @@ def test_copy_blocks_bit_exact(kind):
     perm = rng.permutation(200)
     pairs = np.stack([perm[:40], perm[40:80]], 1).astype(np.int32)   # sources and destinations disjoint
     P.copy_blocks(g["k_cache"], g["v_cache"], torch.as_tensor(pairs, device=DEV), g.get("k_scale"),
-                  g.get("v_scale"), k_zero=g.get("k_zero"), v_zero=g.get("v_zero"))
+                  g.get("v_scale"), k_zero=g.get("k_zero"), v_zero=g.get("v_zero"), kv_format=fmt(kind))
     torch.cuda.synchronize()
     arrays = [bits(case["k_cache"]), bits(case["v_cache"])]
     got = [bits(g["k_cache"]), bits(g["v_cache"])]
@@ -279,7 +297,7 @@ def test_decode_sweep_16bit(dtype, d, group, ptok):
     np.testing.assert_allclose(got[1], np.repeat(v0, group, axis=0), atol=1e-2)
 
 
-@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym"])
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym", "int4", "fp4"])
 @pytest.mark.parametrize("qdtype", ["bf16", "f16"])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("group", [1, 8, 16])
@@ -336,7 +354,8 @@ def _sample_pairs(B, hq, n, seed):
 
 @pytest.mark.parametrize("name,kind,n", [("llama3_8b", None, 48), ("llama3_70b_32k", None, 16),
                                          ("prefix_shared", None, 40), ("quant_mha", "int8", 40),
-                                         ("quant_mha", "fp8", 40), ("quant_mha", "u8asym", 40)])
+                                         ("quant_mha", "fp8", 40), ("quant_mha", "u8asym", 40),
+                                         ("quant_mha", "int4", 24), ("quant_mha", "fp4", 24)])
 def test_decode_full_workload_sampled(name, kind, n):
     g = I.device_decode_case(name, DEV, cache_kind=kind)
     maxc = int(g["context_lens_cpu"].max())
@@ -418,7 +437,7 @@ def test_prefix_sharing_copy_on_write_end_to_end():
     check_attn(np64(out)[sample], ref[sample])
 
 
-@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym"])
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym", "int4", "fp4"])
 def test_quantised_write_then_decode_end_to_end(kind):
     """bf16 token rows are quantised by the write kernel and attended by the
     decode kernel; against the oracle on the unquantised rows (6e-2) and on
@@ -434,7 +453,7 @@ def test_quantised_write_then_decode_end_to_end(kind):
     T = slots.numel()
     k, v = I.new_tokens(T, hkv, d, "bf16", seed=92)
     cdt, _, quant = QUANT[kind]
-    gk = torch.zeros((nb, hkv, 16, d), dtype=cdt, device=DEV)
+    gk = torch.zeros((nb, hkv, 16, d // 2 if kind in FOUR_BIT else d), dtype=cdt, device=DEV)
     gv = torch.zeros_like(gk)
     gks = torch.zeros((nb, hkv, 16), dtype=torch.float32, device=DEV)
     gvs = torch.zeros_like(gks)
@@ -442,22 +461,26 @@ def test_quantised_write_then_decode_end_to_end(kind):
     if kind == "u8asym":
         gkz = torch.zeros((nb, hkv, 16), dtype=torch.uint8, device=DEV)
         gvz = torch.zeros_like(gkz)
-    P.kv_cache_write(k.to(DEV), v.to(DEV), gk, gv, slots.to(DEV), gks, gvs, k_zero=gkz, v_zero=gvz)
+    P.kv_cache_write(k.to(DEV), v.to(DEV), gk, gv, slots.to(DEV), gks, gvs, k_zero=gkz, v_zero=gvz,
+                     kv_format=fmt(kind))
     q = I.randn((B, hq, d), gen, "bf16")
     out = np64(P.paged_attention_decode(q.to(DEV), gk, gv, bt.to(DEV), ctx.to(DEV), 1 / math.sqrt(d), gks, gvs,
-                                        max_context_len=int(ctx.max()), k_zero=gkz, v_zero=gvz))
+                                        max_context_len=int(ctx.max()), k_zero=gkz, v_zero=gvz,
+                                        kv_format=fmt(kind)))
     # (i) against attention over the unquantised bf16 rows
     raw_k = OC.kv_write(np.zeros((nb, hkv, 16, d)), k.double().numpy(), slots.numpy())
     raw_v = OC.kv_write(np.zeros((nb, hkv, 16, d)), v.double().numpy(), slots.numpy())
     ref_raw = OA.paged_decode_attention(np64(q), raw_k, raw_v, bt.numpy(), ctx.numpy(), 1 / math.sqrt(d))
-    check_attn(out, ref_raw, atol=QATOL, meanrel=None)
+    check_attn(out, ref_raw, atol=Q4ATOL if kind in FOUR_BIT else QATOL, meanrel=None)
     # (ii) against the oracle's own quantisation of the same rows
-    dec = OQ.e4m3_decode if kind == "fp8" else (lambda c: c.astype(np.float64))
+    dec = {"fp8": OQ.e4m3_decode, "int4": OQ.int4_values, "fp4": OQ.fp4_values}.get(
+        kind, lambda c: c.astype(np.float64))
     ck, sk, zk = quant(k.float().numpy())
     cv, sv, zv = quant(v.float().numpy())
     zc = np.zeros((nb, hkv, 16, d))
     zs = np.zeros((nb, hkv, 16), np.float32)
     zz = np.zeros((nb, hkv, 16), np.uint8)
+    # (the 4-bit codes are unpacked by ``dec`` before the scatter)
     sl = slots.numpy()
     ref_q = OA.paged_decode_attention(np64(q), OC.kv_write(zc, dec(ck), sl), OC.kv_write(zc, dec(cv), sl),
                                       bt.numpy(), ctx.numpy(), 1 / math.sqrt(d), OC.scale_write(zs, sk, sl),
