@@ -92,8 +92,10 @@ def tensor_peak():
 
 
 def kernel_source_hash():
+    """Hash of the decode kernel's device code (the traffic record is valid
+    only for the kernel it was captured on)."""
     h = hashlib.sha256()
-    for f in ("pkv_decode.cuh", "pkv_device.cuh", "pkv_api.cu"):
+    for f in ("pkv_decode.cuh", "pkv_device.cuh"):
         with open(os.path.join(ROOT, "paged_kv_cache_438_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
