@@ -558,6 +558,21 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
     const int valid = ctx - kpos0;    // >= 1 tokens of this block count
     // sliding window: tokens before position ctx - window are not seen
     const int lowv = p.window > 0 ? ctx - p.window - kpos0 : -32;
+    // Rows of a sequence's last block at or beyond its context were never
+    // written and may hold anything, NaN included; P is 0 there, but 0 * NaN
+    // is not, so those V rows are zeroed in the stage first (and their
+    // scales replaced by 0 below).
+    const bool tail = valid < 16;
+    if (tail) {
+      uint8_t* vrow = base_ptr + (st - smem_base) + Tr::kKVBytes;
+      constexpr int kChunks = Tr::kNumColTiles * Tr::kChunksPerTileRow;  // 16-byte chunks per row
+      for (int e = lane; e < (16 - valid) * kChunks; e += 32) {
+        const int t = valid + e / kChunks, c = e % kChunks;
+        *reinterpret_cast<uint4*>(vrow + (c / Tr::kChunksPerTileRow) * Tr::kColTileBytes + t * Tr::kTileBytes +
+                                  (c % Tr::kChunksPerTileRow) * 16) = make_uint4(0u, 0u, 0u, 0u);
+      }
+      __syncwarp();
+    }
 
     // ---- S^T = K . Q^T (two independent accumulation chains, summed) ----
     float sacc[kNT][4], sacc2[kNT][4];
@@ -650,8 +665,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       const float* sc = reinterpret_cast<const float*>(base_ptr + (st - smem_base) + 2 * Tr::kKVBytes);
       f_r *= sc[r];
       f_r8 *= sc[r + 8];
-      vs_r = sc[16 + r];
-      vs_r8 = sc[16 + r + 8];
+      vs_r = r < valid ? sc[16 + r] : 0.0f;
+      vs_r8 = r + 8 < valid ? sc[16 + r + 8] : 0.0f;
     }
     const bool ok_r = r < valid && r >= lowv;
     const bool ok_r8 = r + 8 < valid && r + 8 >= lowv;
@@ -799,6 +814,9 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 
     // ---- refill this stage with item k + kR ----
     __syncwarp();
+    // the zeroed rows were generic-proxy writes; order them before the TMA
+    // (async-proxy) refill of the same stage
+    if (tail) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     const int kn = k + kR;
     if (kn < count) {
       const int chunk = kn >> 5;

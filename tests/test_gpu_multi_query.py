@@ -185,3 +185,17 @@ def test_validation_rejects_inconsistent_query_runs():
             run_mq(bad)
     finally:
         P.set_validation(False)
+
+
+def test_multi_query_never_written_tail_positions_do_not_leak():
+    case = I.multi_query_case("spec_verify", seed=17, ctx_override=CTX, q_lens=NQ, hq=8, hkv=2, d=128)
+    g = gpu_case(case)
+    for s, c in enumerate(CTX):
+        if c == 0 or c % 16 == 0:
+            continue
+        b = int(case["block_tables"][s, (c - 1) // 16])
+        g["k_cache"][b, :, c % 16:] = float("nan")
+        g["v_cache"][b, :, c % 16:] = float("nan")
+    got = np64(run_mq(g))
+    assert np.all(np.isfinite(got))
+    check_attn(got, oracle_mq(case))

@@ -537,3 +537,29 @@ def test_workspace_reused_across_shapes_matches_fresh_workspaces():
         torch.cuda.synchronize()
         assert torch.equal(got, ref) and torch.equal(got, again)
     assert P.device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("kind", ["float", "fp8", "u8asym", "fp4"])
+def test_never_written_tail_positions_do_not_leak(kind):
+    """Positions of a sequence's last block at or beyond its context were
+    never written and may hold NaN bit patterns (codes and scales alike):
+    the output must be the oracle's, which never reads them."""
+    case = I.decode_case("llama3_8b", seed=13, ctx_override=CTX_MIX, hq=8, hkv=2, d=128,
+                         cache_kind=None if kind == "float" else kind)
+    g = gpu_case(case)
+    for s, c in enumerate(CTX_MIX):
+        if c == 0 or c % 16 == 0:
+            continue
+        b = int(case["block_tables"][s, (c - 1) // 16])
+        for key in ("k_cache", "v_cache"):
+            t = g[key]
+            if kind == "float":
+                t[b, :, c % 16:] = float("nan")
+            else:
+                t[b, :, c % 16:] = 0x7F if kind == "fp8" else 0xFF     # e4m3 NaN / arbitrary codes
+        for key in ("k_scale", "v_scale"):
+            if key in g:
+                g[key][b, :, c % 16:] = float("nan")
+    got = np64(run_decode(g))
+    assert np.all(np.isfinite(got))
+    check_attn(got, oracle_full(case))
