@@ -10,7 +10,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libpagedkv.so")
 SOURCES = ["pkv_api.cu", "pkv_allocator.cpp"]
-HEADERS = ["pkv_device.cuh", "pkv_decode.cuh", "pkv_write.cuh", "pkv_error.h", "pkv_blake2b.h"]
+HEADERS = ["pkv_device.cuh", "pkv_decode.cuh", "pkv_write.cuh", "pkv_error.h", "pkv_blake2b.h", "pkv_prefill.cuh"]
 
 
 def nvcc():

@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "pkv_decode.cuh"
+#include "pkv_prefill.cuh"
 #include "pkv_error.h"
 #include "pkv_write.cuh"
 
@@ -164,6 +165,17 @@ int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int r
   return PKV_OK;
 }
 
+// Multi-query calls whose runs of new tokens fill at least one tile of 128
+// (token, head) rows, on 16-bit caches, with the automatic plan, go to the
+// query-major tcgen05 kernel (paged_prefill_kernel); the rest stay on the
+// decode kernel's multi-query mode.
+bool prefill_eligible(int cache_dtype, int head_dim, int G, int max_q, int num_seqs, int partition_tokens) {
+  return is16(cache_dtype) && (head_dim == 64 || head_dim == 128) && G >= 1 && 128 % G == 0 &&
+         static_cast<long long>(max_q) * G >= 128 && num_seqs <= 65535 && partition_tokens == 0;
+}
+
+int prefill_tiles(int max_q, int G) { return static_cast<int>((static_cast<long long>(max_q) * G + 127) / 128); }
+
 // Monotonic epoch of decode calls (40 bits, never 0): tags the arrival
 // counters so a workspace needs zeroing only before its first use.
 unsigned long long next_epoch() {
@@ -249,6 +261,27 @@ int dispatch_nt_q(const CUtensorMap& km, const CUtensorMap& vm, const pkv::Decod
     return nt2 ? launch_decode<kD, kCT, 2, kQ, kMQ>(km, vm, p, st)
                : launch_decode<kD, kCT, 1, kQ, kMQ>(km, vm, p, st);
   }
+}
+
+template <int kD, bool kBF16>
+int launch_prefill(const CUtensorMap& km, const CUtensorMap& vm, const pkv::PrefillParams& p, cudaStream_t st) {
+  auto kernel = pkv::paged_prefill_kernel<kD, kBF16>;
+  const size_t smem = pkv::PrefillTraits<kD>::kSmem;
+  int rc = set_smem(kernel, smem);
+  if (rc != PKV_OK) return rc;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.max_tiles, p.num_kv_heads, p.num_seqs);
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, km, vm, p);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return PKV_OK;
 }
 
 template <int kD, bool kMQ>
@@ -438,7 +471,9 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
   int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens,
                      &pl, mq ? max_query_len : 0);
   if (rc != PKV_OK) return rc;
-  if (pl.num_streams > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned(workspace, 256)))
+  const bool prefill = mq && prefill_eligible(cache_dtype, head_dim, G, max_query_len, num_seqs, partition_tokens) &&
+                       aligned(q, 16) && aligned(out, 16);
+  if (!prefill && pl.num_streams > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned(workspace, 256)))
     return fail(PKV_ERR_INVALID_ARG, "workspace of %zu bytes (256-byte aligned) required, got %zu", pl.workspace,
                 workspace ? workspace_bytes : 0);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -472,6 +507,35 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
   rc = make_cache_map(&km, k_cache, row_bytes(cache_dtype, head_dim), elt_size(cache_dtype), rows);
   if (rc == PKV_OK) rc = make_cache_map(&vm, v_cache, row_bytes(cache_dtype, head_dim), elt_size(cache_dtype), rows);
   if (rc != PKV_OK) return rc;
+
+  if (prefill) {
+    pkv::PrefillParams pp{};
+    pp.out = out;
+    pp.q = q;
+    pp.block_tables = block_tables;
+    pp.context_lens = context_lens;
+    pp.query_start_loc = query_start_loc;
+    pp.num_seqs = num_seqs;
+    pp.num_q_tokens = num_q_tokens;
+    pp.max_query_len = max_query_len;
+    pp.num_q_heads = num_q_heads;
+    pp.num_kv_heads = num_kv_heads;
+    pp.group = G;
+    pp.max_blocks_per_seq = max_blocks_per_seq;
+    pp.num_blocks = num_blocks;
+    pp.max_context_len = max_context_len;
+    pp.window = sliding_window;
+    pp.max_tiles = prefill_tiles(max_query_len, G);
+    pp.oob_row = static_cast<int>(rows);
+    pp.qk_scale_log2 = scale * 1.4426950408889634f;
+    const bool bf = cache_dtype == PKV_BF16;
+    if (head_dim == 128)
+      rc = bf ? launch_prefill<128, true>(km, vm, pp, st) : launch_prefill<128, false>(km, vm, pp, st);
+    else
+      rc = bf ? launch_prefill<64, true>(km, vm, pp, st) : launch_prefill<64, false>(km, vm, pp, st);
+    if (rc != PKV_OK) return rc;
+    return ok();
+  }
 
   pkv::DecodeParams p{};
   p.out = out;
@@ -545,8 +609,17 @@ int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int he
   int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens,
                      &pl, std::max(max_query_len, 1));
   if (rc != PKV_OK) return rc;
-  if (num_streams_out) *num_streams_out = pl.num_streams;
-  if (partition_tokens_out) *partition_tokens_out = pl.stream_tokens;
+  const int G = num_q_heads / num_kv_heads;
+  if (prefill_eligible(cache_dtype, head_dim, G, max_query_len, num_seqs, partition_tokens)) {
+    // one CTA per (sequence, KV head, 128-row tile), each over all its keys;
+    // the workspace of the other path is still reported (it is used when q
+    // or out is not 16-byte aligned)
+    if (num_streams_out) *num_streams_out = num_seqs * num_kv_heads * prefill_tiles(max_query_len, G);
+    if (partition_tokens_out) *partition_tokens_out = (max_context_len + 15) / 16 * 16;
+  } else {
+    if (num_streams_out) *num_streams_out = pl.num_streams;
+    if (partition_tokens_out) *partition_tokens_out = pl.stream_tokens;
+  }
   if (workspace_bytes_out) *workspace_bytes_out = pl.workspace;
   return ok();
 }

@@ -154,7 +154,14 @@ def test_multi_query_plan_tiles(lib):
     nw, per, ws = P.multi_query_plan(64, 32, 8, 128, 4096, 4, P.PKV_BF16)
     nwd, _, _ = P.decode_plan(64, 32, 8, 128, 4096, P.PKV_BF16)
     assert nw == nwd
-    # 512 new tokens x G 4 = 2048 columns = 128 tiles: one stream per (sequence, head, tile)
+    # 512 new tokens x G 4 = 2048 rows on a 16-bit cache: the query-major
+    # kernel, one CTA per (sequence, head, 128-row tile) over all its keys
     nw, per, ws = P.multi_query_plan(8, 32, 8, 128, 4096, 512, P.PKV_BF16)
-    assert nw == 8 * 8 * 128 and per == 4096
-    assert ws >= 8 * 8 * 128 * 8 + 2 * nw * (32 + 16 * 128) * 4
+    assert nw == 8 * 8 * 16 and per == 4096
+    # an explicit partition keeps the decode kernel's multi-query mode: one
+    # stream per (sequence, head, 16-column tile)... capped by the partition
+    nw2, per2, ws2 = P.multi_query_plan(8, 32, 8, 128, 4096, 512, P.PKV_BF16, partition_tokens=4096)
+    assert per2 == 4096 and nw2 == 8 * 8 * 128 and ws2 == ws
+    # 8-bit caches never take the query-major kernel
+    nw3, _, _ = P.multi_query_plan(8, 32, 8, 128, 4096, 512, P.PKV_I8)
+    assert nw3 == 8 * 8 * 128

@@ -199,3 +199,23 @@ def test_multi_query_never_written_tail_positions_do_not_leak():
     got = np64(run_mq(g))
     assert np.all(np.isfinite(got))
     check_attn(got, oracle_mq(case))
+
+
+@pytest.mark.parametrize("dtype,d,group", [("bf16", 128, 8), ("f16", 128, 4), ("bf16", 64, 16), ("f16", 64, 2)])
+def test_query_major_kernel_against_oracle_and_decode_mode(dtype, d, group):
+    """Runs long enough for the query-major tcgen05 kernel (>= 128 rows of
+    (token, head)): against the oracle, and against the decode kernel's
+    multi-query mode (forced with an explicit partition)."""
+    hkv = 2
+    ctx = [700, 130, 257, 64, 1, 300]
+    nq = [300, 130, 17, 64, 1, 0]
+    case = I.multi_query_case("chunked_prefill", seed=d + group, ctx_override=ctx, q_lens=nq, hq=hkv * group,
+                              hkv=hkv, d=d, dtype=dtype)
+    g = gpu_case(case)
+    nw, _, _ = P.multi_query_plan(len(ctx), hkv * group, hkv, d, max(ctx), max(nq), g["k_cache"].dtype)
+    assert nw == len(ctx) * hkv * ((max(nq) * group + 127) // 128)     # the query-major plan
+    fast = np64(run_mq(g))
+    ref = oracle_mq(case)
+    check_attn(fast, ref)
+    slow = np64(run_mq(g, partition_tokens=64))
+    check_attn(fast, slow, atol=1e-2, meanrel=5e-3)
