@@ -218,4 +218,4 @@ def test_query_major_kernel_against_oracle_and_decode_mode(dtype, d, group):
     ref = oracle_mq(case)
     check_attn(fast, ref)
     slow = np64(run_mq(g, partition_tokens=64))
-    check_attn(fast, slow, atol=1e-2, meanrel=5e-3)
+    check_attn(fast, slow, atol=2e-2, meanrel=5e-3)        # two bf16-rounded outputs: within 2 ulps
