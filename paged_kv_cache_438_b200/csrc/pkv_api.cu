@@ -270,8 +270,8 @@ int launch_prefill(const CUtensorMap& km, const CUtensorMap& vm, const pkv::Pref
   int rc = set_smem(kernel, smem);
   if (rc != PKV_OK) return rc;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.max_tiles, p.num_kv_heads, p.num_seqs);
-  cfg.blockDim = dim3(128);
+  cfg.gridDim = dim3((p.max_tiles + 1) / 2, p.num_kv_heads, p.num_seqs);  // two tiles per CTA
+  cfg.blockDim = dim3(pkv::PrefillTraits<kD>::kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
@@ -472,7 +472,7 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
                      &pl, mq ? max_query_len : 0);
   if (rc != PKV_OK) return rc;
   const bool prefill = mq && prefill_eligible(cache_dtype, head_dim, G, max_query_len, num_seqs, partition_tokens) &&
-                       aligned(q, 16) && aligned(out, 16);
+                       aligned(q, 16) && aligned(out, 16) && scale > 0.0f;
   if (!prefill && pl.num_streams > 1 && (!workspace || workspace_bytes < pl.workspace || !aligned(workspace, 256)))
     return fail(PKV_ERR_INVALID_ARG, "workspace of %zu bytes (256-byte aligned) required, got %zu", pl.workspace,
                 workspace ? workspace_bytes : 0);
@@ -611,10 +611,10 @@ int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int he
   if (rc != PKV_OK) return rc;
   const int G = num_q_heads / num_kv_heads;
   if (prefill_eligible(cache_dtype, head_dim, G, max_query_len, num_seqs, partition_tokens)) {
-    // one CTA per (sequence, KV head, 128-row tile), each over all its keys;
-    // the workspace of the other path is still reported (it is used when q
-    // or out is not 16-byte aligned)
-    if (num_streams_out) *num_streams_out = num_seqs * num_kv_heads * prefill_tiles(max_query_len, G);
+    // one CTA per (sequence, KV head, two 128-row tiles), each over all its
+    // keys; the workspace of the other path is still reported (it is used
+    // when q or out is not 16-byte aligned, or the scale is not positive)
+    if (num_streams_out) *num_streams_out = num_seqs * num_kv_heads * ((prefill_tiles(max_query_len, G) + 1) / 2);
     if (partition_tokens_out) *partition_tokens_out = (max_context_len + 15) / 16 * 16;
   } else {
     if (num_streams_out) *num_streams_out = pl.num_streams;

@@ -10,24 +10,25 @@
 // real matrix product.
 //
 // Design (sm_100a):
-//   * One CTA of 4 warps per (sequence, KV head, tile of 128 query rows); a
-//     row is a (new token, query head of the group) pair, row = t * G + g,
-//     so the GQA group shares every K/V tile.  Thread i owns row i: TMEM lane
-//     i holds its scores and its output accumulator, and the whole softmax of
-//     a row runs in one thread (no shuffles).
+//   * One CTA per (sequence, KV head, pair of tiles of 128 query rows); a row
+//     is a (new token, query head of the group) pair, row = t * G + g, so the
+//     GQA group shares every K/V tile.  Warpgroup A (warps 0-3) and B (warps
+//     4-7) own one tile each; thread i of a warpgroup owns row i, i.e. TMEM
+//     lane i: the whole online softmax of a row runs in one thread.  Warp 8
+//     loads K/V and issues every MMA.
 //   * Keys stream in tiles of 64 (four 16-token cache blocks found through
-//     the block table) by TMA into a 2-stage ring (128-byte swizzle); K tiles
+//     the block table) by TMA into a 3-stage ring (128-byte swizzle); K tiles
 //     are K-major B operands, V tiles MN-major B operands of the same layout.
 //   * S = Q K^T: tcgen05.mma M=128, N=64, K=16 steps over head_dim into TMEM
-//     (fp32); P = exp2(S - m) in bf16/fp16 written to shared memory
-//     (K-major, swizzled; at head_dim 128 over the stage's K tile, which S
-//     no longer needs) as the A operand of O += P V (M=128, N=head_dim).
-//     One thread issues the MMAs; completion is signalled by tcgen05.commit
-//     on an mbarrier; every wait is bounded.
-//   * Online softmax with a lazy rescale: the running max used for the
-//     exponentials only moves when a row's max grows by more than 8 (log2
-//     units), and only then is that row's O rescaled in TMEM.  Two CTAs fit
-//     on an SM, so one CTA's softmax overlaps the other's MMAs.
+//     (fp32); P = exp2(S - m) in bf16/fp16 written to shared memory (K-major,
+//     swizzled) as the A operand of O += P V (M=128, N=head_dim).  The tensor
+//     core alternates between the two tiles, so one warpgroup's softmax runs
+//     while the other tile's MMAs do; completion is signalled by
+//     tcgen05.commit on mbarriers; every wait is bounded.
+//   * Online softmax with a lazy rescale: the exponent base of a row only
+//     moves when its max grows by more than 8 (log2 units), and only then is
+//     that row's O rescaled in TMEM.  Unmasked tiles skip the mask; the
+//     softmax scale is folded into one FMA per score.
 //   * Tokens of a sequence's last block beyond its context were never
 //     written: their V rows are zeroed in the stage, blocks past the context
 //     are loaded from outside the tensor (TMA fills zeros).
@@ -143,29 +144,27 @@ struct PrefillParams {
   int num_blocks;
   int max_context_len;
   int window;
-  int max_tiles;   // tiles of 128 rows of the longest query run (grid.x)
+  int max_tiles;   // tiles of 128 rows of the longest query run (grid.x = pairs of them)
   int oob_row;     // a TMA row coordinate past the cache (zero fill)
   float qk_scale_log2;
 };
 
 template <int kD>
 struct PrefillTraits {
-  static constexpr int kRows = 128;                    // query rows per CTA (M)
-  static constexpr int kKeys = 64;                     // keys per tile (N of S)
+  static constexpr int kRows = 128;                    // query rows per tile (M)
+  static constexpr int kTiles = 2;                     // query tiles per CTA (ping-pong)
+  static constexpr int kKeys = 64;                     // keys per K/V tile (N of S)
   static constexpr int kRegions = kD / 64;             // 128-byte column regions of a row
   static constexpr int kQBytes = kRegions * kRows * 128;
   static constexpr int kKVRegion = kKeys * 128;        // 64 rows x 128 B
   static constexpr int kStageBytes = 2 * kRegions * kKVRegion;  // K regions, then V regions
-  static constexpr int kStages = 2;
+  static constexpr int kStages = 3;
   static constexpr int kPBytes = kRows * 128;          // 128 rows x 64 keys x 2 B
-  // at head_dim 128 the stage's K tile (16 KB) holds P once S is computed;
-  // otherwise P has its own buffer
-  static constexpr bool kPInK = kRegions * kKVRegion >= kPBytes;
-  static constexpr int kTmemCols = 256;                // S: columns [0, 64); O: [128, 128 + kD)
-  // two CTAs per SM (TMEM: 2 x 256 columns of 512), never three: the smem
-  // request is padded above a third of the SM's 228 KB
-  static constexpr int kSmemUsed = 1024 + kQBytes + kStages * kStageBytes + (kPInK ? 0 : kPBytes) + 128;
-  static constexpr int kSmem = kSmemUsed > 80 * 1024 ? kSmemUsed : 80 * 1024;
+  static constexpr int kThreads = 9 * 32;              // 2 softmax warpgroups + 1 control warp
+  static constexpr int kTmemCols = 512;                // S_A [0,64) S_B [64,128) O_A [128,..) O_B [256,..)
+  static constexpr int kSmemUsed = 1024 + kTiles * kQBytes + kStages * kStageBytes + kTiles * kPBytes + 256;
+  // one CTA per SM (it holds all 512 TMEM columns): ask for more than half
+  static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
 };
 
 template <bool kBF16>
@@ -179,28 +178,41 @@ __device__ __forceinline__ uint32_t pack_p2(float a, float b) {
   }
 }
 
+// Sum of the two 16-bit values packed in u, as the MMA will multiply them.
 template <bool kBF16>
-__device__ __forceinline__ float2 unpack_p2(uint32_t u) {
+__device__ __forceinline__ float sum_p2(uint32_t u) {
   if constexpr (kBF16) {
-    return __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&u));
+    return __uint_as_float(u << 16) + __uint_as_float(u & 0xFFFF0000u);
   } else {
-    return __half22float2(*reinterpret_cast<__half2*>(&u));
+    const float2 f = __half22float2(*reinterpret_cast<__half2*>(&u));
+    return f.x + f.y;
   }
 }
 
+// One CTA: two tiles of 128 (token, head) rows of one (sequence, KV head)
+// ("A" = the later tokens, "B" = the 128 rows before them), warpgroup A
+// (warps 0-3) and B (warps 4-7) each owning one tile's softmax, warp 8
+// loading K/V and issuing every MMA.  The tensor core alternates between
+// the tiles: while one warpgroup turns its scores into P, the MMAs of the
+// other run.  Per K/V tile j the issue order is S_A(j), S_B(j) (j = 0 only),
+// then PV_A(j), S_A(j+1) once P_A(j) is written, PV_B(j), S_B(j+1) once
+// P_B(j) is; a commit after each pair tells the warpgroup that its next
+// scores are ready and that its previous P and O are free.
 template <int kD, bool kBF16>
-__global__ void __launch_bounds__(128, 2)
+__global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                          const PrefillParams p) {
   using Tr = PrefillTraits<kD>;
   constexpr int kR = Tr::kRegions;
+  constexpr int kS = Tr::kStages;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
+  const int lane = tid & 31;
   const int s = blockIdx.z;
   const int h = blockIdx.y;
   const int G = p.group;
 
-  // ---- this CTA's rows: tile qt of sequence s's new tokens ----
+  // ---- rows of this CTA ----
   int ctx = p.context_lens[s];
   {
     const int cap = min(p.max_context_len, p.max_blocks_per_seq * 16);
@@ -213,15 +225,19 @@ __global__ void __launch_bounds__(128, 2)
   const int q0 = min(max(qa, 0), p.num_q_tokens);
   const int q1 = min(max(qb, q0), p.num_q_tokens);
   const int n = min(min(q1 - q0, ctx), p.max_query_len);
-  const int toks = Tr::kRows / G;                  // new tokens per tile
+  const int toks = Tr::kRows / G;                    // new tokens per tile
   const int ntiles = (n * G + Tr::kRows - 1) / Tr::kRows;
-  if (blockIdx.x >= ntiles) return;                // whole CTA, before any TMEM use
-  const int qt = ntiles - 1 - blockIdx.x;          // longest (latest) tiles start first
-  const int t0 = qt * toks;
-  const int nt = min(toks, n - t0);
-  // keys: row of token t (0-based in the run) sees positions < ctx - n + t + 1
-  const int klim = ctx - n + t0 + nt;              // exclusive bound of the tile's last token
-  const int kfirst = p.window > 0 ? max(0, ctx - n + t0 + 1 - p.window) : 0;
+  const int pairs = (ntiles + 1) / 2;
+  if (static_cast<int>(blockIdx.x) >= pairs) return;  // whole CTA, before any TMEM use
+  // tile A: the later one (more keys); tile B: the one before it (may not exist)
+  const int tile_a = ntiles - 1 - 2 * static_cast<int>(blockIdx.x);
+  const int tile_b = tile_a - 1;
+  const int ta0 = tile_a * toks, nta = min(toks, n - ta0);
+  const int tb0 = tile_b * toks, ntb = tile_b >= 0 ? min(toks, n - tb0) : 0;
+  // keys: token t (0-based in the run) sees positions < ctx - n + t + 1
+  const int klim = ctx - n + ta0 + nta;
+  const int t_first = tile_b >= 0 ? tb0 : ta0;
+  const int kfirst = p.window > 0 ? max(0, ctx - n + t_first + 1 - p.window) : 0;
   const int kbeg = kfirst & ~15;
   const int nk = (klim - kbeg + Tr::kKeys - 1) / Tr::kKeys;
 
@@ -229,39 +245,57 @@ __global__ void __launch_bounds__(128, 2)
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* const sptr = smem_raw + (sbase - raw);
-  const uint32_t q_s = sbase;
-  const uint32_t kv_s = q_s + Tr::kQBytes;
-  const uint32_t p_own = kv_s + Tr::kStages * Tr::kStageBytes;        // P buffer when not in the K tile
-  const uint32_t bars = p_own + (Tr::kPInK ? 0 : Tr::kPBytes);  // full[0], full[1], s_done, o_done
-  const uint32_t bar_sdone = bars + 16, bar_odone = bars + 24;
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sptr + (bars - sbase) + 32);
-  int* const abort_flag = reinterpret_cast<int*>(sptr + (bars - sbase) + 36);
+  const uint32_t q_s = sbase;                                  // Q_A, Q_B
+  const uint32_t kv_s = q_s + Tr::kTiles * Tr::kQBytes;       // kS stages of K then V
+  const uint32_t p_s = kv_s + kS * Tr::kStageBytes;           // P_A, P_B
+  const uint32_t bars = p_s + Tr::kTiles * Tr::kPBytes;
+  // barriers: full[kS], empty[kS], s_full[2], p_full[2], o_done[2]
+  const uint32_t b_full = bars, b_empty = bars + 8 * kS, b_sfull = bars + 16 * kS;
+  const uint32_t b_pfull = b_sfull + 16, b_odone = b_sfull + 32;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sptr + (bars - sbase) + 16 * kS + 48);
+  int* const abort_flag = reinterpret_cast<int*>(sptr + (bars - sbase) + 16 * kS + 52);
+  auto aborted = [&]() { return *reinterpret_cast<volatile int*>(abort_flag) != 0; };
+  auto wait_or_abort = [&](uint32_t bar, uint32_t parity) {
+    if (!mbar_wait(bar, parity)) atomicExch(abort_flag, 1);
+  };
 
   if (warp == 0) {
     tmem_alloc(smem_addr(tmem_slot), Tr::kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < 4; ++i) mbar_init(bars + 8 * i, 1);
+    for (int i = 0; i < kS; ++i) {
+      mbar_init(b_full + 8 * i, 1);
+      mbar_init(b_empty + 8 * i, 1);
+    }
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(b_sfull + 8 * x, 1);
+      mbar_init(b_pfull + 8 * x, Tr::kRows);
+      mbar_init(b_odone + 8 * x, 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
 
-  // ---- Q tile -> shared memory, K-major with the 128-byte swizzle ----
-  const int row = tid;
+  // ---- Q tiles -> shared memory, K-major with the 128-byte swizzle ----
+  const int wg = warp >> 2;          // 0: tile A, 1: tile B, 2: control warp
+  const int row = tid & 127;         // row of the warpgroup's tile / TMEM lane
+  const int t0x = wg == 0 ? ta0 : tb0;
+  const int ntx = wg == 0 ? nta : ntb;
   const int rt = row / G, rg = row - (row / G) * G;
-  const bool row_ok = rt < nt;
-  {
+  const bool row_ok = wg < 2 && rt < ntx;
+  if (wg < 2) {
     const uint4* src = reinterpret_cast<const uint4*>(
         reinterpret_cast<const uint16_t*>(p.q) +
-        (static_cast<long long>(q0 + t0 + (row_ok ? rt : 0)) * p.num_q_heads + static_cast<long long>(h) * G +
+        (static_cast<long long>(q0 + (row_ok ? t0x + rt : ta0)) * p.num_q_heads + static_cast<long long>(h) * G +
          rg) * kD);
+    const uint32_t qx = q_s + wg * Tr::kQBytes;
 #pragma unroll
     for (int c = 0; c < kD / 8; ++c) {
       const uint4 v = row_ok ? src[c] : make_uint4(0u, 0u, 0u, 0u);
       const int reg = c >> 3, cc = c & 7;
-      *reinterpret_cast<uint4*>(sptr + (q_s - sbase) + reg * (Tr::kRows * 128) + row * 128 +
-                                ((cc ^ (row & 7)) << 4)) = v;
+      *reinterpret_cast<uint4*>(sptr + (qx - sbase) + reg * (Tr::kRows * 128) + row * 128 + ((cc ^ (row & 7)) << 4)) =
+          v;
     }
   }
   fence_async_smem();
@@ -269,200 +303,231 @@ __global__ void __launch_bounds__(128, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;          // 64 columns of scores
-  const uint32_t tO = tmem + 128;    // kD columns of output accumulator
-  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-
-  // ---- K/V tile producer (thread 0) ----
-  int issued = 0;  // tiles whose loads thread 0 has issued
-  auto load_tile = [&](int j) {
-    ++issued;
-    const int stage = j & 1;
-    const uint32_t st = kv_s + stage * Tr::kStageBytes;
-    const uint32_t bar = bars + 8 * stage;
-    mbar_arrive_expect_tx(bar, Tr::kStageBytes);
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const int kb = (kbeg >> 4) + 4 * j + b;  // logical block
-      int row0 = p.oob_row;                    // past the context: zero fill
-      if (kb * 16 < ctx) {
-        int id = p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + kb];
-        if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
-          raise_status(PKV_DEV_BAD_BLOCK);
-          id = 0;
-        }
-        row0 = (id * p.num_kv_heads + h) * 16;
-      }
-#pragma unroll
-      for (int r = 0; r < kR; ++r) {
-        tma_load_2d(st + r * Tr::kKVRegion + b * 2048, &kmap, r * 64, row0, bar);
-        tma_load_2d(st + (kR + r) * Tr::kKVRegion + b * 2048, &vmap, r * 64, row0, bar);
-      }
-    }
-  };
-
   // the cache may still be being written by the preceding kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  if (tid == 0) {
-    load_tile(0);
-    if (nk > 1) load_tile(1);
-  }
 
   constexpr uint32_t kIdescS = umma_idesc(128, Tr::kKeys, kBF16, false);
   constexpr uint32_t kIdescO = umma_idesc(128, kD, kBF16, true);
-  const int lim = row_ok ? ctx - n + t0 + rt + 1 : kbeg + 1;  // exclusive key bound of this row
-  const int lo = p.window > 0 ? lim - p.window : -1;          // keys < lo are outside the window
-  float m_used = -INFINITY, l = 0.0f;
-  uint32_t ph_s = 0, ph_o = 0;
-  int consumed = 0;  // tiles whose loads were waited for
 
-#pragma unroll 1
-  for (int j = 0; j < nk; ++j) {
-    const int stage = j & 1;
-    const uint32_t st = kv_s + stage * Tr::kStageBytes;
-    const uint32_t p_s = Tr::kPInK ? st : p_own;
-    const int kt0 = kbeg + j * Tr::kKeys;  // first key of the tile
-    if (!mbar_wait(bars + 8 * stage, (j >> 1) & 1)) atomicExch(abort_flag, 1);
-    consumed = j + 1;
-    // keys of the tile at or past the context: zero their V rows (never
-    // written, or zero-filled already)
-    if (kt0 + Tr::kKeys > ctx) {
-      const int r0 = max(ctx - kt0, 0);
-      for (int e = tid; e < (Tr::kKeys - r0) * kR * 8; e += 128) {
-        const int rr = r0 + e / (kR * 8), reg = (e / 8) % kR, c = e % 8;
-        *reinterpret_cast<uint4*>(sptr + (st - sbase) + (kR + reg) * Tr::kKVRegion + rr * 128 + c * 16) =
-            make_uint4(0u, 0u, 0u, 0u);
+  if (wg == 2) {
+    // =================== control warp: K/V loads and all MMAs ===================
+    int issued = 0, consumed = 0;
+    auto load_tile = [&](int j) {
+      const int st_i = j % kS;
+      const uint32_t st = kv_s + st_i * Tr::kStageBytes;
+      const uint32_t bar = b_full + 8 * st_i;
+      ++issued;
+      mbar_arrive_expect_tx(bar, Tr::kStageBytes);
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int kb = (kbeg >> 4) + 4 * j + b;  // logical block
+        int row0 = p.oob_row;                    // past the context: zero fill
+        if (kb * 16 < ctx) {
+          int id = p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + kb];
+          if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
+            raise_status(PKV_DEV_BAD_BLOCK);
+            id = 0;
+          }
+          row0 = (id * p.num_kv_heads + h) * 16;
+        }
+#pragma unroll
+        for (int r = 0; r < kR; ++r) {
+          tma_load_2d(st + r * Tr::kKVRegion + b * 2048, &kmap, r * 64, row0, bar);
+          tma_load_2d(st + (kR + r) * Tr::kKVRegion + b * 2048, &vmap, r * 64, row0, bar);
+        }
       }
-      fence_async_smem();
-    }
-    tc_fence_before();
-    __syncthreads();
-    if (*reinterpret_cast<volatile int*>(abort_flag)) break;
-
-    // ---- S = Q K^T ----
-    if (tid == 0) {
-      tc_fence_after();
+    };
+    auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T into S_x's TMEM columns
+      const uint32_t st = kv_s + (j % kS) * Tr::kStageBytes;
+      const uint32_t qx = q_s + x * Tr::kQBytes;
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
         const int reg = ks >> 2, off = (ks & 3) * 32;
-        umma_f16(tS, smem_desc_sw128(q_s + reg * (Tr::kRows * 128) + off, 16),
+        umma_f16(tmem + 64 * x, smem_desc_sw128(qx + reg * (Tr::kRows * 128) + off, 16),
                  smem_desc_sw128(st + reg * Tr::kKVRegion + off, 16), kIdescS, ks > 0 ? 1u : 0u);
       }
-      umma_commit(bar_sdone);
-    }
-    if (!mbar_wait(bar_sdone, ph_s)) atomicExch(abort_flag, 1);
-    ph_s ^= 1u;
-    tc_fence_after();
-
-    // ---- scores of this row, mask, online softmax ----
-    float sv[64];
-    {
-      float a[32], b[32];
-      tmem_ld32(tS + lane_off, a);
-      tmem_ld32(tS + lane_off + 32, b);
-      tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        sv[c] = a[c];
-        sv[32 + c] = b[c];
-      }
-    }
-    float mx = -INFINITY;
-#pragma unroll
-    for (int c = 0; c < 64; ++c) {
-      const int key = kt0 + c;
-      const bool ok = key < lim && key >= lo;
-      sv[c] = ok ? sv[c] * p.qk_scale_log2 : -INFINITY;
-      mx = fmaxf(mx, sv[c]);
-    }
-    float factor = 1.0f;
-    bool rescale = false;
-    if (mx > m_used + 8.0f) {
-      // the base moves; O and l were accumulated against the old one
-      factor = m_used == -INFINITY ? 0.0f : fast_exp2(m_used - mx);
-      rescale = m_used != -INFINITY;
-      m_used = mx;
-    }
-    const float base = m_used == -INFINITY ? 0.0f : m_used;
-    float sum = 0.0f;
-#pragma unroll
-    for (int c8 = 0; c8 < 8; ++c8) {
-      uint32_t w[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        w[k] = pack_p2<kBF16>(fast_exp2(sv[8 * c8 + 2 * k] - base), fast_exp2(sv[8 * c8 + 2 * k + 1] - base));
-        const float2 f = unpack_p2<kBF16>(w[k]);  // sum what the MMA multiplies
-        sum += f.x + f.y;
-      }
-      *reinterpret_cast<uint4*>(sptr + (p_s - sbase) + row * 128 + ((c8 ^ (row & 7)) << 4)) =
-          make_uint4(w[0], w[1], w[2], w[3]);
-    }
-    l = l * factor + sum;
-    if (__any_sync(0xffffffffu, rescale)) {
-      // O of the previous tiles is complete (waited below); rescale this
-      // warp's rows in TMEM
-      const float f = rescale ? factor : 1.0f;
-#pragma unroll 1
-      for (int cb = 0; cb < kD / 32; ++cb) {
-        float o[32];
-        tmem_ld32(tO + lane_off + 32 * cb, o);
-        tmem_wait_ld();
-#pragma unroll
-        for (int c = 0; c < 32; ++c) o[c] *= f;
-        tmem_st32(tO + lane_off + 32 * cb, o);
-      }
-      tmem_wait_st();
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- O += P V ----
-    if (tid == 0) {
-      tc_fence_after();
+    };
+    auto issue_pv = [&](int x, int j) {  // O_x += P_x V_j
+      const uint32_t st = kv_s + (j % kS) * Tr::kStageBytes;
+      const uint32_t px = p_s + x * Tr::kPBytes;
 #pragma unroll
       for (int ks = 0; ks < Tr::kKeys / 16; ++ks) {
-        umma_f16(tO, smem_desc_sw128(p_s + ks * 32, 16),
+        umma_f16(tmem + 128 * (x + 1), smem_desc_sw128(px + ks * 32, 16),
                  smem_desc_sw128(st + kR * Tr::kKVRegion + ks * 2048, Tr::kKVRegion), kIdescO,
                  (j > 0 || ks > 0) ? 1u : 0u);
       }
-      umma_commit(bar_odone);
+    };
+    if (lane == 0) {
+      for (int j = 0; j < kS && j < nk; ++j) load_tile(j);
     }
-    if (!mbar_wait(bar_odone, ph_o)) atomicExch(abort_flag, 1);
-    ph_o ^= 1u;
-    tc_fence_after();
-    // this stage is free again: prefetch tile j + 2 into it
-    if (tid == 0 && j + 2 < nk) {
-      fence_async_smem();
-      load_tile(j + 2);
-    }
-  }
-
-  // after an abort, let loads still in flight land (bounded) before exit
-  if (tid == 0) {
-    for (int j = consumed; j < issued; ++j) mbar_wait(bars + 8 * (j & 1), (j >> 1) & 1);
-  }
-
-  // ---- epilogue: O / l -> out ----
-  if (!*reinterpret_cast<volatile int*>(abort_flag)) {
-    const float inv = l > 0.0f ? 1.0f / l : 0.0f;
-    uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) +
-                    (static_cast<long long>(q0 + t0 + (row_ok ? rt : 0)) * p.num_q_heads +
-                     static_cast<long long>(h) * G + rg) * kD;
 #pragma unroll 1
-    for (int cb = 0; cb < kD / 32; ++cb) {
-      float o[32];
-      tmem_ld32(tO + lane_off + 32 * cb, o);
-      tmem_wait_ld();
-      if (row_ok) {
+    for (int j = 0; j < nk; ++j) {
+      const int st_i = j % kS;
+      const uint32_t st = kv_s + st_i * Tr::kStageBytes;
+      const int kt0 = kbeg + j * Tr::kKeys;
+      wait_or_abort(b_full + 8 * st_i, (j / kS) & 1);
+      consumed = j + 1;
+      if (aborted()) break;
+      // keys of the tile at or past the context: zero their V rows (never
+      // written there, or zero-filled already) before any P . V reads them
+      if (kt0 + Tr::kKeys > ctx) {
+        const int r0 = max(ctx - kt0, 0);
+        for (int e = lane; e < (Tr::kKeys - r0) * kR * 8; e += 32) {
+          const int rr = r0 + e / (kR * 8), reg = (e / 8) % kR, c = e % 8;
+          *reinterpret_cast<uint4*>(sptr + (st - sbase) + (kR + reg) * Tr::kKVRegion + rr * 128 + c * 16) =
+              make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        tc_fence_after();
+        if (j == 0) {
+          issue_s(0, 0);
+          umma_commit(b_sfull);
+          issue_s(1, 0);
+          umma_commit(b_sfull + 8);
+        }
+        const bool more = j + 1 < nk;
+        if (more) {  // the next tile must have landed before its S is issued
+          wait_or_abort(b_full + 8 * ((j + 1) % kS), ((j + 1) / kS) & 1);
+        }
+#pragma unroll 1
+        for (int x = 0; x < 2; ++x) {
+          wait_or_abort(b_pfull + 8 * x, j & 1);  // P_x(j) written
+          tc_fence_after();
+          issue_pv(x, j);
+          if (more) {
+            issue_s(x, j + 1);
+            umma_commit(b_sfull + 8 * x);
+          } else {
+            umma_commit(b_odone + 8 * x);
+          }
+        }
+        umma_commit(b_empty + 8 * st_i);  // the stage is read once both P . V are done
+        if (j + kS < nk) {
+          wait_or_abort(b_empty + 8 * st_i, (j / kS) & 1);
+          fence_async_smem();
+          load_tile(j + kS);
+        }
+      }
+      __syncwarp();
+    }
+    // loads still in flight after an abort land (bounded) before exit
+    if (lane == 0) {
+      for (int j = consumed; j < issued; ++j) mbar_wait(b_full + 8 * (j % kS), (j / kS) & 1);
+    }
+  } else {
+    // =================== softmax warpgroup x = wg ===================
+    const int x = wg;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + 64 * x + lane_off;
+    const uint32_t tO = tmem + 128 * (x + 1) + lane_off;
+    const uint32_t px = p_s + x * Tr::kPBytes;
+    // exclusive key bound and window start of this row; rows past the run
+    // see one key so that their (discarded) math stays finite
+    const int lim = row_ok ? ctx - n + t0x + rt + 1 : kbeg + 1;
+    const int lo = p.window > 0 ? lim - p.window : -1;
+    // a tile is unmasked for the whole warpgroup when it lies between the
+    // largest window start and the smallest bound of the tile's rows
+    const int wmin_lim = ctx - n + t0x + 1;
+    const int wmax_lo = p.window > 0 ? ctx - n + t0x + max(ntx, 1) - p.window : -1;
+    const float c = p.qk_scale_log2;  // > 0 (checked by the host)
+    float m_used = -INFINITY, l = 0.0f;
+#pragma unroll 1
+    for (int j = 0; j < nk; ++j) {
+      wait_or_abort(b_sfull + 8 * x, j & 1);
+      if (aborted()) break;
+      tc_fence_after();
+      float sv[64];
+      {
+        float a[32], b[32];
+        tmem_ld32(tS, a);
+        tmem_ld32(tS + 32, b);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c8 = 0; c8 < 4; ++c8) {
-          uint4 v;
-          v.x = pack_p2<kBF16>(o[8 * c8 + 0] * inv, o[8 * c8 + 1] * inv);
-          v.y = pack_p2<kBF16>(o[8 * c8 + 2] * inv, o[8 * c8 + 3] * inv);
-          v.z = pack_p2<kBF16>(o[8 * c8 + 4] * inv, o[8 * c8 + 5] * inv);
-          v.w = pack_p2<kBF16>(o[8 * c8 + 6] * inv, o[8 * c8 + 7] * inv);
-          *reinterpret_cast<uint4*>(dst + 32 * cb + 8 * c8) = v;
+        for (int k = 0; k < 32; ++k) {
+          sv[k] = a[k];
+          sv[32 + k] = b[k];
+        }
+      }
+      const int kt0 = kbeg + j * Tr::kKeys;
+      const bool full = kt0 + Tr::kKeys <= wmin_lim && kt0 >= wmax_lo && row_ok;
+      if (!full) {
+#pragma unroll
+        for (int k = 0; k < 64; ++k) {
+          const int key = kt0 + k;
+          sv[k] = (key < lim && key >= lo) ? sv[k] : -INFINITY;
+        }
+      }
+      float mr = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < 64; ++k) mr = fmaxf(mr, sv[k]);
+      const float mx = mr * c;  // scores are used as s * c (log2 units)
+      float factor = 1.0f;
+      bool rescale = false;
+      if (mx > m_used + 8.0f) {
+        factor = m_used == -INFINITY ? 0.0f : fast_exp2(m_used - mx);
+        rescale = m_used != -INFINITY;
+        m_used = mx;
+      }
+      const float nbase = m_used == -INFINITY ? 0.0f : -m_used;
+      float sum = 0.0f;
+#pragma unroll
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[8 * c8 + 2 * k], c, nbase)),
+                                fast_exp2(fmaf(sv[8 * c8 + 2 * k + 1], c, nbase)));
+          sum += sum_p2<kBF16>(w[k]);
+        }
+        *reinterpret_cast<uint4*>(sptr + (px - sbase) + row * 128 + ((c8 ^ (row & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      l = l * factor + sum;
+      if (__any_sync(0xffffffffu, rescale)) {
+        // O_x up to tile j - 1 is complete (the commit that released these
+        // scores came after it)
+        const float f = rescale ? factor : 1.0f;
+#pragma unroll 1
+        for (int cb = 0; cb < kD / 32; ++cb) {
+          float o[32];
+          tmem_ld32(tO + 32 * cb, o);
+          tmem_wait_ld();
+#pragma unroll
+          for (int k = 0; k < 32; ++k) o[k] *= f;
+          tmem_st32(tO + 32 * cb, o);
+        }
+        tmem_wait_st();
+      }
+      fence_async_smem();
+      tc_fence_before();
+      mbar_arrive(b_pfull + 8 * x);
+    }
+    // ---- epilogue: O / l -> out ----
+    wait_or_abort(b_odone + 8 * x, 0);
+    tc_fence_after();
+    if (!aborted()) {
+      const float inv = l > 0.0f ? 1.0f / l : 0.0f;
+      uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) +
+                      (static_cast<long long>(q0 + (row_ok ? t0x + rt : ta0)) * p.num_q_heads +
+                       static_cast<long long>(h) * G + rg) * kD;
+#pragma unroll 1
+      for (int cb = 0; cb < kD / 32; ++cb) {
+        float o[32];
+        tmem_ld32(tO + 32 * cb, o);
+        tmem_wait_ld();
+        if (row_ok) {
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) {
+            uint4 v;
+            v.x = pack_p2<kBF16>(o[8 * c8 + 0] * inv, o[8 * c8 + 1] * inv);
+            v.y = pack_p2<kBF16>(o[8 * c8 + 2] * inv, o[8 * c8 + 3] * inv);
+            v.z = pack_p2<kBF16>(o[8 * c8 + 4] * inv, o[8 * c8 + 5] * inv);
+            v.w = pack_p2<kBF16>(o[8 * c8 + 6] * inv, o[8 * c8 + 7] * inv);
+            *reinterpret_cast<uint4*>(dst + 32 * cb + 8 * c8) = v;
+          }
         }
       }
     }

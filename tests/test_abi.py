@@ -157,7 +157,7 @@ def test_multi_query_plan_tiles(lib):
     # 512 new tokens x G 4 = 2048 rows on a 16-bit cache: the query-major
     # kernel, one CTA per (sequence, head, 128-row tile) over all its keys
     nw, per, ws = P.multi_query_plan(8, 32, 8, 128, 4096, 512, P.PKV_BF16)
-    assert nw == 8 * 8 * 16 and per == 4096
+    assert nw == 8 * 8 * 16 // 2 and per == 4096          # one CTA per pair of 128-row tiles
     # an explicit partition keeps the decode kernel's multi-query mode: one
     # stream per (sequence, head, 16-column tile)... capped by the partition
     nw2, per2, ws2 = P.multi_query_plan(8, 32, 8, 128, 4096, 512, P.PKV_BF16, partition_tokens=4096)
