@@ -17,13 +17,14 @@
 //     lane i: the whole online softmax of a row runs in one thread.  Warp 8
 //     loads K/V and issues every MMA.
 //   * Keys stream in tiles of 64 (four 16-token cache blocks found through
-//     the block table) by TMA into a 3-stage ring (128-byte swizzle); K tiles
+//     the block table) by TMA into a 4-stage ring (128-byte swizzle); K tiles
 //     are K-major B operands, V tiles MN-major B operands of the same layout.
 //   * S = Q K^T: tcgen05.mma M=128, N=64, K=16 steps over head_dim into TMEM
 //     (fp32); P = exp2(S - m) in bf16/fp16 written to shared memory (K-major,
-//     swizzled) as the A operand of O += P V (M=128, N=head_dim).  The tensor
-//     core alternates between the two tiles, so one warpgroup's softmax runs
-//     while the other tile's MMAs do; completion is signalled by
+//     swizzled) as the A operand of O += P V (M=128, N=head_dim).  Scores are
+//     double-buffered in TMEM and issued two K/V tiles ahead, and the tensor
+//     core alternates between the two query tiles, so the softmax of one
+//     warpgroup overlaps MMAs of both; completion is signalled by
 //     tcgen05.commit on mbarriers; every wait is bounded.
 //   * Online softmax with a lazy rescale: the exponent base of a row only
 //     moves when its max grows by more than 8 (log2 units), and only then is
@@ -158,10 +159,12 @@ struct PrefillTraits {
   static constexpr int kQBytes = kRegions * kRows * 128;
   static constexpr int kKVRegion = kKeys * 128;        // 64 rows x 128 B
   static constexpr int kStageBytes = 2 * kRegions * kKVRegion;  // K regions, then V regions
-  static constexpr int kStages = 3;
+  static constexpr int kStages = 4;
   static constexpr int kPBytes = kRows * 128;          // 128 rows x 64 keys x 2 B
   static constexpr int kThreads = 9 * 32;              // 2 softmax warpgroups + 1 control warp
-  static constexpr int kTmemCols = 512;                // S_A [0,64) S_B [64,128) O_A [128,..) O_B [256,..)
+  // TMEM: S of tile x, buffer b at 128 x + 64 b (two buffers each), O of
+  // tile x at 256 + 128 x
+  static constexpr int kTmemCols = 512;
   static constexpr int kSmemUsed = 1024 + kTiles * kQBytes + kStages * kStageBytes + kTiles * kPBytes + 256;
   // one CTA per SM (it holds all 512 TMEM columns): ask for more than half
   static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
@@ -192,12 +195,11 @@ __device__ __forceinline__ float sum_p2(uint32_t u) {
 // One CTA: two tiles of 128 (token, head) rows of one (sequence, KV head)
 // ("A" = the later tokens, "B" = the 128 rows before them), warpgroup A
 // (warps 0-3) and B (warps 4-7) each owning one tile's softmax, warp 8
-// loading K/V and issuing every MMA.  The tensor core alternates between
-// the tiles: while one warpgroup turns its scores into P, the MMAs of the
-// other run.  Per K/V tile j the issue order is S_A(j), S_B(j) (j = 0 only),
-// then PV_A(j), S_A(j+1) once P_A(j) is written, PV_B(j), S_B(j+1) once
-// P_B(j) is; a commit after each pair tells the warpgroup that its next
-// scores are ready and that its previous P and O are free.
+// loading K/V and issuing every MMA.  S_x(0), S_x(1) are issued up front;
+// then, for K/V tile j and x = A, B: once P_x(j) is written, P_x(j) . V_j
+// (committed to pv_done[x]) and S_x(j+2) into the score buffer just released
+// (committed to s_full[x][j % 2]).  A warpgroup waits for pv_done before it
+// overwrites P or rescales O, which P_x(j-1) . V_{j-1} has long finished.
 template <int kD, bool kBF16>
 __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -249,11 +251,11 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
   const uint32_t kv_s = q_s + Tr::kTiles * Tr::kQBytes;       // kS stages of K then V
   const uint32_t p_s = kv_s + kS * Tr::kStageBytes;           // P_A, P_B
   const uint32_t bars = p_s + Tr::kTiles * Tr::kPBytes;
-  // barriers: full[kS], empty[kS], s_full[2], p_full[2], o_done[2]
+  // barriers: full[kS], empty[kS], s_full[2 tiles][2 buffers], p_full[2], pv_done[2]
   const uint32_t b_full = bars, b_empty = bars + 8 * kS, b_sfull = bars + 16 * kS;
-  const uint32_t b_pfull = b_sfull + 16, b_odone = b_sfull + 32;
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sptr + (bars - sbase) + 16 * kS + 48);
-  int* const abort_flag = reinterpret_cast<int*>(sptr + (bars - sbase) + 16 * kS + 52);
+  const uint32_t b_pfull = b_sfull + 32, b_pvdone = b_sfull + 48;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sptr + (bars - sbase) + 16 * kS + 64);
+  int* const abort_flag = reinterpret_cast<int*>(sptr + (bars - sbase) + 16 * kS + 68);
   auto aborted = [&]() { return *reinterpret_cast<volatile int*>(abort_flag) != 0; };
   auto wait_or_abort = [&](uint32_t bar, uint32_t parity) {
     if (!mbar_wait(bar, parity)) atomicExch(abort_flag, 1);
@@ -269,9 +271,10 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       mbar_init(b_empty + 8 * i, 1);
     }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(b_sfull + 8 * x, 1);
+      mbar_init(b_sfull + 16 * x, 1);
+      mbar_init(b_sfull + 16 * x + 8, 1);
       mbar_init(b_pfull + 8 * x, Tr::kRows);
-      mbar_init(b_odone + 8 * x, 1);
+      mbar_init(b_pvdone + 8 * x, 1);
     }
     *abort_flag = 0;
     fence_barrier_init();
@@ -337,13 +340,13 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
         }
       }
     };
-    auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T into S_x's TMEM columns
+    auto issue_s = [&](int x, int j) {  // S_x(j) = Q_x K_j^T into score buffer j % 2 of tile x
       const uint32_t st = kv_s + (j % kS) * Tr::kStageBytes;
       const uint32_t qx = q_s + x * Tr::kQBytes;
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
         const int reg = ks >> 2, off = (ks & 3) * 32;
-        umma_f16(tmem + 64 * x, smem_desc_sw128(qx + reg * (Tr::kRows * 128) + off, 16),
+        umma_f16(tmem + 128 * x + 64 * (j & 1), smem_desc_sw128(qx + reg * (Tr::kRows * 128) + off, 16),
                  smem_desc_sw128(st + reg * Tr::kKVRegion + off, 16), kIdescS, ks > 0 ? 1u : 0u);
       }
     };
@@ -352,21 +355,31 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       const uint32_t px = p_s + x * Tr::kPBytes;
 #pragma unroll
       for (int ks = 0; ks < Tr::kKeys / 16; ++ks) {
-        umma_f16(tmem + 128 * (x + 1), smem_desc_sw128(px + ks * 32, 16),
+        umma_f16(tmem + 256 + 128 * x, smem_desc_sw128(px + ks * 32, 16),
                  smem_desc_sw128(st + kR * Tr::kKVRegion + ks * 2048, Tr::kKVRegion), kIdescO,
                  (j > 0 || ks > 0) ? 1u : 0u);
       }
     };
     if (lane == 0) {
       for (int j = 0; j < kS && j < nk; ++j) load_tile(j);
+      // scores of the first two K/V tiles for both query tiles
+      for (int j = 0; j < 2 && j < nk; ++j) {
+        wait_or_abort(b_full + 8 * (j % kS), (j / kS) & 1);
+        tc_fence_after();
+        for (int x = 0; x < 2; ++x) {
+          issue_s(x, j);
+          umma_commit(b_sfull + 16 * x + 8 * (j & 1));
+        }
+      }
     }
+    __syncwarp();
 #pragma unroll 1
     for (int j = 0; j < nk; ++j) {
       const int st_i = j % kS;
       const uint32_t st = kv_s + st_i * Tr::kStageBytes;
       const int kt0 = kbeg + j * Tr::kKeys;
-      wait_or_abort(b_full + 8 * st_i, (j / kS) & 1);
-      consumed = j + 1;
+      wait_or_abort(b_full + 8 * st_i, (j / kS) & 1);  // (already complete: its scores were issued)
+      consumed = max(consumed, j + 1);
       if (aborted()) break;
       // keys of the tile at or past the context: zero their V rows (never
       // written there, or zero-filled already) before any P . V reads them
@@ -381,35 +394,32 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        tc_fence_after();
-        if (j == 0) {
-          issue_s(0, 0);
-          umma_commit(b_sfull);
-          issue_s(1, 0);
-          umma_commit(b_sfull + 8);
-        }
-        const bool more = j + 1 < nk;
-        if (more) {  // the next tile must have landed before its S is issued
-          wait_or_abort(b_full + 8 * ((j + 1) % kS), ((j + 1) / kS) & 1);
+        const bool ahead = j + 2 < nk;
+        if (ahead) {
+          wait_or_abort(b_full + 8 * ((j + 2) % kS), ((j + 2) / kS) & 1);
+          consumed = max(consumed, j + 3);
         }
 #pragma unroll 1
         for (int x = 0; x < 2; ++x) {
-          wait_or_abort(b_pfull + 8 * x, j & 1);  // P_x(j) written
+          wait_or_abort(b_pfull + 8 * x, j & 1);  // P_x(j) written, score buffer j % 2 read
           tc_fence_after();
           issue_pv(x, j);
-          if (more) {
-            issue_s(x, j + 1);
-            umma_commit(b_sfull + 8 * x);
-          } else {
-            umma_commit(b_odone + 8 * x);
+          umma_commit(b_pvdone + 8 * x);
+          if (ahead) {
+            issue_s(x, j + 2);
+            umma_commit(b_sfull + 16 * x + 8 * (j & 1));
+          }
+          if (x == 0 && j >= 1 && j - 1 + kS < nk) {
+            // refill the stage of tile j - 1 with tile j + 3: its last
+            // reader, P_B(j-1) . V, finished while warpgroup A worked on
+            // tile j, so this wait is normally already satisfied
+            const int sp = (j - 1) % kS;
+            wait_or_abort(b_empty + 8 * sp, ((j - 1) / kS) & 1);
+            fence_async_smem();
+            load_tile(j - 1 + kS);
           }
         }
         umma_commit(b_empty + 8 * st_i);  // the stage is read once both P . V are done
-        if (j + kS < nk) {
-          wait_or_abort(b_empty + 8 * st_i, (j / kS) & 1);
-          fence_async_smem();
-          load_tile(j + kS);
-        }
       }
       __syncwarp();
     }
@@ -421,8 +431,8 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     // =================== softmax warpgroup x = wg ===================
     const int x = wg;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + 64 * x + lane_off;
-    const uint32_t tO = tmem + 128 * (x + 1) + lane_off;
+    const uint32_t tS0 = tmem + 128 * x + lane_off;
+    const uint32_t tO = tmem + 256 + 128 * x + lane_off;
     const uint32_t px = p_s + x * Tr::kPBytes;
     // exclusive key bound and window start of this row; rows past the run
     // see one key so that their (discarded) math stays finite
@@ -436,9 +446,10 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     float m_used = -INFINITY, l = 0.0f;
 #pragma unroll 1
     for (int j = 0; j < nk; ++j) {
-      wait_or_abort(b_sfull + 8 * x, j & 1);
+      wait_or_abort(b_sfull + 16 * x + 8 * (j & 1), (j >> 1) & 1);
       if (aborted()) break;
       tc_fence_after();
+      const uint32_t tS = tS0 + 64 * (j & 1);
       float sv[64];
       {
         float a[32], b[32];
@@ -460,9 +471,14 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
           sv[k] = (key < lim && key >= lo) ? sv[k] : -INFINITY;
         }
       }
-      float mr = -INFINITY;
+      // independent partial maxima / sums keep the dependency chains short
+      float mp[8];
 #pragma unroll
-      for (int k = 0; k < 64; ++k) mr = fmaxf(mr, sv[k]);
+      for (int k = 0; k < 8; ++k) mp[k] = fmaxf(sv[k], sv[k + 8]);
+#pragma unroll
+      for (int k = 16; k < 64; ++k) mp[k & 7] = fmaxf(mp[k & 7], sv[k]);
+      const float mr = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float mx = mr * c;  // scores are used as s * c (log2 units)
       float factor = 1.0f;
       bool rescale = false;
@@ -472,23 +488,25 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
         m_used = mx;
       }
       const float nbase = m_used == -INFINITY ? 0.0f : -m_used;
-      float sum = 0.0f;
+      float sp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      uint32_t w[32];
+#pragma unroll
+      for (int k = 0; k < 32; ++k) {
+        w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[2 * k], c, nbase)), fast_exp2(fmaf(sv[2 * k + 1], c, nbase)));
+        sp[k & 3] += sum_p2<kBF16>(w[k]);
+      }
+      const float sum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
+      l = l * factor + sum;
+      // P_x(j-1) . V_{j-1} must be done before P_x is overwritten or O_x
+      // rescaled (issued right after P_x(j-1) was written, long ago)
+      if (j > 0) wait_or_abort(b_pvdone + 8 * x, (j - 1) & 1);
+      tc_fence_after();
 #pragma unroll
       for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t w[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[8 * c8 + 2 * k], c, nbase)),
-                                fast_exp2(fmaf(sv[8 * c8 + 2 * k + 1], c, nbase)));
-          sum += sum_p2<kBF16>(w[k]);
-        }
         *reinterpret_cast<uint4*>(sptr + (px - sbase) + row * 128 + ((c8 ^ (row & 7)) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+            make_uint4(w[4 * c8], w[4 * c8 + 1], w[4 * c8 + 2], w[4 * c8 + 3]);
       }
-      l = l * factor + sum;
       if (__any_sync(0xffffffffu, rescale)) {
-        // O_x up to tile j - 1 is complete (the commit that released these
-        // scores came after it)
         const float f = rescale ? factor : 1.0f;
 #pragma unroll 1
         for (int cb = 0; cb < kD / 32; ++cb) {
@@ -506,7 +524,7 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       mbar_arrive(b_pfull + 8 * x);
     }
     // ---- epilogue: O / l -> out ----
-    wait_or_abort(b_odone + 8 * x, 0);
+    wait_or_abort(b_pvdone + 8 * x, (nk - 1) & 1);
     tc_fence_after();
     if (!aborted()) {
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;
