@@ -315,7 +315,16 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
   if (wg == 2) {
     // =================== control warp: K/V loads and all MMAs ===================
     int issued = 0, consumed = 0;
-    auto load_tile = [&](int j) {
+    // Block ids of K/V tile j, read well before they are needed: the four
+    // loads are independent, and their first use comes after a long wait.
+    auto fetch_ids = [&](int j, int (&ids)[4]) {
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const int kb = (kbeg >> 4) + 4 * j + b;  // logical block
+        ids[b] = kb * 16 < ctx ? p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + kb] : -1;
+      }
+    };
+    auto load_tile = [&](int j, const int (&ids)[4]) {
       const int st_i = j % kS;
       const uint32_t st = kv_s + st_i * Tr::kStageBytes;
       const uint32_t bar = b_full + 8 * st_i;
@@ -323,10 +332,9 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       mbar_arrive_expect_tx(bar, Tr::kStageBytes);
 #pragma unroll
       for (int b = 0; b < 4; ++b) {
-        const int kb = (kbeg >> 4) + 4 * j + b;  // logical block
-        int row0 = p.oob_row;                    // past the context: zero fill
-        if (kb * 16 < ctx) {
-          int id = p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + kb];
+        int row0 = p.oob_row;  // past the context: zero fill
+        int id = ids[b];
+        if (id != -1) {
           if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
             raise_status(PKV_DEV_BAD_BLOCK);
             id = 0;
@@ -361,7 +369,9 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       }
     };
     if (lane == 0) {
-      for (int j = 0; j < kS && j < nk; ++j) load_tile(j);
+      int ids0[kS][4];
+      for (int j = 0; j < kS && j < nk; ++j) fetch_ids(j, ids0[j]);
+      for (int j = 0; j < kS && j < nk; ++j) load_tile(j, ids0[j]);
       // scores of the first two K/V tiles for both query tiles
       for (int j = 0; j < 2 && j < nk; ++j) {
         wait_or_abort(b_full + 8 * (j % kS), (j / kS) & 1);
@@ -394,6 +404,9 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
+        const bool refill = j >= 1 && j - 1 + kS < nk;
+        int nids[4];
+        if (refill) fetch_ids(j - 1 + kS, nids);  // used after the waits below
         const bool ahead = j + 2 < nk;
         if (ahead) {
           wait_or_abort(b_full + 8 * ((j + 2) % kS), ((j + 2) / kS) & 1);
@@ -409,14 +422,14 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
             issue_s(x, j + 2);
             umma_commit(b_sfull + 16 * x + 8 * (j & 1));
           }
-          if (x == 0 && j >= 1 && j - 1 + kS < nk) {
+          if (x == 0 && refill) {
             // refill the stage of tile j - 1 with tile j + 3: its last
             // reader, P_B(j-1) . V, finished while warpgroup A worked on
             // tile j, so this wait is normally already satisfied
             const int sp = (j - 1) % kS;
             wait_or_abort(b_empty + 8 * sp, ((j - 1) / kS) & 1);
             fence_async_smem();
-            load_tile(j - 1 + kS);
+            load_tile(j - 1 + kS, nids);
           }
         }
         umma_commit(b_empty + 8 * st_i);  // the stage is read once both P . V are done
