@@ -161,7 +161,7 @@ struct PrefillTraits {
   static constexpr int kStageBytes = 2 * kRegions * kKVRegion;  // K regions, then V regions
   static constexpr int kStages = 4;
   static constexpr int kPBytes = kRows * 128;          // 128 rows x 64 keys x 2 B
-  static constexpr int kThreads = 9 * 32;              // 2 softmax warpgroups + 1 control warp
+  static constexpr int kThreads = 10 * 32;             // 2 softmax warpgroups, MMA warp, load warp
   // TMEM: S of tile x, buffer b at 128 x + 64 b (two buffers each), O of
   // tile x at 256 + 128 x
   static constexpr int kTmemCols = 512;
@@ -195,11 +195,12 @@ __device__ __forceinline__ float sum_p2(uint32_t u) {
 // One CTA: two tiles of 128 (token, head) rows of one (sequence, KV head)
 // ("A" = the later tokens, "B" = the 128 rows before them), warpgroup A
 // (warps 0-3) and B (warps 4-7) each owning one tile's softmax, warp 8
-// loading K/V and issuing every MMA.  S_x(0), S_x(1) are issued up front;
-// then, for K/V tile j and x = A, B: once P_x(j) is written, P_x(j) . V_j
-// (committed to pv_done[x]) and S_x(j+2) into the score buffer just released
-// (committed to s_full[x][j % 2]).  A warpgroup waits for pv_done before it
-// overwrites P or rescales O, which P_x(j-1) . V_{j-1} has long finished.
+// issuing every MMA and warp 9 loading K/V into a ring of stages (a stage is
+// refilled once both P . V of its tile are done).  S_x(0), S_x(1) are issued
+// up front; then, for K/V tile j and x = A, B: once P_x(j) is written,
+// P_x(j) . V_j (committed to pv_done[x]) and S_x(j+2) into the score buffer
+// just released (committed to s_full[x][j % 2]).  A warpgroup waits for
+// pv_done before it overwrites P or rescales O.
 template <int kD, bool kBF16>
 __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
@@ -281,7 +282,7 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
   }
 
   // ---- Q tiles -> shared memory, K-major with the 128-byte swizzle ----
-  const int wg = warp >> 2;          // 0: tile A, 1: tile B, 2: control warp
+  const int wg = warp >> 2;          // 0: tile A, 1: tile B, 2: MMA warp (8) and load warp (9)
   const int row = tid & 127;         // row of the warpgroup's tile / TMEM lane
   const int t0x = wg == 0 ? ta0 : tb0;
   const int ntx = wg == 0 ? nta : ntb;
@@ -312,66 +313,90 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
   constexpr uint32_t kIdescS = umma_idesc(128, Tr::kKeys, kBF16, false);
   constexpr uint32_t kIdescO = umma_idesc(128, kD, kBF16, true);
 
-  if (wg == 2) {
-    // =================== control warp: K/V loads and all MMAs ===================
-    int issued = 0, consumed = 0;
-    // Block ids of K/V tile j, read well before they are needed: the four
-    // loads are independent, and their first use comes after a long wait.
-    auto fetch_ids = [&](int j, int (&ids)[4]) {
+  if (warp == 9) {
+    // =================== load warp: K/V tiles through the stage ring ===================
+    if (lane == 0) {
+      // Block ids of K/V tile j; those of the next tile are read before the
+      // wait for a free stage, so their latency hides behind it.
+      auto fetch_ids = [&](int j, int (&ids)[4]) {
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const int kb = (kbeg >> 4) + 4 * j + b;  // logical block
-        ids[b] = kb * 16 < ctx ? p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + kb] : -1;
-      }
-    };
-    auto load_tile = [&](int j, const int (&ids)[4]) {
-      const int st_i = j % kS;
-      const uint32_t st = kv_s + st_i * Tr::kStageBytes;
-      const uint32_t bar = b_full + 8 * st_i;
-      ++issued;
-      mbar_arrive_expect_tx(bar, Tr::kStageBytes);
+        for (int b = 0; b < 4; ++b) {
+          const int kb = (kbeg >> 4) + 4 * j + b;  // logical block
+          ids[b] = kb * 16 < ctx ? p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + kb] : -1;
+        }
+      };
+      int issued = 0;
+      int ids[4], nxt[4];
+      if (nk > 0) fetch_ids(0, ids);
+#pragma unroll 1
+      for (int j = 0; j < nk; ++j) {
+        if (j + 1 < nk) fetch_ids(j + 1, nxt);
+        const int st_i = j % kS;
+        if (j >= kS) {
+          // the stage's previous tile (j - kS) has been read by both P . V
+          wait_or_abort(b_empty + 8 * st_i, ((j - kS) / kS) & 1);
+          if (aborted()) break;
+          fence_async_smem();
+        }
+        const uint32_t st = kv_s + st_i * Tr::kStageBytes;
+        const uint32_t bar = b_full + 8 * st_i;
+        mbar_arrive_expect_tx(bar, Tr::kStageBytes);
+        ++issued;
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        int row0 = p.oob_row;  // past the context: zero fill
-        int id = ids[b];
-        if (id != -1) {
-          if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
-            raise_status(PKV_DEV_BAD_BLOCK);
-            id = 0;
+        for (int b = 0; b < 4; ++b) {
+          int row0 = p.oob_row;  // past the context: zero fill
+          int id = ids[b];
+          if (id != -1) {
+            if (static_cast<unsigned>(id) >= static_cast<unsigned>(p.num_blocks)) {
+              raise_status(PKV_DEV_BAD_BLOCK);
+              id = 0;
+            }
+            row0 = (id * p.num_kv_heads + h) * 16;
           }
-          row0 = (id * p.num_kv_heads + h) * 16;
+#pragma unroll
+          for (int r = 0; r < kR; ++r) {
+            tma_load_2d(st + r * Tr::kKVRegion + b * 2048, &kmap, r * 64, row0, bar);
+            tma_load_2d(st + (kR + r) * Tr::kKVRegion + b * 2048, &vmap, r * 64, row0, bar);
+          }
         }
 #pragma unroll
-        for (int r = 0; r < kR; ++r) {
-          tma_load_2d(st + r * Tr::kKVRegion + b * 2048, &kmap, r * 64, row0, bar);
-          tma_load_2d(st + (kR + r) * Tr::kKVRegion + b * 2048, &vmap, r * 64, row0, bar);
-        }
+        for (int b = 0; b < 4; ++b) ids[b] = nxt[b];
       }
-    };
+      // loads still in flight after an abort land (bounded) before exit; the
+      // last tile of each stage is the only one that can still be pending
+      for (int j = max(issued - kS, 0); j < issued; ++j) mbar_wait(b_full + 8 * (j % kS), (j / kS) & 1);
+    }
+  } else if (warp == 8) {
+    // =================== MMA warp: every tcgen05.mma, issued by lane 0 ===================
+    // Descriptors are computed once; a K-step or a stage moves only the
+    // start-address field (bits 0-13, 16-byte units), so each MMA adds a
+    // small constant instead of rebuilding its descriptors.
+    const uint64_t dq0 = smem_desc_sw128(q_s, 16);
+    const uint64_t dk0 = smem_desc_sw128(kv_s, 16);
+    const uint64_t dv0 = smem_desc_sw128(kv_s + kR * Tr::kKVRegion, Tr::kKVRegion);
+    const uint64_t dp0 = smem_desc_sw128(p_s, 16);
     auto issue_s = [&](int x, int j) {  // S_x(j) = Q_x K_j^T into score buffer j % 2 of tile x
-      const uint32_t st = kv_s + (j % kS) * Tr::kStageBytes;
-      const uint32_t qx = q_s + x * Tr::kQBytes;
+      const uint64_t dq = dq0 + static_cast<uint32_t>(x * (Tr::kQBytes >> 4));
+      const uint64_t dk = dk0 + static_cast<uint32_t>((j % kS) * (Tr::kStageBytes >> 4));
+      const uint32_t d = tmem + 128 * x + 64 * (j & 1);
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
-        const int reg = ks >> 2, off = (ks & 3) * 32;
-        umma_f16(tmem + 128 * x + 64 * (j & 1), smem_desc_sw128(qx + reg * (Tr::kRows * 128) + off, 16),
-                 smem_desc_sw128(st + reg * Tr::kKVRegion + off, 16), kIdescS, ks > 0 ? 1u : 0u);
+        constexpr int kQReg = Tr::kRows * 128 / 16, kKReg = Tr::kKVRegion / 16;
+        const uint32_t qo = (ks >> 2) * kQReg + (ks & 3) * 2, ko = (ks >> 2) * kKReg + (ks & 3) * 2;
+        umma_f16(d, dq + qo, dk + ko, kIdescS, ks > 0 ? 1u : 0u);
       }
     };
     auto issue_pv = [&](int x, int j) {  // O_x += P_x V_j
-      const uint32_t st = kv_s + (j % kS) * Tr::kStageBytes;
-      const uint32_t px = p_s + x * Tr::kPBytes;
+      const uint64_t dp = dp0 + static_cast<uint32_t>(x * (Tr::kPBytes >> 4));
+      const uint64_t dv = dv0 + static_cast<uint32_t>((j % kS) * (Tr::kStageBytes >> 4));
+      const uint32_t d = tmem + 256 + 128 * x;
 #pragma unroll
       for (int ks = 0; ks < Tr::kKeys / 16; ++ks) {
-        umma_f16(tmem + 256 + 128 * x, smem_desc_sw128(px + ks * 32, 16),
-                 smem_desc_sw128(st + kR * Tr::kKVRegion + ks * 2048, Tr::kKVRegion), kIdescO,
+        umma_f16(d, dp + static_cast<uint32_t>(ks * 2), dv + static_cast<uint32_t>(ks * 128), kIdescO,
                  (j > 0 || ks > 0) ? 1u : 0u);
       }
     };
     if (lane == 0) {
-      int ids0[kS][4];
-      for (int j = 0; j < kS && j < nk; ++j) fetch_ids(j, ids0[j]);
-      for (int j = 0; j < kS && j < nk; ++j) load_tile(j, ids0[j]);
       // scores of the first two K/V tiles for both query tiles
       for (int j = 0; j < 2 && j < nk; ++j) {
         wait_or_abort(b_full + 8 * (j % kS), (j / kS) & 1);
@@ -389,7 +414,6 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       const uint32_t st = kv_s + st_i * Tr::kStageBytes;
       const int kt0 = kbeg + j * Tr::kKeys;
       wait_or_abort(b_full + 8 * st_i, (j / kS) & 1);  // (already complete: its scores were issued)
-      consumed = max(consumed, j + 1);
       if (aborted()) break;
       // keys of the tile at or past the context: zero their V rows (never
       // written there, or zero-filled already) before any P . V reads them
@@ -404,41 +428,26 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       }
       __syncwarp();
       if (lane == 0) {
-        const bool refill = j >= 1 && j - 1 + kS < nk;
-        int nids[4];
-        if (refill) fetch_ids(j - 1 + kS, nids);  // used after the waits below
         const bool ahead = j + 2 < nk;
-        if (ahead) {
-          wait_or_abort(b_full + 8 * ((j + 2) % kS), ((j + 2) / kS) & 1);
-          consumed = max(consumed, j + 3);
-        }
 #pragma unroll 1
         for (int x = 0; x < 2; ++x) {
           wait_or_abort(b_pfull + 8 * x, j & 1);  // P_x(j) written, score buffer j % 2 read
           tc_fence_after();
           issue_pv(x, j);
           umma_commit(b_pvdone + 8 * x);
+          // the stage is free once both P . V of this tile are done
+          if (x == 1) umma_commit(b_empty + 8 * st_i);
           if (ahead) {
+            if (x == 0) {
+              wait_or_abort(b_full + 8 * ((j + 2) % kS), ((j + 2) / kS) & 1);
+              tc_fence_after();
+            }
             issue_s(x, j + 2);
             umma_commit(b_sfull + 16 * x + 8 * (j & 1));
           }
-          if (x == 0 && refill) {
-            // refill the stage of tile j - 1 with tile j + 3: its last
-            // reader, P_B(j-1) . V, finished while warpgroup A worked on
-            // tile j, so this wait is normally already satisfied
-            const int sp = (j - 1) % kS;
-            wait_or_abort(b_empty + 8 * sp, ((j - 1) / kS) & 1);
-            fence_async_smem();
-            load_tile(j - 1 + kS, nids);
-          }
         }
-        umma_commit(b_empty + 8 * st_i);  // the stage is read once both P . V are done
       }
       __syncwarp();
-    }
-    // loads still in flight after an abort land (bounded) before exit
-    if (lane == 0) {
-      for (int j = consumed; j < issued; ++j) mbar_wait(b_full + 8 * (j % kS), (j / kS) & 1);
     }
   } else {
     // =================== softmax warpgroup x = wg ===================
