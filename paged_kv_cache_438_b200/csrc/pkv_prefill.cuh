@@ -65,6 +65,18 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t adesc, uint64
       : "memory");
 }
 
+// D[tmem] (+)= A[tmem] . B[smem]^T: A (M rows = TMEM lanes, K along the
+// columns, two 16-bit elements per column) is read from tensor memory.
+__device__ __forceinline__ void umma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
 // Arrive once on the mbarrier when every MMA this thread issued so far is done.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
@@ -102,6 +114,16 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float (&v)[32]) 
       "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])), "r"(__float_as_uint(v[26])),
       "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])), "r"(__float_as_uint(v[29])),
       "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+      : "memory");
+}
+
+// 16 consecutive 32-bit columns of the calling thread's TMEM lane (warp-wide).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]), "r"(w[8]), "r"(w[9]),
+      "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]), "r"(w[15])
       : "memory");
 }
 
@@ -154,27 +176,44 @@ template <int kD>
 struct PrefillTraits {
   static constexpr int kRows = 128;                    // query rows per tile (M)
   static constexpr int kTiles = 2;                     // query tiles per CTA (ping-pong)
-  static constexpr int kKeys = 64;                     // keys per K/V tile (N of S)
+  static constexpr int kKeys = 128;                    // keys per K/V tile (N of S, K of P . V)
+  static constexpr int kBlocks = kKeys / 16;           // cache blocks per K/V tile
   static constexpr int kRegions = kD / 64;             // 128-byte column regions of a row
   static constexpr int kQBytes = kRegions * kRows * 128;
-  static constexpr int kKVRegion = kKeys * 128;        // 64 rows x 128 B
-  static constexpr int kStageBytes = 2 * kRegions * kKVRegion;  // K regions, then V regions
-  static constexpr int kStages = 4;
-  static constexpr int kPBytes = kRows * 128;          // 128 rows x 64 keys x 2 B
+  static constexpr int kRegionBytes = kKeys * 128;     // 128 rows x 128 B
+  static constexpr int kEntryBytes = kRegions * kRegionBytes;  // one K tile or one V tile
+  static constexpr int kBarBytes = 256;
+  static constexpr int kFit = (227 * 1024 - 1024 - kTiles * kQBytes - kBarBytes) / kEntryBytes;
+  static constexpr int kEntries = kFit > 8 ? 8 : kFit;  // ring of K and V tiles: K0 V0 K1 V1 ...
   static constexpr int kThreads = 10 * 32;             // 2 softmax warpgroups, MMA warp, load warp
-  // TMEM: S of tile x, buffer b at 128 x + 64 b (two buffers each), O of
-  // tile x at 256 + 128 x
+  // TMEM: S of tile x at 128 x (P of tile x, 16-bit, over its upper half at
+  // 128 x + 64), O of tile x at 256 + 128 x
   static constexpr int kTmemCols = 512;
-  static constexpr int kSmemUsed = 1024 + kTiles * kQBytes + kStages * kStageBytes + kTiles * kPBytes + 256;
+  static constexpr int kSmemUsed = 1024 + kTiles * kQBytes + kEntries * kEntryBytes + kBarBytes;
   // one CTA per SM (it holds all 512 TMEM columns): ask for more than half
   static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
 };
 
+// Two output values, round to nearest.
 template <bool kBF16>
-__device__ __forceinline__ uint32_t pack_p2(float a, float b) {
+__device__ __forceinline__ uint32_t pack_out(float a, float b) {
   if constexpr (kBF16) {
     __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    __half2 v = __floats2half2_rn(a, b);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+}
+
+// Two probabilities packed as the MMA's 16-bit operand pair (a in the low
+// half).  bf16 keeps the top 16 bits (rounding toward zero: one byte permute
+// instead of a conversion); the row sum is taken over the same packed values,
+// so the normalisation matches what the MMA multiplies.
+template <bool kBF16>
+__device__ __forceinline__ uint32_t pack_p2(float a, float b) {
+  if constexpr (kBF16) {
+    return __byte_perm(__float_as_uint(a), __float_as_uint(b), 0x7632);
   } else {
     __half2 v = __floats2half2_rn(a, b);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -195,19 +234,23 @@ __device__ __forceinline__ float sum_p2(uint32_t u) {
 // One CTA: two tiles of 128 (token, head) rows of one (sequence, KV head)
 // ("A" = the later tokens, "B" = the 128 rows before them), warpgroup A
 // (warps 0-3) and B (warps 4-7) each owning one tile's softmax, warp 8
-// issuing every MMA and warp 9 loading K/V into a ring of stages (a stage is
-// refilled once both P . V of its tile are done).  S_x(0), S_x(1) are issued
-// up front; then, for K/V tile j and x = A, B: once P_x(j) is written,
-// P_x(j) . V_j (committed to pv_done[x]) and S_x(j+2) into the score buffer
-// just released (committed to s_full[x][j % 2]).  A warpgroup waits for
-// pv_done before it overwrites P or rescales O.
+// issuing every MMA and warp 9 loading K and V tiles into a ring of entries
+// (an entry is refilled once the MMAs that read it are done).  For K/V tile
+// j and x = A, B, once P_x(j) is in TMEM: O_x += P_x(j) . V_j, then
+// S_x(j+1) = Q_x K_{j+1}^T into the same TMEM columns (the tensor core runs
+// one thread's MMAs in issue order, so P_x(j) is read before it is
+// overwritten), committed to s_full[x].  That commit also covers every
+// earlier MMA, so a warpgroup that sees S_x(j+1) may rescale O_x and write
+// P_x(j+1) without further waits.
 template <int kD, bool kBF16>
 __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     paged_prefill_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                          const PrefillParams p) {
   using Tr = PrefillTraits<kD>;
   constexpr int kR = Tr::kRegions;
-  constexpr int kS = Tr::kStages;
+  constexpr int kE = Tr::kEntries;
+  constexpr int kN = Tr::kKeys;
+  constexpr int kBlk = Tr::kBlocks;
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
@@ -242,21 +285,20 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
   const int t_first = tile_b >= 0 ? tb0 : ta0;
   const int kfirst = p.window > 0 ? max(0, ctx - n + t_first + 1 - p.window) : 0;
   const int kbeg = kfirst & ~15;
-  const int nk = (klim - kbeg + Tr::kKeys - 1) / Tr::kKeys;
+  const int nk = (klim - kbeg + kN - 1) / kN;
 
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_addr(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t* const sptr = smem_raw + (sbase - raw);
   const uint32_t q_s = sbase;                                  // Q_A, Q_B
-  const uint32_t kv_s = q_s + Tr::kTiles * Tr::kQBytes;       // kS stages of K then V
-  const uint32_t p_s = kv_s + kS * Tr::kStageBytes;           // P_A, P_B
-  const uint32_t bars = p_s + Tr::kTiles * Tr::kPBytes;
-  // barriers: full[kS], empty[kS], s_full[2 tiles][2 buffers], p_full[2], pv_done[2]
-  const uint32_t b_full = bars, b_empty = bars + 8 * kS, b_sfull = bars + 16 * kS;
-  const uint32_t b_pfull = b_sfull + 32, b_pvdone = b_sfull + 48;
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sptr + (bars - sbase) + 16 * kS + 64);
-  int* const abort_flag = reinterpret_cast<int*>(sptr + (bars - sbase) + 16 * kS + 68);
+  const uint32_t kv_s = q_s + Tr::kTiles * Tr::kQBytes;       // kE ring entries
+  const uint32_t bars = kv_s + kE * Tr::kEntryBytes;
+  // barriers: full[kE], empty[kE], s_full[2], p_full[2], o_full
+  const uint32_t b_full = bars, b_empty = bars + 8 * kE, b_sfull = bars + 16 * kE;
+  const uint32_t b_pfull = b_sfull + 16, b_ofull = b_sfull + 32;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sptr + (bars - sbase) + 16 * kE + 40);
+  int* const abort_flag = reinterpret_cast<int*>(sptr + (bars - sbase) + 16 * kE + 44);
   auto aborted = [&]() { return *reinterpret_cast<volatile int*>(abort_flag) != 0; };
   auto wait_or_abort = [&](uint32_t bar, uint32_t parity) {
     if (!mbar_wait(bar, parity)) atomicExch(abort_flag, 1);
@@ -267,16 +309,15 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int i = 0; i < kS; ++i) {
+    for (int i = 0; i < kE; ++i) {
       mbar_init(b_full + 8 * i, 1);
       mbar_init(b_empty + 8 * i, 1);
     }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(b_sfull + 16 * x, 1);
-      mbar_init(b_sfull + 16 * x + 8, 1);
+      mbar_init(b_sfull + 8 * x, 1);
       mbar_init(b_pfull + 8 * x, Tr::kRows);
-      mbar_init(b_pvdone + 8 * x, 1);
     }
+    mbar_init(b_ofull, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -310,40 +351,45 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
   // the cache may still be being written by the preceding kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
 
-  constexpr uint32_t kIdescS = umma_idesc(128, Tr::kKeys, kBF16, false);
+  constexpr uint32_t kIdescS = umma_idesc(128, kN, kBF16, false);
   constexpr uint32_t kIdescO = umma_idesc(128, kD, kBF16, true);
 
   if (warp == 9) {
-    // =================== load warp: K/V tiles through the stage ring ===================
+    // =================== load warp: K_0 V_0 K_1 V_1 ... through the ring ===================
     if (lane == 0) {
       // Block ids of K/V tile j; those of the next tile are read before the
-      // wait for a free stage, so their latency hides behind it.
-      auto fetch_ids = [&](int j, int (&ids)[4]) {
+      // waits for free entries, so their latency hides behind them.
+      auto fetch_ids = [&](int j, int (&ids)[kBlk]) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
-          const int kb = (kbeg >> 4) + 4 * j + b;  // logical block
+        for (int b = 0; b < kBlk; ++b) {
+          const int kb = (kbeg >> 4) + kBlk * j + b;  // logical block
           ids[b] = kb * 16 < ctx ? p.block_tables[static_cast<long long>(s) * p.max_blocks_per_seq + kb] : -1;
         }
       };
       int issued = 0;
-      int ids[4], nxt[4];
+      int ids[kBlk], nxt[kBlk];
+#pragma unroll
+      for (int b = 0; b < kBlk; ++b) nxt[b] = -1;
       if (nk > 0) fetch_ids(0, ids);
 #pragma unroll 1
-      for (int j = 0; j < nk; ++j) {
-        if (j + 1 < nk) fetch_ids(j + 1, nxt);
-        const int st_i = j % kS;
-        if (j >= kS) {
-          // the stage's previous tile (j - kS) has been read by both P . V
-          wait_or_abort(b_empty + 8 * st_i, ((j - kS) / kS) & 1);
+      for (int i = 0; i < 2 * nk; ++i) {
+        const int j = i >> 1;
+        const bool is_v = (i & 1) != 0;
+        if (!is_v && j + 1 < nk) fetch_ids(j + 1, nxt);
+        const int slot = i % kE;
+        if (i >= kE) {
+          // the entry's previous tile (i - kE) has been read by its MMAs
+          wait_or_abort(b_empty + 8 * slot, ((i - kE) / kE) & 1);
           if (aborted()) break;
           fence_async_smem();
         }
-        const uint32_t st = kv_s + st_i * Tr::kStageBytes;
-        const uint32_t bar = b_full + 8 * st_i;
-        mbar_arrive_expect_tx(bar, Tr::kStageBytes);
+        const uint32_t dst = kv_s + slot * Tr::kEntryBytes;
+        const uint32_t bar = b_full + 8 * slot;
+        const CUtensorMap* map = is_v ? &vmap : &kmap;
+        mbar_arrive_expect_tx(bar, Tr::kEntryBytes);
         ++issued;
 #pragma unroll
-        for (int b = 0; b < 4; ++b) {
+        for (int b = 0; b < kBlk; ++b) {
           int row0 = p.oob_row;  // past the context: zero fill
           int id = ids[b];
           if (id != -1) {
@@ -354,98 +400,93 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
             row0 = (id * p.num_kv_heads + h) * 16;
           }
 #pragma unroll
-          for (int r = 0; r < kR; ++r) {
-            tma_load_2d(st + r * Tr::kKVRegion + b * 2048, &kmap, r * 64, row0, bar);
-            tma_load_2d(st + (kR + r) * Tr::kKVRegion + b * 2048, &vmap, r * 64, row0, bar);
-          }
+          for (int r = 0; r < kR; ++r) tma_load_2d(dst + r * Tr::kRegionBytes + b * 2048, map, r * 64, row0, bar);
         }
+        if (is_v) {
 #pragma unroll
-        for (int b = 0; b < 4; ++b) ids[b] = nxt[b];
+          for (int b = 0; b < kBlk; ++b) ids[b] = nxt[b];
+        }
       }
       // loads still in flight after an abort land (bounded) before exit; the
-      // last tile of each stage is the only one that can still be pending
-      for (int j = max(issued - kS, 0); j < issued; ++j) mbar_wait(b_full + 8 * (j % kS), (j / kS) & 1);
+      // last tile of each entry is the only one that can still be pending
+      for (int i = max(issued - kE, 0); i < issued; ++i) mbar_wait(b_full + 8 * (i % kE), (i / kE) & 1);
     }
   } else if (warp == 8) {
     // =================== MMA warp: every tcgen05.mma, issued by lane 0 ===================
-    // Descriptors are computed once; a K-step or a stage moves only the
+    // Descriptors are computed once; a K-step or an entry moves only the
     // start-address field (bits 0-13, 16-byte units), so each MMA adds a
     // small constant instead of rebuilding its descriptors.
     const uint64_t dq0 = smem_desc_sw128(q_s, 16);
-    const uint64_t dk0 = smem_desc_sw128(kv_s, 16);
-    const uint64_t dv0 = smem_desc_sw128(kv_s + kR * Tr::kKVRegion, Tr::kKVRegion);
-    const uint64_t dp0 = smem_desc_sw128(p_s, 16);
-    auto issue_s = [&](int x, int j) {  // S_x(j) = Q_x K_j^T into score buffer j % 2 of tile x
+    const uint64_t dk0 = smem_desc_sw128(kv_s, 16);                  // K tiles: K-major
+    const uint64_t dv0 = smem_desc_sw128(kv_s, Tr::kRegionBytes);    // V tiles: MN-major
+    auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T
       const uint64_t dq = dq0 + static_cast<uint32_t>(x * (Tr::kQBytes >> 4));
-      const uint64_t dk = dk0 + static_cast<uint32_t>((j % kS) * (Tr::kStageBytes >> 4));
-      const uint32_t d = tmem + 128 * x + 64 * (j & 1);
+      const uint64_t dk = dk0 + static_cast<uint32_t>(((2 * j) % kE) * (Tr::kEntryBytes >> 4));
+      const uint32_t d = tmem + 128 * x;
 #pragma unroll
       for (int ks = 0; ks < kD / 16; ++ks) {
-        constexpr int kQReg = Tr::kRows * 128 / 16, kKReg = Tr::kKVRegion / 16;
+        constexpr int kQReg = Tr::kRows * 128 / 16, kKReg = Tr::kRegionBytes / 16;
         const uint32_t qo = (ks >> 2) * kQReg + (ks & 3) * 2, ko = (ks >> 2) * kKReg + (ks & 3) * 2;
         umma_f16(d, dq + qo, dk + ko, kIdescS, ks > 0 ? 1u : 0u);
       }
     };
-    auto issue_pv = [&](int x, int j) {  // O_x += P_x V_j
-      const uint64_t dp = dp0 + static_cast<uint32_t>(x * (Tr::kPBytes >> 4));
-      const uint64_t dv = dv0 + static_cast<uint32_t>((j % kS) * (Tr::kStageBytes >> 4));
+    auto issue_pv = [&](int x, int j) {  // O_x += P_x V_j, P_x read from TMEM
+      const uint64_t dv = dv0 + static_cast<uint32_t>(((2 * j + 1) % kE) * (Tr::kEntryBytes >> 4));
+      const uint32_t a = tmem + 128 * x + 64;
       const uint32_t d = tmem + 256 + 128 * x;
 #pragma unroll
-      for (int ks = 0; ks < Tr::kKeys / 16; ++ks) {
-        umma_f16(d, dp + static_cast<uint32_t>(ks * 2), dv + static_cast<uint32_t>(ks * 128), kIdescO,
-                 (j > 0 || ks > 0) ? 1u : 0u);
+      for (int ks = 0; ks < kN / 16; ++ks) {
+        umma_f16_ts(d, a + 8 * ks, dv + static_cast<uint32_t>(ks * 128), kIdescO, (j > 0 || ks > 0) ? 1u : 0u);
       }
     };
-    if (lane == 0) {
-      // scores of the first two K/V tiles for both query tiles
-      for (int j = 0; j < 2 && j < nk; ++j) {
-        wait_or_abort(b_full + 8 * (j % kS), (j / kS) & 1);
-        tc_fence_after();
-        for (int x = 0; x < 2; ++x) {
-          issue_s(x, j);
-          umma_commit(b_sfull + 16 * x + 8 * (j & 1));
-        }
-      }
+    if (lane == 0 && nk > 0) {
+      wait_or_abort(b_full, 0);  // K_0 sits in entry 0
+      tc_fence_after();
+      issue_s(0, 0);
+      umma_commit(b_sfull);
+      issue_s(1, 0);
+      umma_commit(b_sfull + 8);
+      umma_commit(b_empty);
     }
     __syncwarp();
 #pragma unroll 1
     for (int j = 0; j < nk; ++j) {
-      const int st_i = j % kS;
-      const uint32_t st = kv_s + st_i * Tr::kStageBytes;
-      const int kt0 = kbeg + j * Tr::kKeys;
-      wait_or_abort(b_full + 8 * st_i, (j / kS) & 1);  // (already complete: its scores were issued)
+      const int vi = 2 * j + 1, vslot = vi % kE;
+      const int kt0 = kbeg + j * kN;
+      wait_or_abort(b_full + 8 * vslot, (vi / kE) & 1);
       if (aborted()) break;
       // keys of the tile at or past the context: zero their V rows (never
       // written there, or zero-filled already) before any P . V reads them
-      if (kt0 + Tr::kKeys > ctx) {
+      if (kt0 + kN > ctx) {
         const int r0 = max(ctx - kt0, 0);
-        for (int e = lane; e < (Tr::kKeys - r0) * kR * 8; e += 32) {
+        uint8_t* const ve = sptr + (kv_s + vslot * Tr::kEntryBytes - sbase);
+        for (int e = lane; e < (kN - r0) * kR * 8; e += 32) {
           const int rr = r0 + e / (kR * 8), reg = (e / 8) % kR, c = e % 8;
-          *reinterpret_cast<uint4*>(sptr + (st - sbase) + (kR + reg) * Tr::kKVRegion + rr * 128 + c * 16) =
-              make_uint4(0u, 0u, 0u, 0u);
+          *reinterpret_cast<uint4*>(ve + reg * Tr::kRegionBytes + rr * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
         }
         fence_async_smem();
       }
       __syncwarp();
       if (lane == 0) {
-        const bool ahead = j + 2 < nk;
+        const bool more = j + 1 < nk;
+        const int ki = 2 * (j + 1), kslot = ki % kE;
 #pragma unroll 1
         for (int x = 0; x < 2; ++x) {
-          wait_or_abort(b_pfull + 8 * x, j & 1);  // P_x(j) written, score buffer j % 2 read
+          wait_or_abort(b_pfull + 8 * x, j & 1);  // P_x(j) in TMEM, O_x rescaled
           tc_fence_after();
           issue_pv(x, j);
-          umma_commit(b_pvdone + 8 * x);
-          // the stage is free once both P . V of this tile are done
-          if (x == 1) umma_commit(b_empty + 8 * st_i);
-          if (ahead) {
+          if (x == 1) umma_commit(b_empty + 8 * vslot);  // V_j read by both P . V
+          if (more) {
             if (x == 0) {
-              wait_or_abort(b_full + 8 * ((j + 2) % kS), ((j + 2) / kS) & 1);
+              wait_or_abort(b_full + 8 * kslot, (ki / kE) & 1);
               tc_fence_after();
             }
-            issue_s(x, j + 2);
-            umma_commit(b_sfull + 16 * x + 8 * (j & 1));
+            issue_s(x, j + 1);
+            umma_commit(b_sfull + 8 * x);
+            if (x == 1) umma_commit(b_empty + 8 * kslot);  // K_{j+1} read by both S
           }
         }
+        if (!more) umma_commit(b_ofull);  // every MMA of the CTA done
       }
       __syncwarp();
     }
@@ -453,9 +494,9 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     // =================== softmax warpgroup x = wg ===================
     const int x = wg;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS0 = tmem + 128 * x + lane_off;
+    const uint32_t tS = tmem + 128 * x + lane_off;
+    const uint32_t tP = tS + 64;
     const uint32_t tO = tmem + 256 + 128 * x + lane_off;
-    const uint32_t px = p_s + x * Tr::kPBytes;
     // exclusive key bound and window start of this row; rows past the run
     // see one key so that their (discarded) math stays finite
     const int lim = row_ok ? ctx - n + t0x + rt + 1 : kbeg + 1;
@@ -468,27 +509,18 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
     float m_used = -INFINITY, l = 0.0f;
 #pragma unroll 1
     for (int j = 0; j < nk; ++j) {
-      wait_or_abort(b_sfull + 16 * x + 8 * (j & 1), (j >> 1) & 1);
+      wait_or_abort(b_sfull + 8 * x, j & 1);
       if (aborted()) break;
       tc_fence_after();
-      const uint32_t tS = tS0 + 64 * (j & 1);
-      float sv[64];
-      {
-        float a[32], b[32];
-        tmem_ld32(tS, a);
-        tmem_ld32(tS + 32, b);
-        tmem_wait_ld();
+      float sv[kN];
 #pragma unroll
-        for (int k = 0; k < 32; ++k) {
-          sv[k] = a[k];
-          sv[32 + k] = b[k];
-        }
-      }
-      const int kt0 = kbeg + j * Tr::kKeys;
-      const bool full = kt0 + Tr::kKeys <= wmin_lim && kt0 >= wmax_lo && row_ok;
+      for (int q = 0; q < kN / 32; ++q) tmem_ld32(tS + 32 * q, *reinterpret_cast<float(*)[32]>(sv + 32 * q));
+      tmem_wait_ld();
+      const int kt0 = kbeg + j * kN;
+      const bool full = kt0 + kN <= wmin_lim && kt0 >= wmax_lo && row_ok;
       if (!full) {
 #pragma unroll
-        for (int k = 0; k < 64; ++k) {
+        for (int k = 0; k < kN; ++k) {
           const int key = kt0 + k;
           sv[k] = (key < lim && key >= lo) ? sv[k] : -INFINITY;
         }
@@ -498,7 +530,7 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
 #pragma unroll
       for (int k = 0; k < 8; ++k) mp[k] = fmaxf(sv[k], sv[k + 8]);
 #pragma unroll
-      for (int k = 16; k < 64; ++k) mp[k & 7] = fmaxf(mp[k & 7], sv[k]);
+      for (int k = 16; k < kN; ++k) mp[k & 7] = fmaxf(mp[k & 7], sv[k]);
       const float mr = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
                              fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
       const float mx = mr * c;  // scores are used as s * c (log2 units)
@@ -511,42 +543,38 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       }
       const float nbase = m_used == -INFINITY ? 0.0f : -m_used;
       float sp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      uint32_t w[32];
+      // P over the upper half of S (already read into registers)
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[2 * k], c, nbase)), fast_exp2(fmaf(sv[2 * k + 1], c, nbase)));
-        sp[k & 3] += sum_p2<kBF16>(w[k]);
+      for (int q = 0; q < kN / 32; ++q) {
+        uint32_t w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const int e = 32 * q + 2 * k;
+          w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[e], c, nbase)), fast_exp2(fmaf(sv[e + 1], c, nbase)));
+          sp[k & 3] += sum_p2<kBF16>(w[k]);
+        }
+        tmem_st16(tP + 16 * q, w);
       }
       const float sum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
       l = l * factor + sum;
-      // P_x(j-1) . V_{j-1} must be done before P_x is overwritten or O_x
-      // rescaled (issued right after P_x(j-1) was written, long ago)
-      if (j > 0) wait_or_abort(b_pvdone + 8 * x, (j - 1) & 1);
-      tc_fence_after();
-#pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        *reinterpret_cast<uint4*>(sptr + (px - sbase) + row * 128 + ((c8 ^ (row & 7)) << 4)) =
-            make_uint4(w[4 * c8], w[4 * c8 + 1], w[4 * c8 + 2], w[4 * c8 + 3]);
-      }
-      if (__any_sync(0xffffffffu, rescale)) {
-        const float f = rescale ? factor : 1.0f;
+      // O_x holds every P . V before this tile (S_x(j) was committed after them)
+      if (rescale) {
 #pragma unroll 1
         for (int cb = 0; cb < kD / 32; ++cb) {
           float o[32];
           tmem_ld32(tO + 32 * cb, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= f;
+          for (int k = 0; k < 32; ++k) o[k] *= factor;
           tmem_st32(tO + 32 * cb, o);
         }
-        tmem_wait_st();
       }
-      fence_async_smem();
+      tmem_wait_st();
       tc_fence_before();
       mbar_arrive(b_pfull + 8 * x);
     }
     // ---- epilogue: O / l -> out ----
-    wait_or_abort(b_pvdone + 8 * x, (nk - 1) & 1);
+    wait_or_abort(b_ofull, 0);
     tc_fence_after();
     if (!aborted()) {
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;
@@ -562,10 +590,10 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
 #pragma unroll
           for (int c8 = 0; c8 < 4; ++c8) {
             uint4 v;
-            v.x = pack_p2<kBF16>(o[8 * c8 + 0] * inv, o[8 * c8 + 1] * inv);
-            v.y = pack_p2<kBF16>(o[8 * c8 + 2] * inv, o[8 * c8 + 3] * inv);
-            v.z = pack_p2<kBF16>(o[8 * c8 + 4] * inv, o[8 * c8 + 5] * inv);
-            v.w = pack_p2<kBF16>(o[8 * c8 + 6] * inv, o[8 * c8 + 7] * inv);
+            v.x = pack_out<kBF16>(o[8 * c8 + 0] * inv, o[8 * c8 + 1] * inv);
+            v.y = pack_out<kBF16>(o[8 * c8 + 2] * inv, o[8 * c8 + 3] * inv);
+            v.z = pack_out<kBF16>(o[8 * c8 + 4] * inv, o[8 * c8 + 5] * inv);
+            v.w = pack_out<kBF16>(o[8 * c8 + 6] * inv, o[8 * c8 + 7] * inv);
             *reinterpret_cast<uint4*>(dst + 32 * cb + 8 * c8) = v;
           }
         }
