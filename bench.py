@@ -91,11 +91,22 @@ def tensor_peak():
     return FALLBACK_BF16_TFLOPS, "fallback"
 
 
-def kernel_source_hash():
-    """Hash of the decode kernel's device code (the traffic record is valid
-    only for the kernel it was captured on)."""
+DECODE_SOURCES = ("pkv_decode.cuh", "pkv_device.cuh")
+PREFILL_SOURCES = ("pkv_prefill.cuh", "pkv_device.cuh")
+
+
+def uses_prefill_kernel(workload):
+    """True when the workload's calls go to the query-major tcgen05 kernel:
+    runs of new tokens filling a tile of 128 (token, head) rows."""
+    spec = I.WORKLOADS[workload]
+    return spec.get("q_len", 1) * (spec["hq"] // spec["hkv"]) >= 128
+
+
+def kernel_source_hash(files=DECODE_SOURCES):
+    """Hash of a kernel's device code (a traffic record is valid only for the
+    kernel it was captured on)."""
     h = hashlib.sha256()
-    for f in ("pkv_decode.cuh", "pkv_device.cuh"):
+    for f in files:
         with open(os.path.join(ROOT, "paged_kv_cache_438_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -113,7 +124,8 @@ def recorded_traffic(workload, cache, alg_bytes):
         d = json.load(f)
     key = workload + ("" if cache is None else "_" + cache)
     e = d.get(key)
-    if not e or e.get("source_hash") != kernel_source_hash():
+    files = PREFILL_SOURCES if uses_prefill_kernel(workload) else DECODE_SOURCES
+    if not e or e.get("source_hash") != kernel_source_hash(files):
         return None
     return int(e["dram_bytes_per_call"] * alg_bytes / e["alg_bytes_per_call"])
 
@@ -775,7 +787,9 @@ def main():
                       "achieved": round(achieved, 1), "peak": peak, "unit": "GB/s",
                       "frac": round(achieved / peak, 4), "peak_source": f"{peak_kind} hbm_gbs (copy, burst)"}
                      if not tensor_bound else
-                     {"kernel": "paged_decode_kernel, multi-query mode (one launch per call)", "bound": "tensor",
+                     {"kernel": ("paged_prefill_kernel (query-major, tcgen05; one launch per call)"
+                                 if uses_prefill_kernel(args.workload) else
+                                 "paged_decode_kernel, multi-query mode (one launch per call)"), "bound": "tensor",
                       "achieved": round(flops_call / (dec_ms * 1e-3) / 1e12, 2), "peak": tflops_peak,
                       "unit": "TFLOP/s", "frac": round(flops_call / (dec_ms * 1e-3) / 1e12 / tflops_peak, 4),
                       "peak_source": f"{tflops_kind} bf16_tflops (cuBLAS, burst)",
