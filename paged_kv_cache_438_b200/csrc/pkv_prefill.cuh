@@ -186,6 +186,7 @@ struct PrefillTraits {
   static constexpr int kFit = (227 * 1024 - 1024 - kTiles * kQBytes - kBarBytes) / kEntryBytes;
   static constexpr int kEntries = kFit > 8 ? 8 : kFit;  // ring of K and V tiles: K0 V0 K1 V1 ...
   static constexpr int kThreads = 10 * 32;             // 2 softmax warpgroups, MMA warp, load warp
+  static constexpr int kRankMax = 64;                  // sequences ranked by context length per launch
   // TMEM: S of tile x at 128 x (P of tile x, 16-bit, over its upper half at
   // 128 x + 64), O of tile x at 256 + 128 x
   static constexpr int kTmemCols = 512;
@@ -254,14 +255,38 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
   const int lane = tid & 31;
-  const int s = blockIdx.z;
   const int h = blockIdx.y;
   const int G = p.group;
+  const int cap = min(p.max_context_len, p.max_blocks_per_seq * 16);
+
+  // ---- sequence of this CTA ----
+  // Sequences are taken in decreasing context length (ties by index): the
+  // hardware starts CTAs in blockIdx order, so the longest runs of key tiles
+  // start first and short pairs fill the tail.  Beyond kRankMax sequences the
+  // launch order stays as it is (many sequences balance by themselves).
+  int s = blockIdx.z;
+  if (p.num_seqs <= Tr::kRankMax) {
+    __shared__ int seq_of_rank;
+    auto ctx_of = [&](int t) {
+      const int c = p.context_lens[t];
+      return c < 0 ? 0 : (c > cap ? cap : c);
+    };
+    for (int t = tid; t < p.num_seqs; t += blockDim.x) {
+      const int ct = ctx_of(t);
+      int r = 0;
+      for (int u = 0; u < p.num_seqs; ++u) {
+        const int cu = ctx_of(u);
+        r += (cu > ct || (cu == ct && u < t)) ? 1 : 0;
+      }
+      if (r == static_cast<int>(blockIdx.z)) seq_of_rank = t;  // ranks are a permutation of 0 .. num_seqs - 1
+    }
+    __syncthreads();
+    s = seq_of_rank;
+  }
 
   // ---- rows of this CTA ----
   int ctx = p.context_lens[s];
   {
-    const int cap = min(p.max_context_len, p.max_blocks_per_seq * 16);
     if (ctx < 0 || ctx > cap) {
       if (tid == 0 && h == 0 && blockIdx.x == 0) raise_status(PKV_DEV_BAD_CONTEXT);
       ctx = ctx < 0 ? 0 : cap;
