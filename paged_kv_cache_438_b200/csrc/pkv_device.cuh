@@ -197,16 +197,24 @@ __device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
 
 // Eight signed INT4 codes n0..n7 of w (n0 in the lowest nibble) -> four
 // fp16x2 pairs x[k] = (n_k, n_{k+4}), exactly.  u = w ^ 0x88888888 turns
-// code x into x + 8; a nibble placed under the fp16 pattern 0x6400 reads as
-// 1024 + (x + 8); subtracting 1032 leaves x.
+// code x into x + 8.  A nibble placed under the fp16 pattern 0x6400 in bits
+// 0-3 reads as 1024 + (x + 8): subtracting 1032 leaves x.  One placed in bits
+// 4-7 (no shift needed) reads as 1024 + 16 (x + 8): times 1/16 minus 72 leaves
+// x, in one fused multiply-add (every step exact in fp16).  Ten operations
+// per eight codes.
 __device__ __forceinline__ void i4x8_to_h2x4(uint32_t w, uint32_t (&x)[4]) {
   const uint32_t u = w ^ 0x88888888u;
-  const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));
+  const uint32_t v = u >> 8;
+  const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));        // 1032
+  const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));   // 1/16
+  const __half2 minus72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));     // -72
+  uint32_t t[4] = {and_or(u, 0x000F000Fu, 0x64006400u), and_or(u, 0x00F000F0u, 0x64006400u),
+                   and_or(v, 0x000F000Fu, 0x64006400u), and_or(v, 0x00F000F0u, 0x64006400u)};
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    uint32_t t = and_or(u >> (4 * k), 0x000F000Fu, 0x64006400u);
-    __half2 h = __hsub2(*reinterpret_cast<__half2*>(&t), bias);
-    x[k] = *reinterpret_cast<uint32_t*>(&h);
+    const __half2 a = *reinterpret_cast<__half2*>(&t[k]);
+    const __half2 h = (k & 1) ? __hfma2(a, sixteenth, minus72) : __hsub2(a, bias);
+    x[k] = *reinterpret_cast<const uint32_t*>(&h);
   }
 }
 
