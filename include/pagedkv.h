@@ -251,12 +251,15 @@ int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int he
  * [0, num_q_tokens] are clamped to it.  With every n_s = 1 the result equals
  * decode.
  * Kernels: when max_query_len * (num_q_heads / num_kv_heads) >= 128, the
- * cache is 16-bit, 128 is a multiple of the group, partition_tokens is 0 and
- * q and out are 16-byte aligned, a query-major kernel on the tcgen05 tensor
- * cores runs (128 (token, head) rows per CTA, 64-key tiles, accumulators in
- * TMEM; no workspace used); otherwise the decode kernel's multi-query mode
- * (16 (token, head) columns per pass).  Both give the same result up to
- * rounding.
+ * cache is 16-bit, head_dim is 64 or 128, 128 is a multiple of the group,
+ * partition_tokens is 0, scale > 0 and q and out are 16-byte aligned, a
+ * query-major kernel on the tcgen05 tensor cores runs (two tiles of 128
+ * (token, head) rows per CTA sharing 128-key K/V tiles; scores,
+ * probabilities and outputs in TMEM; sequences started longest first; no
+ * workspace used); otherwise the decode kernel's multi-query mode (16
+ * (token, head) columns per pass).  Both give the same result up to
+ * rounding (bf16 probabilities are rounded toward zero in the first, to
+ * nearest in the second).
  */
 int pkv_paged_attention_multi_query(void* out, const void* q,
                                     const void* k_cache, const void* v_cache,
