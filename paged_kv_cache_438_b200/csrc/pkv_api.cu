@@ -143,7 +143,14 @@ int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int r
     const long long per = req_tokens / 16;
     nw = (t_max + per - 1) / per;
   } else {
-    nw = std::min(static_cast<long long>(warps) * sms, (t_max + 15) / 16);
+    // Streams of at least 16 blocks (a merge contributor costs about one
+    // block) while the work fills a wave of warps; below that the warps'
+    // copy rings, not HBM, set the time (each stream waits for its copies one
+    // after another), so shorter streams of at least 4 blocks spread a small
+    // batch over more SMs.
+    const long long wave = static_cast<long long>(warps) * sms;
+    nw = std::min(wave, (t_max + 15) / 16);
+    if (nw < wave) nw = std::min(wave, (t_max + 3) / 4);
     if (max_tiles > 1) {
       // Several column tiles per KV head re-read the same K/V blocks: one
       // stream per (sequence, head, tile) bound makes the warps of a CTA (and
