@@ -319,11 +319,11 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
   const uint32_t q_s = sbase;                                  // Q_A, Q_B
   const uint32_t kv_s = q_s + Tr::kTiles * Tr::kQBytes;       // kE ring entries
   const uint32_t bars = kv_s + kE * Tr::kEntryBytes;
-  // barriers: full[kE], empty[kE], s_full[2], p_full[2], o_full
+  // barriers: full[kE], empty[kE], s_full[2], p_full[2], o_full, v_tail
   const uint32_t b_full = bars, b_empty = bars + 8 * kE, b_sfull = bars + 16 * kE;
-  const uint32_t b_pfull = b_sfull + 16, b_ofull = b_sfull + 32;
-  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sptr + (bars - sbase) + 16 * kE + 40);
-  int* const abort_flag = reinterpret_cast<int*>(sptr + (bars - sbase) + 16 * kE + 44);
+  const uint32_t b_pfull = b_sfull + 16, b_ofull = b_sfull + 32, b_vtail = b_sfull + 40;
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(sptr + (bars - sbase) + 16 * kE + 48);
+  int* const abort_flag = reinterpret_cast<int*>(sptr + (bars - sbase) + 16 * kE + 52);
   auto aborted = [&]() { return *reinterpret_cast<volatile int*>(abort_flag) != 0; };
   auto wait_or_abort = [&](uint32_t bar, uint32_t parity) {
     if (!mbar_wait(bar, parity)) atomicExch(abort_flag, 1);
@@ -343,6 +343,7 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       mbar_init(b_pfull + 8 * x, Tr::kRows);
     }
     mbar_init(b_ofull, 1);
+    mbar_init(b_vtail, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -436,6 +437,26 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       // last tile of each entry is the only one that can still be pending
       for (int i = max(issued - kE, 0); i < issued; ++i) mbar_wait(b_full + 8 * (i % kE), (i / kE) & 1);
     }
+    __syncwarp();
+    // The last K/V tile may reach past the context: once it has landed, its V
+    // rows there (never written, or zero-filled already) are zeroed before
+    // any P . V reads them, and v_tail tells the MMA warp so.
+    const int kt_last = kbeg + (nk - 1) * kN;
+    if (nk > 0 && kt_last + kN > ctx) {
+      const int vi = 2 * nk - 1, vslot = vi % kE;
+      wait_or_abort(b_full + 8 * vslot, (vi / kE) & 1);
+      if (!aborted()) {
+        const int r0 = max(ctx - kt_last, 0);
+        uint8_t* const ve = sptr + (kv_s + vslot * Tr::kEntryBytes - sbase);
+        for (int e = lane; e < (kN - r0) * kR * 8; e += 32) {
+          const int rr = r0 + e / (kR * 8), reg = (e / 8) % kR, c = e % 8;
+          *reinterpret_cast<uint4*>(ve + reg * Tr::kRegionBytes + rr * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        fence_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(b_vtail);
+    }
   } else if (warp == 8) {
     // =================== MMA warp: every tcgen05.mma, issued by lane 0 ===================
     // Descriptors are computed once; a K-step or an entry moves only the
@@ -464,6 +485,7 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
         umma_f16_ts(d, a + 8 * ks, dv + static_cast<uint32_t>(ks * 128), kIdescO, (j > 0 || ks > 0) ? 1u : 0u);
       }
     };
+    // lane 0 alone runs the loop (no warp-wide waits between tiles)
     if (lane == 0 && nk > 0) {
       wait_or_abort(b_full, 0);  // K_0 sits in entry 0
       tc_fence_after();
@@ -472,27 +494,14 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       issue_s(1, 0);
       umma_commit(b_sfull + 8);
       umma_commit(b_empty);
-    }
-    __syncwarp();
 #pragma unroll 1
-    for (int j = 0; j < nk; ++j) {
-      const int vi = 2 * j + 1, vslot = vi % kE;
-      const int kt0 = kbeg + j * kN;
-      wait_or_abort(b_full + 8 * vslot, (vi / kE) & 1);
-      if (aborted()) break;
-      // keys of the tile at or past the context: zero their V rows (never
-      // written there, or zero-filled already) before any P . V reads them
-      if (kt0 + kN > ctx) {
-        const int r0 = max(ctx - kt0, 0);
-        uint8_t* const ve = sptr + (kv_s + vslot * Tr::kEntryBytes - sbase);
-        for (int e = lane; e < (kN - r0) * kR * 8; e += 32) {
-          const int rr = r0 + e / (kR * 8), reg = (e / 8) % kR, c = e % 8;
-          *reinterpret_cast<uint4*>(ve + reg * Tr::kRegionBytes + rr * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
-        }
-        fence_async_smem();
-      }
-      __syncwarp();
-      if (lane == 0) {
+      for (int j = 0; j < nk; ++j) {
+        const int vi = 2 * j + 1, vslot = vi % kE;
+        const int kt0 = kbeg + j * kN;
+        wait_or_abort(b_full + 8 * vslot, (vi / kE) & 1);
+        // a tile past the context: its V rows there are zeroed by the load warp
+        if (kt0 + kN > ctx) wait_or_abort(b_vtail, 0);
+        if (aborted()) break;
         const bool more = j + 1 < nk;
         const int ki = 2 * (j + 1), kslot = ki % kE;
 #pragma unroll 1
@@ -513,8 +522,8 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
         }
         if (!more) umma_commit(b_ofull);  // every MMA of the CTA done
       }
-      __syncwarp();
     }
+    __syncwarp();
   } else {
     // =================== softmax warpgroup x = wg ===================
     const int x = wg;
