@@ -219,3 +219,24 @@ def test_query_major_kernel_against_oracle_and_decode_mode(dtype, d, group):
     check_attn(fast, ref)
     slow = np64(run_mq(g, partition_tokens=64))
     check_attn(fast, slow, atol=2e-2, meanrel=5e-3)        # two bf16-rounded outputs: within 2 ulps
+
+
+@pytest.mark.parametrize("ctx,nq", [
+    ([300] * 5, [300, 129, 64, 200, 32]),                       # every context length equal
+    ([500, 200, 500, 200, 64, 500], [200, 150, 40, 200, 64, 1]),  # repeated lengths
+    ([int(32 + (97 * i) % 170) for i in range(70)],               # more sequences than are ranked
+     [min(40, int(32 + (97 * i) % 170)) for i in range(70)]),
+])
+def test_query_major_launch_order_covers_every_sequence(ctx, nq):
+    """The query-major kernel starts sequences in decreasing context length
+    (ties by index; beyond 64 sequences in launch order): every run of every
+    sequence must still be computed exactly once."""
+    hkv, group = 2, 4
+    case = I.multi_query_case("chunked_prefill", seed=len(ctx) + sum(nq), ctx_override=ctx, q_lens=nq,
+                              hq=hkv * group, hkv=hkv, d=128, dtype="bf16")
+    g = gpu_case(case)
+    nw, _, _ = P.multi_query_plan(len(ctx), hkv * group, hkv, 128, max(ctx), max(nq), g["k_cache"].dtype)
+    assert nw == len(ctx) * hkv * (((max(nq) * group + 127) // 128 + 1) // 2)     # the query-major plan
+    got = np64(run_mq(g))
+    assert np.all(np.isfinite(got))
+    check_attn(got, oracle_mq(case))
