@@ -102,13 +102,37 @@ def uses_prefill_kernel(workload):
     return spec.get("q_len", 1) * (spec["hq"] // spec["hkv"]) >= 128
 
 
+def strip_comments(src):
+    """C++ source without its comments (string literals kept) and with runs of
+    whitespace collapsed: what the compiler sees of the code."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c == '"':
+            j = i + 1
+            while j < n and src[j] != '"':
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash(files=DECODE_SOURCES):
-    """Hash of a kernel's device code (a traffic record is valid only for the
-    kernel it was captured on)."""
+    """Hash of a kernel's device code, comments and layout aside (a traffic
+    record is valid only for the kernel it was captured on)."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, "paged_kv_cache_438_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "paged_kv_cache_438_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -12,27 +12,35 @@
 // Design (sm_100a):
 //   * One CTA per (sequence, KV head, pair of tiles of 128 query rows); a row
 //     is a (new token, query head of the group) pair, row = t * G + g, so the
-//     GQA group shares every K/V tile.  Warpgroup A (warps 0-3) and B (warps
-//     4-7) own one tile each; thread i of a warpgroup owns row i, i.e. TMEM
-//     lane i: the whole online softmax of a row runs in one thread.  Warp 8
-//     loads K/V and issues every MMA.
-//   * Keys stream in tiles of 64 (four 16-token cache blocks found through
-//     the block table) by TMA into a 4-stage ring (128-byte swizzle); K tiles
-//     are K-major B operands, V tiles MN-major B operands of the same layout.
-//   * S = Q K^T: tcgen05.mma M=128, N=64, K=16 steps over head_dim into TMEM
-//     (fp32); P = exp2(S - m) in bf16/fp16 written to shared memory (K-major,
-//     swizzled) as the A operand of O += P V (M=128, N=head_dim).  Scores are
-//     double-buffered in TMEM and issued two K/V tiles ahead, and the tensor
-//     core alternates between the two query tiles, so the softmax of one
-//     warpgroup overlaps MMAs of both; completion is signalled by
+//     GQA group shares every K/V tile, and so do the CTA's two query tiles.
+//     Warpgroup A (warps 0-3) and B (warps 4-7) own one tile each; thread i
+//     of a warpgroup owns row i, i.e. TMEM lane i: the whole online softmax of
+//     a row runs in one thread.  Lane 0 of warp 8 issues every MMA; warp 9
+//     loads K and V.  Sequences start in decreasing context length (the
+//     hardware launches CTAs in blockIdx order), so long runs of key tiles do
+//     not form the tail of the launch.
+//   * Keys stream in tiles of 128 (eight 16-token cache blocks found through
+//     the block table) by TMA into a ring of entries holding K_0, V_0, K_1,
+//     V_1, ... (128-byte swizzle); K tiles are K-major B operands, V tiles
+//     MN-major B operands of the same layout.
+//   * S = Q K^T: tcgen05.mma M=128, N=128, K=16 steps over head_dim, both
+//     operands in shared memory, into TMEM (fp32).  P = exp2(S - m) in
+//     bf16/fp16 is written by the softmax threads over the upper half of S in
+//     TMEM and read from there by O += P V (the TS form, M=128,
+//     N=head_dim), so P never goes through shared memory.  After P_x(j) . V_j
+//     the same thread issues S_x(j+1) into S's columns; the tensor core runs
+//     one thread's MMAs in issue order, so P is read before it is
+//     overwritten.  The two query tiles ping-pong: one warpgroup's softmax
+//     overlaps the other tile's MMAs.  Completion is signalled by
 //     tcgen05.commit on mbarriers; every wait is bounded.
 //   * Online softmax with a lazy rescale: the exponent base of a row only
 //     moves when its max grows by more than 8 (log2 units), and only then is
 //     that row's O rescaled in TMEM.  Unmasked tiles skip the mask; the
 //     softmax scale is folded into one FMA per score.
 //   * Tokens of a sequence's last block beyond its context were never
-//     written: their V rows are zeroed in the stage, blocks past the context
-//     are loaded from outside the tensor (TMA fills zeros).
+//     written: the load warp zeroes their V rows in the entry before P . V
+//     reads them; blocks past the context are loaded from outside the tensor
+//     (TMA fills zeros).
 #pragma once
 
 #include "pkv_device.cuh"
