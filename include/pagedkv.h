@@ -219,7 +219,13 @@ int pkv_paged_attention_decode(void* out, const void* q,
  * pkv_multi_query_plan -- the work division pkv_paged_attention_multi_query
  *   will use (as pkv_decode_plan; the (token, head) columns of one KV head
  *   are cut into tiles of 8 or 16, each tile a pair of its own in the work
- *   list).  max_query_len bounds the new tokens of any sequence.
+ *   list).  max_query_len bounds the new tokens of any sequence.  When the
+ *   query-major kernel applies (see pkv_paged_attention_multi_query),
+ *   *num_streams_out is its CTA count, num_seqs * num_kv_heads * the pairs
+ *   of 128-row tiles of the longest run, and *partition_tokens_out the
+ *   context bound rounded up to whole blocks (each CTA walks all its keys);
+ *   *workspace_bytes_out is still the other kernel's need, used when q or
+ *   out is not 16-byte aligned or the scale is not positive.
  */
 int pkv_multi_query_plan(int num_seqs, int num_q_heads, int num_kv_heads, int head_dim,
                          int max_context_len, int max_query_len, int cache_dtype,
