@@ -23,6 +23,7 @@ import os
 import statistics
 import subprocess
 import sys
+import tempfile
 import time
 
 import numpy as np
@@ -167,7 +168,10 @@ class ClockSampler:
         self.proc = None
         self.path = None
         try:
-            self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+            # raw samples go to PKV_CLOCKS_DIR when set (to keep them), else
+            # to the temporary directory; the JSON line carries the summary
+            self.path = os.path.join(os.environ.get("PKV_CLOCKS_DIR") or tempfile.gettempdir(),
+                                     f"pkv_clocks_{os.getpid()}.csv")
             os.makedirs(os.path.dirname(self.path), exist_ok=True)
             self.fh = open(self.path, "w")
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
