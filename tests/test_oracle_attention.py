@@ -39,6 +39,19 @@ def test_worked_example_batch16_is_32gb():
     assert got == g["batch16_kv_gb_printed"] * 2 ** 30
 
 
+def test_per_token_per_layer_form_reproduces_the_worked_example():
+    # "KV Cache 与 PagedAttention" (ai-infra-wiki) §KV cache 有多大: one token adds
+    # 2 x n_kv x head_dim x 2 bytes to one layer (16-bit values); times the
+    # layers and tokens of the worked example it must give the printed total
+    g = _golden("kv_size_worked_example.json")
+    per = K.kv_bytes_per_token_per_layer(g["n_kv_heads"], g["head_dim"], g["bytes_per_elt"])
+    assert per == 2 * 32 * 128 * 2
+    assert per * g["n_layers"] * g["seq_len"] * g["batch"] == g["kv_bytes"]
+    # and it agrees with the product form for other shapes and element sizes
+    for L, H, D, S, B, e in [(80, 8, 128, 32768, 1, 2), (32, 8, 128, 4096, 64, 1), (1, 1, 64, 1, 1, 4)]:
+        assert K.kv_cache_bytes(L, H, D, S, B, e) == L * S * B * K.kv_bytes_per_token_per_layer(H, D, e)
+
+
 def test_decode_bound_about_140():
     g = _golden("decode_bound.json")
     v = K.decode_tokens_per_s_bound(g["bandwidth_gb_s"], g["weights_gb"])

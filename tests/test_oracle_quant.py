@@ -76,6 +76,18 @@ def test_int8_ties_round_half_to_even():
     assert q[0].tolist() == [127, 2, 4, -2, -4, 0, 0, 2, 126]
 
 
+def test_int8_dequantize_is_code_times_scale_within_half_a_step():
+    # hand case: codes times the row's scale, exactly
+    y = Q.dequantize_int8(np.array([[127, -3, 0]], np.int8), np.array([0.5], np.float32))
+    assert y.tolist() == [[63.5, -1.5, 0.0]]
+    # round trip through the quantiser: within half a quantisation step
+    rng = np.random.default_rng(11)
+    x = rng.standard_normal((200, 4, 64)).astype(np.float32)
+    q, s = Q.quantize_int8(x)
+    err = np.abs(x.astype(np.float64) - Q.dequantize_int8(q, s))
+    assert np.all(err <= s[..., None].astype(np.float64) * (0.5 + 1e-5))
+
+
 def test_int8_zero_row():
     q, s = Q.quantize_int8(np.zeros((2, 8), np.float32))
     assert np.all(q == 0) and np.all(s == 0)
