@@ -165,3 +165,18 @@ def test_multi_query_plan_tiles(lib):
     # 8-bit caches never take the query-major kernel
     nw3, _, _ = P.multi_query_plan(8, 32, 8, 128, 4096, 512, P.PKV_I8)
     assert nw3 == 8 * 8 * 128
+
+
+def test_small_batches_get_shorter_streams(lib):
+    # without a GPU the plan assumes the B200's 148 SMs (as on one): 8 warps each
+    wave = 8 * 148
+    # 4 sequences x 2 heads x 16 blocks = 128 blocks, far below a wave of
+    # 16-block streams: streams of 4 blocks (64 tokens) spread it over 32 warps
+    nw, per, _ = P.decode_plan(4, 8, 2, 64, 256, P.PKV_BF16)
+    assert (nw, per) == (32, 64)
+    # 16 x 8 x 128 blocks: a full wave of shorter streams rather than 128 of 16 blocks
+    nw, per, _ = P.decode_plan(16, 32, 8, 128, 2048, P.PKV_BF16)
+    assert nw == wave and per < 16 * 16
+    # enough work for a wave of 16-block streams: unchanged
+    nw, per, _ = P.decode_plan(64, 32, 8, 128, 4096, P.PKV_BF16)
+    assert nw == wave and per >= 16 * 16
