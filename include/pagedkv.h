@@ -290,8 +290,11 @@ int pkv_paged_attention_multi_query(void* out, const void* q,
  * for pkv_paged_attention_decode; there is no workspace argument.
  *   - The split-KV partials go to one library-owned device array of
  *     PKV_NOALLOC_SCRATCH_BYTES (a file-scope __device__ array: every GPU that
- *     loads the library holds it until the process exits).  A call whose plan
- *     needs more (pkv_decode_plan's workspace_bytes_out) is rejected with
+ *     loads the library holds it until the process exits).  With
+ *     partition_tokens = 0, when the automatic plan needs more
+ *     (pkv_decode_plan's workspace_bytes_out), the call runs the same work in
+ *     fewer, longer warp streams, as many as the array holds; a call that
+ *     still needs more (or whose explicit partition does) is rejected with
  *     PKV_ERR_INVALID_ARG before anything is launched.
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress, with that device current) and caches it; make

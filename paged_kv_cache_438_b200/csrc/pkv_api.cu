@@ -749,6 +749,24 @@ extern "C" int pkv_paged_attention_decode_noalloc(void* out, const void* q, cons
   Plan pl{};
   int rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, partition_tokens, &pl);
   if (rc != PKV_OK) return rc;
+  int pt = partition_tokens;
+  if (pt == 0 && pl.num_streams > 1 && pl.workspace > kNoAllocScratchBytes &&
+      pl.counter_bytes < kNoAllocScratchBytes) {
+    // The automatic plan needs more partials than the array holds: the same
+    // work in fewer, longer warp streams, as many as fit.
+    const long long per_stream = 2LL * pl.slot_floats * 4;
+    const long long fit = static_cast<long long>(kNoAllocScratchBytes - pl.counter_bytes) / per_stream;
+    const long long blocks = static_cast<long long>(std::max(num_seqs, 1)) * num_kv_heads *
+                             std::max(1, (max_context_len + 15) / 16);
+    if (fit >= 1) {
+      const long long per = (blocks + fit - 1) / fit;  // blocks per stream
+      if (per * 16 <= (1LL << 30)) {
+        pt = static_cast<int>(per * 16);
+        rc = make_plan(num_seqs, num_q_heads, num_kv_heads, head_dim, max_context_len, cache_dtype, pt, &pl);
+        if (rc != PKV_OK) return rc;
+      }
+    }
+  }
   const bool needs_scratch = pl.num_streams > 1;
   if (needs_scratch && pl.workspace > kNoAllocScratchBytes)
     return fail(PKV_ERR_INVALID_ARG,
@@ -765,5 +783,5 @@ extern "C" int pkv_paged_attention_decode_noalloc(void* out, const void* q, cons
                                     context_lens,
                                     num_seqs, num_q_heads, num_kv_heads, head_dim, block_size, num_blocks,
                                     max_blocks_per_seq, max_context_len, scale, sliding_window, q_dtype, cache_dtype,
-                                    partition_tokens, scratch, needs_scratch ? kNoAllocScratchBytes : 0, stream);
+                                    pt, scratch, needs_scratch ? kNoAllocScratchBytes : 0, stream);
 }

@@ -368,8 +368,10 @@ def paged_attention_decode_noalloc(q, k_cache, v_cache, block_tables, context_le
     (for instance a plugin whose host framework owns every allocation and
     hands it only input and output buffers): ``out`` must be given, no
     workspace is taken, and the split-KV partials use the library's own
-    device array of NOALLOC_SCRATCH_BYTES.  Work that needs more scratch is
-    rejected with an error.  Calls that overlap on the GPU share that array
+    device array of NOALLOC_SCRATCH_BYTES.  With partition_tokens 0 the work
+    is cut into fewer, longer warp streams when the automatic plan needs more
+    scratch; work that needs more even then, or whose explicit partition
+    does, is rejected with an error.  Calls that overlap on the GPU share that array
     and race; keep them on one stream.  The first call on a device looks up
     the array's address, so make it before any stream capture."""
     dev = q.device

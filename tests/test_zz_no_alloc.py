@@ -76,3 +76,22 @@ def test_noalloc_rejects_work_beyond_its_scratch():
         P.paged_attention_decode_noalloc(q, kc, kc, bt, cl, 1 / math.sqrt(d), maxc, torch.empty_like(q),
                                          partition_tokens=256)
     del c
+
+
+def test_noalloc_lengthens_streams_when_the_automatic_plan_needs_more_scratch():
+    # a GQA group of 16 (128 q / 8 KV heads): with the automatic plan the
+    # partials of a full wave of warp streams need ~19.7 MB, more than the
+    # built-in array; the call runs the same work in fewer, longer streams
+    case = I.decode_case("llama3_8b", seed=31, batch=16, hq=128, hkv=8)
+    g = {k: (v.to(DEV) if isinstance(v, torch.Tensor) else v) for k, v in case.items()}
+    maxc = int(case["context_lens"].max())
+    _, _, ws = P.decode_plan(16, 128, 8, 128, maxc, g["k_cache"].dtype)
+    assert ws > P.NOALLOC_SCRATCH_BYTES
+    out = torch.empty_like(g["q"])
+    P.paged_attention_decode_noalloc(g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"],
+                                     g["scale"], maxc, out)
+    ref = P.paged_attention_decode(g["q"], g["k_cache"], g["v_cache"], g["block_tables"], g["context_lens"],
+                                   g["scale"], max_context_len=maxc)
+    torch.cuda.synchronize()
+    _close(out, ref)
+    assert P.device_status(clear=True) == 0
