@@ -142,7 +142,7 @@ def recorded_traffic(workload, cache, alg_bytes):
     record, or None when absent or taken on a different kernel source.  A
     record captured on a smaller slice of the workload is scaled to this
     call by its algorithmic bytes (traffic grows in proportion)."""
-    p = os.path.join(ROOT, "profiles", "decode_traffic.json")
+    p = os.path.join(ROOT, "profiles", "kernel_traffic.json")
     if not os.path.exists(p):
         return None
     with open(p) as f:

@@ -33,7 +33,7 @@ def test_workloads_map_to_their_kernel():
 
 
 def test_traffic_records_are_well_formed():
-    path = os.path.join(bench.ROOT, "profiles", "decode_traffic.json")
+    path = os.path.join(bench.ROOT, "profiles", "kernel_traffic.json")
     with open(path) as f:
         records = json.load(f)
     for key, rec in records.items():
