@@ -180,3 +180,16 @@ def test_small_batches_get_shorter_streams(lib):
     # enough work for a wave of 16-block streams: unchanged
     nw, per, _ = P.decode_plan(64, 32, 8, 128, 4096, P.PKV_BF16)
     assert nw == wave and per >= 16 * 16
+
+
+def test_query_major_routing_threshold_and_group(lib):
+    def mq(hq, d, n, cd=P.PKV_BF16):
+        return P.multi_query_plan(2, hq, 8, d, 1024, n, cd)[0]
+    # the query-major plan: 2 sequences x 8 KV heads x pairs of 128-row tiles
+    assert mq(32, 128, 32) == 2 * 8 * 1             # 32 new tokens x G 4 = 128 rows: one tile
+    assert mq(32, 64, 512) == 2 * 8 * 8             # head_dim 64 qualifies (16 tiles, 8 pairs)
+    assert mq(32, 128, 512, P.PKV_F16) == 2 * 8 * 8  # so does an fp16 cache
+    # below 128 rows, or a group that does not divide 128: the decode kernel's
+    # multi-query mode, one stream per (sequence, head, 16-column tile)
+    assert mq(32, 128, 31) == 2 * 8 * ((31 * 4 + 15) // 16)
+    assert mq(24, 128, 512) == 2 * 8 * ((512 * 3 + 15) // 16)
