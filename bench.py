@@ -8,12 +8,17 @@ attends each sequence's query heads over its whole cache.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-``value`` is the effective KV-read bandwidth (KV bytes the step's attention
-must read / device time of the step, inputs resident in HBM); ``e2e`` is the
-same metric measured through the Python API with host buffers (allocator on
-the host, pinned H2D of the step's inputs, D2H of the output, every step).
-Multi-GPU runs are independent replicas (one batch per rank, weak scaling,
-no data-path collective); time is the max over ranks.
+The default workload is the long-context one (Llama-3-70B-shaped, 64 q / 8 KV
+heads, batch 32, 32768 tokens each, bf16).  ``value`` is the effective
+KV-read bandwidth (KV bytes the step's attention must read / device time of
+the step, inputs resident in HBM); ``e2e`` is the same metric measured
+through the Python API with host buffers (allocator on the host, pinned H2D
+of the step's inputs, D2H and a host read of the output, every step,
+pipelined over two buffer sets).  At N = 1 the line also carries
+``other_workloads``: the decode-call roofline of every other workload and
+cache format (and the oracle timed on the quantised ones).  Multi-GPU runs
+are independent replicas (one batch per rank, weak scaling, no data-path
+collective); time is the max over ranks.
 """
 import argparse
 import hashlib
@@ -60,11 +65,13 @@ def parse():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="llama3_8b", choices=sorted(I.WORKLOADS))
+    ap.add_argument("--workload", default="llama3_70b_32k", choices=sorted(I.WORKLOADS))
     ap.add_argument("--cache", default=None, choices=[None, "int8", "fp8", "u8asym", "int4", "fp4"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the decode-call records of the other workloads (N = 1 only)")
     ap.add_argument("--batch", type=int, default=None, help="override the workload's batch (profiling)")
     return ap.parse_args()
 
@@ -590,78 +597,224 @@ def roll(wl, steps, out, ws, flush, scrub, device, seconds):
 
 
 def run_e2e(wl, K, W, device, world):
-    """The same steps through the public API with host buffers: every step the
-    C++ allocator appends one token per sequence on the host (slots, CoW pairs,
-    block tables, context lengths written into pinned buffers), the step's
-    inputs (q, new K/V rows, slots, tables, lengths, pairs) are copied
-    host-to-device, the kernels run, and the output is copied back and waited
-    for."""
+    """The same steps through the public API with host buffers, pipelined the
+    way a serving loop runs them.  Every step: the C++ allocator appends one
+    token per sequence on the host (slots, CoW pairs, block tables, context
+    lengths written into pinned buffers), the step's inputs (q, new K/V rows,
+    slots, tables, lengths, pairs) are copied host-to-device on a copy stream,
+    the kernels run on the compute stream, and the output is copied back on a
+    second copy stream and read on the host.  Two sets of pinned and device
+    buffers alternate, so step i+1's allocator work and input copies overlap
+    step i's kernels, and step i's output is read while step i+1 runs; events
+    (not a device synchronisation) guard each buffer before it is reused."""
     P = wl.P
     B, MB, T = wl.B, wl.max_blocks, wl.q_rows
-    pin = dict(q=torch.empty((T, wl.hq, wl.d), dtype=wl.dtype).pin_memory(),
-               k=torch.empty((T, wl.hkv, wl.d), dtype=wl.dtype).pin_memory(),
-               v=torch.empty((T, wl.hkv, wl.d), dtype=wl.dtype).pin_memory(),
-               out=torch.empty((T, wl.hq, wl.d), dtype=wl.dtype).pin_memory(),
-               slots=torch.empty(T, dtype=torch.int64).pin_memory(),
-               pairs=torch.empty((B, 2), dtype=torch.int32).pin_memory(),
-               bt=torch.empty((B, MB), dtype=torch.int32).pin_memory(),
-               cl=torch.empty(B, dtype=torch.int32).pin_memory())
-    dev = {k: torch.empty_like(v, device=device) for k, v in pin.items() if k != "out"}
-    out = torch.empty((T, wl.hq, wl.d), dtype=wl.dtype, device=device)
-    ids = torch.arange(B, dtype=torch.int64)
     g = I.generator(4242)
-    for key in ("q", "k", "v"):
-        pin[key].copy_(torch.randn(pin[key].shape, generator=g).to(wl.dtype))
+
+    def pinned_set():
+        pin = dict(q=torch.empty((T, wl.hq, wl.d), dtype=wl.dtype).pin_memory(),
+                   k=torch.empty((T, wl.hkv, wl.d), dtype=wl.dtype).pin_memory(),
+                   v=torch.empty((T, wl.hkv, wl.d), dtype=wl.dtype).pin_memory(),
+                   out=torch.empty((T, wl.hq, wl.d), dtype=wl.dtype).pin_memory(),
+                   slots=torch.empty(T, dtype=torch.int64).pin_memory(),
+                   pairs=torch.empty((B, 2), dtype=torch.int32).pin_memory(),
+                   bt=torch.empty((B, MB), dtype=torch.int32).pin_memory(),
+                   cl=torch.empty(B, dtype=torch.int32).pin_memory())
+        for key in ("q", "k", "v"):
+            pin[key].copy_(torch.randn(pin[key].shape, generator=g).to(wl.dtype))
+        if wl.mq:
+            # the new tokens' slots are fixed; the query layout travels every step
+            pin["qsl"] = wl.qsl.clone().pin_memory()
+            pin["slots"].copy_(wl.new_slots)
+        return pin
+
+    pins = [pinned_set(), pinned_set()]
+    devs = [{k: torch.empty_like(v, device=device) for k, v in pin.items() if k != "out"} for pin in pins]
+    outs = [torch.empty((T, wl.hq, wl.d), dtype=wl.dtype, device=device) for _ in range(2)]
+    ids = torch.arange(B, dtype=torch.int64)
     _, _, wsb = wl.plan(MB * 16)
     ws = P.new_workspace(device, wsb)
-    if wl.mq:
-        # the new tokens' slots are fixed; the query layout travels every step
-        pin["qsl"] = wl.qsl.clone().pin_memory()
-        dev["qsl"] = torch.empty_like(pin["qsl"], device=device)
-        pin["slots"].copy_(wl.new_slots)
-    stream = torch.cuda.current_stream(device)
+    comp = torch.cuda.current_stream(device)
+    h2d_stream = torch.cuda.Stream(device)
+    d2h_stream = torch.cuda.Stream(device)
     keys = ("q", "k", "v", "slots", "bt", "cl") + (("qsl",) if wl.mq else ())
-    fixed = sum(pin[k].numel() * pin[k].element_size() for k in keys)
-    d2h = pin["out"].numel() * pin["out"].element_size()
+    fixed = sum(pins[0][k].numel() * pins[0][k].element_size() for k in keys)
+    d2h = pins[0]["out"].numel() * pins[0]["out"].element_size()
+    h2d_done = [None, None]    # the H2D copies that read pins[b] have finished
+    comp_done = [None, None]   # the kernels that read devs[b] and wrote outs[b] have finished
+    d2h_done = [None, None]    # outs[b] has reached pins[b]["out"]
+    checksum = [0.0]
 
-    def one():
+    def consume(b):
+        """Waits for buffer b's output on the host and reads it."""
+        if d2h_done[b] is not None:
+            d2h_done[b].synchronize()
+            checksum[0] += float(pins[b]["out"][0, 0, 0])
+            d2h_done[b] = None
+
+    def one(i):
+        b = i & 1
+        pin, dev, out = pins[b], devs[b], outs[b]
+        if h2d_done[b] is not None:
+            h2d_done[b].synchronize()          # pins[b] is free to be rewritten
+        consume(b)                             # (and its last output has been read)
         if wl.mq:
-            pairs = pin["pairs"][:0]
+            npairs = 0
         else:
-            slots, pairs = wl.alloc.batch_append(ids, slots_out=pin["slots"], pairs_out=pin["pairs"])
+            _, pairs = wl.alloc.batch_append(ids, slots_out=pin["slots"], pairs_out=pin["pairs"])
+            npairs = pairs.shape[0]
         wl.alloc.batch_tables(ids, MB, out_tables=pin["bt"], out_lens=pin["cl"])
-        npairs = pairs.shape[0]
-        for key in keys:
-            dev[key].copy_(pin[key], non_blocking=True)
-        gp = None
-        if npairs:
-            gp = dev["pairs"][:npairs]
-            gp.copy_(pin["pairs"][:npairs], non_blocking=True)
         maxc = int(pin["cl"].max())
+        with torch.cuda.stream(h2d_stream):
+            if comp_done[b] is not None:
+                h2d_stream.wait_event(comp_done[b])   # the kernels of step i-2 no longer read devs[b]
+            for key in keys:
+                dev[key].copy_(pin[key], non_blocking=True)
+            gp = None
+            if npairs:
+                gp = dev["pairs"][:npairs]
+                gp.copy_(pin["pairs"][:npairs], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(h2d_stream)
+            h2d_done[b] = ev
+        comp.wait_event(ev)
         if wl.mq:
             wl.qsl_dev = dev["qsl"]
         wl.device_step(dev["q"], dev["k"], dev["v"], dev["slots"], gp, dev["bt"], dev["cl"], maxc, out, ws)
-        pin["out"].copy_(out, non_blocking=True)
-        stream.synchronize()
+        ev = torch.cuda.Event()
+        ev.record(comp)
+        comp_done[b] = ev
+        with torch.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(ev)
+            pin["out"].copy_(out, non_blocking=True)
+            ev2 = torch.cuda.Event()
+            ev2.record(d2h_stream)
+            d2h_done[b] = ev2
+        consume(b ^ 1)                         # the previous step's output, read while this one runs
         return fixed + npairs * 8, wl.kv_bytes(pin["cl"])
 
-    for _ in range(W):
-        one()
+    for i in range(W):
+        one(i)
+    consume(0)
+    consume(1)
     torch.cuda.synchronize(device)
     if world > 1:
         torch.distributed.barrier()
     h2d = kv = 0
     t0 = time.perf_counter()
-    for _ in range(K):
-        a, c = one()
+    for i in range(W, W + K):
+        a, c = one(i)
         h2d += a
         kv += c
-    torch.cuda.synchronize(device)
+    consume(0)
+    consume(1)
     ms = (time.perf_counter() - t0) * 1e3
+    torch.cuda.synchronize(device)
     ms, kv, _ = aggregate_ranks(ms, kv, 0, world, device)
     return {"value": round(kv / (ms * 1e-3) / 1e9, 2), "unit": "GB/s", "ms_per_step": round(ms / K, 4),
             "h2d_bytes_per_step": h2d // K, "d2h_bytes_per_step": d2h,
-            "timing": "host wall clock per step: allocator + H2D + kernels + D2H + stream sync"}
+            "timing": "host wall clock over the steps: allocator + H2D + kernels + D2H + host read of every "
+                      "step's output; two buffer sets, step i+1's host work and copies overlap step i's kernels"}
+
+
+# ------------------------------------------------- the other workloads --
+
+EXTRA_WORKLOADS = (("llama3_8b", None), ("prefix_shared", None), ("quant_mha", "int8"), ("quant_mha", "fp8"),
+                   ("quant_mha", "u8asym"), ("quant_mha", "int4"), ("quant_mha", "fp4"), ("spec_verify", None),
+                   ("chunked_prefill", None), ("tiny", None))
+# quantised workloads whose oracle is also timed on the host cores
+EXTRA_ORACLE = (("quant_mha", "int8"), ("quant_mha", "fp8"))
+
+
+def decode_call_ms(wl, staged, out, ws, flush, scrub, stream, device, reps=3):
+    """Mean CUDA-event time of decode-only calls over the staged inputs
+    (``reps`` passes), with an L2 scrub before each call when ``flush``."""
+    ev = []
+    for _ in range(reps):
+        for st in staged:
+            if flush:
+                scrub.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            wl.decode(st["q"], st["bt"], st["cl"], st["maxc"], out, ws)
+            b.record(stream)
+            ev.append((a, b))
+    torch.cuda.synchronize(device)
+    return sum(a.elapsed_time(b) for a, b in ev) / len(ev)
+
+
+def extra_record(name, cache, device, peak, tflops_peak, steps=8, warmup=3):
+    """Decode-call roofline of one more workload at N = 1: the workload is
+    built through the public API, ``warmup + steps`` whole steps run (write +
+    decode), then the staged steps' decode calls are timed alone."""
+    from paged_kv_cache_438_b200 import pagedkv as P
+    wl = make_workload(name, cache, device)
+    staged = []
+    for _ in range(warmup + steps):
+        slots, pairs, bt, cl = wl.host_step()
+        q, k, v = wl.new_rows()
+        staged.append(dict(slots=slots.to(device), pairs=pairs.to(device) if pairs.numel() else None,
+                           bt=bt.to(device), cl=cl.to(device), maxc=int(cl.max()), q=q, k=k, v=v,
+                           kv=wl.kv_bytes(cl), flops=wl.flops(cl)))
+    maxc_all = max(st["maxc"] for st in staged)
+    _, _, ws_bytes = wl.plan(maxc_all)
+    ws = P.new_workspace(device, ws_bytes)
+    out = torch.empty((wl.q_rows, wl.hq, wl.d), dtype=wl.dtype, device=device)
+    stream = torch.cuda.current_stream(device)
+    scrub = torch.empty(512 * 2 ** 20, dtype=torch.uint8, device=device)
+    step_ev = []
+    for st in staged:
+        scrub.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        wl.device_step(st["q"], st["k"], st["v"], st["slots"], st["pairs"], st["bt"], st["cl"], st["maxc"], out, ws)
+        b.record(stream)
+        step_ev.append((a, b))
+    torch.cuda.synchronize(device)
+    step_ms = sum(a.elapsed_time(b) for a, b in step_ev[warmup:]) / steps
+    timed = staged[warmup:]
+    kv_call = sum(st["kv"] for st in timed) / steps
+    flops_call = sum(st["flops"] for st in timed) / steps
+    small = wl.q_rows * wl.hq * wl.d * 2 * 2 + (kv_call // (wl.per_tok * 16)) * 4
+    alg = kv_call + small
+    flushed_ms = decode_call_ms(wl, timed, out, ws, True, scrub, stream, device)
+    rec = {"workload": name, "cache": cache or ("bf16" if wl.dtype == torch.bfloat16 else "f16"),
+           "batch": wl.B, "kv_bytes_per_call": int(kv_call), "algorithmic_bytes_per_call": int(alg),
+           "ms_per_call": round(flushed_ms, 4), "l2": "scrubbed (512 MiB) before every call",
+           "achieved_gbs": round(alg / (flushed_ms * 1e-3) / 1e9, 1),
+           "frac_of_hbm": round(alg / (flushed_ms * 1e-3) / 1e9 / peak, 4),
+           "ms_per_step": round(step_ms, 4), "seq_steps_per_s": round(wl.B / (step_ms * 1e-3), 1),
+           "traffic": recorded_traffic(name, cache, alg)}
+    if flops_call / (tflops_peak * 1e12) > alg / (peak * 1e9):
+        rec["bound"] = "tensor"
+        rec["achieved_tflops"] = round(flops_call / (flushed_ms * 1e-3) / 1e12, 2)
+        rec["frac_of_tensor"] = round(flops_call / (flushed_ms * 1e-3) / 1e12 / tflops_peak, 4)
+    else:
+        rec["bound"] = "hbm"
+    if wl.mq:
+        rec["query_tokens_per_s"] = round(wl.q_rows / (step_ms * 1e-3), 1)
+    if name == "prefix_shared":
+        # every sequence reads the shared prefix; its blocks are stored once
+        unique = sum((int(st["cl"].sum()) - (wl.B - 1) * wl.prefix) * wl.per_tok for st in timed) / steps
+        warm_ms = decode_call_ms(wl, timed, out, ws, False, scrub, stream, device)
+        rec.update({"unique_kv_bytes_per_call": int(unique),
+                    "unique_gbs": round(unique / (flushed_ms * 1e-3) / 1e9, 1),
+                    "unflushed": {"ms_per_call": round(warm_ms, 4), "l2": "calls back to back, no scrub",
+                                  "achieved_gbs": round(alg / (warm_ms * 1e-3) / 1e9, 1),
+                                  "unique_gbs": round(unique / (warm_ms * 1e-3) / 1e9, 1)},
+                    "note": "achieved_gbs counts logical bytes (the prefix once per sequence); the repeats "
+                            "of the 8 MiB prefix are L2 hits, so it may exceed the HBM figure"})
+    status = P.device_status(clear=True)
+    if status:
+        raise RuntimeError(f"device status {status} raised during the {name} record")
+    if (name, cache) in EXTRA_ORACLE:
+        sec, kvb, seqs = oracle_sample(name, cache, budget_s=6.0)
+        rec["cpu_baseline"] = {"value": round(kvb / sec / 1e9, 4), "unit": "GB/s", "cores": oracle_threads(),
+                               "kind": "oracle", "sample": f"{seqs} of {wl.B} sequences of one step "
+                                                           f"(fp64 numpy oracle, ~6 s, inputs drawn on the CPU)"}
+    del wl, staged, ws, out, scrub
+    torch.cuda.empty_cache()
+    return rec
 
 
 # ----------------------------------------------------------- oracle (CPU) --
@@ -841,6 +994,15 @@ def main():
                                 "sample": f"{seqs} of {wl.B} sequences of one step (fp64 numpy oracle, ~12 s, "
                                           f"inputs drawn on the CPU)",
                                 "seq_steps_per_s": round(seqs / sec, 3)}
+    if world == 1 and not args.no_extra:
+        del r, wl
+        torch.cuda.empty_cache()
+        others = []
+        for name, cache in EXTRA_WORKLOADS:
+            if (name, cache) == (args.workload, args.cache):
+                continue
+            others.append(extra_record(name, cache, device, peak, tflops_peak))
+        line["other_workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -190,12 +190,18 @@ int pkv_decode_workspace_size(int num_seqs, int num_q_heads, int num_kv_heads, i
  * num_q_heads / num_kv_heads = G must be an integer in [1, 16].
  * partition_tokens: as for pkv_decode_plan.
  * workspace      : device scratch of at least the planned bytes, 256-byte
- *                  aligned (may be NULL when the plan has one stream).  It
- *                  must be zero-filled before its first use; afterwards the
- *                  library leaves it valid for the next call (its counters are
- *                  tagged with a per-call epoch).  One workspace serves one
- *                  call at a time: calls that overlap on the GPU need separate
- *                  workspaces.
+ *                  aligned (may be NULL when the plan has one stream).  Its
+ *                  contents need no preparation: it starts with the arrival
+ *                  counters (tagged with a per-call epoch) and the partials
+ *                  follow them.  The library keeps a host-side record, per
+ *                  (device, workspace address), of how many leading bytes hold
+ *                  counters since the last call, and clears the rest of a
+ *                  call's counter area with an asynchronous memset on the
+ *                  call's stream: on the first use of an address, and when a
+ *                  call has more (sequence, KV head) pairs than the previous
+ *                  one on it.  Nothing else may write the workspace between
+ *                  calls.  One workspace serves one call at a time: calls that
+ *                  overlap on the GPU need separate workspaces.
  * The kernel is launched with programmatic stream serialisation: it may
  * start while the immediately preceding kernel on the stream is finishing,
  * and waits for that kernel to complete before it reads q, the caches, or
@@ -297,15 +303,17 @@ int pkv_paged_attention_multi_query(void* out, const void* q,
  *     still needs more (or whose explicit partition does) is rejected with
  *     PKV_ERR_INVALID_ARG before anything is launched.
  *   - The first call on a device looks up the array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make
- *     that first call before any stream capture.
+ *     (cudaGetSymbolAddress, with that device current) and caches it for the
+ *     device's current CUDA context (after a device reset, the first call
+ *     looks it up again); make that first call before any stream capture.
  *   - Nothing is allocated: no cudaMalloc, cudaFree or allocating library call.
  *   - All calls on a device share the one array and it keeps the last call's
- *     contents.  The array starts zero-filled (as a __device__ array does at
- *     load), which is the only state its arrival counters need; partials are
- *     written before they are read.  Calls that overlap on the GPU (concurrent
- *     streams, or other threads) race on it and give wrong results; serialise
- *     them, e.g. on one stream.
+ *     contents.  Its arrival counters are cleared like those of a caller's
+ *     workspace (see pkv_paged_attention_decode: an asynchronous memset on
+ *     the first call and whenever a call has more (sequence, KV head) pairs
+ *     than the one before); partials are written before they are read.
+ *     Calls that overlap on the GPU (concurrent streams, or other threads)
+ *     race on it and give wrong results; serialise them, e.g. on one stream.
  */
 #define PKV_NOALLOC_SCRATCH_BYTES (16u << 20)
 

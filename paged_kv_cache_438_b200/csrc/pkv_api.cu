@@ -8,6 +8,7 @@
 #include <algorithm>
 #include <atomic>
 #include <cmath>
+#include <map>
 #include <mutex>
 #include <unordered_map>
 #include <unordered_set>
@@ -56,17 +57,21 @@ int fetch(std::vector<T>* dst, const T* src, size_t n, cudaStream_t st) {
   return e == cudaSuccess ? PKV_OK : cuda_fail(e, "validation copy");
 }
 
+// A driver API function by name and ABI version (nullptr if unavailable);
+// the library links only the runtime.
+void* driver_entry(const char* name, unsigned int version) {
+  void* p = nullptr;
+  cudaDriverEntryPointQueryResult q{};
+  if (cudaGetDriverEntryPointByVersion(name, &p, version, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return p;
+}
+
 // ---------------------------------------------------------- tensor maps --
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q{};
-    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
-            cudaSuccess ||
-        q != cudaDriverEntryPointSuccess)
-      return static_cast<PFN_cuTensorMapEncodeTiled_v12000>(nullptr);
-    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }();
+  static PFN_cuTensorMapEncodeTiled_v12000 fn =
+      reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(driver_entry("cuTensorMapEncodeTiled", 12000));
   return fn;
 }
 
@@ -192,6 +197,35 @@ unsigned long long next_epoch() {
     e = (epoch.fetch_add(1) + 1) & ((1ull << 40) - 1);
   } while (e == 0);
   return e;
+}
+
+// A workspace holds the arrival counters at its head and the partials after
+// them, and the boundary moves with the call's shape (sequences x KV heads x
+// column tiles).  Bytes that an earlier call used for partials may hold any
+// float pair, and a float pair can read as a counter of the current epoch.
+// So the library records, per (device, workspace address), how many leading
+// bytes hold counters or zeros since the last call, and clears the rest of a
+// call's counter area (an asynchronous memset on the call's stream, not an
+// allocation) before the launch.  A workspace the record does not know has
+// its whole counter area cleared on its first use.
+int prepare_counters(void* ws, size_t counter_bytes, cudaStream_t st) {
+  static std::mutex mu;
+  static std::map<std::pair<int, uintptr_t>, size_t> clean;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const auto key = std::make_pair(dev, reinterpret_cast<uintptr_t>(ws));
+  std::lock_guard<std::mutex> lk(mu);
+  auto it = clean.find(key);
+  const size_t have = it == clean.end() ? 0 : it->second;
+  if (counter_bytes > have) {
+    e = cudaMemsetAsync(static_cast<uint8_t*>(ws) + have, 0, counter_bytes - have, st);
+    if (e != cudaSuccess) return cuda_fail(e, "clearing the workspace's arrival counters");
+  }
+  // bounded: a workspace dropped from the record is cleared again on its next use
+  if (it == clean.end() && clean.size() >= 4096) clean.clear();
+  clean[key] = counter_bytes;  // this call's partials start right after its counters
+  return PKV_OK;
 }
 
 template <class T>
@@ -556,6 +590,8 @@ int attention_call(void* out, const void* q, const void* k_cache, const void* v_
   p.query_start_loc = mq ? query_start_loc : nullptr;
   if (pl.num_streams > 1) {
     auto* ws = static_cast<uint8_t*>(workspace);
+    rc = prepare_counters(workspace, pl.counter_bytes, st);
+    if (rc != PKV_OK) return rc;
     p.counters = reinterpret_cast<unsigned long long*>(ws);
     p.slots = reinterpret_cast<float*>(ws + pl.counter_bytes);
   }
@@ -710,25 +746,41 @@ constexpr size_t kNoAllocScratchBytes = static_cast<size_t>(PKV_NOALLOC_SCRATCH_
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
+// Unique ID of the calling thread's current CUDA context, or 0 when there is
+// none or the driver cannot say.  A device reset ends the primary context
+// (and the module holding the array); the next context has a new ID.
+unsigned long long current_context_id() {
+  static auto get_current = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(driver_entry("cuCtxGetCurrent", 4000));
+  static auto get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(driver_entry("cuCtxGetId", 12000));
+  CUcontext ctx = nullptr;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  return get_id(ctx, &id) == CUDA_SUCCESS ? id : 0;
+}
+
 // Device address of g_noalloc_scratch on the current device, looked up on
-// the first call for that device (with that device current) and cached.
+// the first call for that device (with that device current) and cached per
+// (device, context): after a device reset the address is looked up again.
 int noalloc_scratch_address(void** out) {
   static std::mutex mu;
-  static std::vector<void*> by_device;
+  static std::vector<std::pair<unsigned long long, void*>> by_device;  // (context ID, address)
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  const unsigned long long ctx = current_context_id();
   std::lock_guard<std::mutex> lk(mu);
-  if (static_cast<size_t>(dev) < by_device.size() && by_device[dev] != nullptr) {
-    *out = by_device[dev];
+  if (ctx != 0 && static_cast<size_t>(dev) < by_device.size() && by_device[dev].first == ctx &&
+      by_device[dev].second != nullptr) {
+    *out = by_device[dev].second;
     return PKV_OK;
   }
   void* p = nullptr;
   e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(no-alloc scratch)");
   if (p == nullptr) return fail(PKV_ERR_CUDA, "cudaGetSymbolAddress returned NULL for the no-alloc scratch");
-  if (by_device.size() <= static_cast<size_t>(dev)) by_device.resize(dev + 1, nullptr);
-  by_device[dev] = p;
+  if (by_device.size() <= static_cast<size_t>(dev)) by_device.resize(dev + 1, {0ull, nullptr});
+  // with no context ID to check against, the address is looked up on every call
+  by_device[dev] = {ctx, ctx != 0 ? p : nullptr};
   *out = p;
   return PKV_OK;
 }

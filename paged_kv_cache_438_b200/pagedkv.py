@@ -242,9 +242,9 @@ _WORKSPACES = {}
 
 
 def _cached_workspace(device, stream, nbytes):
-    """A decode workspace for (device, stream): zero-filled when created (the
-    library needs zeros only before a workspace's first use) and grown on
-    demand.  One per stream, so calls on different streams never share one."""
+    """A decode workspace for (device, stream), grown on demand (the library
+    prepares its counter area itself).  One per stream, so calls on different
+    streams never share one."""
     s = torch.cuda.current_stream(device) if stream is None else stream
     key = (device.index, s.cuda_stream)
     ws = _WORKSPACES.get(key)
@@ -255,7 +255,8 @@ def _cached_workspace(device, stream, nbytes):
 
 
 def new_workspace(device, nbytes):
-    """A zero-filled decode workspace of at least ``nbytes`` (see decode_plan)."""
+    """A decode workspace of at least ``nbytes`` (see decode_plan); the library
+    clears its counter area itself, so the zero fill here is only tidiness."""
     return torch.zeros(max(int(nbytes), 256), dtype=torch.uint8, device=device)
 
 
@@ -267,8 +268,8 @@ def paged_attention_decode(q, k_cache, v_cache, block_tables, context_lens, scal
     q [B, Hq, D] fp16/bf16; caches [NB, Hkv, 16, D]; block_tables [B, MB]
     int32; context_lens [B] int32.  ``max_context_len`` is a host-side upper
     bound on context_lens (if None it is read from the device, which
-    synchronises).  ``workspace`` (uint8, from ``new_workspace``) must be
-    zero-filled before its first use and serve one call at a time; when None
+    synchronises).  ``workspace`` (uint8, from ``new_workspace``) serves one
+    call at a time and is written by nothing else between calls; when None
     a cached per-stream workspace is used.  A uint8 cache with ``k_zero`` /
     ``v_zero`` is the asymmetric format, read as (code - zero) * scale.
     ``sliding_window`` W > 0 limits each query to its W most recent keys.

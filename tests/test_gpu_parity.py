@@ -539,6 +539,33 @@ def test_workspace_reused_across_shapes_matches_fresh_workspaces():
     assert P.device_status(clear=True) == 0
 
 
+def test_workspace_needs_no_zero_fill_and_survives_a_growing_counter_area():
+    """A workspace holding arbitrary bytes, and one whose next call has more
+    (sequence, KV head) pairs than the last (its counter area then covers
+    bytes that held the last call's partial floats), give the same bits as a
+    fresh workspace: the library clears whatever part of a call's counter
+    area it has not seen hold counters."""
+    small = I.device_decode_case("llama3_8b", DEV, batch=4, seed=21)
+    large = I.device_decode_case("quant_mha", DEV, batch=96, cache_kind="fp8", seed=22)
+    runs = []
+    for c in (small, large, small, large):
+        maxc = int(c["context_lens_cpu"].max())
+        nw, _, wsb = P.decode_plan(c["batch"], c["hq"], c["hkv"], c["d"], maxc, c["k_cache"].dtype, 256)
+        assert nw > 1
+        runs.append((c, maxc, wsb))
+    wsb_max = max(w for _, _, w in runs)
+    garbage = torch.randint(0, 256, (wsb_max,), dtype=torch.uint8, device=DEV)
+    for c, maxc, wsb in runs:
+        run = lambda ws: P.paged_attention_decode(c["q"], c["k_cache"], c["v_cache"], c["block_tables"],
+                                                  c["context_lens"], c["scale"], c.get("k_scale"), c.get("v_scale"),
+                                                  max_context_len=maxc, workspace=ws, partition_tokens=256)
+        got = run(garbage)
+        ref = run(P.new_workspace(DEV, wsb))
+        torch.cuda.synchronize()
+        assert torch.equal(got, ref)
+    assert P.device_status(clear=True) == 0
+
+
 @pytest.mark.parametrize("kind", ["float", "fp8", "u8asym", "fp4"])
 def test_never_written_tail_positions_do_not_leak(kind):
     """Positions of a sequence's last block at or beyond its context were
