@@ -135,13 +135,15 @@ int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int r
   const long long blocks_max = std::max(1, (max_ctx + 15) / 16);
   const long long t_max = static_cast<long long>(std::max(B, 1)) * Hkv * max_tiles * blocks_max;
   if (t_max >= (1LL << 31)) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31 (sequence, head, block) items");
-  // One CTA per SM.  8-bit caches always use 8 warps (more conversion work per
-  // byte); 16-bit caches use 4 warps with twice the ring depth when each of 8
-  // warps per SM would still get at least kLongStreamBlocks blocks (measured:
-  // long contexts keep HBM busiest that way, short or L2-resident work wants
-  // the extra warps).
+  // One CTA per SM.  Quantised caches use 12 warps (8 when a pair has more
+  // than 8 columns): their conversion work per byte, not HBM, sets the pace
+  // and more warps hide its latency.  16-bit caches use 4 warps with twice
+  // the ring depth when each of 8 warps per SM would still get at least
+  // kLongStreamBlocks blocks (measured: long contexts keep HBM busiest that
+  // way, short or L2-resident work wants the extra warps).
   const long long sms = sm_count();
-  const int warps = (!isq(cache_dtype) && t_max / (8 * sms) >= kLongStreamBlocks) ? 4 : 8;
+  const bool wide = tile_cols > 8;
+  const int warps = isq(cache_dtype) ? (wide ? 8 : 12) : (t_max / (8 * sms) >= kLongStreamBlocks ? 4 : 8);
   long long nw;
   if (req_tokens > 0) {
     if (req_tokens % 16 != 0) return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d is not a multiple of 16", req_tokens);
@@ -259,7 +261,7 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::Decod
   using Tr = pkv::DecodeTraits<kD, kCT>;
   auto kernel = pkv::paged_decode_kernel<kD, kCT, kNT, kQBF16, kMQ>;
   const int warps = p.ring_warps;
-  if (warps < 1 || warps > Tr::kMaxWarps) return fail(PKV_ERR_INVALID_ARG, "bad warp count %d", warps);
+  if (warps < 1 || warps > Tr::max_warps(kNT)) return fail(PKV_ERR_INVALID_ARG, "bad warp count %d", warps);
   pkv::DecodeParams q = p;
   q.ring = Tr::ring_depth(warps);
   const size_t smem = decode_smem_bytes<kD, kCT>(p.num_seqs, warps);

@@ -80,11 +80,17 @@ struct DecodeTraits {
   // stage layout: K tile, V tile, K scales, V scales, K zero points, V zero points
   static constexpr int kStageTx = 2 * kKVBytes + 2 * kScaleBytes + 2 * kZeroBytes;  // bytes landing per stage
   static constexpr int kStageBytes = round_up_c(kStageTx, 1024);    // keeps every tile 1024-aligned
-  static constexpr int kMaxWarps = 8;
+  // Quantised caches with up to 8 columns per pair run 12 warps per CTA
+  // (registers capped at 168 by the launch bounds, three warps per SM
+  // sub-partition): their per-block instruction stream, not HBM, sets the
+  // pace, so more warps hide more of its latency.  16-bit caches run 4 or 8,
+  // and so do 16-column pairs, whose accumulators do not fit 168 registers.
+  static constexpr int max_warps(int nt) { return kQuant && nt == 1 ? 12 : 8; }
   // One CTA per SM.  Its warps (4 or 8, chosen per call) share this many
   // bytes of copy ring: 4 warps x 4 stages or 8 warps x 2 stages of 8 KiB for
-  // bf16 / fp16 at head_dim 128; 8-bit caches keep 8 warps and more stages.
-  static constexpr int kRingBudget = kQuant ? 160 * 1024 : 128 * 1024;
+  // bf16 / fp16 at head_dim 128; quantised caches 12 warps x 3 stages of
+  // 5 KiB (8-bit) or x 5 stages of 3 KiB (4-bit).
+  static constexpr int kRingBudget = kQuant ? 180 * 1024 : 128 * 1024;
   static int ring_depth(int warps) {
     const int r = kRingBudget / (warps * kStageBytes);
     return r < 2 ? 2 : (r > 8 ? 8 : r);
@@ -329,7 +335,7 @@ __device__ __forceinline__ int stream_of(long long T, long long g, long long nw)
 }
 
 template <int kD, int kCT, int kNT, bool kQBF16, bool kMQ>
-__global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
+__global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
     paged_decode_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
                         const DecodeParams p) {
   using Tr = DecodeTraits<kD, kCT>;
@@ -479,7 +485,14 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
   auto col_token = [&](int c) { return (tile * p.tile_cols + c) / G; };
   auto col_head = [&](int c) { return (tile * p.tile_cols + c) % G; };
 
+  // Integer K codes (INT8, uint8, INT4) are widened with their bias left in
+  // (e.g. 1152 + c for INT8); the bias times the sum of the query elements
+  // it multiplies is subtracted when the block's scores start.  kqs holds,
+  // for this lane's two accumulator columns, that sum (uint8: the plain
+  // query sum, scaled per token row by 1024 + its zero point).
+  constexpr bool kBiasK = (kCT == kI8 || kCT == kU8 || kCT == kI4);
   uint32_t qf[kNT][kKS][2];
+  float kqs[kNT][2];
   float o[kMT][kNT][4];
   float m_run[kNT][2], l_run[kNT][2];
   int colv[kNT][2];  // multi-query: visible keys of the lane's accumulator columns
@@ -521,6 +534,12 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
           }
           qf[nt][jj][0] = valid ? load_q_two<kQBF16>(p.q, b8 + e0, b8 + e1) : 0u;
           qf[nt][jj][1] = valid ? load_q_two<kQBF16>(p.q, b8 + e2, b8 + e3) : 0u;
+          if constexpr (kCT == kI4) {
+            // slots 2q+8, 2q+9 meet odd nibbles, widened at 16x: q / 16 (exact)
+            const __half2 h = __hmul2(*reinterpret_cast<const __half2*>(&qf[nt][jj][1]),
+                                      __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00)));
+            qf[nt][jj][1] = *reinterpret_cast<const uint32_t*>(&h);
+          }
         } else {
           // 16-bit K: k-index 2q,2q+1 -> d 16jj+2q.. ; 2q+8.. -> d 16jj+8+2q..
           // 8-bit K:  k-index 2q,2q+1 -> d 16jj+4q.. ; 2q+8.. -> d 16jj+4q+2..
@@ -534,6 +553,29 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       l_run[nt][0] = l_run[nt][1] = 0.0f;
 #pragma unroll
       for (int i = 0; i < kMT; ++i) o[i][nt][0] = o[i][nt][1] = o[i][nt][2] = o[i][nt][3] = 0.0f;
+      if constexpr (kBiasK) {
+        // this lane holds column r's query elements at its k-slots: sum them
+        // in the weights the biases give them, over the four lanes of the
+        // column, then fetch the sums of the lane's accumulator columns
+        // 2q and 2q+1 (held by lanes 8q and 8q + 4)
+        float sb = 0.0f;
+#pragma unroll
+        for (int jj = 0; jj < kKS; ++jj) {
+          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&qf[nt][jj][0]));
+          const float2 b = __half22float2(*reinterpret_cast<const __half2*>(&qf[nt][jj][1]));
+          if constexpr (kCT == kI4) {
+            sb += 1032.0f * (a.x + a.y) + 1152.0f * (b.x + b.y);
+          } else {
+            sb += (a.x + a.y) + (b.x + b.y);
+          }
+        }
+        sb += __shfl_xor_sync(0xffffffffu, sb, 1);
+        sb += __shfl_xor_sync(0xffffffffu, sb, 2);
+        const float s0 = __shfl_sync(0xffffffffu, sb, 8 * q4);
+        const float s1 = __shfl_sync(0xffffffffu, sb, 8 * q4 + 4);
+        kqs[nt][0] = kCT == kI8 ? 1152.0f * s0 : s0;
+        kqs[nt][1] = kCT == kI8 ? 1152.0f * s1 : s1;
+      }
     }
   };
   begin_pair();
@@ -576,10 +618,24 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 
     // ---- S^T = K . Q^T (two independent accumulation chains, summed) ----
     float sacc[kNT][4], sacc2[kNT][4];
+    // uint8: the bias of token row r (r + 8) is 1024 + its zero point
+    float zb_r = 1.0f, zb_r8 = 1.0f;
+    if constexpr (kCT == kU8) {
+      const uint8_t* zk = base_ptr + (st - smem_base) + 2 * Tr::kKVBytes + 128;
+      zb_r = 1024.0f + static_cast<float>(zk[r]);
+      zb_r8 = 1024.0f + static_cast<float>(zk[r + 8]);
+    }
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0.0f;
+      for (int e = 0; e < 4; ++e) {
+        sacc2[nt][e] = 0.0f;
+        if constexpr (kBiasK) {
+          sacc[nt][e] = -kqs[nt][e & 1] * (e < 2 ? zb_r : zb_r8);
+        } else {
+          sacc[nt][e] = 0.0f;
+        }
+      }
     if constexpr (!kQt) {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
@@ -601,8 +657,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
         for (int c2 = 0; c2 < 2; ++c2) {
           uint32_t x[4], y[4];  // fp16 pairs of token r (x) and token r + 8 (y)
           if constexpr (kCT == kI4) {
-            i4x8_to_h2x4(w[2 * c2], x);
-            i4x8_to_h2x4(w[2 * c2 + 1], y);
+            i4x8_to_h2x4_biased(w[2 * c2], x);
+            i4x8_to_h2x4_biased(w[2 * c2 + 1], y);
           } else {
             e2m1x8_to_h2x4(w[2 * c2], x);
             e2m1x8_to_h2x4(w[2 * c2 + 1], y);
@@ -617,13 +673,6 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
       }
     } else {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
-      // uint8: fp16 pairs (1024 + z) of this lane's two tokens r and r + 8
-      uint32_t zk_r = 0, zk_r8 = 0;
-      if constexpr (kCT == kU8) {
-        const uint8_t* zk = base_ptr + (st - smem_base) + 2 * Tr::kKVBytes + 128;
-        zk_r = (0x6400u + zk[r]) * 0x10001u;
-        zk_r8 = (0x6400u + zk[r + 8]) * 0x10001u;
-      }
 #pragma unroll
       for (int jj = 0; jj < kKS; jj += 2) {
         uint32_t w[4];
@@ -632,16 +681,18 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
         for (int j2 = 0; j2 < 2; ++j2) {
           uint32_t lo_r, hi_r, lo_r8, hi_r8;  // (d 4q,4q+1) and (d 4q+2,4q+3) of tokens r and r+8
           if constexpr (kCT == kI8) {
+            // fp16 1152 + c (the bias is taken out through kqs)
             const uint32_t u0 = w[2 * j2] ^ 0x80808080u, u1 = w[2 * j2 + 1] ^ 0x80808080u;
-            lo_r = i8pair_to_h2(u0, 0x4140u);
-            hi_r = i8pair_to_h2(u0, 0x4342u);
-            lo_r8 = i8pair_to_h2(u1, 0x4140u);
-            hi_r8 = i8pair_to_h2(u1, 0x4342u);
+            lo_r = prmt(u0, 0x64646464u, 0x4140u);
+            hi_r = prmt(u0, 0x64646464u, 0x4342u);
+            lo_r8 = prmt(u1, 0x64646464u, 0x4140u);
+            hi_r8 = prmt(u1, 0x64646464u, 0x4342u);
           } else if constexpr (kCT == kU8) {
-            lo_r = u8pair_minus_zero(w[2 * j2], 0x4140u, zk_r);
-            hi_r = u8pair_minus_zero(w[2 * j2], 0x4342u, zk_r);
-            lo_r8 = u8pair_minus_zero(w[2 * j2 + 1], 0x4140u, zk_r8);
-            hi_r8 = u8pair_minus_zero(w[2 * j2 + 1], 0x4342u, zk_r8);
+            // fp16 1024 + c (the bias 1024 + z is taken out through kqs)
+            lo_r = prmt(w[2 * j2], 0x64646464u, 0x4140u);
+            hi_r = prmt(w[2 * j2], 0x64646464u, 0x4342u);
+            lo_r8 = prmt(w[2 * j2 + 1], 0x64646464u, 0x4140u);
+            hi_r8 = prmt(w[2 * j2 + 1], 0x64646464u, 0x4342u);
           } else {
             e4m3x4_to_h2x2(w[2 * j2], lo_r, hi_r);
             e4m3x4_to_h2x2(w[2 * j2 + 1], lo_r8, hi_r8);
@@ -930,16 +981,19 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
             const int idx = 2 * w + (stream_start(T, w, nw) >= gp0 ? 0 : 1);
             return p.slots + static_cast<long long>(idx) * p.slot_floats;
           };
-          // One pass over the contributors per group of 8 heads, with a
+          // One pass over the contributors per group of kMG heads, with a
           // running max per head: every load of a contributor is independent
           // of the others, and two contributors are in flight at once.  Each
-          // lane owns kD / 32 output columns of every head.
+          // lane owns kD / 32 output columns of every head.  (Groups of 4 for
+          // quantised caches keep this rarely run code within their 168
+          // registers.)
           constexpr int kV = kD / 32;
+          constexpr int kMG = kQt ? 4 : 8;
 #pragma unroll 1
-          for (int c0 = 0; c0 < ncols; c0 += 8) {
-            float Mg[8], Lg[8], acc[8][kV];
+          for (int c0 = 0; c0 < ncols; c0 += kMG) {
+            float Mg[kMG], Lg[kMG], acc[kMG][kV];
 #pragma unroll
-            for (int gg = 0; gg < 8; ++gg) {
+            for (int gg = 0; gg < kMG; ++gg) {
               Mg[gg] = -INFINITY;
               Lg[gg] = 0.0f;
 #pragma unroll
@@ -948,9 +1002,9 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
 #pragma unroll 2
             for (int c = 0; c < n_c; ++c) {
               const float* sl = slot_of(c);
-              float mc[8], lc[8], ov[8][kV];
+              float mc[kMG], lc[kMG], ov[kMG][kV];
 #pragma unroll
-              for (int gg = 0; gg < 8; ++gg) {
+              for (int gg = 0; gg < kMG; ++gg) {
                 const int g = c0 + gg;
                 if (g < ncols) {
                   mc[gg] = __ldcg(sl + g);
@@ -970,7 +1024,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
                 }
               }
 #pragma unroll
-              for (int gg = 0; gg < 8; ++gg) {
+              for (int gg = 0; gg < kMG; ++gg) {
                 // multi-query: skip a share that saw no visible key of the column
                 if (c0 + gg < ncols && (!kMQ || mc[gg] != -INFINITY)) {
                   const float mn = fmaxf(Mg[gg], mc[gg]);
@@ -984,7 +1038,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::kMaxWarps * 32)
               }
             }
 #pragma unroll
-            for (int gg = 0; gg < 8; ++gg) {
+            for (int gg = 0; gg < kMG; ++gg) {
               const int g = c0 + gg;
               if (g < ncols) {
                 const float inv = Lg[gg] > 0.0f ? 1.0f / Lg[gg] : 0.0f;

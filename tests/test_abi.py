@@ -182,6 +182,19 @@ def test_small_batches_get_shorter_streams(lib):
     assert nw == wave and per >= 16 * 16
 
 
+def test_quantised_caches_run_twelve_warps_per_sm_unless_pairs_are_wide(lib):
+    # quantised caches: 12 warps per SM (168 registers each) for pairs of up
+    # to 8 columns; 16-column pairs (a GQA group of 16) keep 8
+    for code in (P.PKV_I8, P.PKV_FP8E4M3, P.PKV_U8ASYM, P.PKV_I4, P.PKV_FP4E2M1):
+        nw, _, _ = P.decode_plan(256, 32, 32, 128, 8192, code)
+        assert nw == 12 * 148
+        nw, _, _ = P.decode_plan(64, 256, 16, 128, 8192, code)
+        assert nw == 8 * 148
+    # a 16-bit cache of the same shape: long streams, 4 warps per SM
+    nw, _, _ = P.decode_plan(256, 32, 32, 128, 8192, P.PKV_BF16)
+    assert nw == 4 * 148
+
+
 def test_query_major_routing_threshold_and_group(lib):
     def mq(hq, d, n, cd=P.PKV_BF16):
         return P.multi_query_plan(2, hq, 8, d, 1024, n, cd)[0]
