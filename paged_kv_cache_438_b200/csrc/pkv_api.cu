@@ -248,12 +248,22 @@ int set_smem(T* kernel, size_t bytes) {
   return PKV_OK;
 }
 
+// Shared memory of a decode CTA: alignment slack, the warps' copy rings and
+// their barriers, and the context-length scan (num_seqs + 1 entries).
 template <int kD, int kCT>
-size_t decode_smem_bytes(int num_seqs, int warps) {
+size_t decode_smem_bytes(int num_seqs, int warps, int ring) {
   using Tr = pkv::DecodeTraits<kD, kCT>;
-  const int ring = Tr::ring_depth(warps);
-  return 1024 + static_cast<size_t>(warps) * ring * Tr::kStageBytes + static_cast<size_t>(warps) * ring * 8 +
-         (static_cast<size_t>(num_seqs) + 1) * 4;
+  return 1024 + static_cast<size_t>(warps) * ring * (Tr::kStageBytes + 8) + (static_cast<size_t>(num_seqs) + 1) * 4;
+}
+
+// Copy stages per warp: as many as the ring budget holds (2 to 8), fewer
+// when the scan of a large batch would not leave room for them.
+template <int kD, int kCT>
+int decode_ring(int num_seqs, int warps) {
+  using Tr = pkv::DecodeTraits<kD, kCT>;
+  int r = std::max(2, std::min(8, Tr::ring_budget(warps) / (warps * Tr::kStageBytes)));
+  while (r > 2 && decode_smem_bytes<kD, kCT>(num_seqs, warps, r) > static_cast<size_t>(kMaxCtaSmem)) --r;
+  return r;
 }
 
 template <int kD, int kCT, int kNT, bool kQBF16, bool kMQ>
@@ -263,8 +273,8 @@ int launch_decode(const CUtensorMap& km, const CUtensorMap& vm, const pkv::Decod
   const int warps = p.ring_warps;
   if (warps < 1 || warps > Tr::max_warps(kNT)) return fail(PKV_ERR_INVALID_ARG, "bad warp count %d", warps);
   pkv::DecodeParams q = p;
-  q.ring = Tr::ring_depth(warps);
-  const size_t smem = decode_smem_bytes<kD, kCT>(p.num_seqs, warps);
+  q.ring = decode_ring<kD, kCT>(p.num_seqs, warps);
+  const size_t smem = decode_smem_bytes<kD, kCT>(p.num_seqs, warps, q.ring);
   if (smem > static_cast<size_t>(kMaxCtaSmem))
     return fail(PKV_ERR_UNSUPPORTED, "batch of %d sequences needs %zu bytes of shared memory", p.num_seqs, smem);
   int rc = set_smem(kernel, smem);

@@ -63,6 +63,12 @@ enum CacheType : int {
 
 constexpr int round_up_c(int x, int m) { return (x + m - 1) / m * m; }
 
+// A compile-time int carried as a value (selects a generic lambda's instance).
+template <int N>
+struct IntC {
+  static constexpr int value = N;
+};
+
 template <int kD, int kCT>
 struct DecodeTraits {
   static constexpr bool k8bit = (kCT == kI8 || kCT == kFP8 || kCT == kU8);
@@ -86,15 +92,14 @@ struct DecodeTraits {
   // pace, so more warps hide more of its latency.  16-bit caches run 4 or 8,
   // and so do 16-column pairs, whose accumulators do not fit 168 registers.
   static constexpr int max_warps(int nt) { return kQuant && nt == 1 ? 12 : 8; }
-  // One CTA per SM.  Its warps (4 or 8, chosen per call) share this many
-  // bytes of copy ring: 4 warps x 4 stages or 8 warps x 2 stages of 8 KiB for
-  // bf16 / fp16 at head_dim 128; quantised caches 12 warps x 3 stages of
-  // 5 KiB (8-bit) or x 5 stages of 3 KiB (4-bit).
-  static constexpr int kRingBudget = kQuant ? 180 * 1024 : 128 * 1024;
-  static int ring_depth(int warps) {
-    const int r = kRingBudget / (warps * kStageBytes);
-    return r < 2 ? 2 : (r > 8 ? 8 : r);
-  }
+  // One CTA per SM.  Its warps (chosen per call) share up to this many bytes
+  // of copy ring: 4 warps x 6 stages or 8 warps x 2 stages of 8 KiB for
+  // bf16 / fp16 at head_dim 128 (measured: the long-context stream gains
+  // from the deeper ring, the 8-warp plan loses with 3 stages); quantised
+  // caches 12 warps x 3 stages of 5 KiB (8-bit) or x 5 stages of 3 KiB
+  // (4-bit).  The host trims the depth when a large batch's context-length
+  // scan needs the shared memory.
+  static constexpr int ring_budget(int warps) { return kQuant ? 180 * 1024 : (warps <= 4 ? 192 : 128) * 1024; }
 };
 
 // Epoch-tagged arrival counters: bits 63..24 hold the epoch of the call that
@@ -494,10 +499,22 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
   uint32_t qf[kNT][kKS][2];
   float kqs[kNT][2];
   float o[kMT][kNT][4];
+  // Integer V codes are widened with their bias left in as well (INT8
+  // 1152 + c, uint8 1024 + c, INT4 1032 + c at even d and 1152 + 16c at odd
+  // d).  One more MMA per block accumulates, per column, the weight that
+  // bias carries into O^T (wacc = sum over tokens of bias x P), and it is
+  // taken out of O^T every kFoldBlocks blocks and when the pair ends; so the
+  // bias never builds up over a long context (the cancellation stays within
+  // 128 tokens), and O^T is exact up to that rounding.
+  constexpr bool kBiasV = kBiasK;
+  constexpr int kFoldBlocks = 8;
+  float wacc[kNT][4];
+  int since_fold = 0;
   float m_run[kNT][2], l_run[kNT][2];
   int colv[kNT][2];  // multi-query: visible keys of the lane's accumulator columns
 
   auto begin_pair = [&]() {
+    since_fold = 0;
     const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
 #pragma unroll
     for (int nt = 0; nt < kNT; ++nt) {
@@ -553,6 +570,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
       l_run[nt][0] = l_run[nt][1] = 0.0f;
 #pragma unroll
       for (int i = 0; i < kMT; ++i) o[i][nt][0] = o[i][nt][1] = o[i][nt][2] = o[i][nt][3] = 0.0f;
+      wacc[nt][0] = wacc[nt][1] = wacc[nt][2] = wacc[nt][3] = 0.0f;
       if constexpr (kBiasK) {
         // this lane holds column r's query elements at its k-slots: sum them
         // in the weights the biases give them, over the four lanes of the
@@ -580,62 +598,12 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
   };
   begin_pair();
 
-  int cstage = 0;        // ring stage of item k
+  int cstage = 0;        // ring stage of the next item
   uint32_t cphase = 0;   // its barrier phase
-#pragma unroll 1
-  for (int k = 0; k < count; ++k) {
-    const int stage = cstage;
-    const uint32_t st = ring + stage * Tr::kStageBytes;
-    const bool landed = mbar_wait(bars + stage * 8, cphase);
-    if (++cstage == kR) {
-      cstage = 0;
-      cphase ^= 1u;
-    }
-    if (__any_sync(0xffffffffu, !landed)) {  // warp-uniform: never split the warp before ldmatrix/mma
-      // let copies already in flight land (bounded) before the warp leaves
-      for (int kk = k + 1; kk < count && kk < k + kR; ++kk) mbar_wait(bars + (kk % kR) * 8, (kk / kR) & 1);
-      return;
-    }
-    const int kpos0 = (jb + j) * 16;  // position of the block's first token
-    const int valid = ctx - kpos0;    // >= 1 tokens of this block count
-    // sliding window: tokens before position ctx - window are not seen
-    const int lowv = p.window > 0 ? ctx - p.window - kpos0 : -32;
-    // Rows of a sequence's last block at or beyond its context were never
-    // written and may hold anything, NaN included; P is 0 there, but 0 * NaN
-    // is not, so those V rows are zeroed in the stage first (and their
-    // scales replaced by 0 below).
-    const bool tail = valid < 16;
-    if (tail) {
-      uint8_t* vrow = base_ptr + (st - smem_base) + Tr::kKVBytes;
-      constexpr int kChunks = Tr::kNumColTiles * Tr::kChunksPerTileRow;  // 16-byte chunks per row
-      for (int e = lane; e < (16 - valid) * kChunks; e += 32) {
-        const int t = valid + e / kChunks, c = e % kChunks;
-        *reinterpret_cast<uint4*>(vrow + (c / Tr::kChunksPerTileRow) * Tr::kColTileBytes + t * Tr::kTileBytes +
-                                  (c % Tr::kChunksPerTileRow) * 16) = make_uint4(0u, 0u, 0u, 0u);
-      }
-      __syncwarp();
-    }
 
-    // ---- S^T = K . Q^T (two independent accumulation chains, summed) ----
-    float sacc[kNT][4], sacc2[kNT][4];
-    // uint8: the bias of token row r (r + 8) is 1024 + its zero point
-    float zb_r = 1.0f, zb_r8 = 1.0f;
-    if constexpr (kCT == kU8) {
-      const uint8_t* zk = base_ptr + (st - smem_base) + 2 * Tr::kKVBytes + 128;
-      zb_r = 1024.0f + static_cast<float>(zk[r]);
-      zb_r8 = 1024.0f + static_cast<float>(zk[r + 8]);
-    }
-#pragma unroll
-    for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        sacc2[nt][e] = 0.0f;
-        if constexpr (kBiasK) {
-          sacc[nt][e] = -kqs[nt][e & 1] * (e < 2 ? zb_r : zb_r8);
-        } else {
-          sacc[nt][e] = 0.0f;
-        }
-      }
+  // Scores S^T = K . Q^T of the block in stage `st`: even k-steps accumulate
+  // into `ae`, odd ones into `ao` (the same array for one chain per block).
+  auto scores = [&](uint32_t st, float (&ae)[kNT][4], float (&ao)[kNT][4]) {
     if constexpr (!kQt) {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
@@ -644,7 +612,7 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
         ldsm_x4(st + swz<Tr>(t, 2 * jj + (lane >> 4)), a0, a1, a2, a3);
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt)
-          mma_16816<kMmaBF16>((jj & 1) ? sacc2[nt] : sacc[nt], a0, a1, a2, a3, qf[nt][jj][0], qf[nt][jj][1]);
+          mma_16816<kMmaBF16>((jj & 1) ? ao[nt] : ae[nt], a0, a1, a2, a3, qf[nt][jj][0], qf[nt][jj][1]);
       }
     } else if constexpr (k4) {
       // one ldmatrix.x4 = tokens 0-7 / 8-15 of two 32-code chunks (4 k-steps)
@@ -666,8 +634,8 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
           const int jj = 2 * (c + c2);
 #pragma unroll
           for (int nt = 0; nt < kNT; ++nt) {
-            mma_16816<false>(sacc[nt], x[0], y[0], x[1], y[1], qf[nt][jj][0], qf[nt][jj][1]);
-            mma_16816<false>(sacc2[nt], x[2], y[2], x[3], y[3], qf[nt][jj + 1][0], qf[nt][jj + 1][1]);
+            mma_16816<false>(ae[nt], x[0], y[0], x[1], y[1], qf[nt][jj][0], qf[nt][jj][1]);
+            mma_16816<false>(ao[nt], x[2], y[2], x[3], y[3], qf[nt][jj + 1][0], qf[nt][jj + 1][1]);
           }
         }
       }
@@ -699,84 +667,14 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
           }
 #pragma unroll
           for (int nt = 0; nt < kNT; ++nt)
-            mma_16816<false>(j2 ? sacc2[nt] : sacc[nt], lo_r, lo_r8, hi_r, hi_r8, qf[nt][jj + j2][0],
-                             qf[nt][jj + j2][1]);
+            mma_16816<false>(j2 ? ao[nt] : ae[nt], lo_r, lo_r8, hi_r, hi_r8, qf[nt][jj + j2][0], qf[nt][jj + j2][1]);
         }
       }
     }
-#pragma unroll
-    for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
+  };
 
-    // ---- scale, mask, online softmax (base 2) ----
-    float f_r = p.qk_scale_log2, f_r8 = p.qk_scale_log2;
-    float vs_r = 1.0f, vs_r8 = 1.0f;
-    if constexpr (kQt) {
-      const float* sc = reinterpret_cast<const float*>(base_ptr + (st - smem_base) + 2 * Tr::kKVBytes);
-      f_r *= sc[r];
-      f_r8 *= sc[r + 8];
-      vs_r = r < valid ? sc[16 + r] : 0.0f;
-      vs_r8 = r + 8 < valid ? sc[16 + r + 8] : 0.0f;
-    }
-    const bool ok_r = r < valid && r >= lowv;
-    const bool ok_r8 = r + 8 < valid && r + 8 >= lowv;
-    uint32_t pb[kNT][2];
-    bool grow = false;
-    float alpha[kNT][2];
-#pragma unroll
-    for (int nt = 0; nt < kNT; ++nt) {
-      bool ok0 = ok_r, ok1 = ok_r, ok2 = ok_r8, ok3 = ok_r8;
-      if constexpr (kMQ) {
-        const int va = colv[nt][0] - kpos0, vb = colv[nt][1] - kpos0;
-        const int la = p.window > 0 ? va - p.window : -32, lb = p.window > 0 ? vb - p.window : -32;
-        ok0 = r < va && r >= la;
-        ok1 = r < vb && r >= lb;
-        ok2 = r + 8 < va && r + 8 >= la;
-        ok3 = r + 8 < vb && r + 8 >= lb;
-      }
-      const float s0 = ok0 ? sacc[nt][0] * f_r : -INFINITY;
-      const float s1 = ok1 ? sacc[nt][1] * f_r : -INFINITY;
-      const float s2 = ok2 ? sacc[nt][2] * f_r8 : -INFINITY;
-      const float s3 = ok3 ? sacc[nt][3] * f_r8 : -INFINITY;
-      float mx_a = fmaxf(s0, s2), mx_b = fmaxf(s1, s3);
-#pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
-        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
-      }
-      const float mn_a = fmaxf(m_run[nt][0], mx_a);
-      const float mn_b = fmaxf(m_run[nt][1], mx_b);
-      grow |= (mn_a > m_run[nt][0]) || (mn_b > m_run[nt][1]);
-      alpha[nt][0] = mn_a == m_run[nt][0] ? 1.0f : fast_exp2(m_run[nt][0] - mn_a);
-      alpha[nt][1] = mn_b == m_run[nt][1] ? 1.0f : fast_exp2(m_run[nt][1] - mn_b);
-      m_run[nt][0] = mn_a;
-      m_run[nt][1] = mn_b;
-      // a column with no visible key yet keeps m = -inf: exponentiate
-      // against 0 instead, which gives p = 0 for its masked entries
-      const float b_a = (kMQ && mn_a == -INFINITY) ? 0.0f : mn_a;
-      const float b_b = (kMQ && mn_b == -INFINITY) ? 0.0f : mn_b;
-      const float p0 = fast_exp2(s0 - b_a), p1 = fast_exp2(s1 - b_b);
-      const float p2 = fast_exp2(s2 - b_a), p3 = fast_exp2(s3 - b_b);
-      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (p0 + p2);
-      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (p1 + p3);
-      // P^T operand: rows = tokens of the block, columns = query heads
-      pb[nt][0] = movmatrix_t(pack2<kMmaBF16>(p0 * vs_r, p1 * vs_r));
-      pb[nt][1] = movmatrix_t(pack2<kMmaBF16>(p2 * vs_r8, p3 * vs_r8));
-    }
-    if (__any_sync(0xffffffffu, grow)) {
-#pragma unroll
-      for (int i = 0; i < kMT; ++i)
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt) {
-          o[i][nt][0] *= alpha[nt][0];
-          o[i][nt][1] *= alpha[nt][1];
-          o[i][nt][2] *= alpha[nt][0];
-          o[i][nt][3] *= alpha[nt][1];
-        }
-    }
-
-    // ---- O^T += V^T . P^T ----
+  // O^T += V^T . P^T for the block in stage `st`.
+  auto values = [&](uint32_t st, const uint32_t (&pb)[kNT][2]) {
     const uint32_t vt = st + Tr::kKVBytes;
     if constexpr (!kQt) {
       const int t = (lane & 7) + (lane >> 4) * 8;
@@ -801,8 +699,9 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
         for (int c2 = 0; c2 < 2; ++c2) {
           uint32_t x[4], y[4];  // x: tokens 0-7 of the block, y: tokens 8-15
           if constexpr (kCT == kI4) {
-            i4x8_to_h2x4(w[2 * c2], x);
-            i4x8_to_h2x4(w[2 * c2 + 1], y);
+            // rows r (even d) read 1032 + c, rows r + 8 (odd d) 1152 + 16c
+            i4x8_to_h2x4_biased(w[2 * c2], x);
+            i4x8_to_h2x4_biased(w[2 * c2 + 1], y);
           } else {
             uint32_t a[4], b[4];
             e2m1x8_to_h2x4(w[2 * c2], a);
@@ -826,14 +725,6 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
       }
     } else {
       const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
-      // uint8: fp16 pairs (1024 + z) of this lane's tokens (2q, 2q + 1) and
-      // (2q + 8, 2q + 9)
-      uint32_t zv_x = 0, zv_y = 0;
-      if constexpr (kCT == kU8) {
-        const uint8_t* zv = base_ptr + (st - smem_base) + 2 * Tr::kKVBytes + 144;
-        zv_x = (0x6400u + zv[2 * q4]) | ((0x6400u + zv[2 * q4 + 1]) << 16);
-        zv_y = (0x6400u + zv[2 * q4 + 8]) | ((0x6400u + zv[2 * q4 + 9]) << 16);
-      }
 #pragma unroll
       for (int i = 0; i < kMT; i += 2) {
         uint32_t w[4];
@@ -843,16 +734,18 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
           // w = [A0 A1 B0 B1]: tokens 2q (A) and 2q+1 (B) at d 16(i+ii)+2r (0) and +1 (1)
           uint32_t x0, x1, y0, y1;  // x: tokens 0-7 of the block, y: tokens 8-15
           if constexpr (kCT == kI8) {
+            // fp16 1152 + c (the bias leaves through wacc)
             const uint32_t u0 = w[2 * ii] ^ 0x80808080u, u1 = w[2 * ii + 1] ^ 0x80808080u;
-            x0 = i8pair_to_h2(u0, 0x4240u);
-            x1 = i8pair_to_h2(u0, 0x4341u);
-            y0 = i8pair_to_h2(u1, 0x4240u);
-            y1 = i8pair_to_h2(u1, 0x4341u);
+            x0 = prmt(u0, 0x64646464u, 0x4240u);
+            x1 = prmt(u0, 0x64646464u, 0x4341u);
+            y0 = prmt(u1, 0x64646464u, 0x4240u);
+            y1 = prmt(u1, 0x64646464u, 0x4341u);
           } else if constexpr (kCT == kU8) {
-            x0 = u8pair_minus_zero(w[2 * ii], 0x4240u, zv_x);
-            x1 = u8pair_minus_zero(w[2 * ii], 0x4341u, zv_x);
-            y0 = u8pair_minus_zero(w[2 * ii + 1], 0x4240u, zv_y);
-            y1 = u8pair_minus_zero(w[2 * ii + 1], 0x4341u, zv_y);
+            // fp16 1024 + c (the bias 1024 + z leaves through wacc)
+            x0 = prmt(w[2 * ii], 0x64646464u, 0x4240u);
+            x1 = prmt(w[2 * ii], 0x64646464u, 0x4341u);
+            y0 = prmt(w[2 * ii + 1], 0x64646464u, 0x4240u);
+            y1 = prmt(w[2 * ii + 1], 0x64646464u, 0x4341u);
           } else {
             e4m3x4_to_h2x2(prmt(w[2 * ii], w[2 * ii], 0x3120u), x0, x1);
             e4m3x4_to_h2x2(prmt(w[2 * ii + 1], w[2 * ii + 1], 0x3120u), y0, y1);
@@ -862,210 +755,806 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
         }
       }
     }
+    if constexpr (kBiasV) {
+      // every row of the A operand holds the bias of each token: INT8 1152,
+      // uint8 1024 + z, INT4 1 (its two row biases are applied at the fold)
+      uint32_t ax = 0x3C003C00u, ay = 0x3C003C00u;
+      if constexpr (kCT == kI8) {
+        ax = ay = 0x64806480u;
+      } else if constexpr (kCT == kU8) {
+        const uint8_t* zv = base_ptr + (st - smem_base) + 2 * Tr::kKVBytes + 144;
+        ax = (0x6400u + zv[2 * q4]) | ((0x6400u + zv[2 * q4 + 1]) << 16);
+        ay = (0x6400u + zv[2 * q4 + 8]) | ((0x6400u + zv[2 * q4 + 9]) << 16);
+      }
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) mma_16816<false>(wacc[nt], ax, ax, ay, ay, pb[nt][0], pb[nt][1]);
+    }
+  };
 
-    // ---- refill this stage with item k + kR ----
+  // Takes the accumulated bias weight out of O^T (integer V codes).
+  auto fold_v = [&]() {
+    if constexpr (kBiasV) {
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+#pragma unroll
+        for (int i = 0; i < kMT; ++i)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            if constexpr (kCT == kI4) {
+              o[i][nt][e] -= (e < 2 ? 1032.0f : 1152.0f) * wacc[nt][e];
+            } else {
+              o[i][nt][e] -= wacc[nt][e];
+            }
+          }
+        wacc[nt][0] = wacc[nt][1] = wacc[nt][2] = wacc[nt][3] = 0.0f;
+      }
+      since_fold = 0;
+    }
+  };
+
+  // Items k .. k + NB - 1: NB consecutive blocks of the current pair (NB = 2
+  // only when both belong to it), whose scores share one softmax update.
+  // False when a copy wait timed out (the warp then leaves).
+  auto blocks = [&](int k, auto nb_tag) -> bool {
+    constexpr int NB = decltype(nb_tag)::value;
+    uint32_t stb[NB];
+    bool landed = true;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      stb[b] = ring + cstage * Tr::kStageBytes;
+      landed = mbar_wait(bars + cstage * 8, cphase) && landed;
+      if (++cstage == kR) {
+        cstage = 0;
+        cphase ^= 1u;
+      }
+    }
+    if (__any_sync(0xffffffffu, !landed)) {  // warp-uniform: never split the warp before ldmatrix/mma
+      // let copies already in flight land (bounded) before the warp leaves
+      for (int kk = k + NB; kk < count && kk < k + kR; ++kk) mbar_wait(bars + (kk % kR) * 8, (kk / kR) & 1);
+      return false;
+    }
+    const int kpos0 = (jb + j) * 16;  // position of the first block's first token
+    const int valid = ctx - kpos0;    // >= 1 tokens of these blocks count
+    // sliding window: tokens before position ctx - window are not seen
+    const int lowv = p.window > 0 ? ctx - p.window - kpos0 : -32;
+    // Rows of a sequence's last block at or beyond its context were never
+    // written and may hold anything, NaN included; P is 0 there, but 0 * NaN
+    // is not, so those V rows are zeroed in the stage first (and their
+    // scales replaced by 0 below).  Only the last block of a pair can have
+    // such rows.
+    bool any_tail = false;
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int vb = valid - 16 * b;
+      if (vb < 16) {
+        any_tail = true;
+        uint8_t* vrow = base_ptr + (stb[b] - smem_base) + Tr::kKVBytes;
+        constexpr int kChunks = Tr::kNumColTiles * Tr::kChunksPerTileRow;  // 16-byte chunks per row
+        for (int e = lane; e < (16 - vb) * kChunks; e += 32) {
+          const int t = vb + e / kChunks, c = e % kChunks;
+          *reinterpret_cast<uint4*>(vrow + (c / Tr::kChunksPerTileRow) * Tr::kColTileBytes + t * Tr::kTileBytes +
+                                    (c % Tr::kChunksPerTileRow) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    }
+    if (any_tail) __syncwarp();
+
+    // ---- S^T = K . Q^T: two independent accumulation chains (one per block
+    // when NB = 2, even and odd k-steps of the one block otherwise) ----
+    float sacc[NB][kNT][4];
+    float sacc2[kNT][4];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      if constexpr (kBiasK) {
+        // uint8: the bias of token row r (r + 8) is 1024 + its zero point
+        float zb_r = 1.0f, zb_r8 = 1.0f;
+        if constexpr (kCT == kU8) {
+          const uint8_t* zk = base_ptr + (stb[b] - smem_base) + 2 * Tr::kKVBytes + 128;
+          zb_r = 1024.0f + static_cast<float>(zk[r]);
+          zb_r8 = 1024.0f + static_cast<float>(zk[r + 8]);
+        }
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[b][nt][e] = -kqs[nt][e & 1] * (e < 2 ? zb_r : zb_r8);
+      } else {
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) sacc[b][nt][e] = 0.0f;
+      }
+    }
+    if constexpr (NB == 1) {
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc2[nt][e] = 0.0f;
+      scores(stb[0], sacc[0], sacc2);
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[0][nt][e] += sacc2[nt][e];
+    } else {
+#pragma unroll
+      for (int b = 0; b < NB; ++b) scores(stb[b], sacc[b], sacc[b]);
+    }
+
+    // ---- scale, mask, online softmax (base 2) over the NB blocks ----
+    float f_r[NB], f_r8[NB], vs_r[NB], vs_r8[NB];
+    bool ok_r[NB], ok_r8[NB];
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int vb = valid - 16 * b, lb = lowv - 16 * b;
+      f_r[b] = p.qk_scale_log2;
+      f_r8[b] = p.qk_scale_log2;
+      vs_r[b] = 1.0f;
+      vs_r8[b] = 1.0f;
+      if constexpr (kQt) {
+        const float* sc = reinterpret_cast<const float*>(base_ptr + (stb[b] - smem_base) + 2 * Tr::kKVBytes);
+        f_r[b] *= sc[r];
+        f_r8[b] *= sc[r + 8];
+        vs_r[b] = r < vb ? sc[16 + r] : 0.0f;
+        vs_r8[b] = r + 8 < vb ? sc[16 + r + 8] : 0.0f;
+      }
+      ok_r[b] = r < vb && r >= lb;
+      ok_r8[b] = r + 8 < vb && r + 8 >= lb;
+    }
+    uint32_t pb[NB][kNT][2];
+    bool grow = false;
+    float alpha[kNT][2];
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      float sv[NB][4];
+      float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        bool ok0 = ok_r[b], ok1 = ok_r[b], ok2 = ok_r8[b], ok3 = ok_r8[b];
+        if constexpr (kMQ) {
+          const int va = colv[nt][0] - kpos0 - 16 * b, vb = colv[nt][1] - kpos0 - 16 * b;
+          const int la = p.window > 0 ? va - p.window : -32, lb = p.window > 0 ? vb - p.window : -32;
+          ok0 = r < va && r >= la;
+          ok1 = r < vb && r >= lb;
+          ok2 = r + 8 < va && r + 8 >= la;
+          ok3 = r + 8 < vb && r + 8 >= lb;
+        }
+        sv[b][0] = ok0 ? sacc[b][nt][0] * f_r[b] : -INFINITY;
+        sv[b][1] = ok1 ? sacc[b][nt][1] * f_r[b] : -INFINITY;
+        sv[b][2] = ok2 ? sacc[b][nt][2] * f_r8[b] : -INFINITY;
+        sv[b][3] = ok3 ? sacc[b][nt][3] * f_r8[b] : -INFINITY;
+        mx_a = fmaxf(mx_a, fmaxf(sv[b][0], sv[b][2]));
+        mx_b = fmaxf(mx_b, fmaxf(sv[b][1], sv[b][3]));
+      }
+#pragma unroll
+      for (int off = 4; off < 32; off <<= 1) {
+        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+      }
+      const float mn_a = fmaxf(m_run[nt][0], mx_a);
+      const float mn_b = fmaxf(m_run[nt][1], mx_b);
+      grow |= (mn_a > m_run[nt][0]) || (mn_b > m_run[nt][1]);
+      alpha[nt][0] = mn_a == m_run[nt][0] ? 1.0f : fast_exp2(m_run[nt][0] - mn_a);
+      alpha[nt][1] = mn_b == m_run[nt][1] ? 1.0f : fast_exp2(m_run[nt][1] - mn_b);
+      m_run[nt][0] = mn_a;
+      m_run[nt][1] = mn_b;
+      // a column with no visible key yet keeps m = -inf: exponentiate
+      // against 0 instead, which gives p = 0 for its masked entries
+      const float b_a = (kMQ && mn_a == -INFINITY) ? 0.0f : mn_a;
+      const float b_b = (kMQ && mn_b == -INFINITY) ? 0.0f : mn_b;
+      float la = 0.0f, lbs = 0.0f;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float p0 = fast_exp2(sv[b][0] - b_a), p1 = fast_exp2(sv[b][1] - b_b);
+        const float p2 = fast_exp2(sv[b][2] - b_a), p3 = fast_exp2(sv[b][3] - b_b);
+        la += p0 + p2;
+        lbs += p1 + p3;
+        // P^T operand: rows = tokens of the block, columns = query heads
+        pb[b][nt][0] = movmatrix_t(pack2<kMmaBF16>(p0 * vs_r[b], p1 * vs_r[b]));
+        pb[b][nt][1] = movmatrix_t(pack2<kMmaBF16>(p2 * vs_r8[b], p3 * vs_r8[b]));
+      }
+      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + la;
+      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + lbs;
+    }
+    if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+      for (int i = 0; i < kMT; ++i)
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          o[i][nt][0] *= alpha[nt][0];
+          o[i][nt][1] *= alpha[nt][1];
+          o[i][nt][2] *= alpha[nt][0];
+          o[i][nt][3] *= alpha[nt][1];
+        }
+      if constexpr (kBiasV) {
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          wacc[nt][0] *= alpha[nt][0];
+          wacc[nt][1] *= alpha[nt][1];
+          wacc[nt][2] *= alpha[nt][0];
+          wacc[nt][3] *= alpha[nt][1];
+        }
+      }
+    }
+
+    // ---- O^T += V^T . P^T ----
+#pragma unroll
+    for (int b = 0; b < NB; ++b) values(stb[b], pb[b]);
+    if constexpr (kBiasV) {
+      since_fold += NB;
+      if (since_fold >= kFoldBlocks) fold_v();
+    }
+
+    // ---- refill these stages with items k + kR .. ----
     __syncwarp();
     // the zeroed rows were generic-proxy writes; order them before the TMA
     // (async-proxy) refill of the same stage
-    if (tail) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    const int kn = k + kR;
-    if (kn < count) {
-      const int chunk = kn >> 5;
-      if ((kn & 31) == 0) {
-        // entering chunk `chunk` (held in pre[chunk & 1]); chunk - 1 is spent,
-        // so its register takes chunk + 1
-        const int ki = (chunk + 1) * 32 + lane;
-        const int nxt = ki < count ? item_row<kMQ>(p, cum, item_of(ki)) : 0;
-        if (chunk & 1) pre0 = nxt; else pre1 = nxt;
+    if (any_tail) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+#pragma unroll
+    for (int b = 0; b < NB; ++b) {
+      const int kn = k + b + kR;
+      if (kn < count) {
+        const int chunk = kn >> 5;
+        if ((kn & 31) == 0) {
+          // entering chunk `chunk` (held in pre[chunk & 1]); chunk - 1 is
+          // spent, so its register takes chunk + 1
+          const int ki = (chunk + 1) * 32 + lane;
+          const int nxt = ki < count ? item_row<kMQ>(p, cum, item_of(ki)) : 0;
+          if (chunk & 1) pre0 = nxt; else pre1 = nxt;
+        }
+        const int row0 = __shfl_sync(0xffffffffu, (chunk & 1) ? pre1 : pre0, kn & 31);
+        if (lane == 0) issue(row0);
       }
-      const int row0 = __shfl_sync(0xffffffffu, (chunk & 1) ? pre1 : pre0, kn & 31);
-      if (lane == 0) issue(row0);
     }
+    return true;
+  };
 
-    // ---- advance; finish the (sequence, head) pair at its end or the stream's ----
-    ++j;
-    const bool wrap_next = offset > 0 && k + 1 == count - offset;  // next item is g0
-    if (j == nb || wrap_next || k == count - 1) {
-      float lsum[kNT][2];
-#pragma unroll
-      for (int nt = 0; nt < kNT; ++nt) {
-        float la = l_run[nt][0], lb = l_run[nt][1];
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-          la += __shfl_xor_sync(0xffffffffu, la, off);
-          lb += __shfl_xor_sync(0xffffffffu, lb, off);
-        }
-        lsum[nt][0] = la;
-        lsum[nt][1] = lb;
-      }
-      const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
-      // columns of this pair: G heads (decode) or a tile of (token, head)
-      const int C = kMQ ? p.tile_cols : G;
-      const int ncols = kMQ ? min(p.tile_cols, n_new * G - tile * p.tile_cols) : G;
-      auto out_row = [&](int c) -> long long {
-        if constexpr (kMQ) {
-          return static_cast<long long>(q0 + col_token(c)) * Hq + static_cast<long long>(h) * G + col_head(c);
-        } else {
-          return head_row0 + c;
-        }
-      };
-      const int gp0 = cum[s] + pr * nb;  // the pair's first and last items
-      const int gpe = gp0 + nb - 1;
-      if (gp0 >= g0 && gpe < g1) {
-        // the whole pair went through this warp: write the output
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int g = nt * 8 + 2 * q4 + c;
-            if (g >= ncols) continue;
-            const float inv = 1.0f / lsum[nt][c];
-            const long long row = out_row(g);
-#pragma unroll
-            for (int i = 0; i < kMT; ++i) {
-              const int d0 = k4 ? 32 * (i >> 1) + 4 * r + 2 * (i & 1) : (k8 ? 16 * i + 2 * r : 16 * i + r);
-              const int d1 = kQt ? d0 + 1 : d0 + 8;
-              store_out<kOutBF16>(p.out, row * kD + d0, o[i][nt][c] * inv);
-              store_out<kOutBF16>(p.out, row * kD + d1, o[i][nt][2 + c] * inv);
-            }
-          }
-      } else {
-        // a share of a split pair: publish (m, l, o / l), then count arrivals
-        const int ml = p.slot_floats - C * kD;
-        float* slot = p.slots + static_cast<long long>(2 * gw + (gp0 <= g0 && g0 <= gpe ? 0 : 1)) * p.slot_floats;
-#pragma unroll
-        for (int nt = 0; nt < kNT; ++nt)
-#pragma unroll
-          for (int c = 0; c < 2; ++c) {
-            const int g = nt * 8 + 2 * q4 + c;
-            if (g >= ncols) continue;
-            // multi-query: a share may hold no visible key of a column (l = 0)
-            const float inv = (kMQ && lsum[nt][c] == 0.0f) ? 0.0f : 1.0f / lsum[nt][c];
-            if (r == 0) {
-              slot[g] = m_run[nt][c];
-              slot[C + g] = lsum[nt][c];
-            }
-            float* og = slot + ml + g * kD;
-#pragma unroll
-            for (int i = 0; i < kMT; ++i) {
-              const int d0 = k4 ? 32 * (i >> 1) + 4 * r + 2 * (i & 1) : (k8 ? 16 * i + 2 * r : 16 * i + r);
-              const int d1 = kQt ? d0 + 1 : d0 + 8;
-              og[d0] = o[i][nt][c] * inv;
-              og[d1] = o[i][nt][2 + c] * inv;
-            }
-          }
-        __threadfence();
-        __syncwarp();
-        const int w_first = stream_of(T, gp0, nw);
-        const int n_c = stream_of(T, gpe, nw) - w_first + 1;
-        int last = 0;
-        if (lane == 0) {
-          unsigned long long* ctr =
-              p.counters + (static_cast<long long>(s) * Hkv + h) * (kMQ ? p.max_tiles : 1) + (kMQ ? tile : 0);
-          const unsigned long long E = p.epoch;
-          unsigned long long old = atomicAdd(ctr, 0ull), assumed, next;
-          do {
-            assumed = old;
-            next = ((assumed >> kEpochShift) == E) ? assumed + 1 : ((E << kEpochShift) | 1ull);
-            old = atomicCAS(ctr, assumed, next);
-          } while (old != assumed);
-          last = static_cast<int>(next & kCountMask) == n_c;
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          __threadfence();
-          // contributor c = w_first + c keeps its share in slot 2w (the pair
-          // holds the stream's first item) or 2w + 1 (it does not)
-          auto slot_of = [&](int c) -> const float* {
-            const int w = w_first + c;
-            const int idx = 2 * w + (stream_start(T, w, nw) >= gp0 ? 0 : 1);
-            return p.slots + static_cast<long long>(idx) * p.slot_floats;
-          };
-          // One pass over the contributors per group of kMG heads, with a
-          // running max per head: every load of a contributor is independent
-          // of the others, and two contributors are in flight at once.  Each
-          // lane owns kD / 32 output columns of every head.  (Groups of 4 for
-          // quantised caches keep this rarely run code within their 168
-          // registers.)
-          constexpr int kV = kD / 32;
-          constexpr int kMG = kQt ? 4 : 8;
+  constexpr bool kPairBlocks = kQt;
+  if constexpr (kPairBlocks) {
+    // Quantised caches take two blocks of a pair per iteration: their
+    // per-block bookkeeping (softmax reduction and update, rescale test, loop
+    // and pair tests) is shared, and the two blocks' independent work
+    // interleaves.
 #pragma unroll 1
-          for (int c0 = 0; c0 < ncols; c0 += kMG) {
-            float Mg[kMG], Lg[kMG], acc[kMG][kV];
+    for (int k = 0; k < count;) {
+      const int nbk = (k + 1 < count && j + 1 < nb && !(offset > 0 && k + 1 == count - offset)) ? 2 : 1;
+      if (!(nbk == 2 ? blocks(k, IntC<2>{}) : blocks(k, IntC<1>{}))) return;
+      k += nbk;
+      const int kl = k - 1;  // the last item processed
+
+      // ---- advance; finish the (sequence, head) pair at its end or the stream's ----
+      j += nbk;
+      const bool wrap_next = offset > 0 && kl + 1 == count - offset;  // next item is g0
+      if (j == nb || wrap_next || kl == count - 1) {
+        fold_v();
+        if constexpr (kCT == kI4) {
+          // rows r + 8 (odd d) were widened at 16x
 #pragma unroll
-            for (int gg = 0; gg < kMG; ++gg) {
-              Mg[gg] = -INFINITY;
-              Lg[gg] = 0.0f;
+          for (int i = 0; i < kMT; ++i)
 #pragma unroll
-              for (int e = 0; e < kV; ++e) acc[gg][e] = 0.0f;
+            for (int nt = 0; nt < kNT; ++nt) {
+              o[i][nt][2] *= 0.0625f;
+              o[i][nt][3] *= 0.0625f;
             }
-#pragma unroll 2
-            for (int c = 0; c < n_c; ++c) {
-              const float* sl = slot_of(c);
-              float mc[kMG], lc[kMG], ov[kMG][kV];
+        }
+        float lsum[kNT][2];
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          float la = l_run[nt][0], lb = l_run[nt][1];
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            la += __shfl_xor_sync(0xffffffffu, la, off);
+            lb += __shfl_xor_sync(0xffffffffu, lb, off);
+          }
+          lsum[nt][0] = la;
+          lsum[nt][1] = lb;
+        }
+        const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
+        // columns of this pair: G heads (decode) or a tile of (token, head)
+        const int C = kMQ ? p.tile_cols : G;
+        const int ncols = kMQ ? min(p.tile_cols, n_new * G - tile * p.tile_cols) : G;
+        auto out_row = [&](int c) -> long long {
+          if constexpr (kMQ) {
+            return static_cast<long long>(q0 + col_token(c)) * Hq + static_cast<long long>(h) * G + col_head(c);
+          } else {
+            return head_row0 + c;
+          }
+        };
+        const int gp0 = cum[s] + pr * nb;  // the pair's first and last items
+        const int gpe = gp0 + nb - 1;
+        if (gp0 >= g0 && gpe < g1) {
+          // the whole pair went through this warp: write the output
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int g = nt * 8 + 2 * q4 + c;
+              if (g >= ncols) continue;
+              const float inv = 1.0f / lsum[nt][c];
+              const long long row = out_row(g);
+#pragma unroll
+              for (int i = 0; i < kMT; ++i) {
+                const int d0 = k4 ? 32 * (i >> 1) + 4 * r + 2 * (i & 1) : (k8 ? 16 * i + 2 * r : 16 * i + r);
+                const int d1 = kQt ? d0 + 1 : d0 + 8;
+                store_out<kOutBF16>(p.out, row * kD + d0, o[i][nt][c] * inv);
+                store_out<kOutBF16>(p.out, row * kD + d1, o[i][nt][2 + c] * inv);
+              }
+            }
+        } else {
+          // a share of a split pair: publish (m, l, o / l), then count arrivals
+          const int ml = p.slot_floats - C * kD;
+          float* slot = p.slots + static_cast<long long>(2 * gw + (gp0 <= g0 && g0 <= gpe ? 0 : 1)) * p.slot_floats;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int g = nt * 8 + 2 * q4 + c;
+              if (g >= ncols) continue;
+              // multi-query: a share may hold no visible key of a column (l = 0)
+              const float inv = (kMQ && lsum[nt][c] == 0.0f) ? 0.0f : 1.0f / lsum[nt][c];
+              if (r == 0) {
+                slot[g] = m_run[nt][c];
+                slot[C + g] = lsum[nt][c];
+              }
+              float* og = slot + ml + g * kD;
+#pragma unroll
+              for (int i = 0; i < kMT; ++i) {
+                const int d0 = k4 ? 32 * (i >> 1) + 4 * r + 2 * (i & 1) : (k8 ? 16 * i + 2 * r : 16 * i + r);
+                const int d1 = kQt ? d0 + 1 : d0 + 8;
+                og[d0] = o[i][nt][c] * inv;
+                og[d1] = o[i][nt][2 + c] * inv;
+              }
+            }
+          __threadfence();
+          __syncwarp();
+          const int w_first = stream_of(T, gp0, nw);
+          const int n_c = stream_of(T, gpe, nw) - w_first + 1;
+          int last = 0;
+          if (lane == 0) {
+            unsigned long long* ctr =
+                p.counters + (static_cast<long long>(s) * Hkv + h) * (kMQ ? p.max_tiles : 1) + (kMQ ? tile : 0);
+            const unsigned long long E = p.epoch;
+            unsigned long long old = atomicAdd(ctr, 0ull), assumed, next;
+            do {
+              assumed = old;
+              next = ((assumed >> kEpochShift) == E) ? assumed + 1 : ((E << kEpochShift) | 1ull);
+              old = atomicCAS(ctr, assumed, next);
+            } while (old != assumed);
+            last = static_cast<int>(next & kCountMask) == n_c;
+          }
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            __threadfence();
+            // contributor c = w_first + c keeps its share in slot 2w (the pair
+            // holds the stream's first item) or 2w + 1 (it does not)
+            auto slot_of = [&](int c) -> const float* {
+              const int w = w_first + c;
+              const int idx = 2 * w + (stream_start(T, w, nw) >= gp0 ? 0 : 1);
+              return p.slots + static_cast<long long>(idx) * p.slot_floats;
+            };
+            // One pass over the contributors per group of kMG heads, with a
+            // running max per head: every load of a contributor is independent
+            // of the others, and two contributors are in flight at once.  Each
+            // lane owns kD / 32 output columns of every head.  (Groups of 4 for
+            // quantised caches keep this rarely run code within their 168
+            // registers.)
+            constexpr int kV = kD / 32;
+            constexpr int kMG = kQt ? 4 : 8;
+#pragma unroll 1
+            for (int c0 = 0; c0 < ncols; c0 += kMG) {
+              float Mg[kMG], Lg[kMG], acc[kMG][kV];
 #pragma unroll
               for (int gg = 0; gg < kMG; ++gg) {
-                const int g = c0 + gg;
-                if (g < ncols) {
-                  mc[gg] = __ldcg(sl + g);
-                  lc[gg] = __ldcg(sl + C + g);
-                  const float* og = sl + ml + g * kD + lane * kV;
-                  if constexpr (kV == 4) {
-                    const float4 v = __ldcg(reinterpret_cast<const float4*>(og));
-                    ov[gg][0] = v.x;
-                    ov[gg][1] = v.y;
-                    ov[gg][2] = v.z;
-                    ov[gg][3] = v.w;
-                  } else {
-                    const float2 v = __ldcg(reinterpret_cast<const float2*>(og));
-                    ov[gg][0] = v.x;
-                    ov[gg][1] = v.y;
+                Mg[gg] = -INFINITY;
+                Lg[gg] = 0.0f;
+#pragma unroll
+                for (int e = 0; e < kV; ++e) acc[gg][e] = 0.0f;
+              }
+#pragma unroll 2
+              for (int c = 0; c < n_c; ++c) {
+                const float* sl = slot_of(c);
+                float mc[kMG], lc[kMG], ov[kMG][kV];
+#pragma unroll
+                for (int gg = 0; gg < kMG; ++gg) {
+                  const int g = c0 + gg;
+                  if (g < ncols) {
+                    mc[gg] = __ldcg(sl + g);
+                    lc[gg] = __ldcg(sl + C + g);
+                    const float* og = sl + ml + g * kD + lane * kV;
+                    if constexpr (kV == 4) {
+                      const float4 v = __ldcg(reinterpret_cast<const float4*>(og));
+                      ov[gg][0] = v.x;
+                      ov[gg][1] = v.y;
+                      ov[gg][2] = v.z;
+                      ov[gg][3] = v.w;
+                    } else {
+                      const float2 v = __ldcg(reinterpret_cast<const float2*>(og));
+                      ov[gg][0] = v.x;
+                      ov[gg][1] = v.y;
+                    }
+                  }
+                }
+#pragma unroll
+                for (int gg = 0; gg < kMG; ++gg) {
+                  // multi-query: skip a share that saw no visible key of the column
+                  if (c0 + gg < ncols && (!kMQ || mc[gg] != -INFINITY)) {
+                    const float mn = fmaxf(Mg[gg], mc[gg]);
+                    const float a = fast_exp2(Mg[gg] - mn);  // 0 for the first contributor
+                    const float w = fast_exp2(mc[gg] - mn) * lc[gg];
+                    Lg[gg] = Lg[gg] * a + w;
+#pragma unroll
+                    for (int e = 0; e < kV; ++e) acc[gg][e] = acc[gg][e] * a + w * ov[gg][e];
+                    Mg[gg] = mn;
                   }
                 }
               }
 #pragma unroll
               for (int gg = 0; gg < kMG; ++gg) {
-                // multi-query: skip a share that saw no visible key of the column
-                if (c0 + gg < ncols && (!kMQ || mc[gg] != -INFINITY)) {
-                  const float mn = fmaxf(Mg[gg], mc[gg]);
-                  const float a = fast_exp2(Mg[gg] - mn);  // 0 for the first contributor
-                  const float w = fast_exp2(mc[gg] - mn) * lc[gg];
-                  Lg[gg] = Lg[gg] * a + w;
+                const int g = c0 + gg;
+                if (g < ncols) {
+                  const float inv = Lg[gg] > 0.0f ? 1.0f / Lg[gg] : 0.0f;
+                  const long long row = out_row(g);
 #pragma unroll
-                  for (int e = 0; e < kV; ++e) acc[gg][e] = acc[gg][e] * a + w * ov[gg][e];
-                  Mg[gg] = mn;
+                  for (int e = 0; e < kV; ++e)
+                    store_out<kOutBF16>(p.out, row * kD + lane * kV + e, acc[gg][e] * inv);
                 }
               }
             }
+          }
+        }
+        if (kl + 1 < count) {  // the stream continues: back to g0, or the next non-empty pair
+          if (wrap_next) {
+            locate(g0);
+          } else {
+            j = 0;
+            if (++pr == Hkv * ntile) {
+              pr = 0;
+              do {
+                ++s;
+              } while (cum[s + 1] == cum[s]);
+              enter_seq();
+            }
+            set_pair();
+          }
+          begin_pair();
+        }
+      }
+    }
+  } else {
+    // 16-bit caches: one block per iteration (this loop is kept as it is:
+    // with one warp per SM sub-partition the HBM stream is sensitive to the
+    // instruction schedule, and a shared body with the quantised path
+    // measured 7 % slower on the long-context workload)
+#pragma unroll 1
+    for (int k = 0; k < count; ++k) {
+      const int stage = cstage;
+      const uint32_t st = ring + stage * Tr::kStageBytes;
+      const bool landed = mbar_wait(bars + stage * 8, cphase);
+      if (++cstage == kR) {
+        cstage = 0;
+        cphase ^= 1u;
+      }
+      if (__any_sync(0xffffffffu, !landed)) {  // warp-uniform: never split the warp before ldmatrix/mma
+        // let copies already in flight land (bounded) before the warp leaves
+        for (int kk = k + 1; kk < count && kk < k + kR; ++kk) mbar_wait(bars + (kk % kR) * 8, (kk / kR) & 1);
+        return;
+      }
+      const int kpos0 = (jb + j) * 16;  // position of the block's first token
+      const int valid = ctx - kpos0;    // >= 1 tokens of this block count
+      // sliding window: tokens before position ctx - window are not seen
+      const int lowv = p.window > 0 ? ctx - p.window - kpos0 : -32;
+      // Rows of a sequence's last block at or beyond its context were never
+      // written and may hold anything, NaN included; P is 0 there, but 0 * NaN
+      // is not, so those V rows are zeroed in the stage first.
+      const bool tail = valid < 16;
+      if (tail) {
+        uint8_t* vrow = base_ptr + (st - smem_base) + Tr::kKVBytes;
+        constexpr int kChunks = Tr::kNumColTiles * Tr::kChunksPerTileRow;  // 16-byte chunks per row
+        for (int e = lane; e < (16 - valid) * kChunks; e += 32) {
+          const int t = valid + e / kChunks, c = e % kChunks;
+          *reinterpret_cast<uint4*>(vrow + (c / Tr::kChunksPerTileRow) * Tr::kColTileBytes + t * Tr::kTileBytes +
+                                    (c % Tr::kChunksPerTileRow) * 16) = make_uint4(0u, 0u, 0u, 0u);
+        }
+        __syncwarp();
+      }
+
+      // ---- S^T = K . Q^T (two independent accumulation chains, summed) ----
+      float sacc[kNT][4], sacc2[kNT][4];
 #pragma unroll
-            for (int gg = 0; gg < kMG; ++gg) {
-              const int g = c0 + gg;
-              if (g < ncols) {
-                const float inv = Lg[gg] > 0.0f ? 1.0f / Lg[gg] : 0.0f;
-                const long long row = out_row(g);
+      for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
-                for (int e = 0; e < kV; ++e)
-                  store_out<kOutBF16>(p.out, row * kD + lane * kV + e, acc[gg][e] * inv);
+        for (int e = 0; e < 4; ++e) sacc[nt][e] = sacc2[nt][e] = 0.0f;
+      {
+        const int t = (lane & 7) + ((lane >> 3) & 1) * 8;
+#pragma unroll
+        for (int jj = 0; jj < kKS; ++jj) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(st + swz<Tr>(t, 2 * jj + (lane >> 4)), a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+            mma_16816<kMmaBF16>((jj & 1) ? sacc2[nt] : sacc[nt], a0, a1, a2, a3, qf[nt][jj][0], qf[nt][jj][1]);
+        }
+      }
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) sacc[nt][e] += sacc2[nt][e];
+
+      // ---- scale, mask, online softmax (base 2) ----
+      const float f_r = p.qk_scale_log2, f_r8 = p.qk_scale_log2;
+      const float vs_r = 1.0f, vs_r8 = 1.0f;
+      const bool ok_r = r < valid && r >= lowv;
+      const bool ok_r8 = r + 8 < valid && r + 8 >= lowv;
+      uint32_t pb[kNT][2];
+      bool grow = false;
+      float alpha[kNT][2];
+#pragma unroll
+      for (int nt = 0; nt < kNT; ++nt) {
+        bool ok0 = ok_r, ok1 = ok_r, ok2 = ok_r8, ok3 = ok_r8;
+        if constexpr (kMQ) {
+          const int va = colv[nt][0] - kpos0, vb = colv[nt][1] - kpos0;
+          const int la = p.window > 0 ? va - p.window : -32, lb = p.window > 0 ? vb - p.window : -32;
+          ok0 = r < va && r >= la;
+          ok1 = r < vb && r >= lb;
+          ok2 = r + 8 < va && r + 8 >= la;
+          ok3 = r + 8 < vb && r + 8 >= lb;
+        }
+        const float s0 = ok0 ? sacc[nt][0] * f_r : -INFINITY;
+        const float s1 = ok1 ? sacc[nt][1] * f_r : -INFINITY;
+        const float s2 = ok2 ? sacc[nt][2] * f_r8 : -INFINITY;
+        const float s3 = ok3 ? sacc[nt][3] * f_r8 : -INFINITY;
+        float mx_a = fmaxf(s0, s2), mx_b = fmaxf(s1, s3);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+          mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+        }
+        const float mn_a = fmaxf(m_run[nt][0], mx_a);
+        const float mn_b = fmaxf(m_run[nt][1], mx_b);
+        grow |= (mn_a > m_run[nt][0]) || (mn_b > m_run[nt][1]);
+        alpha[nt][0] = mn_a == m_run[nt][0] ? 1.0f : fast_exp2(m_run[nt][0] - mn_a);
+        alpha[nt][1] = mn_b == m_run[nt][1] ? 1.0f : fast_exp2(m_run[nt][1] - mn_b);
+        m_run[nt][0] = mn_a;
+        m_run[nt][1] = mn_b;
+        // a column with no visible key yet keeps m = -inf: exponentiate
+        // against 0 instead, which gives p = 0 for its masked entries
+        const float b_a = (kMQ && mn_a == -INFINITY) ? 0.0f : mn_a;
+        const float b_b = (kMQ && mn_b == -INFINITY) ? 0.0f : mn_b;
+        const float p0 = fast_exp2(s0 - b_a), p1 = fast_exp2(s1 - b_b);
+        const float p2 = fast_exp2(s2 - b_a), p3 = fast_exp2(s3 - b_b);
+        l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + (p0 + p2);
+        l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + (p1 + p3);
+        // P^T operand: rows = tokens of the block, columns = query heads
+        pb[nt][0] = movmatrix_t(pack2<kMmaBF16>(p0 * vs_r, p1 * vs_r));
+        pb[nt][1] = movmatrix_t(pack2<kMmaBF16>(p2 * vs_r8, p3 * vs_r8));
+      }
+      if (__any_sync(0xffffffffu, grow)) {
+#pragma unroll
+        for (int i = 0; i < kMT; ++i)
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) {
+            o[i][nt][0] *= alpha[nt][0];
+            o[i][nt][1] *= alpha[nt][1];
+            o[i][nt][2] *= alpha[nt][0];
+            o[i][nt][3] *= alpha[nt][1];
+          }
+      }
+
+      // ---- O^T += V^T . P^T ----
+      const uint32_t vt = st + Tr::kKVBytes;
+      {
+        const int t = (lane & 7) + (lane >> 4) * 8;
+#pragma unroll
+        for (int i = 0; i < kMT; ++i) {
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_t(vt + swz<Tr>(t, 2 * i + ((lane >> 3) & 1)), a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt) mma_16816<kMmaBF16>(o[i][nt], a0, a1, a2, a3, pb[nt][0], pb[nt][1]);
+        }
+      }
+
+      // ---- refill this stage with item k + kR ----
+      __syncwarp();
+      // the zeroed rows were generic-proxy writes; order them before the TMA
+      // (async-proxy) refill of the same stage
+      if (tail) asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      const int kn = k + kR;
+      if (kn < count) {
+        const int chunk = kn >> 5;
+        if ((kn & 31) == 0) {
+          // entering chunk `chunk` (held in pre[chunk & 1]); chunk - 1 is spent,
+          // so its register takes chunk + 1
+          const int ki = (chunk + 1) * 32 + lane;
+          const int nxt = ki < count ? item_row<kMQ>(p, cum, item_of(ki)) : 0;
+          if (chunk & 1) pre0 = nxt; else pre1 = nxt;
+        }
+        const int row0 = __shfl_sync(0xffffffffu, (chunk & 1) ? pre1 : pre0, kn & 31);
+        if (lane == 0) issue(row0);
+      }
+
+      // ---- advance; finish the (sequence, head) pair at its end or the stream's ----
+      ++j;
+      const bool wrap_next = offset > 0 && k + 1 == count - offset;  // next item is g0
+      if (j == nb || wrap_next || k == count - 1) {
+        float lsum[kNT][2];
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+          float la = l_run[nt][0], lb = l_run[nt][1];
+#pragma unroll
+          for (int off = 4; off < 32; off <<= 1) {
+            la += __shfl_xor_sync(0xffffffffu, la, off);
+            lb += __shfl_xor_sync(0xffffffffu, lb, off);
+          }
+          lsum[nt][0] = la;
+          lsum[nt][1] = lb;
+        }
+        const long long head_row0 = static_cast<long long>(s) * Hq + static_cast<long long>(h) * G;
+        // columns of this pair: G heads (decode) or a tile of (token, head)
+        const int C = kMQ ? p.tile_cols : G;
+        const int ncols = kMQ ? min(p.tile_cols, n_new * G - tile * p.tile_cols) : G;
+        auto out_row = [&](int c) -> long long {
+          if constexpr (kMQ) {
+            return static_cast<long long>(q0 + col_token(c)) * Hq + static_cast<long long>(h) * G + col_head(c);
+          } else {
+            return head_row0 + c;
+          }
+        };
+        const int gp0 = cum[s] + pr * nb;  // the pair's first and last items
+        const int gpe = gp0 + nb - 1;
+        if (gp0 >= g0 && gpe < g1) {
+          // the whole pair went through this warp: write the output
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int g = nt * 8 + 2 * q4 + c;
+              if (g >= ncols) continue;
+              const float inv = 1.0f / lsum[nt][c];
+              const long long row = out_row(g);
+#pragma unroll
+              for (int i = 0; i < kMT; ++i) {
+                const int d0 = k4 ? 32 * (i >> 1) + 4 * r + 2 * (i & 1) : (k8 ? 16 * i + 2 * r : 16 * i + r);
+                const int d1 = kQt ? d0 + 1 : d0 + 8;
+                store_out<kOutBF16>(p.out, row * kD + d0, o[i][nt][c] * inv);
+                store_out<kOutBF16>(p.out, row * kD + d1, o[i][nt][2 + c] * inv);
+              }
+            }
+        } else {
+          // a share of a split pair: publish (m, l, o / l), then count arrivals
+          const int ml = p.slot_floats - C * kD;
+          float* slot = p.slots + static_cast<long long>(2 * gw + (gp0 <= g0 && g0 <= gpe ? 0 : 1)) * p.slot_floats;
+#pragma unroll
+          for (int nt = 0; nt < kNT; ++nt)
+#pragma unroll
+            for (int c = 0; c < 2; ++c) {
+              const int g = nt * 8 + 2 * q4 + c;
+              if (g >= ncols) continue;
+              // multi-query: a share may hold no visible key of a column (l = 0)
+              const float inv = (kMQ && lsum[nt][c] == 0.0f) ? 0.0f : 1.0f / lsum[nt][c];
+              if (r == 0) {
+                slot[g] = m_run[nt][c];
+                slot[C + g] = lsum[nt][c];
+              }
+              float* og = slot + ml + g * kD;
+#pragma unroll
+              for (int i = 0; i < kMT; ++i) {
+                const int d0 = k4 ? 32 * (i >> 1) + 4 * r + 2 * (i & 1) : (k8 ? 16 * i + 2 * r : 16 * i + r);
+                const int d1 = kQt ? d0 + 1 : d0 + 8;
+                og[d0] = o[i][nt][c] * inv;
+                og[d1] = o[i][nt][2 + c] * inv;
+              }
+            }
+          __threadfence();
+          __syncwarp();
+          const int w_first = stream_of(T, gp0, nw);
+          const int n_c = stream_of(T, gpe, nw) - w_first + 1;
+          int last = 0;
+          if (lane == 0) {
+            unsigned long long* ctr =
+                p.counters + (static_cast<long long>(s) * Hkv + h) * (kMQ ? p.max_tiles : 1) + (kMQ ? tile : 0);
+            const unsigned long long E = p.epoch;
+            unsigned long long old = atomicAdd(ctr, 0ull), assumed, next;
+            do {
+              assumed = old;
+              next = ((assumed >> kEpochShift) == E) ? assumed + 1 : ((E << kEpochShift) | 1ull);
+              old = atomicCAS(ctr, assumed, next);
+            } while (old != assumed);
+            last = static_cast<int>(next & kCountMask) == n_c;
+          }
+          last = __shfl_sync(0xffffffffu, last, 0);
+          if (last) {
+            __threadfence();
+            // contributor c = w_first + c keeps its share in slot 2w (the pair
+            // holds the stream's first item) or 2w + 1 (it does not)
+            auto slot_of = [&](int c) -> const float* {
+              const int w = w_first + c;
+              const int idx = 2 * w + (stream_start(T, w, nw) >= gp0 ? 0 : 1);
+              return p.slots + static_cast<long long>(idx) * p.slot_floats;
+            };
+            // One pass over the contributors per group of kMG heads, with a
+            // running max per head: every load of a contributor is independent
+            // of the others, and two contributors are in flight at once.  Each
+            // lane owns kD / 32 output columns of every head.  (Groups of 4 for
+            // quantised caches keep this rarely run code within their 168
+            // registers.)
+            constexpr int kV = kD / 32;
+            constexpr int kMG = kQt ? 4 : 8;
+#pragma unroll 1
+            for (int c0 = 0; c0 < ncols; c0 += kMG) {
+              float Mg[kMG], Lg[kMG], acc[kMG][kV];
+#pragma unroll
+              for (int gg = 0; gg < kMG; ++gg) {
+                Mg[gg] = -INFINITY;
+                Lg[gg] = 0.0f;
+#pragma unroll
+                for (int e = 0; e < kV; ++e) acc[gg][e] = 0.0f;
+              }
+#pragma unroll 2
+              for (int c = 0; c < n_c; ++c) {
+                const float* sl = slot_of(c);
+                float mc[kMG], lc[kMG], ov[kMG][kV];
+#pragma unroll
+                for (int gg = 0; gg < kMG; ++gg) {
+                  const int g = c0 + gg;
+                  if (g < ncols) {
+                    mc[gg] = __ldcg(sl + g);
+                    lc[gg] = __ldcg(sl + C + g);
+                    const float* og = sl + ml + g * kD + lane * kV;
+                    if constexpr (kV == 4) {
+                      const float4 v = __ldcg(reinterpret_cast<const float4*>(og));
+                      ov[gg][0] = v.x;
+                      ov[gg][1] = v.y;
+                      ov[gg][2] = v.z;
+                      ov[gg][3] = v.w;
+                    } else {
+                      const float2 v = __ldcg(reinterpret_cast<const float2*>(og));
+                      ov[gg][0] = v.x;
+                      ov[gg][1] = v.y;
+                    }
+                  }
+                }
+#pragma unroll
+                for (int gg = 0; gg < kMG; ++gg) {
+                  // multi-query: skip a share that saw no visible key of the column
+                  if (c0 + gg < ncols && (!kMQ || mc[gg] != -INFINITY)) {
+                    const float mn = fmaxf(Mg[gg], mc[gg]);
+                    const float a = fast_exp2(Mg[gg] - mn);  // 0 for the first contributor
+                    const float w = fast_exp2(mc[gg] - mn) * lc[gg];
+                    Lg[gg] = Lg[gg] * a + w;
+#pragma unroll
+                    for (int e = 0; e < kV; ++e) acc[gg][e] = acc[gg][e] * a + w * ov[gg][e];
+                    Mg[gg] = mn;
+                  }
+                }
+              }
+#pragma unroll
+              for (int gg = 0; gg < kMG; ++gg) {
+                const int g = c0 + gg;
+                if (g < ncols) {
+                  const float inv = Lg[gg] > 0.0f ? 1.0f / Lg[gg] : 0.0f;
+                  const long long row = out_row(g);
+#pragma unroll
+                  for (int e = 0; e < kV; ++e)
+                    store_out<kOutBF16>(p.out, row * kD + lane * kV + e, acc[gg][e] * inv);
+                }
               }
             }
           }
         }
-      }
-      if (k + 1 < count) {  // the stream continues: back to g0, or the next non-empty pair
-        if (wrap_next) {
-          locate(g0);
-        } else {
-          j = 0;
-          if (++pr == Hkv * ntile) {
-            pr = 0;
-            do {
-              ++s;
-            } while (cum[s + 1] == cum[s]);
-            enter_seq();
+        if (k + 1 < count) {  // the stream continues: back to g0, or the next non-empty pair
+          if (wrap_next) {
+            locate(g0);
+          } else {
+            j = 0;
+            if (++pr == Hkv * ntile) {
+              pr = 0;
+              do {
+                ++s;
+              } while (cum[s + 1] == cum[s]);
+              enter_seq();
+            }
+            set_pair();
           }
-          set_pair();
+          begin_pair();
         }
-        begin_pair();
       }
     }
   }
