@@ -899,13 +899,16 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
       ok_r[b] = r < vb && r >= lb;
       ok_r8[b] = r + 8 < vb && r + 8 >= lb;
     }
-    uint32_t pb[NB][kNT][2];
-    bool grow = false;
-    float alpha[kNT][2];
+    // Lazy exponent base: a column's base m_run moves only when one of its
+    // scores exceeds it by more than 8 (log2 units), so p = 2^(s - m_run)
+    // stays below 256 and the common block needs no cross-lane maximum and
+    // no rescale, only one warp vote.  When a column's base must move, the
+    // whole warp takes the block maximum and rescales (the first block of a
+    // pair always does: its base starts at -inf).
+    float sv[NB][kNT][4];
+    bool up = false;
 #pragma unroll
-    for (int nt = 0; nt < kNT; ++nt) {
-      float sv[NB][4];
-      float mx_a = -INFINITY, mx_b = -INFINITY;
+    for (int nt = 0; nt < kNT; ++nt)
 #pragma unroll
       for (int b = 0; b < NB; ++b) {
         bool ok0 = ok_r[b], ok1 = ok_r[b], ok2 = ok_r8[b], ok3 = ok_r8[b];
@@ -917,44 +920,37 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
           ok2 = r + 8 < va && r + 8 >= la;
           ok3 = r + 8 < vb && r + 8 >= lb;
         }
-        sv[b][0] = ok0 ? sacc[b][nt][0] * f_r[b] : -INFINITY;
-        sv[b][1] = ok1 ? sacc[b][nt][1] * f_r[b] : -INFINITY;
-        sv[b][2] = ok2 ? sacc[b][nt][2] * f_r8[b] : -INFINITY;
-        sv[b][3] = ok3 ? sacc[b][nt][3] * f_r8[b] : -INFINITY;
-        mx_a = fmaxf(mx_a, fmaxf(sv[b][0], sv[b][2]));
-        mx_b = fmaxf(mx_b, fmaxf(sv[b][1], sv[b][3]));
+        sv[b][nt][0] = ok0 ? sacc[b][nt][0] * f_r[b] : -INFINITY;
+        sv[b][nt][1] = ok1 ? sacc[b][nt][1] * f_r[b] : -INFINITY;
+        sv[b][nt][2] = ok2 ? sacc[b][nt][2] * f_r8[b] : -INFINITY;
+        sv[b][nt][3] = ok3 ? sacc[b][nt][3] * f_r8[b] : -INFINITY;
+        up |= fmaxf(sv[b][nt][0], sv[b][nt][2]) > m_run[nt][0] + 8.0f;
+        up |= fmaxf(sv[b][nt][1], sv[b][nt][3]) > m_run[nt][1] + 8.0f;
       }
+    if (__any_sync(0xffffffffu, up)) {
+      float alpha[kNT][2];
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
-        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
-      }
-      const float mn_a = fmaxf(m_run[nt][0], mx_a);
-      const float mn_b = fmaxf(m_run[nt][1], mx_b);
-      grow |= (mn_a > m_run[nt][0]) || (mn_b > m_run[nt][1]);
-      alpha[nt][0] = mn_a == m_run[nt][0] ? 1.0f : fast_exp2(m_run[nt][0] - mn_a);
-      alpha[nt][1] = mn_b == m_run[nt][1] ? 1.0f : fast_exp2(m_run[nt][1] - mn_b);
-      m_run[nt][0] = mn_a;
-      m_run[nt][1] = mn_b;
-      // a column with no visible key yet keeps m = -inf: exponentiate
-      // against 0 instead, which gives p = 0 for its masked entries
-      const float b_a = (kMQ && mn_a == -INFINITY) ? 0.0f : mn_a;
-      const float b_b = (kMQ && mn_b == -INFINITY) ? 0.0f : mn_b;
-      float la = 0.0f, lbs = 0.0f;
+      for (int nt = 0; nt < kNT; ++nt) {
+        float mx_a = -INFINITY, mx_b = -INFINITY;
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const float p0 = fast_exp2(sv[b][0] - b_a), p1 = fast_exp2(sv[b][1] - b_b);
-        const float p2 = fast_exp2(sv[b][2] - b_a), p3 = fast_exp2(sv[b][3] - b_b);
-        la += p0 + p2;
-        lbs += p1 + p3;
-        // P^T operand: rows = tokens of the block, columns = query heads
-        pb[b][nt][0] = movmatrix_t(pack2<kMmaBF16>(p0 * vs_r[b], p1 * vs_r[b]));
-        pb[b][nt][1] = movmatrix_t(pack2<kMmaBF16>(p2 * vs_r8[b], p3 * vs_r8[b]));
+        for (int b = 0; b < NB; ++b) {
+          mx_a = fmaxf(mx_a, fmaxf(sv[b][nt][0], sv[b][nt][2]));
+          mx_b = fmaxf(mx_b, fmaxf(sv[b][nt][1], sv[b][nt][3]));
+        }
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+          mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, off));
+          mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, off));
+        }
+        const float mn_a = fmaxf(m_run[nt][0], mx_a);
+        const float mn_b = fmaxf(m_run[nt][1], mx_b);
+        alpha[nt][0] = mn_a == m_run[nt][0] ? 1.0f : fast_exp2(m_run[nt][0] - mn_a);
+        alpha[nt][1] = mn_b == m_run[nt][1] ? 1.0f : fast_exp2(m_run[nt][1] - mn_b);
+        m_run[nt][0] = mn_a;
+        m_run[nt][1] = mn_b;
+        l_run[nt][0] *= alpha[nt][0];
+        l_run[nt][1] *= alpha[nt][1];
       }
-      l_run[nt][0] = l_run[nt][0] * alpha[nt][0] + la;
-      l_run[nt][1] = l_run[nt][1] * alpha[nt][1] + lbs;
-    }
-    if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll
       for (int i = 0; i < kMT; ++i)
 #pragma unroll
@@ -973,6 +969,27 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
           wacc[nt][3] *= alpha[nt][1];
         }
       }
+    }
+    uint32_t pb[NB][kNT][2];
+#pragma unroll
+    for (int nt = 0; nt < kNT; ++nt) {
+      // a column with no visible key yet keeps m = -inf: exponentiate
+      // against 0 instead, which gives p = 0 for its masked entries
+      const float b_a = m_run[nt][0] == -INFINITY ? 0.0f : m_run[nt][0];
+      const float b_b = m_run[nt][1] == -INFINITY ? 0.0f : m_run[nt][1];
+      float la = 0.0f, lbs = 0.0f;
+#pragma unroll
+      for (int b = 0; b < NB; ++b) {
+        const float p0 = fast_exp2(sv[b][nt][0] - b_a), p1 = fast_exp2(sv[b][nt][1] - b_b);
+        const float p2 = fast_exp2(sv[b][nt][2] - b_a), p3 = fast_exp2(sv[b][nt][3] - b_b);
+        la += p0 + p2;
+        lbs += p1 + p3;
+        // P^T operand: rows = tokens of the block, columns = query heads
+        pb[b][nt][0] = movmatrix_t(pack2<kMmaBF16>(p0 * vs_r[b], p1 * vs_r[b]));
+        pb[b][nt][1] = movmatrix_t(pack2<kMmaBF16>(p2 * vs_r8[b], p3 * vs_r8[b]));
+      }
+      l_run[nt][0] += la;
+      l_run[nt][1] += lbs;
     }
 
     // ---- O^T += V^T . P^T ----
