@@ -927,6 +927,11 @@ __global__ void __launch_bounds__(DecodeTraits<kD, kCT>::max_warps(kNT) * 32)
         up |= fmaxf(sv[b][nt][0], sv[b][nt][2]) > m_run[nt][0] + 8.0f;
         up |= fmaxf(sv[b][nt][1], sv[b][nt][3]) > m_run[nt][1] + 8.0f;
       }
+    // P enters the MMA as p x (value scale) in fp16: with p up to 2^8 a
+    // value scale above 128 could overflow it, so such blocks move the base
+    // to their maximum (p <= 1 there, as with an exact running maximum)
+#pragma unroll
+    for (int b = 0; b < NB; ++b) up |= fmaxf(vs_r[b], vs_r8[b]) > 128.0f;
     if (__any_sync(0xffffffffu, up)) {
       float alpha[kNT][2];
 #pragma unroll

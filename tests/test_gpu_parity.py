@@ -311,6 +311,24 @@ def test_decode_sweep_quantised(kind, qdtype, d, group, ptok):
     check_attn(got, oracle_full(case))
 
 
+@pytest.mark.parametrize("kind", ["int8", "fp8", "u8asym", "int4", "fp4"])
+def test_decode_quantised_large_value_scales(kind):
+    """Value scales in the hundreds to thousands (values up to ~4e4): the
+    probabilities enter the MMA multiplied by the value scale in fp16, so
+    the kernel must keep them small enough not to overflow; compared with the
+    oracle relative to the output's magnitude."""
+    hkv, group = 2, 4
+    case = I.decode_case("quant_mha", seed=77, ctx_override=CTX_MIX, hq=hkv * group, hkv=hkv, d=128,
+                         dtype="bf16", cache_kind=kind)
+    case["v_scale"] = case["v_scale"] * 1.0e4
+    g = gpu_case(case)
+    got = np64(run_decode(g))
+    ref = oracle_full(case)
+    scale = float(np.abs(ref).max())
+    assert scale > 1e3
+    check_attn(got / scale, ref / scale)
+
+
 @pytest.mark.parametrize("window", [1, 16, 40, 300])
 @pytest.mark.parametrize("group,d", [(4, 128), (16, 128), (8, 64)])
 @pytest.mark.parametrize("ptok", [0, 16])
