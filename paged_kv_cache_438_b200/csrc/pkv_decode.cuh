@@ -8,8 +8,8 @@
 //
 // Design for sm_100a (HBM-bound: every K/V byte is read once):
 //   * Work list.  All (sequence, KV head, block) triples form one ordered
-//     list (sequence-major).  Each warp of a persistent grid (one CTA of four
-//     warps per SM for 16-bit caches, two for 8-bit) owns an equal contiguous
+//     list (sequence-major).  Each warp of a persistent grid (one CTA per SM:
+//     4 or 8 warps for 16-bit caches, 12 for quantised ones) owns an equal contiguous
 //     share of it and streams
 //     through that share, crossing (sequence, head) boundaries without
 //     stopping its copy pipeline.  The G query heads of a KV head are served
