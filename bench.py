@@ -1033,7 +1033,12 @@ def main():
         for name, cache in EXTRA_WORKLOADS:
             if (name, cache) == (args.workload, args.cache):
                 continue
-            others.append(extra_record(name, cache, device, peak, tflops_peak))
+            try:
+                others.append(extra_record(name, cache, device, peak, tflops_peak))
+            except Exception as e:  # the headline line must still print; the failure is recorded
+                others.append({"workload": name, "cache": cache, "error": f"{type(e).__name__}: {e}"[:300]})
+                torch.cuda.synchronize(device)
+                torch.cuda.empty_cache()
         line["other_workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)
