@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
 #pragma unroll 1
     for (int j = 0; j < nk; ++j) {
       wait_or_abort(b_sfull + 8 * x, j & 1);
-      if (aborted()) break;
+      if (__any_sync(0xFFFFFFFFu, aborted())) break;  // the warp leaves together
       tc_fence_after();
       float sv[kN];
 #pragma unroll
@@ -567,47 +567,70 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
           sv[k] = (key < lim && key >= lo) ? sv[k] : -INFINITY;
         }
       }
-      // independent partial maxima / sums keep the dependency chains short
-      float mp[8];
+      // P over the upper half of S (already read into registers) with the
+      // exponent base -nb; returns the row sum of the packed values
+      auto emit_p = [&](float nb) {
+        float sp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int k = 0; k < 8; ++k) mp[k] = fmaxf(sv[k], sv[k + 8]);
+        for (int q = 0; q < kN / 32; ++q) {
+          uint32_t w[16];
 #pragma unroll
-      for (int k = 16; k < kN; ++k) mp[k & 7] = fmaxf(mp[k & 7], sv[k]);
-      const float mr = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
-                             fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
-      const float mx = mr * c;  // scores are used as s * c (log2 units)
+          for (int k = 0; k < 16; ++k) {
+            const int e = 32 * q + 2 * k;
+            w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[e], c, nb)), fast_exp2(fmaf(sv[e + 1], c, nb)));
+            sp[k & 3] += sum_p2<kBF16>(w[k]);
+          }
+          tmem_st16(tP + 16 * q, w);
+        }
+        return (sp[0] + sp[1]) + (sp[2] + sp[3]);
+      };
+      // Common case (bf16): the base of the earlier tiles still serves.  The
+      // row sum bounds every probability, so a sum of at most 2^20
+      // (p <= 2^20, far from overflowing O or l) keeps the tile without ever
+      // taking its maximum; a larger or non-finite sum (a score far above the base, or
+      // no base yet) takes the maximum, moves the base and writes P again.
+      // tcgen05.ld / st / wait are warp-wide instructions, so the choice is
+      // made per warp: it takes the slow way when any of its rows needs it.
+      // fp16 probabilities (largest value 65504) always take the maximum
+      // first.
       float factor = 1.0f;
       bool rescale = false;
-      if (mx > m_used + 8.0f) {
-        factor = m_used == -INFINITY ? 0.0f : fast_exp2(m_used - mx);
-        rescale = m_used != -INFINITY;
-        m_used = mx;
+      float sum = 0.0f;
+      bool need_max = !kBF16 || __any_sync(0xFFFFFFFFu, m_used == -INFINITY);
+      if (!need_max) {
+        sum = emit_p(-m_used);
+        need_max = __any_sync(0xFFFFFFFFu, !(sum <= 1048576.0f));
+        if (need_max) tmem_wait_st();  // the first try has landed before it is overwritten
       }
-      const float nbase = m_used == -INFINITY ? 0.0f : -m_used;
-      float sp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      // P over the upper half of S (already read into registers)
+      if (need_max) {
+        // independent partial maxima keep the dependency chains short
+        float mp[8];
 #pragma unroll
-      for (int q = 0; q < kN / 32; ++q) {
-        uint32_t w[16];
+        for (int k = 0; k < 8; ++k) mp[k] = fmaxf(sv[k], sv[k + 8]);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int e = 32 * q + 2 * k;
-          w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[e], c, nbase)), fast_exp2(fmaf(sv[e + 1], c, nbase)));
-          sp[k & 3] += sum_p2<kBF16>(w[k]);
+        for (int k = 16; k < kN; ++k) mp[k & 7] = fmaxf(mp[k & 7], sv[k]);
+        const float mr = fmaxf(fmaxf(fmaxf(mp[0], mp[1]), fmaxf(mp[2], mp[3])),
+                               fmaxf(fmaxf(mp[4], mp[5]), fmaxf(mp[6], mp[7])));
+        const float mx = mr * c;  // scores are used as s * c (log2 units)
+        if (mx > m_used + 8.0f) {
+          factor = m_used == -INFINITY ? 0.0f : fast_exp2(m_used - mx);
+          rescale = m_used != -INFINITY;
+          m_used = mx;
         }
-        tmem_st16(tP + 16 * q, w);
+        sum = emit_p(m_used == -INFINITY ? 0.0f : -m_used);
       }
-      const float sum = (sp[0] + sp[1]) + (sp[2] + sp[3]);
       l = l * factor + sum;
-      // O_x holds every P . V before this tile (S_x(j) was committed after them)
-      if (rescale) {
+      // O_x holds every P . V before this tile (S_x(j) was committed after
+      // them); the warp rescales together, rows keeping their base by 1
+      if (__any_sync(0xFFFFFFFFu, rescale)) {
+        const float oscale = rescale ? factor : 1.0f;
 #pragma unroll 1
         for (int cb = 0; cb < kD / 32; ++cb) {
           float o[32];
           tmem_ld32(tO + 32 * cb, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] *= factor;
+          for (int k = 0; k < 32; ++k) o[k] *= oscale;
           tmem_st32(tO + 32 * cb, o);
         }
       }
@@ -616,9 +639,9 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       mbar_arrive(b_pfull + 8 * x);
     }
     // ---- epilogue: O / l -> out ----
-    wait_or_abort(b_ofull, 0);
+    if (!__any_sync(0xFFFFFFFFu, aborted())) wait_or_abort(b_ofull, 0);
     tc_fence_after();
-    if (!aborted()) {
+    if (!__any_sync(0xFFFFFFFFu, aborted())) {
       const float inv = l > 0.0f ? 1.0f / l : 0.0f;
       uint16_t* dst = reinterpret_cast<uint16_t*>(p.out) +
                       (static_cast<long long>(q0 + (row_ok ? t0x + rt : ta0)) * p.num_q_heads +

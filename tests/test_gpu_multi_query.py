@@ -240,3 +240,34 @@ def test_query_major_launch_order_covers_every_sequence(ctx, nq):
     got = np64(run_mq(g))
     assert np.all(np.isfinite(got))
     check_attn(got, oracle_mq(case))
+
+
+@pytest.mark.parametrize("dtype,group", [("bf16", 4), ("f16", 4), ("bf16", 16)])
+def test_query_major_kernel_scores_rising_along_the_keys(dtype, group):
+    """Scores that climb by about 65 log2 units over each context (about 12
+    per 128-key tile; q and the K rows share one direction, the K rows scaled
+    by their position): every row keeps moving its exponent base.  A tile
+    whose probabilities against the base in use would pass 2^20 (or overflow
+    fp16) must take its maximum and be written again, the others keep the
+    lagging base; both must match the oracle."""
+    hkv, d = 2, 128
+    ctx, nq = [700, 1100, 300], [300, 200, 140]
+    case = I.multi_query_case("chunked_prefill", seed=77 + group, ctx_override=ctx, q_lens=nq, hq=hkv * group,
+                              hkv=hkv, d=d, dtype=dtype)
+    gen = torch.Generator().manual_seed(5 + group)
+    u = torch.where(torch.rand(d, generator=gen) < 0.5, -1.0, 1.0)
+    case["q"] = (2.0 * u + 0.3 * torch.randn(case["q"].shape, generator=gen)).to(case["q"].dtype)
+    k = case["k_cache"].float()
+    bt = case["block_tables"]
+    for s, c in enumerate(ctx):
+        for lb in range((c + 15) // 16):
+            b = int(bt[s, lb])
+            pos = torch.arange(lb * 16, lb * 16 + 16, dtype=torch.float32)
+            k[b] = (2.0 * pos / c)[None, :, None] * u + 0.3 * torch.randn(k[b].shape, generator=gen)
+    case["k_cache"] = k.to(case["k_cache"].dtype)
+    g = gpu_case(case)
+    nw, _, _ = P.multi_query_plan(len(ctx), hkv * group, hkv, d, max(ctx), max(nq), g["k_cache"].dtype)
+    assert nw == len(ctx) * hkv * (((max(nq) * group + 127) // 128 + 1) // 2)     # the query-major plan
+    got = np64(run_mq(g))
+    assert np.all(np.isfinite(got))
+    check_attn(got, oracle_mq(case))
