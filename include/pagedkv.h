@@ -132,7 +132,7 @@ int pkv_kv_cache_write(const void* k, const void* v, void* k_cache, void* v_cach
  * pkv_decode_plan -- how pkv_paged_attention_decode will divide the work.
  *   The decode streams the ordered list of (sequence, KV head, block) items
  *   through warps that each own an equal contiguous share of it (a persistent
- *   grid of one CTA per SM by default: 4 or 8 warps for 16-bit caches, 12 (8
+ *   grid of one CTA per SM by default: 8 warps for 16-bit caches, 12 (8
  *   for a GQA group above 8) for quantised ones).  A (sequence, head) pair whose
  *   blocks span several warps is merged from per-warp partial softmax results
  *   by a log-sum-exp rule.  This split is the library's choice; the pages do

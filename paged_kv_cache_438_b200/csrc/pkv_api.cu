@@ -97,7 +97,6 @@ int make_cache_map(CUtensorMap* map, const void* cache, int row_bytes, int elt, 
 }
 
 // ------------------------------------------------------------ planning --
-constexpr int kLongStreamBlocks = 256;   // streams at least this long use 4 warps with deep rings
 constexpr int kMaxCtaSmem = 227 * 1024;  // opt-in shared memory per CTA on sm_100
 
 struct Plan {
@@ -137,13 +136,14 @@ int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int r
   if (t_max >= (1LL << 31)) return fail(PKV_ERR_UNSUPPORTED, "more than 2^31 (sequence, head, block) items");
   // One CTA per SM.  Quantised caches use 12 warps (8 when a pair has more
   // than 8 columns): their conversion work per byte, not HBM, sets the pace
-  // and more warps hide its latency.  16-bit caches use 4 warps with twice
-  // the ring depth when each of 8 warps per SM would still get at least
-  // kLongStreamBlocks blocks (measured: long contexts keep HBM busiest that
-  // way, short or L2-resident work wants the extra warps).
+  // and more warps hide its latency.  16-bit caches use 8 warps.  (Measured
+  // on 32 sequences of 32k tokens: 4 warps with twice the ring depth match 8
+  // warps within 0.5 % at the full SM clock, but under the power cap's lower
+  // clocks the longer per-warp chains slow a step by ~10 % for a 6 % lower
+  // clock, where 8 warps lose under 2 % for 9 %.)
   const long long sms = sm_count();
   const bool wide = tile_cols > 8;
-  const int warps = isq(cache_dtype) ? (wide ? 8 : 12) : (t_max / (8 * sms) >= kLongStreamBlocks ? 4 : 8);
+  const int warps = isq(cache_dtype) ? (wide ? 8 : 12) : 8;
   long long nw;
   if (req_tokens > 0) {
     if (req_tokens % 16 != 0) return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d is not a multiple of 16", req_tokens);

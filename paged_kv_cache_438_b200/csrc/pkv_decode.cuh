@@ -9,7 +9,7 @@
 // Design for sm_100a (HBM-bound: every K/V byte is read once):
 //   * Work list.  All (sequence, KV head, block) triples form one ordered
 //     list (sequence-major).  Each warp of a persistent grid (one CTA per SM:
-//     4 or 8 warps for 16-bit caches, 12 for quantised ones) owns an equal contiguous
+//     8 warps for 16-bit caches, 12 for quantised ones) owns an equal contiguous
 //     share of it and streams
 //     through that share, crossing (sequence, head) boundaries without
 //     stopping its copy pipeline.  The G query heads of a KV head are served
@@ -89,13 +89,14 @@ struct DecodeTraits {
   // Quantised caches with up to 8 columns per pair run 12 warps per CTA
   // (registers capped at 168 by the launch bounds, three warps per SM
   // sub-partition): their per-block instruction stream, not HBM, sets the
-  // pace, so more warps hide more of its latency.  16-bit caches run 4 or 8,
-  // and so do 16-column pairs, whose accumulators do not fit 168 registers.
+  // pace, so more warps hide more of its latency.  16-bit caches run 8 (up
+  // to 8 are supported), and so do 16-column pairs, whose accumulators do not
+  // fit 168 registers.
   static constexpr int max_warps(int nt) { return kQuant && nt == 1 ? 12 : 8; }
   // One CTA per SM.  Its warps (chosen per call) share up to this many bytes
-  // of copy ring: 4 warps x 6 stages or 8 warps x 2 stages of 8 KiB for
-  // bf16 / fp16 at head_dim 128 (measured: the long-context stream gains
-  // from the deeper ring, the 8-warp plan loses with 3 stages); quantised
+  // of copy ring: 8 warps x 2 stages of 8 KiB for bf16 / fp16 at head_dim
+  // 128 (measured: 3 stages lose 2-5 %), or 6 stages for a launch of 4
+  // warps, which the host plan no longer chooses; quantised
   // caches 12 warps x 3 stages of 5 KiB (8-bit) or x 5 stages of 3 KiB
   // (4-bit).  The host trims the depth when a large batch's context-length
   // scan needs the shared memory.

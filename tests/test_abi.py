@@ -190,9 +190,11 @@ def test_quantised_caches_run_twelve_warps_per_sm_unless_pairs_are_wide(lib):
         assert nw == 12 * 148
         nw, _, _ = P.decode_plan(64, 256, 16, 128, 8192, code)
         assert nw == 8 * 148
-    # a 16-bit cache of the same shape: long streams, 4 warps per SM
+    # a 16-bit cache of the same shape: 8 warps per SM, long streams included
     nw, _, _ = P.decode_plan(256, 32, 32, 128, 8192, P.PKV_BF16)
-    assert nw == 4 * 148
+    assert nw == 8 * 148
+    nw, _, _ = P.decode_plan(32, 64, 8, 128, 32768, P.PKV_BF16)
+    assert nw == 8 * 148
 
 
 def test_query_major_routing_threshold_and_group(lib):
