@@ -188,49 +188,29 @@ __device__ __forceinline__ uint32_t u8pair_minus_zero(uint32_t w, uint32_t sel, 
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// (a & b) | c in one instruction.
-__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t b, uint32_t c) {
+// (a & b) ^ c in one instruction.
+__device__ __forceinline__ uint32_t and_xor(uint32_t a, uint32_t b, uint32_t c) {
   uint32_t d;
-  asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
   return d;
 }
 
 // Eight signed INT4 codes n0..n7 of w (n0 in the lowest nibble) -> four
-// fp16x2 pairs x[k] = (n_k, n_{k+4}), exactly.  u = w ^ 0x88888888 turns
-// code x into x + 8.  A nibble placed under the fp16 pattern 0x6400 in bits
-// 0-3 reads as 1024 + (x + 8): subtracting 1032 leaves x.  One placed in bits
-// 4-7 (no shift needed) reads as 1024 + 16 (x + 8): times 1/16 minus 72 leaves
-// x, in one fused multiply-add (every step exact in fp16).  Ten operations
-// per eight codes.
-__device__ __forceinline__ void i4x8_to_h2x4(uint32_t w, uint32_t (&x)[4]) {
-  const uint32_t u = w ^ 0x88888888u;
-  const uint32_t v = u >> 8;
-  const __half2 bias = __halves2half2(__ushort_as_half(0x6408), __ushort_as_half(0x6408));        // 1032
-  const __half2 sixteenth = __halves2half2(__ushort_as_half(0x2C00), __ushort_as_half(0x2C00));   // 1/16
-  const __half2 minus72 = __halves2half2(__ushort_as_half(0xD480), __ushort_as_half(0xD480));     // -72
-  uint32_t t[4] = {and_or(u, 0x000F000Fu, 0x64006400u), and_or(u, 0x00F000F0u, 0x64006400u),
-                   and_or(v, 0x000F000Fu, 0x64006400u), and_or(v, 0x00F000F0u, 0x64006400u)};
-#pragma unroll
-  for (int k = 0; k < 4; ++k) {
-    const __half2 a = *reinterpret_cast<__half2*>(&t[k]);
-    const __half2 h = (k & 1) ? __hfma2(a, sixteenth, minus72) : __hsub2(a, bias);
-    x[k] = *reinterpret_cast<const uint32_t*>(&h);
-  }
-}
-
-// The placement step of i4x8_to_h2x4 alone: x[k] = (1032 + n_k, 1032 +
-// n_{k+4}) for even k and (1152 + 16 n_k, 1152 + 16 n_{k+4}) for odd k,
-// exactly, in six operations per eight codes.  For a dot product whose
-// other operand is pre-divided by 16 at the odd positions, the biases add
-// 1032 (even) and 72 (odd) times that operand's sum, a constant the caller
-// subtracts.
+// fp16x2 pairs placed under the fp16 pattern 0x6400, exactly:
+// x[k] = (1032 + n_k, 1032 + n_{k+4}) for even k (a nibble x + 8 in bits
+// 0-3 reads as 1024 + x + 8) and (1152 + 16 n_k, 1152 + 16 n_{k+4}) for odd
+// k (a nibble in bits 4-7, no shift, reads as 1024 + 16 (x + 8)).  Flipping
+// the nibble's top bit turns x into x + 8; since the masks and 0x6400 share
+// no bits, mask, flip and exponent pattern are one three-input operation,
+// so five operations per eight codes.  For a dot product whose other operand
+// is pre-divided by 16 at the odd positions, the biases add 1032 (even) and
+// 72 (odd) times that operand's sum, a constant the caller subtracts.
 __device__ __forceinline__ void i4x8_to_h2x4_biased(uint32_t w, uint32_t (&x)[4]) {
-  const uint32_t u = w ^ 0x88888888u;
-  const uint32_t v = u >> 8;
-  x[0] = and_or(u, 0x000F000Fu, 0x64006400u);
-  x[1] = and_or(u, 0x00F000F0u, 0x64006400u);
-  x[2] = and_or(v, 0x000F000Fu, 0x64006400u);
-  x[3] = and_or(v, 0x00F000F0u, 0x64006400u);
+  const uint32_t v = w >> 8;
+  x[0] = and_xor(w, 0x000F000Fu, 0x64086408u);
+  x[1] = and_xor(w, 0x00F000F0u, 0x64806480u);
+  x[2] = and_xor(v, 0x000F000Fu, 0x64086408u);
+  x[3] = and_xor(v, 0x00F000F0u, 0x64806480u);
 }
 
 // Eight E2M1 codes of w (two per byte, low nibble first) -> four fp16x2
