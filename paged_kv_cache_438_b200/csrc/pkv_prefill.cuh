@@ -203,6 +203,27 @@ struct PrefillTraits {
   static constexpr int kSmem = kSmemUsed > 116 * 1024 ? kSmemUsed : 116 * 1024;
 };
 
+// Packed two-lane fp32 arithmetic: one instruction for two lanes (sm_100),
+// each lane rounded once as its scalar form would be.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // Two output values, round to nearest.
 template <bool kBF16>
 __device__ __forceinline__ uint32_t pack_out(float a, float b) {
@@ -570,19 +591,40 @@ __global__ void __launch_bounds__(PrefillTraits<kD>::kThreads, 1)
       // P over the upper half of S (already read into registers) with the
       // exponent base -nb; returns the row sum of the packed values
       auto emit_p = [&](float nb) {
-        float sp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        if constexpr (kBF16) {
+          // two scores per packed instruction: s * c + nb, and the row sum
+          // over the packed (truncated) probabilities
+          const float2 c2 = make_float2(c, c), nb2 = make_float2(nb, nb);
+          float2 sp2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
-        for (int q = 0; q < kN / 32; ++q) {
-          uint32_t w[16];
+          for (int q = 0; q < kN / 32; ++q) {
+            uint32_t w[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const int e = 32 * q + 2 * k;
-            w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[e], c, nb)), fast_exp2(fmaf(sv[e + 1], c, nb)));
-            sp[k & 3] += sum_p2<kBF16>(w[k]);
+            for (int k = 0; k < 16; ++k) {
+              const int e = 32 * q + 2 * k;
+              const float2 xy = fma2(make_float2(sv[e], sv[e + 1]), c2, nb2);
+              w[k] = pack_p2<true>(fast_exp2(xy.x), fast_exp2(xy.y));
+              sp2[k & 1] = add2(sp2[k & 1], make_float2(__uint_as_float(w[k] << 16),
+                                                        __uint_as_float(w[k] & 0xFFFF0000u)));
+            }
+            tmem_st16(tP + 16 * q, w);
           }
-          tmem_st16(tP + 16 * q, w);
+          return (sp2[0].x + sp2[1].x) + (sp2[0].y + sp2[1].y);
+        } else {
+          float sp[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+          for (int q = 0; q < kN / 32; ++q) {
+            uint32_t w[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              const int e = 32 * q + 2 * k;
+              w[k] = pack_p2<kBF16>(fast_exp2(fmaf(sv[e], c, nb)), fast_exp2(fmaf(sv[e + 1], c, nb)));
+              sp[k & 3] += sum_p2<kBF16>(w[k]);
+            }
+            tmem_st16(tP + 16 * q, w);
+          }
+          return (sp[0] + sp[1]) + (sp[2] + sp[3]);
         }
-        return (sp[0] + sp[1]) + (sp[2] + sp[3]);
       };
       // Common case (bf16): the base of the earlier tiles still serves.  The
       // row sum bounds every probability, so a sum of at most 2^20
