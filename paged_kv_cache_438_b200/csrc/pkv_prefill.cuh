@@ -35,8 +35,13 @@
 //     tcgen05.commit on mbarriers; every wait is bounded.
 //   * Online softmax with a lazy rescale: the exponent base of a row only
 //     moves when its max grows by more than 8 (log2 units), and only then is
-//     that row's O rescaled in TMEM.  Unmasked tiles skip the mask; the
-//     softmax scale is folded into one FMA per score.
+//     that row's O rescaled in TMEM.  With bf16 probabilities a tile is
+//     first computed against the current base without taking its maximum
+//     (the row sum bounds every probability; a sum above 2^20 takes the
+//     maximum and writes P again).  Unmasked tiles skip the mask; the
+//     softmax scale is folded into one FMA per score, two scores per packed
+//     f32x2 instruction.  tcgen05.ld / st / wait are warp-wide, so every
+//     branch around them is decided per warp.
 //   * Tokens of a sequence's last block beyond its context were never
 //     written: the load warp zeroes their V rows in the entry before P . V
 //     reads them; blocks past the context are loaded from outside the tensor
