@@ -122,6 +122,8 @@ size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 // is spread over the warps of the resident CTAs (one CTA per SM: a
 // persistent grid) but never thinner than 16 blocks per warp;
 // partition_tokens > 0 instead caps the items per warp at partition_tokens / 16.
+int decode_warps(int cache_dtype, int D, bool wide, int B);
+
 int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int req_tokens, Plan* out,
               int max_q = 0) {
   const int G = Hq / Hkv;
@@ -140,10 +142,12 @@ int make_plan(int B, int Hq, int Hkv, int D, int max_ctx, int cache_dtype, int r
   // on 32 sequences of 32k tokens: 4 warps with twice the ring depth match 8
   // warps within 0.5 % at the full SM clock, but under the power cap's lower
   // clocks the longer per-warp chains slow a step by ~10 % for a 6 % lower
-  // clock, where 8 warps lose under 2 % for 9 %.)
+  // clock, where 8 warps lose under 2 % for 9 %.)  Fewer warps take a
+  // batch whose context-length scan would not fit beside their smallest
+  // rings (decode_warps).
   const long long sms = sm_count();
   const bool wide = tile_cols > 8;
-  const int warps = isq(cache_dtype) ? (wide ? 8 : 12) : 8;
+  const int warps = decode_warps(cache_dtype, D, wide, B);
   long long nw;
   if (req_tokens > 0) {
     if (req_tokens % 16 != 0) return fail(PKV_ERR_INVALID_ARG, "partition_tokens %d is not a multiple of 16", req_tokens);
@@ -264,6 +268,38 @@ int decode_ring(int num_seqs, int warps) {
   int r = std::max(2, std::min(8, Tr::ring_budget(warps) / (warps * Tr::kStageBytes)));
   while (r > 2 && decode_smem_bytes<kD, kCT>(num_seqs, warps, r) > static_cast<size_t>(kMaxCtaSmem)) --r;
   return r;
+}
+
+// Shared memory of a CTA of `warps` warps with two-stage rings (the fewest
+// the kernel runs with) beside the scan of B sequences.
+template <int kD>
+size_t min_decode_smem(int cache_dtype, int warps, int B) {
+  switch (cache_dtype) {
+    case PKV_F16: return decode_smem_bytes<kD, PKV_F16>(B, warps, 2);
+    case PKV_BF16: return decode_smem_bytes<kD, PKV_BF16>(B, warps, 2);
+    case PKV_I8: return decode_smem_bytes<kD, PKV_I8>(B, warps, 2);
+    case PKV_FP8E4M3: return decode_smem_bytes<kD, PKV_FP8E4M3>(B, warps, 2);
+    case PKV_U8ASYM: return decode_smem_bytes<kD, PKV_U8ASYM>(B, warps, 2);
+    case PKV_I4: return decode_smem_bytes<kD, PKV_I4>(B, warps, 2);
+    case PKV_FP4E2M1: return decode_smem_bytes<kD, PKV_FP4E2M1>(B, warps, 2);
+    default: return 0;
+  }
+}
+
+// Warps per decode CTA: 12 for quantised caches (8 when a pair has more than
+// 8 columns), 8 for 16-bit ones; 4 fewer at a time while the context-length
+// scan of a very large batch would not fit beside those warps' two-stage
+// rings (16-bit caches at head_dim 128: above ~25,000 sequences with 8 warps,
+// ~41,000 with 4).
+int decode_warps(int cache_dtype, int D, bool wide, int B) {
+  int w = isq(cache_dtype) ? (wide ? 8 : 12) : 8;
+  while (w > 4) {
+    const size_t need = D == 128 ? min_decode_smem<128>(cache_dtype, w, std::max(B, 1))
+                                 : min_decode_smem<64>(cache_dtype, w, std::max(B, 1));
+    if (need <= static_cast<size_t>(kMaxCtaSmem)) break;
+    w -= 4;
+  }
+  return w;
 }
 
 template <int kD, int kCT, int kNT, bool kQBF16, bool kMQ>

@@ -197,6 +197,22 @@ def test_quantised_caches_run_twelve_warps_per_sm_unless_pairs_are_wide(lib):
     assert nw == 8 * 148
 
 
+def test_very_large_batches_step_down_to_fewer_warps(lib):
+    # a decode CTA holds the context-length scan ((B + 1) x 4 bytes) beside
+    # its warps' rings: 16-bit caches at head_dim 128 keep 8 warps up to
+    # ~25,000 sequences and run 4 beyond
+    nw, _, _ = P.decode_plan(20000, 8, 8, 128, 1024, P.PKV_BF16)
+    assert nw == 8 * 148
+    nw, _, _ = P.decode_plan(30000, 8, 8, 128, 1024, P.PKV_BF16)
+    assert nw == 4 * 148
+    # head_dim 64 rings are half the size: 8 warps still fit
+    nw, _, _ = P.decode_plan(30000, 8, 8, 64, 1024, P.PKV_BF16)
+    assert nw == 8 * 148
+    # quantised caches step from 12 warps to 8
+    nw, _, _ = P.decode_plan(30000, 32, 32, 128, 1024, P.PKV_I8)
+    assert nw == 8 * 148
+
+
 def test_query_major_routing_threshold_and_group(lib):
     def mq(hq, d, n, cd=P.PKV_BF16):
         return P.multi_query_plan(2, hq, 8, d, 1024, n, cd)[0]

@@ -388,6 +388,24 @@ def test_decode_full_workload_sampled(name, kind, n):
         assert float(o.abs().max()) <= float(g["v_cache"].float().abs().max()) + 1e-2
 
 
+def test_decode_batch_beyond_the_eight_warp_scan_limit():
+    """30,000 sequences of 0-16 tokens (at most one block each, some empty):
+    the context-length scan of the batch no longer fits beside 8 warps'
+    rings at head_dim 128, so the plan runs 4 warps per CTA.  Sampled
+    outputs against the oracle; empty sequences give zero rows."""
+    B = 30000
+    ctx = np.random.default_rng(31).integers(0, 17, B).astype(np.int32)
+    g = I.device_decode_case("llama3_8b", DEV, batch=B, ctx_override=ctx)
+    nw, _, _ = P.decode_plan(B, g["hq"], g["hkv"], g["d"], 16, P.PKV_BF16)
+    assert nw == 4 * 148
+    out = run_decode(g, max_context_len=16)
+    pairs = _sample_pairs(B, g["hq"], 64, seed=5)
+    pairs += [(int(s), 3) for s in np.flatnonzero(ctx == 0)[:4]]
+    got = np.stack([np64(out[s, i]) for s, i in pairs])
+    check_attn(got, oracle_sampled(g, pairs))
+    assert torch.isfinite(out.float()).all()
+
+
 # --------------------------------------------------------- end to end ------
 
 def test_prefix_sharing_copy_on_write_end_to_end():
