@@ -96,10 +96,10 @@ struct DecodeTraits {
   // One CTA per SM.  Its warps (chosen per call) share up to this many bytes
   // of copy ring: 8 warps x 2 stages of 8 KiB for bf16 / fp16 at head_dim
   // 128 (measured: 3 stages lose 2-5 %), or 6 stages for a launch of 4
-  // warps, which the host plan no longer chooses; quantised
-  // caches 12 warps x 3 stages of 5 KiB (8-bit) or x 5 stages of 3 KiB
-  // (4-bit).  The host trims the depth when a large batch's context-length
-  // scan needs the shared memory.
+  // warps (the plan's choice for batches whose scan leaves no room for 8);
+  // quantised caches 12 warps x 3 stages of 5 KiB (8-bit) or x 5 stages of
+  // 3 KiB (4-bit).  The host trims the depth when a large batch's
+  // context-length scan needs the shared memory.
   static constexpr int ring_budget(int warps) { return kQuant ? 180 * 1024 : (warps <= 4 ? 192 : 128) * 1024; }
 };
 
